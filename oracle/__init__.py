@@ -1,0 +1,155 @@
+"""fp64 CPU oracle for exact attention -- TEST INFRASTRUCTURE.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of ``bench.py`` may
+import this package. It shares no code with the CUDA path: the arithmetic lives in
+``oracle.c`` (plain C, fp64, one materialised score row per query); this module only
+marshals numpy arrays.
+
+Tensors cross as raw bf16 bit patterns (``numpy.uint16``), so the oracle sees exactly the
+bits the GPU sees. Results come back as float64.
+"""
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+_LIB = None
+
+
+def _lib(path: str = None):
+    global _LIB
+    if path is not None:
+        lib = ctypes.CDLL(path)
+        _declare(lib)
+        return lib
+    if _LIB is None:
+        _LIB = ctypes.CDLL(_build.build())
+        _declare(_LIB)
+    return _LIB
+
+
+def _declare(lib):
+    p = ctypes.c_void_p
+    i32, i64, f64 = ctypes.c_int, ctypes.c_int64, ctypes.c_double
+    lib.oracle_attention.argtypes = [p, p, p, i32, i32, i32, i32, i32, i32, i32, f64, f64, p, i64,
+                                     p, p, i32]
+    lib.oracle_attention.restype = i32
+    lib.oracle_decode_paged.argtypes = [p, p, p, p, p, i32, i32, i32, i32, i32, i32, i32, f64, p, p,
+                                        i32]
+    lib.oracle_decode_paged.restype = i32
+    lib.oracle_rope_bf16.argtypes = [p, p, i64, i32, f64, p]
+    lib.oracle_rope_bf16.restype = i32
+    lib.oracle_round_bf16_array.argtypes = [p, i64, p]
+    lib.oracle_round_bf16_array.restype = None
+    lib.oracle_max_threads.argtypes = []
+    lib.oracle_max_threads.restype = i32
+
+
+def _ptr(a):
+    return ctypes.c_void_p(a.ctypes.data) if a is not None else None
+
+
+def _bits(a):
+    a = np.ascontiguousarray(a)
+    if a.dtype != np.uint16:
+        raise TypeError("oracle inputs are bf16 bit patterns (numpy.uint16), got %s" % a.dtype)
+    return a
+
+
+class OracleError(RuntimeError):
+    pass
+
+
+def max_threads(lib=None) -> int:
+    return int((lib or _lib()).oracle_max_threads())
+
+
+def attention(q, k, v, causal=False, window=0, rope_base=0.0, scale=None, rows=None,
+              nthreads=0, lib=None):
+    """Exact attention in fp64.
+
+    q: uint16 [B, Hq, N, D]; k, v: uint16 [B, Hkv, N, D] (bf16 bits).
+    rows: None for all rows, else int64 flat row ids ((b*Hq + h)*N + i).
+    Returns (o, lse): float64 [B, Hq, N, D] and [B, Hq, N], or [len(rows), D] and [len(rows)].
+    """
+    lib = lib or _lib()
+    q, k, v = _bits(q), _bits(k), _bits(v)
+    B, Hq, N, D = q.shape
+    Hkv = k.shape[1]
+    if k.shape != (B, Hkv, N, D) or v.shape != k.shape:
+        raise ValueError("k/v shape mismatch")
+    if scale is None:
+        scale = 1.0 / np.sqrt(D)
+    if rows is None:
+        n = B * Hq * N
+        rows_arr = None
+    else:
+        rows_arr = np.ascontiguousarray(rows, dtype=np.int64)
+        n = rows_arr.size
+    o = np.empty((n, D), dtype=np.float64)
+    lse = np.empty((n,), dtype=np.float64)
+    st = lib.oracle_attention(_ptr(q), _ptr(k), _ptr(v), B, Hq, Hkv, N, D, int(causal),
+                              int(window), float(rope_base), float(scale), _ptr(rows_arr),
+                              n, _ptr(o), _ptr(lse), int(nthreads))
+    if st != 0:
+        raise OracleError("oracle_attention failed with status %d" % st)
+    if rows is None:
+        return o.reshape(B, Hq, N, D), lse.reshape(B, Hq, N)
+    return o, lse
+
+
+def decode_paged(q, k_pages, v_pages, block_table, seq_lens, scale=None, nthreads=0, lib=None):
+    """One-token decode over a paged KV cache, in fp64.
+
+    q: uint16 [S, Hq, D]; k_pages, v_pages: uint16 [num_pages, Hkv, page_size, D];
+    block_table: int32 [S, max_blocks]; seq_lens: int32 [S].
+    Returns (o [S, Hq, D], lse [S, Hq]) as float64.
+    """
+    lib = lib or _lib()
+    q, k_pages, v_pages = _bits(q), _bits(k_pages), _bits(v_pages)
+    bt = np.ascontiguousarray(block_table, dtype=np.int32)
+    sl = np.ascontiguousarray(seq_lens, dtype=np.int32)
+    S, Hq, D = q.shape
+    num_pages, Hkv, page_size, D2 = k_pages.shape
+    if D2 != D or v_pages.shape != k_pages.shape or bt.shape[0] != S or sl.shape != (S,):
+        raise ValueError("decode shape mismatch")
+    if scale is None:
+        scale = 1.0 / np.sqrt(D)
+    o = np.empty((S, Hq, D), dtype=np.float64)
+    lse = np.empty((S, Hq), dtype=np.float64)
+    st = lib.oracle_decode_paged(_ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(bt), _ptr(sl), S,
+                                 bt.shape[1], num_pages, page_size, Hq, Hkv, D, float(scale),
+                                 _ptr(o), _ptr(lse), int(nthreads))
+    if st != 0:
+        raise OracleError("oracle_decode_paged failed with status %d" % st)
+    return o, lse
+
+
+def rope_bf16(x, pos, base, lib=None):
+    """Rotate rows of x (uint16 [n, D]) at positions pos (int64 [n]); returns uint16 [n, D]."""
+    lib = lib or _lib()
+    x = _bits(x)
+    n, D = x.shape
+    pos = np.ascontiguousarray(pos, dtype=np.int64)
+    out = np.empty_like(x)
+    st = lib.oracle_rope_bf16(_ptr(x), _ptr(pos), n, D, float(base), _ptr(out))
+    if st != 0:
+        raise OracleError("oracle_rope_bf16 failed with status %d" % st)
+    return out
+
+
+def round_bf16(x, lib=None):
+    """Round float64 values to bf16 (ties to even); returns the uint16 bit patterns."""
+    lib = lib or _lib()
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    out = np.empty(x.shape, dtype=np.uint16)
+    lib.oracle_round_bf16_array(_ptr(x), x.size, _ptr(out))
+    return out
+
+
+def bf16_bits_to_f64(bits):
+    """Exact value of bf16 bit patterns (plain reinterpretation, no arithmetic)."""
+    bits = np.ascontiguousarray(bits, dtype=np.uint16)
+    return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)

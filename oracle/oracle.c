@@ -1,0 +1,310 @@
+/*
+ * oracle.c -- plain, slow, fp64 CPU oracle for exact scaled dot-product attention.
+ *
+ * TEST INFRASTRUCTURE. Only the test suite, the smoke check and the benchmark's CPU-baseline
+ * leg may load this library. The CUDA product path never calls it, and the two share no code.
+ *
+ * What it computes, and the passage each step follows:
+ *   - O_i = sum_j softmax_j(q_i . k_j * scale) v_j, one query head at a time
+ *     ("attention-transformers", Q "How does self-attention work in a transformer?";
+ *      "Transformer Attention Mechanism Interview Deep Dive", "Scaled dot-product attention").
+ *   - Masks enter as -inf on the logits before the softmax
+ *     ("Transformer Attention Mechanism Interview Deep Dive", "Causal masking").
+ *     Causal: key j visible to query i iff j <= i. Sliding window of width w (always together
+ *     with causal): j in [i-w+1, i] ("attention-transformers", Q "What is sparse / sliding-window
+ *     attention?").
+ *   - Grouped-query attention: query head h reads K/V head floor(h / (Hq/Hkv))
+ *     ("Transformer Complexity, Inference Optimization, GQA and FlashAttention", Part 3).
+ *   - RoPE: pairs (2i, 2i+1) of q and k are rotated counter-clockwise by pos * base^(-2i/D)
+ *     ("attention-transformers", Q "How does Rotary Position Embedding (RoPE) work?").
+ *     The rotated values are rounded to bf16 with round-to-nearest-even, because the tensor
+ *     cores that consume them take bf16 operands.
+ *   - The saved row statistic is LSE_i = m_i + ln(l_i), natural log of the scaled scores
+ *     ("Why is attention O(n^2), how does FlashAttention help, ...", "Deep dive: FlashAttention":
+ *     the backward pass recomputes from the saved m and l).
+ *   - Paged decode gathers a sequence's cached keys/values through its block table in logical
+ *     order ("Self-Attention Complexity, FlashAttention, PagedAttention, and RoPE in Code",
+ *     Part 3: fixed-size blocks and block tables) and computes the single query row at the
+ *     sequence's last position over all seq_len cached tokens.
+ *
+ * The score row of every query is materialised in full (masked entries hold -inf), then
+ * max, exp, sum, the weighted sum of V and the logsumexp are taken -- the plain definition,
+ * with no tiling and no online rescaling.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define ORACLE_OK 0
+#define ORACLE_ERR_ARG 1
+#define ORACLE_ERR_INDEX 2
+#define ORACLE_ERR_NOMEM 3
+
+/* bf16 bit pattern -> its exact value. A bf16 number is the top 16 bits of an IEEE binary32. */
+static double bf16_value(uint16_t bits) {
+    uint32_t u = (uint32_t)bits << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/* Round a double to the nearest bf16 (8 significant bits, exponent range of binary32), ties to
+ * even, in one step (no intermediate rounding to binary32). Returns the bf16 bit pattern. */
+uint16_t oracle_round_bf16(double x) {
+    if (isnan(x)) return 0x7FC0u;
+    uint16_t sign = signbit(x) ? 0x8000u : 0u;
+    double ax = fabs(x);
+    if (ax == 0.0) return sign;
+    /* Largest finite bf16 is (2 - 2^-7) * 2^127; halfway to the next binade rounds to inf
+     * because the largest mantissa is odd. */
+    const double max_finite = ldexp(2.0 - ldexp(1.0, -7), 127);
+    const double overflow_edge = ldexp(2.0 - ldexp(1.0, -8), 127);
+    if (ax >= overflow_edge) return (uint16_t)(sign | 0x7F80u);
+    int ex;
+    frexp(ax, &ex);                 /* ax in [2^(ex-1), 2^ex) */
+    int qexp = ex - 8;              /* quantum of an 8-significant-bit number in that binade */
+    if (qexp < -133) qexp = -133;   /* subnormal quantum of binary32/bf16 */
+    double r = nearbyint(ldexp(ax, -qexp));   /* default rounding mode: to nearest, ties even */
+    double y = ldexp(r, qexp);
+    if (y > max_finite) return (uint16_t)(sign | 0x7F80u);
+    float yf = (float)y;            /* exact: y has at most 8 significant bits */
+    uint32_t u;
+    memcpy(&u, &yf, sizeof u);
+    return (uint16_t)(sign | (uint16_t)((u >> 16) & 0x7FFFu));
+}
+
+/* RoPE on one head vector x[0..D) at position pos, pairs (2i, 2i+1), angle pos * base^(-2i/D),
+ * counter-clockwise: (x0 cos - x1 sin, x0 sin + x1 cos). Result rounded to bf16, returned as
+ * exact doubles. base <= 0 means no rotation (values passed through exactly). */
+static void rope_row(const uint16_t* x, int D, long pos, double base, double* out) {
+    if (base <= 0.0) {
+        for (int d = 0; d < D; ++d) out[d] = bf16_value(x[d]);
+        return;
+    }
+    for (int i = 0; i < D / 2; ++i) {
+        double theta = pow(base, -2.0 * (double)i / (double)D);
+        double angle = (double)pos * theta;
+        double c = cos(angle), s = sin(angle);
+        double x0 = bf16_value(x[2 * i]), x1 = bf16_value(x[2 * i + 1]);
+        out[2 * i] = bf16_value(oracle_round_bf16(x0 * c - x1 * s));
+        out[2 * i + 1] = bf16_value(oracle_round_bf16(x0 * s + x1 * c));
+    }
+}
+
+/* Exposed for the pins: rotate n_rows rows of length D; row r sits at position pos[r]. */
+int oracle_rope_bf16(const uint16_t* x, const int64_t* pos, int64_t n_rows, int D, double base,
+                     uint16_t* out) {
+    if (!x || !pos || !out || D <= 0 || (D % 2) != 0 || n_rows < 0) return ORACLE_ERR_ARG;
+    double* tmp = (double*)malloc(sizeof(double) * (size_t)D);
+    if (!tmp) return ORACLE_ERR_NOMEM;
+    for (int64_t r = 0; r < n_rows; ++r) {
+        rope_row(x + r * D, D, (long)pos[r], base, tmp);
+        for (int d = 0; d < D; ++d) out[r * D + d] = oracle_round_bf16(tmp[d]);
+    }
+    free(tmp);
+    return ORACLE_OK;
+}
+
+/* One query row against keys/values already converted to doubles.
+ * q[D]; kk, vv: [N, D]; writes o[D] and *lse. Masked keys get score -inf. */
+static void attend_row(const double* q, const double* kk, const double* vv, int N, int D,
+                       long i, int causal, int window, double scale, double* s_row, double* o,
+                       double* lse) {
+    for (int j = 0; j < N; ++j) {
+        int visible = 1;
+        if (causal && j > i) visible = 0;
+        if (window > 0 && (long)j < i - window + 1) visible = 0;
+        if (!visible) {
+            s_row[j] = -INFINITY;
+            continue;
+        }
+        double acc = 0.0;
+        for (int d = 0; d < D; ++d) acc += q[d] * kk[(size_t)j * D + d];
+        s_row[j] = acc * scale;
+    }
+    double m = -INFINITY;
+    for (int j = 0; j < N; ++j)
+        if (s_row[j] > m) m = s_row[j];
+    for (int d = 0; d < D; ++d) o[d] = 0.0;
+    if (m == -INFINITY) { /* no visible key: defined as O = 0, LSE = -inf */
+        *lse = -INFINITY;
+        return;
+    }
+    double l = 0.0;
+    for (int j = 0; j < N; ++j) {
+        double p = exp(s_row[j] - m); /* exp(-inf) == 0 for masked keys */
+        s_row[j] = p;
+        l += p;
+    }
+    for (int j = 0; j < N; ++j) {
+        double p = s_row[j];
+        if (p == 0.0) continue;
+        const double* vj = vv + (size_t)j * D;
+        for (int d = 0; d < D; ++d) o[d] += p * vj[d];
+    }
+    for (int d = 0; d < D; ++d) o[d] /= l;
+    *lse = m + log(l);
+}
+
+/*
+ * Prefill attention. q: bf16 [B, Hq, N, D]; k, v: bf16 [B, Hkv, N, D] (contiguous).
+ * rows: NULL for every row, else n_rows flat row ids ((b*Hq + h)*N + i).
+ * o: [n_rows, D] (or [B*Hq*N, D]); lse: [n_rows] (or [B*Hq*N]). Query i sits at position i.
+ */
+int oracle_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, int B, int Hq,
+                     int Hkv, int N, int D, int causal, int window, double rope_base,
+                     double scale, const int64_t* rows, int64_t n_rows, double* o, double* lse,
+                     int nthreads) {
+    if (!q || !k || !v || !o || !lse) return ORACLE_ERR_ARG;
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || N <= 0 || D <= 0 || Hq % Hkv != 0) return ORACLE_ERR_ARG;
+    if (window > 0 && !causal) return ORACLE_ERR_ARG;
+    if (rope_base > 0.0 && (D % 2) != 0) return ORACLE_ERR_ARG;
+    const int G = Hq / Hkv;
+    const int64_t total = (int64_t)B * Hq * N;
+    if (rows == NULL) n_rows = total;
+    for (int64_t r = 0; rows && r < n_rows; ++r)
+        if (rows[r] < 0 || rows[r] >= total) return ORACLE_ERR_INDEX;
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#else
+    (void)nthreads;
+#endif
+    double* kk = (double*)malloc(sizeof(double) * (size_t)N * D);
+    double* vv = (double*)malloc(sizeof(double) * (size_t)N * D);
+    if (!kk || !vv) {
+        free(kk);
+        free(vv);
+        return ORACLE_ERR_NOMEM;
+    }
+    int status = ORACLE_OK;
+    /* One K/V head at a time: rotate its keys once, then every requested query row that
+     * reads it. */
+    for (int b = 0; b < B && status == ORACLE_OK; ++b) {
+        for (int g = 0; g < Hkv && status == ORACLE_OK; ++g) {
+            int needed = 0;
+            for (int64_t r = 0; r < n_rows && !needed; ++r) {
+                int64_t id = rows ? rows[r] : r;
+                int rb = (int)(id / ((int64_t)Hq * N));
+                int rh = (int)((id / N) % Hq);
+                if (rb == b && rh / G == g) needed = 1;
+            }
+            if (!needed) continue;
+            const size_t kv_off = ((size_t)b * Hkv + g) * (size_t)N * D;
+#pragma omp parallel for schedule(static)
+            for (int j = 0; j < N; ++j) {
+                rope_row(k + kv_off + (size_t)j * D, D, j, rope_base, kk + (size_t)j * D);
+                for (int d = 0; d < D; ++d) vv[(size_t)j * D + d] = bf16_value(v[kv_off + (size_t)j * D + d]);
+            }
+#pragma omp parallel
+            {
+                double* s_row = (double*)malloc(sizeof(double) * (size_t)N);
+                double* qq = (double*)malloc(sizeof(double) * (size_t)D);
+                if (!s_row || !qq) {
+#pragma omp atomic write
+                    status = ORACLE_ERR_NOMEM;
+                } else {
+#pragma omp for schedule(dynamic, 16)
+                    for (int64_t r = 0; r < n_rows; ++r) {
+                        int64_t id = rows ? rows[r] : r;
+                        int rb = (int)(id / ((int64_t)Hq * N));
+                        int rh = (int)((id / N) % Hq);
+                        long i = (long)(id % N);
+                        if (rb != b || rh / G != g) continue;
+                        rope_row(q + (size_t)id * D, D, i, rope_base, qq);
+                        attend_row(qq, kk, vv, N, D, i, causal, window, scale, s_row,
+                                   o + (size_t)r * D, lse + r);
+                    }
+                }
+                free(s_row);
+                free(qq);
+            }
+        }
+    }
+    free(kk);
+    free(vv);
+    return status;
+}
+
+/*
+ * Paged decode: one query token per sequence, attending to all seq_lens[s] cached tokens.
+ * q: bf16 [S, Hq, D] (taken as already rotated); k_pages, v_pages: bf16
+ * [num_pages, Hkv, page_size, D]; block_table: [S, max_blocks]; seq_lens: [S].
+ * Token t of sequence s lives in page block_table[s][t / page_size], slot t % page_size.
+ * o: [S, Hq, D]; lse: [S, Hq].
+ */
+int oracle_decode_paged(const uint16_t* q, const uint16_t* k_pages, const uint16_t* v_pages,
+                        const int32_t* block_table, const int32_t* seq_lens, int S,
+                        int max_blocks, int num_pages, int page_size, int Hq, int Hkv, int D,
+                        double scale, double* o, double* lse, int nthreads) {
+    if (!q || !k_pages || !v_pages || !block_table || !seq_lens || !o || !lse) return ORACLE_ERR_ARG;
+    if (S <= 0 || max_blocks <= 0 || num_pages <= 0 || page_size <= 0 || Hq <= 0 || Hkv <= 0 ||
+        D <= 0 || Hq % Hkv != 0)
+        return ORACLE_ERR_ARG;
+    const int G = Hq / Hkv;
+    for (int s = 0; s < S; ++s) {
+        int len = seq_lens[s];
+        if (len < 1 || (int64_t)len > (int64_t)max_blocks * page_size) return ORACLE_ERR_INDEX;
+        int pages = (len + page_size - 1) / page_size;
+        for (int p = 0; p < pages; ++p) {
+            int32_t pg = block_table[(size_t)s * max_blocks + p];
+            if (pg < 0 || pg >= num_pages) return ORACLE_ERR_INDEX;
+        }
+    }
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#else
+    (void)nthreads;
+#endif
+    int status = ORACLE_OK;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int sg = 0; sg < S * Hkv; ++sg) {
+        int s = sg / Hkv, g = sg % Hkv;
+        int len = seq_lens[s];
+        double* kk = (double*)malloc(sizeof(double) * (size_t)len * D);
+        double* vv = (double*)malloc(sizeof(double) * (size_t)len * D);
+        double* s_row = (double*)malloc(sizeof(double) * (size_t)len);
+        double* qq = (double*)malloc(sizeof(double) * (size_t)D);
+        if (!kk || !vv || !s_row || !qq) {
+#pragma omp atomic write
+            status = ORACLE_ERR_NOMEM;
+        } else {
+            for (int t = 0; t < len; ++t) {
+                int32_t pg = block_table[(size_t)s * max_blocks + t / page_size];
+                size_t base = (((size_t)pg * Hkv + g) * page_size + (size_t)(t % page_size)) * D;
+                for (int d = 0; d < D; ++d) {
+                    kk[(size_t)t * D + d] = bf16_value(k_pages[base + d]);
+                    vv[(size_t)t * D + d] = bf16_value(v_pages[base + d]);
+                }
+            }
+            for (int hh = 0; hh < G; ++hh) {
+                int h = g * G + hh;
+                for (int d = 0; d < D; ++d) qq[d] = bf16_value(q[((size_t)s * Hq + h) * D + d]);
+                /* the query is the sequence's last token: position len-1, causal over the cache */
+                attend_row(qq, kk, vv, len, D, (long)len - 1, 1, 0, scale, s_row,
+                           o + ((size_t)s * Hq + h) * D, lse + (size_t)s * Hq + h);
+            }
+        }
+        free(kk);
+        free(vv);
+        free(s_row);
+        free(qq);
+    }
+    return status;
+}
+
+int oracle_max_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+/* Vector form of oracle_round_bf16, for the pins. */
+void oracle_round_bf16_array(const double* x, int64_t n, uint16_t* out) {
+    for (int64_t i = 0; i < n; ++i) out[i] = oracle_round_bf16(x[i]);
+}

@@ -1,0 +1,377 @@
+"""Pins of the fp64 oracle against what the pages and the mathematics fix.
+
+Each ``check_*`` function takes an oracle library handle (``oracle._lib()`` or a deliberately
+broken copy built by the mutation tests) and raises AssertionError when the oracle disagrees
+with the pin. None of them re-types the oracle's own formula: they use hand-derived values,
+closed forms of special cases, library routines (torch's float64 scaled_dot_product_attention,
+scipy's logsumexp, torch's bf16 conversion) and invariants.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import torch
+
+import oracle
+from exact_attention_161_b200 import synth
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "hand_cases.json")
+
+
+def _golden():
+    with open(GOLDEN) as f:
+        return json.load(f)
+
+
+def _to_bits(values):
+    """Exact bf16 values -> bit patterns through torch (values must be bf16-representable)."""
+    t = torch.tensor(np.asarray(values, dtype=np.float32)).to(torch.bfloat16)
+    assert np.array_equal(t.float().numpy().astype(np.float64), np.asarray(values, np.float64))
+    return t.view(torch.int16).numpy().view(np.uint16)
+
+
+def _f64(bits):
+    return oracle.bf16_bits_to_f64(bits)
+
+
+def _rand(shape, seed):
+    g = torch.Generator().manual_seed(seed)
+    return synth.bits(synth.randn_bf16(shape, g))
+
+
+def _sdpa64(q, k, v, scale, causal=False, mask=None, gqa=False):
+    """torch's float64 CPU scaled_dot_product_attention (a library routine)."""
+    qt, kt, vt = (torch.from_numpy(_f64(x)) for x in (q, k, v))
+    return torch.nn.functional.scaled_dot_product_attention(
+        qt, kt, vt, attn_mask=mask, is_causal=causal, scale=scale, enable_gqa=gqa).numpy()
+
+
+# ---------------------------------------------------------------------------------- rounding
+
+def check_round_bf16_golden(lib):
+    for case in _golden()["bf16_rounding"]["cases"]:
+        got = int(oracle.round_bf16(np.array([case["x"]]), lib=lib)[0])
+        assert got == case["bits"], (case, got)
+
+
+def check_round_bf16_matches_torch(lib):
+    """On binary32 inputs (no double rounding possible) the result must equal torch's RNE
+    float32 -> bfloat16 conversion, ties included."""
+    rng = np.random.default_rng(7)
+    x = rng.standard_normal(20000).astype(np.float32) * np.float32(3.0)
+    u = x.view(np.uint32).copy()
+    u[:2000] = (u[:2000] & 0xFFFF0000) | 0x8000       # exact ties
+    u[2000:4000] = (u[2000:4000] & 0xFFFF0000) | 0x7FFF
+    u[4000:6000] = (u[4000:6000] & 0xFFFF0000) | 0x8001
+    x = u.view(np.float32)
+    want = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    got = oracle.round_bf16(x.astype(np.float64), lib=lib)
+    assert np.array_equal(got, want)
+
+
+# ---------------------------------------------------------------------------------- RoPE
+
+def check_rope_golden(lib):
+    g = _golden()["rope_d4"]
+    for case in g["cases"]:
+        x = _to_bits(case["x"])[None, :]
+        got = _f64(oracle.rope_bf16(x, np.array([case["pos"]]), g["base"], lib=lib))[0]
+        assert np.array_equal(got, np.asarray(case["bf16"])), (case, got)
+
+
+def check_rope_matches_sinusoid(lib):
+    """Rotating (1,0) gives (cos, sin) of the angle and rotating (0,1) gives (-sin, cos). With
+    base 10000 the angles are those of the sinusoidal encoding PE(pos,2i) = sin(pos/10000^(2i/d))
+    ("attention-transformers", Q "Explain sinusoidal positional encoding"), evaluated here with
+    numpy and rounded to bf16 by torch."""
+    D = 64
+    pos = np.array([0, 1, 7, 100, 2047, 30000], dtype=np.int64)
+    i = np.arange(D // 2)
+    pe_sin = np.sin(pos[:, None] / np.power(10000.0, 2 * i[None, :] / D))
+    pe_cos = np.cos(pos[:, None] / np.power(10000.0, 2 * i[None, :] / D))
+    for x_pair, want0, want1 in (((1.0, 0.0), pe_cos, pe_sin), ((0.0, 1.0), -pe_sin, pe_cos)):
+        x = _to_bits(np.tile(np.array(x_pair), (len(pos), D // 2)))
+        got = _f64(oracle.rope_bf16(x, pos, 10000.0, lib=lib))
+        want = np.empty((len(pos), D))
+        want[:, 0::2], want[:, 1::2] = want0, want1
+        want_bf16 = torch.from_numpy(want).to(torch.bfloat16).double().numpy()
+        # torch rounds float64 -> bf16 directly; allow one bf16 ulp for the last-bit angle
+        # difference between numpy's and libm's sin/cos.
+        assert np.allclose(got, want_bf16, rtol=2.0 ** -7, atol=2.0 ** -14), np.abs(got - want_bf16).max()
+
+
+def check_rope_norm_and_identity(lib):
+    x = _rand((64, 128), 11)
+    pos0 = np.zeros(64, dtype=np.int64)
+    assert np.array_equal(oracle.rope_bf16(x, pos0, 10000.0, lib=lib), x)
+    pos = np.arange(64, dtype=np.int64) * 517
+    y = _f64(oracle.rope_bf16(x, pos, 500000.0, lib=lib))
+    xn = np.linalg.norm(_f64(x).reshape(64, 64, 2), axis=2)
+    yn = np.linalg.norm(y.reshape(64, 64, 2), axis=2)
+    # each pair keeps its length up to the two bf16 roundings
+    assert np.all(np.abs(yn - xn) <= 2.0 ** -7 * xn + 1e-30)
+
+
+def check_rope_relative(lib):
+    """(R_i q).(R_j k) depends only on i - j ("How does Rotary Position Embedding (RoPE) work?");
+    up to the bf16 rounding of the rotated values."""
+    D = 128
+    q = _rand((1, D), 12)
+    k = _rand((1, D), 13)
+    base = 10000.0
+    for i, j, t in ((5, 2, 1000), (100, 0, 7), (40, 90, 3000)):
+        a = _f64(oracle.rope_bf16(q, np.array([i]), base, lib=lib)) @ _f64(oracle.rope_bf16(k, np.array([j]), base, lib=lib)).T
+        b = _f64(oracle.rope_bf16(q, np.array([i + t]), base, lib=lib)) @ _f64(oracle.rope_bf16(k, np.array([j + t]), base, lib=lib)).T
+        bound = 2.0 ** -6 * np.linalg.norm(_f64(q)) * np.linalg.norm(_f64(k))
+        assert abs(a - b) <= bound, (i, j, t, a, b)
+
+
+# ---------------------------------------------------------------------------------- prefill
+
+def check_hand_two_tokens(lib):
+    c = _golden()["sdpa_two_tokens"]
+    q = _to_bits(c["q"]).reshape(1, 1, 1, 2)
+    k = _to_bits(c["k"]).reshape(1, 1, 2, 2)
+    v = _to_bits(c["v"]).reshape(1, 1, 2, 2)
+    # a 2-token sequence whose two queries are both q
+    q2 = np.concatenate([q, q], axis=2)
+    o, lse = oracle.attention(q2, k, v, causal=False, scale=c["scale"], lib=lib)
+    assert np.allclose(o[0, 0, 0], c["o_full"], atol=1e-8) and abs(lse[0, 0, 0] - c["lse_full"]) < 1e-8
+    o, lse = oracle.attention(q2, k, v, causal=True, scale=c["scale"], lib=lib)
+    assert np.allclose(o[0, 0, 0], c["o_causal_row0"], atol=0) and abs(lse[0, 0, 0] - c["lse_causal_row0"]) < 1e-8
+    assert np.allclose(o[0, 0, 1], c["o_full"], atol=1e-8) and abs(lse[0, 0, 1] - c["lse_full"]) < 1e-8
+
+
+def check_library_sdpa(lib):
+    """Without RoPE the oracle must agree with torch's float64 SDPA: the single-head N=128 d=64
+    workload, and a two-batch four-head slice of the N=2048 d=128 causal workload."""
+    q, k, v = (synth.bits(t) for t in synth.prefill_inputs(1, 1, 1, 128, 64, 1001))
+    for causal in (False, True):
+        o, _ = oracle.attention(q, k, v, causal=causal, scale=0.125, lib=lib)
+        ref = _sdpa64(q, k, v, 0.125, causal=causal)
+        assert np.abs(o - ref).max() < 1e-12
+    q, k, v = (synth.bits(t) for t in synth.prefill_inputs(2, 4, 4, 512, 128, 1002))
+    o, _ = oracle.attention(q, k, v, causal=True, scale=128 ** -0.5, lib=lib)
+    ref = _sdpa64(q, k, v, 128 ** -0.5, causal=True)
+    assert np.abs(o - ref).max() < 1e-12
+
+
+def check_library_window(lib):
+    N, w = 200, 37
+    q, k, v = (synth.bits(t) for t in synth.prefill_inputs(1, 2, 2, N, 64, 21))
+    i = np.arange(N)[:, None]
+    j = np.arange(N)[None, :]
+    mask = torch.from_numpy((j <= i) & (j >= i - w + 1))
+    o, _ = oracle.attention(q, k, v, causal=True, window=w, scale=0.125, lib=lib)
+    ref = _sdpa64(q, k, v, 0.125, mask=mask)
+    assert np.abs(o - ref).max() < 1e-12
+
+
+def check_library_gqa(lib):
+    """Query head h reads K/V head h // (Hq/Hkv): the convention of torch's enable_gqa."""
+    q = _rand((2, 8, 96, 64), 31).reshape(2, 8, 96, 64)
+    k = _rand((2, 2, 96, 64), 32).reshape(2, 2, 96, 64)
+    v = _rand((2, 2, 96, 64), 33).reshape(2, 2, 96, 64)
+    o, _ = oracle.attention(q, k, v, causal=True, scale=0.125, lib=lib)
+    ref = _sdpa64(q, k, v, 0.125, causal=True, gqa=True)
+    assert np.abs(o - ref).max() < 1e-12
+
+
+def check_gqa_reduces_to_mha(lib):
+    """GQA equals MHA on K/V repeated per group; Hkv = Hq is MHA; Hkv = 1 is MQA
+    ("Transformer Complexity, Inference Optimization, GQA and FlashAttention", Part 3)."""
+    q = _rand((1, 8, 64, 64), 41).reshape(1, 8, 64, 64)
+    for hkv in (1, 2, 8):
+        k = _rand((1, hkv, 64, 64), 42).reshape(1, hkv, 64, 64)
+        v = _rand((1, hkv, 64, 64), 43).reshape(1, hkv, 64, 64)
+        o, lse = oracle.attention(q, k, v, causal=True, rope_base=10000.0, scale=0.125, lib=lib)
+        kr, vr = np.repeat(k, 8 // hkv, axis=1), np.repeat(v, 8 // hkv, axis=1)
+        o2, lse2 = oracle.attention(q, kr, vr, causal=True, rope_base=10000.0, scale=0.125, lib=lib)
+        assert np.array_equal(o, o2) and np.array_equal(lse, lse2)
+
+
+def check_lse_library(lib):
+    """LSE = ln sum exp(scaled scores) over the visible keys, via scipy's logsumexp."""
+    from scipy.special import logsumexp
+    N, D = 150, 64
+    q, k, v = (synth.bits(t) for t in synth.prefill_inputs(1, 1, 1, N, D, 51))
+    _, lse = oracle.attention(q, k, v, causal=True, window=60, scale=0.125, lib=lib)
+    s = (_f64(q[0, 0]) @ _f64(k[0, 0]).T) * 0.125
+    i = np.arange(N)[:, None]
+    j = np.arange(N)[None, :]
+    s = np.where((j <= i) & (j >= i - 59), s, -np.inf)
+    assert np.abs(lse[0, 0] - logsumexp(s, axis=1)).max() < 1e-12
+
+
+def check_probability_rows(lib):
+    """With V = identity (D = N) row i of O is row i of P. Every row sums to 1 and every masked
+    entry is exactly 0 -- the mask acts on the logits before the softmax
+    ("Transformer Attention Mechanism Interview Deep Dive", "Causal masking")."""
+    N = 32
+    q = _rand((1, 1, N, N), 61).reshape(1, 1, N, N)
+    k = _rand((1, 1, N, N), 62).reshape(1, 1, N, N)
+    v = _to_bits(np.eye(N)).reshape(1, 1, N, N)
+    for causal, window in ((False, 0), (True, 0), (True, 5)):
+        p, _ = oracle.attention(q, k, v, causal=causal, window=window, scale=1 / math.sqrt(N), lib=lib)
+        p = p[0, 0]
+        assert np.abs(p.sum(axis=1) - 1.0).max() < 1e-12
+        i = np.arange(N)[:, None]
+        j = np.arange(N)[None, :]
+        visible = np.ones((N, N), bool)
+        if causal:
+            visible &= j <= i
+        if window:
+            visible &= j >= i - window + 1
+        assert np.all(p[~visible] == 0.0) and np.all(p[visible] > 0.0)
+        # number of attended pairs: N^2, N(N+1)/2, or sum_i min(i+1, w) (window cost O(n*w))
+        want = N * N if not causal else sum(min(r + 1, window or N) for r in range(N))
+        assert int((p > 0).sum()) == want
+
+
+def check_permutation_equivariance(lib):
+    """Without position information and without a mask, permuting the tokens permutes the
+    outputs the same way ("attention-transformers", Q "Why does a transformer need positional
+    encoding?")."""
+    N = 64
+    q, k, v = (synth.bits(t) for t in synth.prefill_inputs(1, 2, 2, N, 64, 71))
+    perm = np.random.default_rng(3).permutation(N)
+    o, lse = oracle.attention(q, k, v, scale=0.125, lib=lib)
+    op, lsep = oracle.attention(q[:, :, perm], k[:, :, perm], v[:, :, perm], scale=0.125, lib=lib)
+    assert np.abs(op - o[:, :, perm]).max() < 1e-13 and np.abs(lsep - lse[:, :, perm]).max() < 1e-13
+
+
+def check_causal_row0_and_window1(lib):
+    N = 48
+    q, k, v = (synth.bits(t) for t in synth.prefill_inputs(1, 3, 3, N, 64, 81))
+    o, lse = oracle.attention(q, k, v, causal=True, rope_base=10000.0, scale=0.125, lib=lib)
+    assert np.array_equal(o[:, :, 0], _f64(v[:, :, 0]))
+    s00 = np.einsum("bhd,bhd->bh", _f64(q[:, :, 0]), _f64(k[:, :, 0])) * 0.125  # pos 0: no rotation
+    assert np.abs(lse[:, :, 0] - s00).max() < 1e-13
+    o1, _ = oracle.attention(q, k, v, causal=True, window=1, rope_base=10000.0, scale=0.125, lib=lib)
+    assert np.array_equal(o1, _f64(v))
+    ow, lsew = oracle.attention(q, k, v, causal=True, window=N, rope_base=10000.0, scale=0.125, lib=lib)
+    assert np.array_equal(ow, o) and np.array_equal(lsew, lse)
+
+
+def check_equal_scores(lib):
+    """q = 0 gives equal scores: O_i is the mean of the visible values, LSE_i = ln(count)."""
+    N = 40
+    _, k, v = (synth.bits(t) for t in synth.prefill_inputs(1, 1, 1, N, 64, 91))
+    q = np.zeros((1, 1, N, 64), dtype=np.uint16)
+    o, lse = oracle.attention(q, k, v, causal=True, scale=0.125, lib=lib)
+    vv = _f64(v[0, 0])
+    means = np.cumsum(vv, axis=0) / np.arange(1, N + 1)[:, None]
+    assert np.abs(o[0, 0] - means).max() < 1e-13
+    assert np.abs(lse[0, 0] - np.log(np.arange(1, N + 1))).max() < 1e-13
+
+
+def check_rows_subset(lib):
+    """Row-sampled evaluation returns exactly the rows of the full evaluation."""
+    q, k, v = (synth.bits(t) for t in synth.prefill_inputs(2, 4, 2, 100, 64, 95))
+    o, lse = oracle.attention(q, k, v, causal=True, window=30, rope_base=10000.0, scale=0.125, lib=lib)
+    rows = np.array([0, 99, 100, 357, 799, 401], dtype=np.int64)
+    os_, ls_ = oracle.attention(q, k, v, causal=True, window=30, rope_base=10000.0, scale=0.125,
+                                rows=rows, lib=lib)
+    assert np.array_equal(os_, o.reshape(-1, 64)[rows]) and np.array_equal(ls_, lse.reshape(-1)[rows])
+
+
+def online_softmax_reference(q, k, v, scale, block, causal):
+    """The pages' streaming recurrence ("Why is attention O(n^2), how does FlashAttention help,
+    ...", "Deep dive: FlashAttention"), in fp64, one K/V block at a time. Test-only."""
+    N = q.shape[0]
+    m = np.full(N, -np.inf)
+    l = np.zeros(N)
+    o = np.zeros_like(q)
+    for j0 in range(0, N, block):
+        kb, vb = k[j0:j0 + block], v[j0:j0 + block]
+        s = q @ kb.T * scale
+        if causal:
+            s = np.where(np.arange(j0, j0 + kb.shape[0])[None, :] <= np.arange(N)[:, None], s, -np.inf)
+        m_new = np.maximum(m, s.max(axis=1))
+        p = np.exp(s - m_new[:, None])
+        alpha = np.exp(m - m_new)
+        l = alpha * l + p.sum(axis=1)
+        o = alpha[:, None] * o + p @ vb
+        m = m_new
+    return o / l[:, None], m + np.log(l)
+
+
+def check_online_recurrence(lib):
+    """The tiled recurrence reaches the materialised result up to rounding, for any block size
+    ("Exact: the rescaling makes the result identical to a full softmax")."""
+    N, D = 130, 64
+    q, k, v = (synth.bits(t) for t in synth.prefill_inputs(1, 1, 1, N, D, 97))
+    o, lse = oracle.attention(q, k, v, causal=True, scale=0.125, lib=lib)
+    for block in (1, 3, 16, 128, N):
+        ob, lseb = online_softmax_reference(_f64(q[0, 0]), _f64(k[0, 0]), _f64(v[0, 0]), 0.125, block, True)
+        assert np.abs(ob - o[0, 0]).max() < 1e-12 and np.abs(lseb - lse[0, 0]).max() < 1e-12
+
+
+# ---------------------------------------------------------------------------------- decode
+
+def _small_cache(seed=5, permute=True, poison=True, lens=(1, 15, 16, 17, 40, 33)):
+    return synth.paged_decode_inputs(len(lens), 8, 2, 64, 16, seq_lens=list(lens), spare_frac=0.5,
+                                     seed=seed, permute=permute, poison=poison)
+
+
+def _decode(cache, lib):
+    return oracle.decode_paged(synth.bits(cache.q), synth.bits(cache.k_pages), synth.bits(cache.v_pages),
+                               cache.block_table.numpy(), cache.seq_lens.numpy(), lib=lib)
+
+
+def _gather(cache, s):
+    n = int(cache.seq_lens[s])
+    pages = cache.block_table[s, :(n + cache.page_size - 1) // cache.page_size].long()
+    k = cache.k_pages[pages].permute(1, 0, 2, 3).reshape(cache.Hkv, -1, cache.D)[:, :n]
+    v = cache.v_pages[pages].permute(1, 0, 2, 3).reshape(cache.Hkv, -1, cache.D)[:, :n]
+    return k, v
+
+
+def check_decode_is_last_prefill_row(lib):
+    """One decode step attends to the T cached keys: it equals the last row of causal prefill
+    over the same sequence ("Why is attention O(n^2), ...", prefill vs. decode)."""
+    cache = _small_cache()
+    o, lse = _decode(cache, lib)
+    for s in range(cache.num_seqs):
+        n = int(cache.seq_lens[s])
+        k, v = _gather(cache, s)
+        qs = np.zeros((1, cache.Hq, n, cache.D), np.uint16)
+        qs[0, :, n - 1] = synth.bits(cache.q[s])
+        op, lsep = oracle.attention(qs, synth.bits(k.contiguous())[None], synth.bits(v.contiguous())[None],
+                                    causal=True, scale=cache.D ** -0.5, lib=lib)
+        assert np.array_equal(o[s], op[0, :, n - 1]) and np.array_equal(lse[s], lsep[0, :, n - 1])
+
+
+def check_decode_library(lib):
+    cache = _small_cache(seed=6)
+    o, _ = _decode(cache, lib)
+    for s in range(cache.num_seqs):
+        k, v = _gather(cache, s)
+        ref = _sdpa64(synth.bits(cache.q[s])[:, None, :], synth.bits(k.contiguous()),
+                      synth.bits(v.contiguous()), cache.D ** -0.5, gqa=True)
+        assert np.abs(o[s] - ref[:, 0]).max() < 1e-12
+
+
+def check_decode_paging_invariance(lib):
+    """Paging is indirection only: the permuted pool and its contiguous copy give the same bits,
+    and NaN in spare pages and page tails never reaches the output."""
+    cache = _small_cache(seed=8)
+    o, lse = _decode(cache, lib)
+    assert np.all(np.isfinite(o)) and np.all(np.isfinite(lse))
+    o2, lse2 = _decode(synth.contiguous_copy(cache), lib)
+    assert np.array_equal(o, o2) and np.array_equal(lse, lse2)
+    ident = _small_cache(seed=8, permute=False)
+    o3, lse3 = _decode(ident, lib)
+    assert np.array_equal(o, o3) and np.array_equal(lse, lse3)
+
+
+ALL_CHECKS = [
+    check_round_bf16_golden, check_round_bf16_matches_torch, check_rope_golden,
+    check_rope_matches_sinusoid, check_rope_norm_and_identity, check_rope_relative,
+    check_hand_two_tokens, check_library_sdpa, check_library_window, check_library_gqa,
+    check_gqa_reduces_to_mha, check_lse_library, check_probability_rows,
+    check_permutation_equivariance, check_causal_row0_and_window1, check_equal_scores,
+    check_rows_subset, check_online_recurrence, check_decode_is_last_prefill_row,
+    check_decode_library, check_decode_paging_invariance,
+]

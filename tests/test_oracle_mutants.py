@@ -1,0 +1,52 @@
+"""Mistakes planted in a copy of the oracle must each be caught by at least one pin.
+
+Each mutant is the oracle's C source with one plausible mistake substituted (a dropped term,
+a wrong sign or index, a transposed operand, an off-by-one mask), compiled on the CPU into a
+temporary library. The shipped oracle is never modified.
+"""
+import os
+
+import pytest
+
+import oracle
+from oracle import build as obuild
+from oracle_checks import ALL_CHECKS
+
+MUTANTS = {
+    "rope_sign": ("out[2 * i + 1] = bf16_value(oracle_round_bf16(x0 * s + x1 * c));",
+                  "out[2 * i + 1] = bf16_value(oracle_round_bf16(x1 * c - x0 * s));"),
+    "rope_theta_exponent": ("pow(base, -2.0 * (double)i / (double)D)", "pow(base, -1.0 * (double)i / (double)D)"),
+    "rope_half_split_pairing": ("double x0 = bf16_value(x[2 * i]), x1 = bf16_value(x[2 * i + 1]);",
+                                "double x0 = bf16_value(x[i]), x1 = bf16_value(x[i + D / 2]);"),
+    "rope_position_offset": ("double angle = (double)pos * theta;", "double angle = (double)(pos + 1) * theta;"),
+    "causal_off_by_one": ("if (causal && j > i) visible = 0;", "if (causal && j >= i + 1 + (i > 3)) visible = 0;"),
+    "window_off_by_one": ("(long)j < i - window + 1", "(long)j < i - window"),
+    "scale_dropped": ("s_row[j] = acc * scale;", "s_row[j] = acc;"),
+    "lse_drops_max": ("*lse = m + log(l);", "*lse = log(l);"),
+    "values_are_keys": ("const double* vj = vv + (size_t)j * D;", "const double* vj = kk + (size_t)j * D;"),
+    "gqa_interleaved_heads": ("if (rb != b || rh / G != g) continue;", "if (rb != b || rh % Hkv != g) continue;"),
+    "round_truncates": ("double r = nearbyint(ldexp(ax, -qexp));", "double r = floor(ldexp(ax, -qexp));"),
+    "decode_slot_index": ("(size_t)(t % page_size)) * D;", "(size_t)((t + 1) % page_size)) * D;"),
+    "decode_query_position": ("attend_row(qq, kk, vv, len, D, (long)len - 1, 1, 0, scale, s_row,",
+                              "attend_row(qq, kk, vv, len, D, (long)len - 2, 1, 0, scale, s_row,"),
+    "normaliser_missing": ("for (int d = 0; d < D; ++d) o[d] /= l;", "for (int d = 0; d < D; ++d) o[d] /= (l + 1e-3);"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_planted_mistake_is_caught(name, tmp_path):
+    old, new = MUTANTS[name]
+    src = open(obuild.SRC).read()
+    assert src.count(old) == 1, "mutation anchor not found exactly once: %r" % old
+    mutant_src = tmp_path / ("oracle_%s.c" % name)
+    mutant_src.write_text(src.replace(old, new))
+    lib_path = str(tmp_path / ("liboracle_%s.so" % name))
+    obuild.build(force=True, src=str(mutant_src), out=lib_path)
+    lib = oracle._lib(lib_path)
+    caught = []
+    for check in ALL_CHECKS:
+        try:
+            check(lib)
+        except Exception as e:  # an AssertionError or an oracle error status
+            caught.append((check.__name__, type(e).__name__))
+    assert caught, "mutant %s passed every pin" % name
