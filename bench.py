@@ -1,0 +1,482 @@
+#!/usr/bin/env python
+"""Benchmark of the exact-attention hot path on B200.
+
+One step is one pass of the whole hot path over one batch of synthetic input:
+  prefill  causal GQA attention with RoPE, B=2, Hq=32, Hkv=8, N=8192, D=128 (attn_fwd: the key
+           rotation pass plus the attention kernel), and
+  decode   one paged-KV decode token for 64 sequences with lengths uniform in [512, 16384],
+           Hq=32, Hkv=8, D=128, 16-token pages (attn_decode_paged: split kernel plus merge).
+The headline value is prefill TFLOP/s (algorithmic FLOPs = 4*D per unmasked (query, key) pair per
+query head) over the device time of the prefill calls; the decode line reports KV-cache GB/s
+(algorithmic bytes = every cached K/V byte of every sequence once, plus q, o, lse, block table and
+lengths) over the decode calls' device time.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+With N > 1 it runs under torchrun, one process per GPU; every rank runs its own copy of the
+workload (weak scaling, no data-path collective) and rank 0 prints one JSON line.
+--impl reference times the fp64 CPU oracle (the reference arm of this benchmark) on a bounded
+sample of the same workload.
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from exact_attention_161_b200 import synth  # noqa: E402
+
+PREFILL = synth.GQA_CAUSAL_N8192
+DECODE = synth.PAGED_DECODE_64
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+DATASHEET_BF16_TFLOPS = 2250.0
+DATASHEET_HBM_GBS = 8000.0
+KERNEL_SOURCES = ["exact_attention_161_b200/csrc/fwd_sm100.cuh", "exact_attention_161_b200/csrc/decode.cuh",
+                  "exact_attention_161_b200/csrc/ptx.cuh", "exact_attention_161_b200/csrc/rope.cuh",
+                  "exact_attention_161_b200/csrc/attn_api.cu"]
+
+
+# ------------------------------------------------------------------------------ workload arithmetic
+def visible_pairs(N, causal, window):
+    """Unmasked (query, key) pairs of one head: N^2, N(N+1)/2, or sum_i min(i+1, w)."""
+    if not causal:
+        return N * N
+    if window <= 0 or window >= N:
+        return N * (N + 1) // 2
+    w = window
+    return w * (w + 1) // 2 + (N - w) * w
+
+
+def prefill_flops(cfg=PREFILL):
+    return 4 * cfg.D * visible_pairs(cfg.N, cfg.causal, cfg.window) * cfg.B * cfg.Hq
+
+
+def decode_bytes(cache):
+    kv = int(cache.seq_lens.to(torch.int64).sum()) * 2 * cache.Hkv * cache.D * 2
+    io = cache.q.numel() * 2 * 2 + cache.num_seqs * cache.Hq * 4
+    tables = cache.num_seqs * 4 + sum(((int(n) + cache.page_size - 1) // cache.page_size)
+                                      for n in cache.seq_lens) * 4
+    return kv + io + tables
+
+
+# ------------------------------------------------------------------------------ ranks
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def init_dist(world, backend):
+    if world > 1 and not torch.distributed.is_initialized():
+        import datetime
+        torch.distributed.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def reduce_max(value, world, device=None):
+    """Max of a float over ranks (every rank takes the same collective steps)."""
+    if world == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_rank, world, seconds):
+    """Whole-job throughput: units processed by all ranks over the slowest rank's time."""
+    return units_per_rank * world / seconds
+
+
+# ------------------------------------------------------------------------------ clocks, peaks
+class ClockSampler:
+    """nvidia-smi sampling of SM clock and throttle reasons during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.device_index = device_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(self.device_index).uuid)
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", uuid, "--query-gpu=" + self.FIELDS,
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, flags in rows for i, f in enumerate(flags) if f.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kind):
+    """DRAM bytes per launch from the committed ncu summary, or None when the kernels changed
+    after the counters were taken."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    if d.get("kernel_source_hash") != kernel_source_hash():
+        return None
+    return d.get(kind, {}).get("dram_bytes_per_launch")
+
+
+# ------------------------------------------------------------------------------ CPU baseline (oracle)
+def oracle_prefill_sample(q, k, v, budget_s):
+    """Time the fp64 oracle on a bounded sample of prefill rows; returns (TFLOP/s, rows, seconds,
+    threads). Rows are spread over all positions of one head so the mix of causal lengths
+    matches the workload."""
+    import oracle
+    qb, kb, vb = synth.bits(q), synth.bits(k), synth.bits(v)
+    N, D = PREFILL.N, PREFILL.D
+
+    def run(n_rows):
+        rows = np.linspace(0, N - 1, n_rows).astype(np.int64)
+        flops = sum(4 * D * (int(i) + 1) for i in rows)
+        t0 = time.perf_counter()
+        oracle.attention(qb, kb, vb, causal=True, rope_base=PREFILL.rope_base, scale=PREFILL.scale, rows=rows)
+        return flops, time.perf_counter() - t0
+
+    f, t = run(64)  # calibration (includes the one-off key rotation)
+    n = int(min(N, max(64, 64 * budget_s / max(t, 1e-3))))
+    f, t = run(n)
+    return f / t / 1e12, n, t, oracle.max_threads()
+
+
+def oracle_decode_sample(cache, budget_s):
+    import oracle
+    S = cache.num_seqs
+
+    def run(n_seq):
+        sub = slice(0, n_seq)
+        c = synth.PagedCache(cache.q[sub], cache.k_pages, cache.v_pages, cache.block_table[sub],
+                             cache.seq_lens[sub], cache.page_size, cache.Hq, cache.Hkv, cache.D)
+        t0 = time.perf_counter()
+        oracle.decode_paged(synth.bits(c.q), synth.bits(c.k_pages), synth.bits(c.v_pages), c.block_table.numpy(),
+                            c.seq_lens.numpy())
+        return decode_bytes(c), time.perf_counter() - t0
+
+    b, t = run(1)
+    n = int(min(S, max(1, budget_s / max(t, 1e-3))))
+    b, t = run(n)
+    return b / t / 1e9, n, t
+
+
+# ------------------------------------------------------------------------------ our arm
+def run_ours(args, rank, world, local):
+    from exact_attention_161_b200 import api
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    init_dist(world, "nccl")
+    stream = torch.cuda.current_stream()
+
+    q_h, k_h, v_h = synth.prefill_inputs_for(PREFILL)
+    cache_h = synth.paged_decode_inputs_for(DECODE)
+    q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((PREFILL.B, PREFILL.Hq, PREFILL.N), dtype=torch.float32, device=dev)
+    dq, kp, vp = cache_h.q.to(dev), cache_h.k_pages.to(dev), cache_h.v_pages.to(dev)
+    bt, sl = cache_h.block_table.to(dev), cache_h.seq_lens.to(dev)
+    do = torch.empty_like(dq)
+    dlse = torch.empty((DECODE.num_seqs, DECODE.Hq), dtype=torch.float32, device=dev)
+    ws = torch.empty(api.decode_workspace_size(DECODE.num_seqs, cache_h.max_blocks, DECODE.page_size, DECODE.Hq,
+                                               DECODE.D), dtype=torch.uint8, device=dev)
+
+    def prefill():
+        api.attn_fwd(q, k, v, causal=PREFILL.causal, window=PREFILL.window, rope_base=PREFILL.rope_base,
+                     o=o, lse=lse, stream=stream)
+
+    def decode():
+        api.attn_decode_paged(dq, kp, vp, bt, sl, o=do, lse=dlse, workspace=ws, stream=stream)
+
+    for _ in range(args.warmup):
+        prefill()
+        decode()
+    torch.cuda.synchronize()
+    if api.device_status() != 0:
+        raise RuntimeError("device status raised during warm-up")
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    clocks = ClockSampler(local)
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)  # let the sampler take its first reading
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for s in range(K):
+        ev[s][0].record(stream)
+        prefill()
+        ev[s][1].record(stream)
+        decode()
+        ev[s][2].record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    total_ms = t_start.elapsed_time(t_end)
+    prefill_ms = [ev[s][0].elapsed_time(ev[s][1]) for s in range(K)]
+    decode_ms = [ev[s][1].elapsed_time(ev[s][2]) for s in range(K)]
+    status = api.device_status()
+
+    total_ms_max = reduce_max(total_ms, world, dev)
+    prefill_sum_max = reduce_max(sum(prefill_ms), world, dev)
+    decode_sum_max = reduce_max(sum(decode_ms), world, dev)
+    flops = prefill_flops()
+    dbytes = decode_bytes(cache_h)
+    value = job_throughput(flops * K, world, prefill_sum_max / 1e3) / 1e12
+    decode_value = job_throughput(dbytes * K, world, decode_sum_max / 1e3) / 1e9
+
+    # ---- end to end through the public API with pinned host buffers
+    E = max(3, min(args.e2e_steps, K))
+    q_p, k_p, v_p = q_h.pin_memory(), k_h.pin_memory(), v_h.pin_memory()
+    o_p = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    lse_p = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    dq_p, bt_p, sl_p = cache_h.q.pin_memory(), cache_h.block_table.pin_memory(), cache_h.seq_lens.pin_memory()
+    do_p = torch.empty(do.shape, dtype=do.dtype).pin_memory()
+    dlse_p = torch.empty(dlse.shape, dtype=dlse.dtype).pin_memory()
+    e_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(E)]
+    for s in range(E + 1):  # the first pass is a warm-up
+        r = e_ev[s - 1] if s > 0 else [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        r[0].record(stream)
+        q.copy_(q_p, non_blocking=True)
+        k.copy_(k_p, non_blocking=True)
+        v.copy_(v_p, non_blocking=True)
+        prefill()
+        o_p.copy_(o, non_blocking=True)
+        lse_p.copy_(lse, non_blocking=True)
+        r[1].record(stream)
+        dq.copy_(dq_p, non_blocking=True)
+        bt.copy_(bt_p, non_blocking=True)
+        sl.copy_(sl_p, non_blocking=True)
+        decode()
+        do_p.copy_(do, non_blocking=True)
+        dlse_p.copy_(dlse, non_blocking=True)
+        r[2].record(stream)
+    torch.cuda.synchronize()
+    e_pre = reduce_max(sum(e[0].elapsed_time(e[1]) for e in e_ev), world, dev)
+    e_dec = reduce_max(sum(e[1].elapsed_time(e[2]) for e in e_ev), world, dev)
+    h2d = sum(t.numel() * t.element_size() for t in (q_h, k_h, v_h))
+    d2h = o.numel() * 2 + lse.numel() * 4
+    dh2d = sum(t.numel() * t.element_size() for t in (cache_h.q, cache_h.block_table, cache_h.seq_lens))
+    dd2h = do.numel() * 2 + dlse.numel() * 4
+    e2e_value = job_throughput(flops * E, world, e_pre / 1e3) / 1e12
+    e2e_decode = job_throughput(dbytes * E, world, e_dec / 1e3) / 1e9
+
+    if rank != 0:
+        return None
+    peaks, peaks_kind = measured_peaks()
+    pre_launch_ms = statistics.mean(prefill_ms)
+    dec_launch_ms = statistics.mean(decode_ms)
+    tflops_launch = flops / (pre_launch_ms / 1e3) / 1e12
+    gbs_launch = dbytes / (dec_launch_ms / 1e3) / 1e9
+    tensor_peak = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
+    line = {
+        "metric": "attn fwd TFLOP/s (causal GQA prefill B2 Hq32 Hkv8 N8192 D128, RoPE 5e5) "
+                  "& paged-decode KV GB/s",
+        "value": round(value, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": round(total_ms_max / K, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) bf16; paged cache from a seeded permutation)",
+        "config": {
+            "workload": "prefill %s + decode %s" % (PREFILL.name, DECODE.name),
+            "prefill": {"B": PREFILL.B, "Hq": PREFILL.Hq, "Hkv": PREFILL.Hkv, "N": PREFILL.N, "D": PREFILL.D,
+                        "causal": PREFILL.causal, "window": PREFILL.window, "rope_base": PREFILL.rope_base,
+                        "flops_per_step": flops},
+            "decode": {"num_seqs": DECODE.num_seqs, "Hq": DECODE.Hq, "Hkv": DECODE.Hkv, "D": DECODE.D,
+                       "page_size": DECODE.page_size, "total_tokens": cache_h.total_tokens,
+                       "bytes_per_step": dbytes},
+            "l2": "inputs larger than L2 (prefill Q/K/V 201 MB, decode KV 2.2 GB); no flush",
+            "parallelism": "replica per GPU" if world > 1 else "single GPU",
+        },
+        "decode": {"metric": "paged-decode KV GB/s", "value": round(decode_value, 1), "unit": "GB/s",
+                   "ms_per_step": round(decode_sum_max / K, 4),
+                   "roofline": {"bound": "hbm", "achieved": round(gbs_launch, 1), "peak": peaks["hbm_gbs"],
+                                "unit": "GB/s", "frac": round(gbs_launch / peaks["hbm_gbs"], 4),
+                                "peak_kind": peaks_kind, "frac_of_8TBs": round(gbs_launch / DATASHEET_HBM_GBS, 4),
+                                "traffic": profiled_traffic("decode_split")},
+                   "e2e": {"value": round(e2e_decode, 2), "unit": "GB/s", "h2d_bytes_per_step": dh2d,
+                           "d2h_bytes_per_step": dd2h}},
+        "roofline": {"bound": "tensor", "achieved": round(tflops_launch, 2), "peak": tensor_peak, "unit": "TFLOP/s",
+                     "frac": round(tflops_launch / tensor_peak, 4),
+                     "peak_kind": "%s bf16 GEMM, sustained" % peaks_kind,
+                     "frac_of_2250": round(tflops_launch / DATASHEET_BF16_TFLOPS, 4),
+                     "traffic": profiled_traffic("attn_fwd"),
+                     "kernel": "attn_fwd_kernel<128> (+ key rotation pass, inside the timed call)"},
+        "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": 4 * K,
+        "device_status": status,
+        "clocks": clk,
+    }
+    return line
+
+
+def add_cpu_baseline(line, args):
+    if args.no_cpu_baseline:
+        line["cpu_baseline"] = None
+        return
+    q, k, v = synth.prefill_inputs_for(PREFILL)
+    tf, n, t, threads = oracle_prefill_sample(q, k, v, args.cpu_budget)
+    cache = synth.paged_decode_inputs_for(DECODE)
+    gbs, ns, td = oracle_decode_sample(cache, args.cpu_budget / 2)
+    line["cpu_baseline"] = {"value": round(tf, 6), "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                            "sample": "%d query rows spread over positions 0..8191 of one head of the prefill "
+                                      "workload (causal, RoPE), %.1f s" % (n, t),
+                            "decode": {"value": round(gbs, 4), "unit": "GB/s",
+                                       "sample": "%d of 64 sequences, %.1f s" % (ns, td)}}
+
+
+# ------------------------------------------------------------------------------ reference arm
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    import oracle
+    q, k, v = synth.prefill_inputs_for(PREFILL)
+    qb, kb, vb = synth.bits(q), synth.bits(k), synth.bits(v)
+    # per-step budget so that warm-up + steps end within a few minutes
+    per_step = max(0.05, min(5.0, 150.0 / (args.steps + args.warmup)))
+    N, D = PREFILL.N, PREFILL.D
+    rows_probe = np.linspace(0, N - 1, 16).astype(np.int64)
+    t0 = time.perf_counter()
+    oracle.attention(qb, kb, vb, causal=True, rope_base=PREFILL.rope_base, scale=PREFILL.scale, rows=rows_probe)
+    t_probe = time.perf_counter() - t0
+    n_rows = int(max(4, min(N, 16 * per_step / max(t_probe, 1e-4))))
+    rng = np.random.default_rng(0)
+    flops_total, secs_total = 0, 0.0
+    for s in range(args.warmup + args.steps):
+        rows = np.sort(rng.choice(N, size=n_rows, replace=False)).astype(np.int64)
+        t0 = time.perf_counter()
+        oracle.attention(qb, kb, vb, causal=True, rope_base=PREFILL.rope_base, scale=PREFILL.scale, rows=rows)
+        dt = time.perf_counter() - t0
+        if s >= args.warmup:
+            flops_total += sum(4 * D * (int(i) + 1) for i in rows)
+            secs_total += dt
+    value = flops_total / secs_total / 1e12
+    sample = ("%d random query rows of one head of the prefill workload per step (causal, RoPE); "
+              "the oracle rotates that head's keys each step" % n_rows)
+    return {
+        "impl": "reference",
+        "metric": "attn fwd TFLOP/s (causal GQA prefill B2 Hq32 Hkv8 N8192 D128, RoPE 5e5) & paged-decode KV GB/s",
+        "value": round(value, 6),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(secs_total / args.steps * 1e3, 3),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": "prefill %s (bounded row sample on the host CPU)" % PREFILL.name},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": oracle.max_threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle time for the CPU baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing (profiling runs)")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    return args
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    rank, world, local = dist_env()
+    if world != args.gpus:
+        print("warning: --gpus %d but WORLD_SIZE %d; using WORLD_SIZE" % (args.gpus, world), file=sys.stderr)
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+    else:
+        line = run_ours(args, rank, world, local)
+        if line is not None and world == 1:
+            add_cpu_baseline(line, args)
+        elif line is not None:
+            line["cpu_baseline"] = None
+    if line is not None:
+        print(json.dumps(line), flush=True)
+    if world > 1 and torch.distributed.is_initialized():
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

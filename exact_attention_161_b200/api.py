@@ -1,0 +1,151 @@
+"""Python binding of the C ABI in ``include/attn.h`` (argument marshalling only).
+
+Every computation runs in ``libattn_b200.so``; this module checks tensor dtypes, shapes and
+devices, allocates outputs when the caller passes none, and forwards raw device pointers and the
+current CUDA stream. Importing it loads the library and raises if it is missing: there is no
+CPU fallback.
+"""
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libattn_b200.so")
+
+ATTN_OK = 0
+ATTN_ERR_INVALID_ARG = 1
+ATTN_ERR_UNSUPPORTED = 2
+ATTN_ERR_CUDA = 3
+ATTN_ERR_DEVICE_CHECK = 4
+ATTN_ERR_TIMEOUT = 5
+STATUS_NAMES = {0: "ATTN_OK", 1: "ATTN_ERR_INVALID_ARG", 2: "ATTN_ERR_UNSUPPORTED", 3: "ATTN_ERR_CUDA",
+                4: "ATTN_ERR_DEVICE_CHECK", 5: "ATTN_ERR_TIMEOUT"}
+DEVICE_TIMEOUT, DEVICE_BAD_PAGE, DEVICE_BAD_SEQLEN = 1, 2, 4
+
+# Every function include/attn.h declares, with its ctypes signature.
+_p, _i, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+SIGNATURES = {
+    "attn_fwd": (_i, [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _f, _f, _p]),
+    "attn_decode_workspace_size": (_sz, [_i, _i, _i, _i, _i]),
+    "attn_decode_paged": (_i, [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _f, _p, _p, _p, _sz, _p]),
+    "attn_get_device_status": (_i, [_p, ctypes.POINTER(ctypes.c_int)]),
+    "attn_last_error": (ctypes.c_char_p, []),
+    "attn_version": (ctypes.c_char_p, []),
+    "attn_shutdown": (None, []),
+}
+
+
+class AttnError(RuntimeError):
+    def __init__(self, status, message):
+        super().__init__("%s: %s" % (STATUS_NAMES.get(status, status), message))
+        self.status = status
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    if not os.path.exists(path):
+        raise ImportError("CUDA library %s is missing; build it with `python -m exact_attention_161_b200.build` "
+                          "(there is no CPU fallback)" % path)
+    lib = ctypes.CDLL(path)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+lib = load()
+
+
+def _check(status):
+    if status != ATTN_OK:
+        raise AttnError(status, lib.attn_last_error().decode())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _dev_tensor(t, name, dtype):
+    if not isinstance(t, torch.Tensor) or t.device.type != "cuda":
+        raise TypeError("%s must be a CUDA tensor" % name)
+    if t.dtype != dtype:
+        raise TypeError("%s must be %s, got %s" % (name, dtype, t.dtype))
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def version() -> str:
+    return lib.attn_version().decode()
+
+
+def last_error() -> str:
+    return lib.attn_last_error().decode()
+
+
+def shutdown() -> None:
+    lib.attn_shutdown()
+
+
+def attn_fwd(q, k, v, causal=False, window=0, rope_base=0.0, scale=0.0, o=None, lse=None, want_lse=True,
+             stream=None):
+    """Exact attention forward. q [B,Hq,N,D], k/v [B,Hkv,N,D] bf16 CUDA tensors.
+    Returns (o [B,Hq,N,D] bf16, lse [B,Hq,N] fp32 or None)."""
+    B, Hq, N, D = q.shape
+    Hkv = k.shape[1]
+    if k.shape != (B, Hkv, N, D) or v.shape != k.shape:
+        raise ValueError("k and v must be [B, Hkv, N, D] matching q")
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device)
+    args = [_dev_tensor(q, "q", torch.bfloat16), _dev_tensor(k, "k", torch.bfloat16),
+            _dev_tensor(v, "v", torch.bfloat16), _dev_tensor(o, "o", torch.bfloat16),
+            _dev_tensor(lse, "lse", torch.float32) if lse is not None else None]
+    _check(lib.attn_fwd(*args, B, Hq, Hkv, N, D, int(bool(causal)), int(window), float(rope_base), float(scale),
+                        _stream(stream)))
+    return o, lse
+
+
+def decode_workspace_size(num_seqs, max_blocks_per_seq, page_size, Hq, D) -> int:
+    return int(lib.attn_decode_workspace_size(num_seqs, max_blocks_per_seq, page_size, Hq, D))
+
+
+def attn_decode_paged(q, k_pages, v_pages, block_table, seq_lens, scale=0.0, o=None, lse=None, want_lse=True,
+                      workspace=None, stream=None):
+    """One decode step per sequence over a paged KV cache.
+    q [S,Hq,D] bf16; k_pages/v_pages [num_pages,Hkv,page_size,D] bf16; block_table [S,max_blocks]
+    int32; seq_lens [S] int32 (all CUDA). Returns (o [S,Hq,D] bf16, lse [S,Hq] fp32 or None)."""
+    S, Hq, D = q.shape
+    num_pages, Hkv, page_size, D2 = k_pages.shape
+    if D2 != D or v_pages.shape != k_pages.shape:
+        raise ValueError("k_pages/v_pages must be [num_pages, Hkv, page_size, D]")
+    max_blocks = block_table.shape[1]
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((S, Hq), dtype=torch.float32, device=q.device)
+    need = decode_workspace_size(S, max_blocks, page_size, Hq, D)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    args = [_dev_tensor(q, "q", torch.bfloat16), _dev_tensor(k_pages, "k_pages", torch.bfloat16),
+            _dev_tensor(v_pages, "v_pages", torch.bfloat16), _dev_tensor(block_table, "block_table", torch.int32),
+            _dev_tensor(seq_lens, "seq_lens", torch.int32)]
+    _check(lib.attn_decode_paged(*args, S, max_blocks, num_pages, page_size, Hq, Hkv, D, float(scale),
+                                 _dev_tensor(o, "o", torch.bfloat16),
+                                 _dev_tensor(lse, "lse", torch.float32) if lse is not None else None,
+                                 _dev_tensor(workspace, "workspace", torch.uint8),
+                                 workspace.numel() * workspace.element_size(), _stream(stream)))
+    return o, lse
+
+
+def device_status(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device status word's bits."""
+    flags = ctypes.c_int(0)
+    st = lib.attn_get_device_status(_stream(stream), ctypes.byref(flags))
+    if st not in (ATTN_OK, ATTN_ERR_DEVICE_CHECK, ATTN_ERR_TIMEOUT):
+        _check(st)
+    return flags.value

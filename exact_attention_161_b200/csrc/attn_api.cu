@@ -1,0 +1,352 @@
+// attn_api.cu -- the C ABI declared in include/attn.h: argument checks, TMA descriptors, the
+// cached RoPE tables and key scratch, and the kernel launches. The whole library is this one
+// translation unit.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <string>
+#include <tuple>
+#include <vector>
+
+#include "../../include/attn.h"
+#include "common.cuh"
+#include "decode.cuh"
+#include "fwd_sm100.cuh"
+#include "rope.cuh"
+
+#define ATTN_VERSION_STRING "exact_attention_161_b200 0.1.0 (sm_100a)"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+attn_status fail(attn_status st, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return st;
+}
+
+#define CUDA_TRY(expr)                                                                          \
+    do {                                                                                        \
+        cudaError_t e_ = (expr);                                                                \
+        if (e_ != cudaSuccess) return fail(ATTN_ERR_CUDA, "%s: %s", #expr, cudaGetErrorString(e_)); \
+    } while (0)
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ------------------------------------------------------------------ cuTensorMapEncodeTiled
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// A rank-3 bf16 tensor map: dims {d0 (contiguous), d1, d2}, box {64, box1, 1}, 128-byte swizzle,
+// out-of-bounds elements read as zero.
+attn_status make_map_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t box1) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return fail(ATTN_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable (no CUDA driver?)");
+    const cuuint64_t dims[3] = {d0, d1, d2};
+    const cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
+    const cuuint32_t box[3] = {64, box1, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(ATTN_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+    return ATTN_OK;
+}
+
+// ------------------------------------------------------------------ caches
+struct DevBuf {
+    void* ptr = nullptr;
+    size_t bytes = 0;
+    int dev = 0;
+};
+
+std::mutex g_cache_mu;
+// (device, base, D) -> cos/sin table covering positions [0, capacity)
+std::map<std::tuple<int, double, int>, std::pair<DevBuf, int>> g_rope_tables;
+// (device, stream) -> rotated-key scratch
+std::map<std::pair<int, void*>, DevBuf> g_key_scratch;
+std::vector<DevBuf> g_retired;  // outgrown buffers; a launch still queued may read them
+
+// (cos, sin) of pos * base^(-2i/D) for pos < n, i < D/2: angles and trigonometry in fp64, stored
+// as fp32 pairs.
+attn_status rope_table(int dev, double base, int D, int n, const float2** out) {
+    std::lock_guard<std::mutex> lock(g_cache_mu);
+    auto key = std::make_tuple(dev, base, D);
+    auto it = g_rope_tables.find(key);
+    if (it != g_rope_tables.end() && it->second.second >= n) {
+        *out = static_cast<const float2*>(it->second.first.ptr);
+        return ATTN_OK;
+    }
+    const int cap = ((n + 1023) / 1024) * 1024;
+    std::vector<float2> host(static_cast<size_t>(cap) * (D / 2));
+    std::vector<double> theta(D / 2);
+    for (int i = 0; i < D / 2; ++i) theta[i] = std::pow(base, -2.0 * i / D);
+    for (int pos = 0; pos < cap; ++pos)
+        for (int i = 0; i < D / 2; ++i) {
+            const double a = pos * theta[i];
+            host[static_cast<size_t>(pos) * (D / 2) + i] = make_float2(static_cast<float>(std::cos(a)),
+                                                                       static_cast<float>(std::sin(a)));
+        }
+    DevBuf buf;
+    buf.dev = dev;
+    buf.bytes = host.size() * sizeof(float2);
+    CUDA_TRY(cudaMalloc(&buf.ptr, buf.bytes));
+    cudaError_t e = cudaMemcpy(buf.ptr, host.data(), buf.bytes, cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) {
+        cudaFree(buf.ptr);
+        return fail(ATTN_ERR_CUDA, "rope table upload: %s", cudaGetErrorString(e));
+    }
+    if (it != g_rope_tables.end()) g_retired.push_back(it->second.first);
+    g_rope_tables[key] = std::make_pair(buf, cap);
+    *out = static_cast<const float2*>(buf.ptr);
+    return ATTN_OK;
+}
+
+attn_status key_scratch(int dev, void* stream, size_t bytes, void** out) {
+    std::lock_guard<std::mutex> lock(g_cache_mu);
+    DevBuf& b = g_key_scratch[std::make_pair(dev, stream)];
+    if (b.bytes < bytes) {
+        if (b.ptr) g_retired.push_back(b);
+        b = DevBuf();
+        CUDA_TRY(cudaMalloc(&b.ptr, bytes));
+        b.bytes = bytes;
+        b.dev = dev;
+    }
+    *out = b.ptr;
+    return ATTN_OK;
+}
+
+// Opt a kernel into more than 48 KB of dynamic shared memory, once per (kernel, device).
+std::mutex g_attr_mu;
+std::map<std::pair<const void*, int>, bool> g_smem_set;
+
+template <typename K>
+attn_status ensure_smem(K kernel, int bytes, int dev) {
+    std::lock_guard<std::mutex> lock(g_attr_mu);
+    const auto key = std::make_pair(reinterpret_cast<const void*>(kernel), dev);
+    if (!g_smem_set[key]) {
+        CUDA_TRY(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
+        g_smem_set[key] = true;
+    }
+    return ATTN_OK;
+}
+
+template <int D>
+attn_status launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                       int N, int causal, int window, float rope_base, float scale, cudaStream_t stream, int dev) {
+    using C = attn::FwdCfg<D>;
+    const void* k_use = k;
+    attn::FwdParams p{};
+    if (rope_base > 0.f) {
+        const float2* table = nullptr;
+        attn_status st = rope_table(dev, static_cast<double>(rope_base), D, N, &table);
+        if (st != ATTN_OK) return st;
+        void* k_rot = nullptr;
+        const size_t kbytes = static_cast<size_t>(B) * Hkv * N * D * 2;
+        st = key_scratch(dev, stream, kbytes, &k_rot);
+        if (st != ATTN_OK) return st;
+        const long long rows = static_cast<long long>(B) * Hkv * N;
+        const long long chunks = rows * (D / 8);
+        int sms = 148;
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        const long long want = (chunks + 255) / 256;
+        const int grid = static_cast<int>(want < 8LL * sms ? want : 8LL * sms);
+        attn::rope_rotate_rows_kernel<D><<<grid, 256, 0, stream>>>(static_cast<const uint4*>(k),
+                                                                   static_cast<uint4*>(k_rot), table, rows, N);
+        CUDA_TRY(cudaGetLastError());
+        k_use = k_rot;
+        p.rope = table;
+    }
+    CUtensorMap tq, tk, tv;
+    attn_status st;
+    if ((st = make_map_3d(&tq, q, D, N, static_cast<uint64_t>(B) * Hq, 128)) != ATTN_OK) return st;
+    if ((st = make_map_3d(&tk, k_use, D, N, static_cast<uint64_t>(B) * Hkv, 128)) != ATTN_OK) return st;
+    if ((st = make_map_3d(&tv, v, D, N, static_cast<uint64_t>(B) * Hkv, 128)) != ATTN_OK) return st;
+    p.o = static_cast<__nv_bfloat16*>(o);
+    p.lse = lse;
+    p.B = B;
+    p.Hq = Hq;
+    p.Hkv = Hkv;
+    p.N = N;
+    p.causal = causal;
+    p.window = window > 0 ? window : 0;
+    p.scale_log2 = scale * attn::kLog2e;
+    if ((st = ensure_smem(attn::attn_fwd_kernel<D>, C::SMEM_BYTES, dev)) != ATTN_OK) return st;
+    const dim3 grid(Hq, B, (N + C::BM - 1) / C::BM);
+    attn::attn_fwd_kernel<D><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+    CUDA_TRY(cudaGetLastError());
+    return ATTN_OK;
+}
+
+size_t decode_chunks(int max_blocks) { return (static_cast<size_t>(max_blocks) + attn::kChunkPages - 1) / attn::kChunkPages; }
+
+template <int D>
+attn_status launch_decode(const void* q, const void* k_pages, const void* v_pages, const int32_t* block_table,
+                          const int32_t* seq_lens, int S, int max_blocks, int num_pages, int Hq, int Hkv,
+                          float scale, void* o, float* lse, void* ws, cudaStream_t stream, int dev) {
+    using C = attn::DecCfg<D>;
+    CUtensorMap tk, tv;
+    attn_status st;
+    const uint64_t slabs = static_cast<uint64_t>(num_pages) * Hkv;
+    if ((st = make_map_3d(&tk, k_pages, D, attn::kPageSize, slabs, attn::kPageSize)) != ATTN_OK) return st;
+    if ((st = make_map_3d(&tv, v_pages, D, attn::kPageSize, slabs, attn::kPageSize)) != ATTN_OK) return st;
+    const int max_chunks = static_cast<int>(decode_chunks(max_blocks));
+    attn::DecodeParams p{};
+    p.q = static_cast<const __nv_bfloat16*>(q);
+    p.block_table = block_table;
+    p.seq_lens = seq_lens;
+    p.o = static_cast<__nv_bfloat16*>(o);
+    p.lse = lse;
+    p.ws_o = static_cast<float*>(ws);
+    p.ws_ml = p.ws_o + static_cast<size_t>(S) * Hq * max_chunks * D;
+    p.S = S;
+    p.Hq = Hq;
+    p.Hkv = Hkv;
+    p.G = Hq / Hkv;
+    p.max_blocks = max_blocks;
+    p.num_pages = num_pages;
+    p.max_chunks = max_chunks;
+    p.scale_log2 = scale * attn::kLog2e;
+    if ((st = ensure_smem(attn::decode_split_kernel<D>, C::SMEM_BYTES, dev)) != ATTN_OK) return st;
+    attn::decode_split_kernel<D><<<dim3(max_chunks, Hkv, S), attn::kDecodeThreads, C::SMEM_BYTES, stream>>>(tk, tv, p);
+    CUDA_TRY(cudaGetLastError());
+    const long long warps = static_cast<long long>(S) * Hq;
+    attn::decode_merge_kernel<D><<<static_cast<unsigned>((warps * 32 + 127) / 128), 128, 0, stream>>>(p);
+    CUDA_TRY(cudaGetLastError());
+    return ATTN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                     int N, int D, int causal, int window, float rope_base, float scale, void* stream) {
+    g_last_error.clear();
+    if (!q || !k || !v || !o) return fail(ATTN_ERR_INVALID_ARG, "q, k, v and o must be non-NULL");
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || (lse && !aligned16(lse)))
+        return fail(ATTN_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+    if (B < 1 || Hq < 1 || Hkv < 1 || N < 1) return fail(ATTN_ERR_INVALID_ARG, "B, Hq, Hkv, N must be >= 1");
+    if (Hq % Hkv != 0) return fail(ATTN_ERR_INVALID_ARG, "Hq (%d) must be a multiple of Hkv (%d)", Hq, Hkv);
+    if (causal != 0 && causal != 1) return fail(ATTN_ERR_INVALID_ARG, "causal must be 0 or 1");
+    if (window > 0 && !causal) return fail(ATTN_ERR_INVALID_ARG, "a sliding window requires causal = 1");
+    if (!std::isfinite(scale) || !std::isfinite(rope_base)) return fail(ATTN_ERR_INVALID_ARG, "scale and rope_base must be finite");
+    if (D != 64 && D != 128) return fail(ATTN_ERR_UNSUPPORTED, "head dim %d not supported (64 or 128)", D);
+    if (B > 65535 || (N + 127) / 128 > 65535) return fail(ATTN_ERR_UNSUPPORTED, "B or N too large for the grid");
+    if (static_cast<double>(B) * Hq * N * D * 2 >= 1099511627776.0)
+        return fail(ATTN_ERR_UNSUPPORTED, "tensor larger than 1 TiB");
+    if (scale <= 0.f) scale = 1.0f / std::sqrt(static_cast<float>(D));
+    int dev = 0;
+    CUDA_TRY(cudaGetDevice(&dev));
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (D == 64) return launch_fwd<64>(q, k, v, o, lse, B, Hq, Hkv, N, causal, window, rope_base, scale, s, dev);
+    return launch_fwd<128>(q, k, v, o, lse, B, Hq, Hkv, N, causal, window, rope_base, scale, s, dev);
+}
+
+size_t attn_decode_workspace_size(int num_seqs, int max_blocks_per_seq, int page_size, int Hq, int D) {
+    if (num_seqs < 1 || max_blocks_per_seq < 1 || page_size < 1 || Hq < 1 || D < 1) return 0;
+    const size_t rows = static_cast<size_t>(num_seqs) * Hq * decode_chunks(max_blocks_per_seq);
+    const size_t bytes = rows * (static_cast<size_t>(D) + 2) * sizeof(float);
+    return (bytes + 255) / 256 * 256;
+}
+
+attn_status attn_decode_paged(const void* q, const void* k_pages, const void* v_pages, const int32_t* block_table,
+                              const int32_t* seq_lens, int num_seqs, int max_blocks_per_seq, int num_pages,
+                              int page_size, int Hq, int Hkv, int D, float scale, void* o, float* lse,
+                              void* workspace, size_t workspace_bytes, void* stream) {
+    g_last_error.clear();
+    if (!q || !k_pages || !v_pages || !block_table || !seq_lens || !o || !workspace)
+        return fail(ATTN_ERR_INVALID_ARG, "q, k_pages, v_pages, block_table, seq_lens, o and workspace must be non-NULL");
+    if (!aligned16(q) || !aligned16(k_pages) || !aligned16(v_pages) || !aligned16(o) || !aligned16(workspace) ||
+        (reinterpret_cast<uintptr_t>(block_table) & 3u) || (reinterpret_cast<uintptr_t>(seq_lens) & 3u) ||
+        (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+        return fail(ATTN_ERR_INVALID_ARG, "misaligned pointer (tensors 16-byte, int32/fp32 arrays 4-byte)");
+    if (num_seqs < 1 || max_blocks_per_seq < 1 || num_pages < 1 || page_size < 1 || Hq < 1 || Hkv < 1)
+        return fail(ATTN_ERR_INVALID_ARG, "sizes must be >= 1");
+    if (Hq % Hkv != 0) return fail(ATTN_ERR_INVALID_ARG, "Hq (%d) must be a multiple of Hkv (%d)", Hq, Hkv);
+    if (!std::isfinite(scale)) return fail(ATTN_ERR_INVALID_ARG, "scale must be finite");
+    if (page_size != attn::kPageSize) return fail(ATTN_ERR_UNSUPPORTED, "page_size %d not supported (16)", page_size);
+    if (D != 64 && D != 128) return fail(ATTN_ERR_UNSUPPORTED, "head dim %d not supported (64 or 128)", D);
+    if (Hq / Hkv > 16) return fail(ATTN_ERR_UNSUPPORTED, "more than 16 query heads per KV head");
+    if (num_seqs > 65535 || Hkv > 65535) return fail(ATTN_ERR_UNSUPPORTED, "num_seqs or Hkv too large for the grid");
+    if (static_cast<double>(num_pages) * Hkv * page_size * D * 2 >= 1099511627776.0)
+        return fail(ATTN_ERR_UNSUPPORTED, "KV pool larger than 1 TiB");
+    const size_t need = attn_decode_workspace_size(num_seqs, max_blocks_per_seq, page_size, Hq, D);
+    if (workspace_bytes < need)
+        return fail(ATTN_ERR_INVALID_ARG, "workspace too small: %zu < %zu bytes", workspace_bytes, need);
+    if (scale <= 0.f) scale = 1.0f / std::sqrt(static_cast<float>(D));
+    int dev = 0;
+    CUDA_TRY(cudaGetDevice(&dev));
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (D == 64)
+        return launch_decode<64>(q, k_pages, v_pages, block_table, seq_lens, num_seqs, max_blocks_per_seq, num_pages,
+                                 Hq, Hkv, scale, o, lse, workspace, s, dev);
+    return launch_decode<128>(q, k_pages, v_pages, block_table, seq_lens, num_seqs, max_blocks_per_seq, num_pages,
+                              Hq, Hkv, scale, o, lse, workspace, s, dev);
+}
+
+attn_status attn_get_device_status(void* stream, int* flags_out) {
+    g_last_error.clear();
+    if (!flags_out) return fail(ATTN_ERR_INVALID_ARG, "flags_out must be non-NULL");
+    *flags_out = 0;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    unsigned int word = 0;
+    CUDA_TRY(cudaMemcpyFromSymbolAsync(&word, attn::g_attn_status, sizeof word, 0, cudaMemcpyDeviceToHost, s));
+    CUDA_TRY(cudaStreamSynchronize(s));
+    if (word) {
+        const unsigned int zero = 0;
+        CUDA_TRY(cudaMemcpyToSymbolAsync(attn::g_attn_status, &zero, sizeof zero, 0, cudaMemcpyHostToDevice, s));
+        CUDA_TRY(cudaStreamSynchronize(s));
+    }
+    *flags_out = static_cast<int>(word);
+    if (word & attn::kStatusTimeout) return fail(ATTN_ERR_TIMEOUT, "a device-side wait timed out (flags 0x%x)", word);
+    if (word) return fail(ATTN_ERR_DEVICE_CHECK, "a device-side check fired (flags 0x%x)", word);
+    return ATTN_OK;
+}
+
+const char* attn_last_error(void) { return g_last_error.c_str(); }
+
+const char* attn_version(void) { return ATTN_VERSION_STRING; }
+
+void attn_shutdown(void) {
+    std::lock_guard<std::mutex> lock(g_cache_mu);
+    int cur = 0;
+    const bool have_dev = cudaGetDevice(&cur) == cudaSuccess;
+    auto release = [](const DevBuf& b) {
+        if (b.ptr && cudaSetDevice(b.dev) == cudaSuccess) cudaFree(b.ptr);
+    };
+    for (auto& kv : g_rope_tables) release(kv.second.first);
+    for (auto& kv : g_key_scratch) release(kv.second);
+    for (auto& b : g_retired) release(b);
+    if (have_dev) cudaSetDevice(cur);
+    g_rope_tables.clear();
+    g_key_scratch.clear();
+    g_retired.clear();
+}
+
+}  // extern "C"

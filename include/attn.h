@@ -1,0 +1,144 @@
+/*
+ * attn.h -- C ABI of libattn_b200.so: exact scaled dot-product attention on NVIDIA B200 (sm_100a).
+ *
+ * Two operations, both computing softmax(Q K^T * scale) V exactly (up to floating-point
+ * rounding), never materialising the n x n score matrix in device memory:
+ *   attn_fwd           prefill over whole sequences (causal / sliding-window / full, GQA, RoPE);
+ *   attn_decode_paged  one new query token per sequence over a paged KV cache.
+ *
+ * Conventions shared by every entry point:
+ *   - Tensor arguments are plain device pointers to caller-owned memory, contiguous, in the
+ *     layouts stated below, each 16-byte aligned. bf16 means IEEE bfloat16 (uint16 storage).
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream). Calls are
+ *     asynchronous on that stream; the return value covers argument validation and launch only.
+ *   - Nothing throws, aborts or traps. Every failure returns a status and sets a thread-local
+ *     message readable with attn_last_error(). Faults detected on the device (a bounded wait
+ *     that gave up, an out-of-range block-table entry) set bits of a device status word read
+ *     with attn_get_device_status().
+ *   - The library owns only its caches (RoPE cos/sin tables per (device, base, head dim); key
+ *     scratch per (device, stream) for the rotated keys; the device status word); attn_shutdown
+ *     releases them.
+ *   - There is no CPU fallback: without a B200 every compute call returns ATTN_ERR_CUDA.
+ */
+#ifndef ATTN_B200_H
+#define ATTN_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    ATTN_OK = 0,
+    ATTN_ERR_INVALID_ARG = 1,  /* a pointer, size or flag violates the contract below */
+    ATTN_ERR_UNSUPPORTED = 2,  /* valid request outside what the kernels implement (e.g. D) */
+    ATTN_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed (no device, launch error) */
+    ATTN_ERR_DEVICE_CHECK = 4, /* reported by attn_get_device_status: a device-side check fired */
+    ATTN_ERR_TIMEOUT = 5       /* reported by attn_get_device_status: a bounded wait gave up */
+} attn_status;
+
+/* Bits of the device status word returned by attn_get_device_status(). */
+#define ATTN_DEVICE_TIMEOUT 1u      /* a pipeline wait exceeded its limit; that CTA bailed out */
+#define ATTN_DEVICE_BAD_PAGE 2u     /* a block-table entry outside [0, num_pages) was skipped */
+#define ATTN_DEVICE_BAD_SEQLEN 4u   /* a seq_len outside [1, max_blocks*page_size]; row set to NaN */
+
+/*
+ * attn_fwd -- attention forward (prefill), FlashAttention-style.
+ *
+ * Computes, for every batch b, query head h and query position i,
+ *   O[b,h,i,:] = sum_j softmax_j(scale * q_i . k_j) v_j,   LSE[b,h,i] = ln sum_j exp(scale * q_i . k_j)
+ * over the visible keys j, where q_i = Q[b,h,i,:] and k_j, v_j come from K/V head h / (Hq/Hkv)
+ * ("attention-transformers", Q "How does self-attention work in a transformer?";
+ * "Transformer Complexity, Inference Optimization, GQA and FlashAttention", Part 3 for
+ * grouped-query attention). The computation tiles Q, K and V through on-chip memory with the
+ * online softmax of "Why is attention O(n^2), how does FlashAttention help, ...",
+ * "Deep dive: FlashAttention"; LSE is the saved row statistic m + ln(l) of that section.
+ *
+ *   q      bf16 [B, Hq,  N, D] device, read only
+ *   k, v   bf16 [B, Hkv, N, D] device, read only
+ *   o      bf16 [B, Hq,  N, D] device, written
+ *   lse    fp32 [B, Hq,  N]    device, written (natural log), or NULL to skip
+ *   causal 1: key j visible to query i iff j <= i (mask on the logits, "Transformer Attention
+ *          Mechanism Interview Deep Dive", "Causal masking"); 0: every key visible.
+ *   window >0: additionally j >= i - window + 1 (sliding window of width `window`,
+ *          "attention-transformers", Q "What is sparse / sliding-window attention?");
+ *          requires causal = 1. <=0: no window.
+ *   rope_base  >0: rotate q and k pairwise, pairs (2t, 2t+1) by pos * rope_base^(-2t/D), pos =
+ *          the token index 0..N-1, counter-clockwise, then round to bf16 ("attention-transformers",
+ *          Q "How does Rotary Position Embedding (RoPE) work?"). <=0: no rotation.
+ *   scale  >0: softmax scale; <=0: 1/sqrt(D) ("Why is attention scaled by 1/sqrt(dk)?").
+ * Constraints: B, Hq, Hkv, N >= 1; Hq % Hkv == 0; D in {64, 128} (else ATTN_ERR_UNSUPPORTED);
+ * B <= 65535 and ceil(N/128) <= 65535. Fully masked key tiles are skipped, not computed.
+ * Errors: ATTN_ERR_INVALID_ARG for NULL/misaligned pointers or inconsistent sizes/flags;
+ * ATTN_ERR_CUDA when a runtime call or the launch fails. With RoPE, the first call for a new
+ * (device, rope_base, D, N) or a new stream allocates cached device memory (cudaMalloc).
+ */
+attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                     int N, int D, int causal, int window, float rope_base, float scale, void* stream);
+
+/*
+ * attn_decode_workspace_size -- bytes of device workspace attn_decode_paged needs: fp32 partial
+ * (max, sum, output) states for every (sequence, query head, 512-token split). Returns 0 for
+ * invalid sizes.
+ */
+size_t attn_decode_workspace_size(int num_seqs, int max_blocks_per_seq, int page_size, int Hq, int D);
+
+/*
+ * attn_decode_paged -- one decode step per sequence over a PagedAttention KV cache.
+ *
+ * The cache is a pool of fixed-size pages; token t of sequence s lives in page
+ * block_table[s][t / page_size], slot t % page_size ("Self-Attention Complexity,
+ * FlashAttention, PagedAttention, and RoPE in Code", Part 3: fixed-size blocks, block tables).
+ * The single query of sequence s (its newest token, position seq_lens[s]-1, already rotated)
+ * attends to all seq_lens[s] cached tokens, which include that token itself. The key range is
+ * split into chunks of 512 tokens whose partial softmax states are merged in ascending order,
+ * so the result depends only on logical token positions: a paged cache and a contiguous copy
+ * of it give bit-identical outputs.
+ *
+ *   q            bf16 [num_seqs, Hq, D] device
+ *   k_pages,
+ *   v_pages      bf16 [num_pages, Hkv, page_size, D] device (RoPE already applied to keys)
+ *   block_table  int32 [num_seqs, max_blocks_per_seq] device; entries past a sequence's last
+ *                page are never read (any value, e.g. -1)
+ *   seq_lens     int32 [num_seqs] device, each in [1, max_blocks_per_seq * page_size]
+ *   o            bf16 [num_seqs, Hq, D] device, written
+ *   lse          fp32 [num_seqs, Hq] device, written (natural log), or NULL
+ *   workspace    device scratch of at least attn_decode_workspace_size(...) bytes, 16-byte
+ *                aligned, owned by the caller; overwritten; calls that overlap on the GPU must
+ *                use different workspaces.
+ *   scale        >0 softmax scale, <=0: 1/sqrt(D)
+ * Constraints: page_size == 16 and D in {64, 128} (else ATTN_ERR_UNSUPPORTED); Hq % Hkv == 0
+ * and Hq / Hkv <= 16; num_seqs, Hkv <= 65535. Slots past seq_len in a sequence's last page may
+ * hold anything (NaN included): they are masked and never reach the output.
+ * Block-table entries and seq_lens are device data and are checked on the device: an invalid
+ * entry sets a bit of the device status word (the page is skipped; the output is then wrong).
+ */
+attn_status attn_decode_paged(const void* q, const void* k_pages, const void* v_pages, const int32_t* block_table,
+                              const int32_t* seq_lens, int num_seqs, int max_blocks_per_seq, int num_pages,
+                              int page_size, int Hq, int Hkv, int D, float scale, void* o, float* lse,
+                              void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * attn_get_device_status -- synchronises `stream` on the current device, returns the device
+ * status word (ATTN_DEVICE_* bits) in *flags_out and clears it. Returns ATTN_ERR_TIMEOUT or
+ * ATTN_ERR_DEVICE_CHECK when a bit was set, ATTN_OK otherwise.
+ */
+attn_status attn_get_device_status(void* stream, int* flags_out);
+
+/* Message of the last failure on the calling thread ("" if none). Owned by the library. */
+const char* attn_last_error(void);
+
+/* Library version string. */
+const char* attn_version(void);
+
+/* Frees every cache the library allocated (RoPE tables, key scratch), on every device.
+ * The caller must ensure no call is still running on the GPU. */
+void attn_shutdown(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATTN_B200_H */

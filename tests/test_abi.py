@@ -1,0 +1,88 @@
+"""The C-ABI library on the CPU: it loads without a GPU, exports every function include/attn.h
+declares, and rejects bad arguments before any CUDA call (no compute call is made here)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from exact_attention_161_b200 import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "attn.h")
+
+
+@pytest.fixture(scope="module")
+def api():
+    build.build()
+    from exact_attention_161_b200 import api as api_mod
+    return api_mod
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(attn_[a-z_]+)\s*\(", text)))
+
+
+def test_header_and_binding_agree(api):
+    assert declared_functions() == sorted(api.SIGNATURES)
+
+
+def test_library_exports_every_declared_symbol(api):
+    lib = ctypes.CDLL(api.LIB_PATH)
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_version_and_error_strings(api):
+    assert "sm_100a" in api.version()
+    assert api.last_error() == ""
+
+
+FAKE = ctypes.c_void_p(0x10000)      # never dereferenced: validation fails first
+MISALIGNED = ctypes.c_void_p(0x10008)
+
+
+def _fwd(api, q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=None, B=1, Hq=4, Hkv=2, N=128, D=128, causal=1, window=0,
+         rope=0.0, scale=0.0):
+    return api.lib.attn_fwd(q, k, v, o, lse, B, Hq, Hkv, N, D, causal, window, rope, scale, None)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(q=None), 1), (dict(o=None), 1), (dict(k=MISALIGNED), 1), (dict(lse=MISALIGNED), 1),
+    (dict(B=0), 1), (dict(N=0), 1), (dict(Hq=3, Hkv=2), 1), (dict(causal=2), 1),
+    (dict(causal=0, window=16), 1), (dict(scale=float("nan")), 1), (dict(rope=float("inf")), 1),
+    (dict(D=96), 2), (dict(D=256), 2), (dict(B=70000), 2), (dict(N=65536 * 128), 2),
+])
+def test_fwd_validation(api, kw, expect):
+    assert _fwd(api, **kw) == expect
+    assert api.last_error() != ""
+
+
+def _dec(api, num_seqs=2, max_blocks=8, num_pages=16, page_size=16, Hq=8, Hkv=2, D=128, ws_bytes=None,
+         ws=FAKE, q=FAKE, bt=FAKE):
+    if ws_bytes is None:
+        ws_bytes = api.decode_workspace_size(num_seqs, max_blocks, page_size, Hq, D)
+    return api.lib.attn_decode_paged(q, FAKE, FAKE, bt, FAKE, num_seqs, max_blocks, num_pages, page_size, Hq, Hkv, D,
+                                     0.0, FAKE, None, ws, ws_bytes, None)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(q=None), 1), (dict(ws=None), 1), (dict(bt=ctypes.c_void_p(0x10002)), 1), (dict(num_seqs=0), 1),
+    (dict(Hq=6, Hkv=4), 1), (dict(ws_bytes=16), 1), (dict(page_size=32), 2), (dict(D=80), 2),
+    (dict(Hq=32, Hkv=1), 2), (dict(num_seqs=70000), 2),
+])
+def test_decode_validation(api, kw, expect):
+    assert _dec(api, **kw) == expect
+
+
+def test_workspace_size(api):
+    # per (sequence, head, 512-token split): D partial outputs plus (max, sum), fp32, 256-B rounded
+    assert api.decode_workspace_size(64, 1024, 16, 32, 128) == 64 * 32 * 32 * 130 * 4
+    assert api.decode_workspace_size(1, 1, 16, 1, 64) == 512
+    assert api.decode_workspace_size(0, 1, 16, 1, 64) == 0
+
+
+def test_device_status_needs_out_pointer(api):
+    assert api.lib.attn_get_device_status(None, None) == 1
