@@ -1,0 +1,67 @@
+"""The benchmark's host logic (CPU only): the pair counts behind its FLOP numbers, and the
+multi-rank path -- barrier, max-over-ranks timing and whole-job throughput -- on two gloo ranks."""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+import bench
+
+
+@pytest.mark.parametrize("N,causal,window", [(1, 0, 0), (7, 0, 0), (128, 1, 0), (300, 1, 7), (300, 1, 1),
+                                             (300, 1, 299), (300, 1, 300), (300, 1, 5000)])
+def test_visible_pairs_closed_form(N, causal, window):
+    i = np.arange(N)[:, None]
+    j = np.arange(N)[None, :]
+    vis = np.ones((N, N), bool)
+    if causal:
+        vis &= j <= i
+    if window > 0:
+        vis &= j >= i - window + 1
+    assert bench.visible_pairs(N, causal, window) == int(vis.sum())
+
+
+def test_headline_flops():
+    # 4 * D * N(N+1)/2 * B * Hq for the causal GQA N=8192 workload
+    assert bench.prefill_flops() == 4 * 128 * (8192 * 8193 // 2) * 2 * 32
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world),
+                      LOCAL_RANK=str(rank))
+    r, w, local = bench.dist_env()
+    bench.init_dist(w, "gloo")
+    bench.barrier(w)
+    elapsed = 10.0 + 5.0 * r          # rank 1 is the slow one
+    mx = bench.reduce_max(elapsed, w)
+    value = bench.job_throughput(units_per_rank=1000.0, world=w, seconds=mx)
+    out[r] = (r, w, local, mx, value)
+    torch.distributed.destroy_process_group()
+
+
+def test_two_gloo_ranks_take_the_max_and_sum_the_work():
+    world = 2
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    mgr = ctx.Manager()
+    out = mgr.dict()
+    procs = [ctx.Process(target=_rank_main, args=(r, world, port, out)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    for r in range(world):
+        rr, w, local, mx, value = out[r]
+        assert (rr, w, local) == (r, world, r)
+        assert mx == 15.0                      # slowest rank
+        assert value == 1000.0 * world / 15.0  # all ranks' units over the slowest time
