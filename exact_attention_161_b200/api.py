@@ -29,6 +29,7 @@ SIGNATURES = {
     "attn_fwd": (_i, [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _f, _f, _p]),
     "attn_decode_workspace_size": (_sz, [_i, _i, _i, _i, _i]),
     "attn_decode_paged": (_i, [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _f, _p, _p, _p, _sz, _p]),
+    "attn_decode_paged_noalloc": (_i, [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _f, _p, _p, _p]),
     "attn_get_device_status": (_i, [_p, ctypes.POINTER(ctypes.c_int)]),
     "attn_last_error": (ctypes.c_char_p, []),
     "attn_version": (ctypes.c_char_p, []),
@@ -139,6 +140,30 @@ def attn_decode_paged(q, k_pages, v_pages, block_table, seq_lens, scale=0.0, o=N
                                  _dev_tensor(lse, "lse", torch.float32) if lse is not None else None,
                                  _dev_tensor(workspace, "workspace", torch.uint8),
                                  workspace.numel() * workspace.element_size(), _stream(stream)))
+    return o, lse
+
+
+DECODE_NOALLOC_MAX_BYTES = 40 << 20
+
+
+def attn_decode_paged_noalloc(q, k_pages, v_pages, block_table, seq_lens, scale=0.0, o=None, lse=None,
+                              want_lse=True, stream=None):
+    """attn_decode_paged without a workspace, for callers that cannot allocate device memory at
+    call time; its scratch is a fixed 40 MiB array inside the library, shared by every call
+    (calls that overlap on the GPU race). Outputs must be passed in to allocate nothing here."""
+    S, Hq, D = q.shape
+    num_pages, Hkv, page_size, _ = k_pages.shape
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((S, Hq), dtype=torch.float32, device=q.device)
+    args = [_dev_tensor(q, "q", torch.bfloat16), _dev_tensor(k_pages, "k_pages", torch.bfloat16),
+            _dev_tensor(v_pages, "v_pages", torch.bfloat16), _dev_tensor(block_table, "block_table", torch.int32),
+            _dev_tensor(seq_lens, "seq_lens", torch.int32)]
+    _check(lib.attn_decode_paged_noalloc(*args, S, block_table.shape[1], num_pages, page_size, Hq, Hkv, D,
+                                         float(scale), _dev_tensor(o, "o", torch.bfloat16),
+                                         _dev_tensor(lse, "lse", torch.float32) if lse is not None else None,
+                                         _stream(stream)))
     return o, lse
 
 

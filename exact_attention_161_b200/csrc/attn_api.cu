@@ -350,3 +350,59 @@ void attn_shutdown(void) {
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------ decode without allocation
+// Some callers cannot allocate device memory when they call in: a plugin hosted by a framework
+// that owns the device's memory pool and hands out no scratch buffers, or a serving loop that
+// cannot afford cudaMalloc's implicit device-wide synchronisation. For them the split-KV decode
+// runs with its partial states in this fixed array instead of a caller workspace. Every GPU that
+// loads the library holds the array until the process exits.
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = ATTN_DECODE_NOALLOC_MAX_BYTES;  // 40 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[64] = {};  // device address of g_noalloc_scratch, per device
+
+// Host code must not use g_noalloc_scratch's name as an address (on the host it is only a
+// stand-in); the device address is looked up once per device with that device current.
+attn_status noalloc_scratch(int dev, void** out) {
+    if (dev < 0 || dev >= 64) return fail(ATTN_ERR_CUDA, "device index %d out of range", dev);
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void* p = nullptr;
+        const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess || p == nullptr)
+            return fail(ATTN_ERR_CUDA, "cudaGetSymbolAddress(no-alloc scratch): %s", cudaGetErrorString(e));
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return ATTN_OK;
+}
+
+}  // namespace
+
+extern "C" attn_status attn_decode_paged_noalloc(const void* q, const void* k_pages, const void* v_pages,
+                                                 const int32_t* block_table, const int32_t* seq_lens, int num_seqs,
+                                                 int max_blocks_per_seq, int num_pages, int page_size, int Hq,
+                                                 int Hkv, int D, float scale, void* o, float* lse, void* stream) {
+    g_last_error.clear();
+    if (num_seqs < 1 || max_blocks_per_seq < 1 || page_size < 1 || Hq < 1 || D < 1)
+        return fail(ATTN_ERR_INVALID_ARG, "sizes must be >= 1");
+    const size_t need = attn_decode_workspace_size(num_seqs, max_blocks_per_seq, page_size, Hq, D);
+    if (need > kNoAllocScratchBytes)
+        return fail(ATTN_ERR_INVALID_ARG,
+                    "decode needs %zu bytes of scratch, above the no-alloc limit of %zu bytes (40 MiB); "
+                    "use attn_decode_paged with a caller workspace",
+                    need, kNoAllocScratchBytes);
+    int dev = 0;
+    CUDA_TRY(cudaGetDevice(&dev));
+    void* scratch = nullptr;
+    const attn_status st = noalloc_scratch(dev, &scratch);
+    if (st != ATTN_OK) return st;
+    // Same checks and kernels as attn_decode_paged; the split kernel writes every partial state
+    // the merge reads within the call, so nothing in the scratch has to start at zero.
+    return attn_decode_paged(q, k_pages, v_pages, block_table, seq_lens, num_seqs, max_blocks_per_seq, num_pages,
+                             page_size, Hq, Hkv, D, scale, o, lse, scratch, kNoAllocScratchBytes, stream);
+}

@@ -121,6 +121,31 @@ attn_status attn_decode_paged(const void* q, const void* k_pages, const void* v_
                               void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * attn_decode_paged_noalloc -- attn_decode_paged for callers that cannot allocate device memory.
+ * The pages have no counterpart to this entry point; it exists for callers that cannot call
+ * cudaMalloc when they call in -- for example a plugin inside a framework that owns the device's
+ * memory pool and hands out no scratch buffers, or a serving loop that cannot afford cudaMalloc's
+ * implicit device-wide synchronisation.
+ *
+ * Same arguments, computation, results and checks as attn_decode_paged, without the workspace:
+ * the partial softmax states live in one fixed device array of ATTN_DECODE_NOALLOC_MAX_BYTES
+ * compiled into the library (every GPU that loads the library holds it until the process exits).
+ * The call allocates nothing. Limits and sharing:
+ *   - requests whose attn_decode_workspace_size(...) exceeds ATTN_DECODE_NOALLOC_MAX_BYTES are
+ *     rejected with ATTN_ERR_INVALID_ARG and a message naming the limit;
+ *   - every call, on every stream, uses the same array and leaves its contents behind; nothing in
+ *     it needs to start at zero (each call writes every partial state it reads), but calls that
+ *     overlap on the GPU race on it and must be serialised by the caller;
+ *   - the first call on each device looks up the array's device address (cudaGetSymbolAddress,
+ *     with that device current); make that first call before any stream capture.
+ */
+#define ATTN_DECODE_NOALLOC_MAX_BYTES ((size_t)40 << 20)
+attn_status attn_decode_paged_noalloc(const void* q, const void* k_pages, const void* v_pages,
+                                      const int32_t* block_table, const int32_t* seq_lens, int num_seqs,
+                                      int max_blocks_per_seq, int num_pages, int page_size, int Hq, int Hkv, int D,
+                                      float scale, void* o, float* lse, void* stream);
+
+/*
  * attn_get_device_status -- synchronises `stream` on the current device, returns the device
  * status word (ATTN_DEVICE_* bits) in *flags_out and clears it. Returns ATTN_ERR_TIMEOUT or
  * ATTN_ERR_DEVICE_CHECK when a bit was set, ATTN_OK otherwise.
