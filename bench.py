@@ -170,7 +170,7 @@ def kernel_source_hash():
 def profiled_traffic(kind):
     """DRAM bytes per launch from the committed ncu summary, or None when the kernels changed
     after the counters were taken."""
-    path = os.path.join(ROOT, "profiles", "traffic.json")
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
     if not os.path.exists(path):
         return None
     with open(path) as f:
@@ -183,21 +183,22 @@ def profiled_traffic(kind):
 # ------------------------------------------------------------------------------ CPU baseline (oracle)
 def oracle_prefill_sample(q, k, v, budget_s):
     """Time the fp64 oracle on a bounded sample of prefill rows; returns (TFLOP/s, rows, seconds,
-    threads). Rows are spread over all positions of one head so the mix of causal lengths
-    matches the workload."""
+    threads). The rows are evenly spaced over every (batch, head, position) of the workload, so
+    the mix of causal lengths matches it."""
     import oracle
     qb, kb, vb = synth.bits(q), synth.bits(k), synth.bits(v)
     N, D = PREFILL.N, PREFILL.D
+    total = PREFILL.B * PREFILL.Hq * N
 
     def run(n_rows):
-        rows = np.linspace(0, N - 1, n_rows).astype(np.int64)
-        flops = sum(4 * D * (int(i) + 1) for i in rows)
+        rows = np.linspace(0, total - 1, n_rows).astype(np.int64)
+        flops = int((4 * D * ((rows % N) + 1)).sum())
         t0 = time.perf_counter()
         oracle.attention(qb, kb, vb, causal=True, rope_base=PREFILL.rope_base, scale=PREFILL.scale, rows=rows)
         return flops, time.perf_counter() - t0
 
-    f, t = run(64)  # calibration (includes the one-off key rotation)
-    n = int(min(N, max(64, 64 * budget_s / max(t, 1e-3))))
+    f, t = run(256)  # calibration (includes the one-off key rotation of every KV head)
+    n = int(min(total, max(256, 256 * budget_s / max(t, 1e-3))))
     f, t = run(n)
     return f / t / 1e12, n, t, oracle.max_threads()
 
@@ -229,17 +230,21 @@ def run_ours(args, rank, world, local):
     init_dist(world, "nccl")
     stream = torch.cuda.current_stream()
 
-    q_h, k_h, v_h = synth.prefill_inputs_for(PREFILL)
-    cache_h = synth.paged_decode_inputs_for(DECODE)
-    q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
-    o = torch.empty_like(q)
-    lse = torch.empty((PREFILL.B, PREFILL.Hq, PREFILL.N), dtype=torch.float32, device=dev)
-    dq, kp, vp = cache_h.q.to(dev), cache_h.k_pages.to(dev), cache_h.v_pages.to(dev)
-    bt, sl = cache_h.block_table.to(dev), cache_h.seq_lens.to(dev)
-    do = torch.empty_like(dq)
-    dlse = torch.empty((DECODE.num_seqs, DECODE.Hq), dtype=torch.float32, device=dev)
-    ws = torch.empty(api.decode_workspace_size(DECODE.num_seqs, cache_h.max_blocks, DECODE.page_size, DECODE.Hq,
-                                               DECODE.D), dtype=torch.uint8, device=dev)
+    do_prefill = args.only in ("all", "prefill")
+    do_decode = args.only in ("all", "decode")
+    if do_prefill:
+        q_h, k_h, v_h = synth.prefill_inputs_for(PREFILL)
+        q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
+        o = torch.empty_like(q)
+        lse = torch.empty((PREFILL.B, PREFILL.Hq, PREFILL.N), dtype=torch.float32, device=dev)
+    if do_decode:
+        cache_h = synth.paged_decode_inputs_for(DECODE)
+        dq, kp, vp = cache_h.q.to(dev), cache_h.k_pages.to(dev), cache_h.v_pages.to(dev)
+        bt, sl = cache_h.block_table.to(dev), cache_h.seq_lens.to(dev)
+        do = torch.empty_like(dq)
+        dlse = torch.empty((DECODE.num_seqs, DECODE.Hq), dtype=torch.float32, device=dev)
+        ws = torch.empty(api.decode_workspace_size(DECODE.num_seqs, cache_h.max_blocks, DECODE.page_size,
+                                                   DECODE.Hq, DECODE.D), dtype=torch.uint8, device=dev)
 
     def prefill():
         api.attn_fwd(q, k, v, causal=PREFILL.causal, window=PREFILL.window, rope_base=PREFILL.rope_base,
@@ -249,8 +254,10 @@ def run_ours(args, rank, world, local):
         api.attn_decode_paged(dq, kp, vp, bt, sl, o=do, lse=dlse, workspace=ws, stream=stream)
 
     for _ in range(args.warmup):
-        prefill()
-        decode()
+        if do_prefill:
+            prefill()
+        if do_decode:
+            decode()
     torch.cuda.synchronize()
     if api.device_status() != 0:
         raise RuntimeError("device status raised during warm-up")
@@ -267,9 +274,11 @@ def run_ours(args, rank, world, local):
     t_start.record(stream)
     for s in range(K):
         ev[s][0].record(stream)
-        prefill()
+        if do_prefill:
+            prefill()
         ev[s][1].record(stream)
-        decode()
+        if do_decode:
+            decode()
         ev[s][2].record(stream)
     t_end.record(stream)
     torch.cuda.synchronize()
@@ -284,20 +293,21 @@ def run_ours(args, rank, world, local):
     prefill_sum_max = reduce_max(sum(prefill_ms), world, dev)
     decode_sum_max = reduce_max(sum(decode_ms), world, dev)
     flops = prefill_flops()
-    dbytes = decode_bytes(cache_h)
-    value = job_throughput(flops * K, world, prefill_sum_max / 1e3) / 1e12
-    decode_value = job_throughput(dbytes * K, world, decode_sum_max / 1e3) / 1e9
+    dbytes = decode_bytes(cache_h) if do_decode else 0
+    value = job_throughput(flops * K, world, prefill_sum_max / 1e3) / 1e12 if do_prefill else None
+    decode_value = job_throughput(dbytes * K, world, decode_sum_max / 1e3) / 1e9 if do_decode else None
 
     # ---- end to end through the public API with pinned host buffers
-    E = max(3, min(args.e2e_steps, K))
-    q_p, k_p, v_p = q_h.pin_memory(), k_h.pin_memory(), v_h.pin_memory()
-    o_p = torch.empty(o.shape, dtype=o.dtype).pin_memory()
-    lse_p = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
-    dq_p, bt_p, sl_p = cache_h.q.pin_memory(), cache_h.block_table.pin_memory(), cache_h.seq_lens.pin_memory()
-    do_p = torch.empty(do.shape, dtype=do.dtype).pin_memory()
-    dlse_p = torch.empty(dlse.shape, dtype=dlse.dtype).pin_memory()
+    E = min(args.e2e_steps, K) if (args.e2e_steps > 0 and args.only == "all") else 0
+    if E:
+        q_p, k_p, v_p = q_h.pin_memory(), k_h.pin_memory(), v_h.pin_memory()
+        o_p = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        lse_p = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+        dq_p, bt_p, sl_p = cache_h.q.pin_memory(), cache_h.block_table.pin_memory(), cache_h.seq_lens.pin_memory()
+        do_p = torch.empty(do.shape, dtype=do.dtype).pin_memory()
+        dlse_p = torch.empty(dlse.shape, dtype=dlse.dtype).pin_memory()
     e_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(E)]
-    for s in range(E + 1):  # the first pass is a warm-up
+    for s in range(E + 1 if E else 0):  # the first pass is a warm-up
         r = e_ev[s - 1] if s > 0 else [torch.cuda.Event(enable_timing=True) for _ in range(3)]
         r[0].record(stream)
         q.copy_(q_p, non_blocking=True)
@@ -315,27 +325,27 @@ def run_ours(args, rank, world, local):
         dlse_p.copy_(dlse, non_blocking=True)
         r[2].record(stream)
     torch.cuda.synchronize()
-    e_pre = reduce_max(sum(e[0].elapsed_time(e[1]) for e in e_ev), world, dev)
-    e_dec = reduce_max(sum(e[1].elapsed_time(e[2]) for e in e_ev), world, dev)
-    h2d = sum(t.numel() * t.element_size() for t in (q_h, k_h, v_h))
-    d2h = o.numel() * 2 + lse.numel() * 4
-    dh2d = sum(t.numel() * t.element_size() for t in (cache_h.q, cache_h.block_table, cache_h.seq_lens))
-    dd2h = do.numel() * 2 + dlse.numel() * 4
-    e2e_value = job_throughput(flops * E, world, e_pre / 1e3) / 1e12
-    e2e_decode = job_throughput(dbytes * E, world, e_dec / 1e3) / 1e9
+    e_pre = reduce_max(sum(e[0].elapsed_time(e[1]) for e in e_ev), world, dev) if E else float("nan")
+    e_dec = reduce_max(sum(e[1].elapsed_time(e[2]) for e in e_ev), world, dev) if E else float("nan")
+    h2d = sum(t.numel() * t.element_size() for t in (q_h, k_h, v_h)) if do_prefill else 0
+    d2h = o.numel() * 2 + lse.numel() * 4 if do_prefill else 0
+    dh2d = sum(t.numel() * t.element_size() for t in (cache_h.q, cache_h.block_table, cache_h.seq_lens)) if do_decode else 0
+    dd2h = do.numel() * 2 + dlse.numel() * 4 if do_decode else 0
+    e2e_value = job_throughput(flops * E, world, e_pre / 1e3) / 1e12 if E else None
+    e2e_decode = job_throughput(dbytes * E, world, e_dec / 1e3) / 1e9 if E else None
 
     if rank != 0:
         return None
     peaks, peaks_kind = measured_peaks()
     pre_launch_ms = statistics.mean(prefill_ms)
     dec_launch_ms = statistics.mean(decode_ms)
-    tflops_launch = flops / (pre_launch_ms / 1e3) / 1e12
-    gbs_launch = dbytes / (dec_launch_ms / 1e3) / 1e9
+    tflops_launch = flops / (pre_launch_ms / 1e3) / 1e12 if do_prefill else float("nan")
+    gbs_launch = dbytes / (dec_launch_ms / 1e3) / 1e9 if do_decode else float("nan")
     tensor_peak = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
     line = {
         "metric": "attn fwd TFLOP/s (causal GQA prefill B2 Hq32 Hkv8 N8192 D128, RoPE 5e5) "
                   "& paged-decode KV GB/s",
-        "value": round(value, 2),
+        "value": round(value, 2) if do_prefill else None,
         "unit": "TFLOP/s",
         "n_gpus": world,
         "steps": K,
@@ -352,18 +362,18 @@ def run_ours(args, rank, world, local):
                         "causal": PREFILL.causal, "window": PREFILL.window, "rope_base": PREFILL.rope_base,
                         "flops_per_step": flops},
             "decode": {"num_seqs": DECODE.num_seqs, "Hq": DECODE.Hq, "Hkv": DECODE.Hkv, "D": DECODE.D,
-                       "page_size": DECODE.page_size, "total_tokens": cache_h.total_tokens,
+                       "page_size": DECODE.page_size, "total_tokens": cache_h.total_tokens if do_decode else None,
                        "bytes_per_step": dbytes},
             "l2": "inputs larger than L2 (prefill Q/K/V 201 MB, decode KV 2.2 GB); no flush",
             "parallelism": "replica per GPU" if world > 1 else "single GPU",
         },
-        "decode": {"metric": "paged-decode KV GB/s", "value": round(decode_value, 1), "unit": "GB/s",
+        "decode": {"metric": "paged-decode KV GB/s", "value": round(decode_value, 1) if do_decode else None, "unit": "GB/s",
                    "ms_per_step": round(decode_sum_max / K, 4),
                    "roofline": {"bound": "hbm", "achieved": round(gbs_launch, 1), "peak": peaks["hbm_gbs"],
                                 "unit": "GB/s", "frac": round(gbs_launch / peaks["hbm_gbs"], 4),
                                 "peak_kind": peaks_kind, "frac_of_8TBs": round(gbs_launch / DATASHEET_HBM_GBS, 4),
                                 "traffic": profiled_traffic("decode_split")},
-                   "e2e": {"value": round(e2e_decode, 2), "unit": "GB/s", "h2d_bytes_per_step": dh2d,
+                   "e2e": {"value": round(e2e_decode, 2) if E else None, "unit": "GB/s", "h2d_bytes_per_step": dh2d,
                            "d2h_bytes_per_step": dd2h}},
         "roofline": {"bound": "tensor", "achieved": round(tflops_launch, 2), "peak": tensor_peak, "unit": "TFLOP/s",
                      "frac": round(tflops_launch / tensor_peak, 4),
@@ -371,9 +381,9 @@ def run_ours(args, rank, world, local):
                      "frac_of_2250": round(tflops_launch / DATASHEET_BF16_TFLOPS, 4),
                      "traffic": profiled_traffic("attn_fwd"),
                      "kernel": "attn_fwd_kernel<128> (+ key rotation pass, inside the timed call)"},
-        "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+        "e2e": {"value": round(e2e_value, 2) if E else None, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
-        "gpu_launches": 4 * K,
+        "gpu_launches": (2 * do_prefill + 2 * do_decode) * K,
         "device_status": status,
         "clocks": clk,
     }
@@ -389,8 +399,8 @@ def add_cpu_baseline(line, args):
     cache = synth.paged_decode_inputs_for(DECODE)
     gbs, ns, td = oracle_decode_sample(cache, args.cpu_budget / 2)
     line["cpu_baseline"] = {"value": round(tf, 6), "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
-                            "sample": "%d query rows spread over positions 0..8191 of one head of the prefill "
-                                      "workload (causal, RoPE), %.1f s" % (n, t),
+                            "sample": "%d query rows evenly spaced over all (batch, head, position) of the "
+                                      "prefill workload (causal, RoPE), %.1f s" % (n, t),
                             "decode": {"value": round(gbs, 4), "unit": "GB/s",
                                        "sample": "%d of 64 sequences, %.1f s" % (ns, td)}}
 
@@ -450,7 +460,9 @@ def parse_args(argv=None):
     ap.add_argument("--steps", type=int, default=400)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--e2e-steps", type=int, default=10, help="0 skips the end-to-end leg")
+    ap.add_argument("--only", choices=["all", "prefill", "decode"], default="all",
+                    help="time one half of the step only (profiling runs); the JSON line is then partial")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle time for the CPU baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing (profiling runs)")
     args = ap.parse_args(argv)
@@ -468,7 +480,7 @@ def main(argv=None):
         line = run_reference(args, rank, world)
     else:
         line = run_ours(args, rank, world, local)
-        if line is not None and world == 1:
+        if line is not None and world == 1 and args.only == "all":
             add_cpu_baseline(line, args)
         elif line is not None:
             line["cpu_baseline"] = None
