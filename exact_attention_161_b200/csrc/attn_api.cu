@@ -14,7 +14,7 @@
 #include <tuple>
 #include <vector>
 
-#include "../../include/attn.h"
+#include "attn.h"
 #include "common.cuh"
 #include "decode.cuh"
 #include "fwd_sm100.cuh"
@@ -197,7 +197,7 @@ attn_status launch_fwd(const void* q, const void* k, const void* v, void* o, flo
     p.window = window > 0 ? window : 0;
     p.scale_log2 = scale * attn::kLog2e;
     if ((st = ensure_smem(attn::attn_fwd_kernel<D>, C::SMEM_BYTES, dev)) != ATTN_OK) return st;
-    const dim3 grid(Hq, B, (N + C::BM - 1) / C::BM);
+    const dim3 grid(Hq, B, (N + C::QT * C::BM - 1) / (C::QT * C::BM));
     attn::attn_fwd_kernel<D><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
     CUDA_TRY(cudaGetLastError());
     return ATTN_OK;
@@ -257,7 +257,7 @@ attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float
     if (window > 0 && !causal) return fail(ATTN_ERR_INVALID_ARG, "a sliding window requires causal = 1");
     if (!std::isfinite(scale) || !std::isfinite(rope_base)) return fail(ATTN_ERR_INVALID_ARG, "scale and rope_base must be finite");
     if (D != 64 && D != 128) return fail(ATTN_ERR_UNSUPPORTED, "head dim %d not supported (64 or 128)", D);
-    if (B > 65535 || (N + 127) / 128 > 65535) return fail(ATTN_ERR_UNSUPPORTED, "B or N too large for the grid");
+    if (B > 65535 || (N + 255) / 256 > 65535) return fail(ATTN_ERR_UNSUPPORTED, "B or N too large for the grid");
     if (static_cast<double>(B) * Hq * N * D * 2 >= 1099511627776.0)
         return fail(ATTN_ERR_UNSUPPORTED, "tensor larger than 1 TiB");
     if (scale <= 0.f) scale = 1.0f / std::sqrt(static_cast<float>(D));

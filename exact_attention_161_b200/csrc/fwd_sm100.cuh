@@ -1,28 +1,33 @@
 // fwd_sm100.cuh -- FlashAttention-style exact attention forward for sm_100a.
 //
-// One CTA computes one 128-row tile of queries of one (batch, query head). It streams the
-// visible 128-key tiles of the matching K/V head through shared memory and keeps the online
-// softmax state per row: running max m, normaliser l and output accumulator o, rescaled as the
-// max grows, then O = o / l and the row logsumexp ("Why is attention O(n^2), how does
-// FlashAttention help, ...", "Deep dive: FlashAttention"). The n x n score matrix never leaves
-// the SM: each 128x128 score tile lives in Tensor Memory only.
+// One CTA computes two 128-row query tiles (256 consecutive queries) of one (batch, query head).
+// Both tiles stream the same visible 128-key tiles of the matching K/V head through shared
+// memory, so each K/V tile loaded serves 256 query rows. Per row the online softmax keeps the
+// running max m, the normaliser l and the output accumulator o, rescaled as the max grows, then
+// O = o / l and the row logsumexp ("Why is attention O(n^2), how does FlashAttention help, ...",
+// "Deep dive: FlashAttention"). The n x n score matrix never leaves the SM: each 128x128 score
+// tile lives in Tensor Memory only.
 //
-// Roles (192 threads):
-//   warps 0-3  softmax: thread r owns query row r of the tile; it rotates its Q row (RoPE) once,
-//              then per key tile reads its 128 scores from TMEM, masks them, updates m and l,
-//              writes P (bf16) back into TMEM over the first half of the scores, rescales its
-//              row of O when the max moved by more than 2^8, and finally writes O and LSE.
-//   warp 4     TMA producer: Q once, then K and V tiles into a NS-stage ring.
-//   warp 5     MMA issuer (one thread) and TMEM owner: S = Q K^T into one of two TMEM score
-//              buffers, O += P V with P read from TMEM, completion signalled by tcgen05.commit.
+// Roles (320 threads):
+//   warps 0-3, 4-7  softmax warpgroup i (i = 0, 1) owns query tile i; thread r owns row r (TMEM
+//              lane r). It rotates its Q row (RoPE) once, then per key tile reads its 128 scores
+//              from TMEM with one load, masks them, updates m and l, writes P (bf16) back into
+//              TMEM over the first half of its score buffer, rescales its row of O when the max
+//              moved by more than 2^8, and finally writes O and LSE.
+//   warp 8     TMA producer: the Q tiles once, then K tiles into a NK-stage ring and V tiles into
+//              a NV-stage ring.
+//   warp 9     MMA issuer (one thread) and TMEM owner.
 //
-// Tensor Memory (512 columns x 128 lanes x 32 bit): S0 at column 0, S1 at 128, O at 256
-// (D columns). The score buffers alternate per key tile, so the tensor core computes the next
-// tile's scores while the softmax works on the current one.
+// Tensor Memory (512 columns): S0 at 0, S1 at 128, O0 at 256, O1 at 256 + D. The MMA thread
+// issues, per key tile j:  O0 += P0(j) V(j);  S0(j+1) = Q0 K(j+1)^T;  O1 += P1(j) V(j);
+// S1(j+1) = Q1 K(j+1)^T. So while warpgroup 0 computes the softmax of S0(j+1), the tensor core
+// works on tile 1's products, and the other way round. tcgen05.mma executes in issue order, so
+// when a warpgroup sees S_i(j+1) complete, the product O_i += P_i(j) V(j) issued before it has
+// completed too: the warpgroup may then overwrite P_i and rescale O_i without a further wait.
 //
 // Masks enter as -inf on the logits before the softmax ("Transformer Attention Mechanism
-// Interview Deep Dive", "Causal masking"); key tiles that are fully masked are never visited
-// (causal: tiles past the diagonal; sliding window: tiles before the window), which is the
+// Interview Deep Dive", "Causal masking"); key tiles fully masked for a query tile are never
+// visited by it (causal: tiles past the diagonal; sliding window: tiles before the window), the
 // block skipping of "Deep dive: FlashAttention".
 #pragma once
 #include "common.cuh"
@@ -44,29 +49,49 @@ struct FwdCfg {
     static_assert(D == 64 || D == 128, "head dim 64 or 128");
     static constexpr int BM = 128;                    // query rows per tile
     static constexpr int BN = 128;                    // keys per tile
+    static constexpr int QT = 2;                      // query tiles per CTA
     static constexpr int NREG = D / 64;               // 128-byte swizzle regions per row
     static constexpr int REGION_BYTES = 128 * 128;    // 128 rows x 128 bytes
     static constexpr int TILE_BYTES = 128 * D * 2;    // one Q, K or V tile in bf16
-    static constexpr int NS = (D == 128) ? 2 : 4;     // K/V pipeline stages
-    static constexpr int SMEM_TILES = 1 + 2 * NS;
+    static constexpr int NK = (D == 128) ? 3 : 4;     // K pipeline stages
+    static constexpr int NV = (D == 128) ? 2 : 4;     // V pipeline stages
+    static constexpr int SMEM_TILES = QT + NK + NV;
     static constexpr int SMEM_BYTES = SMEM_TILES * TILE_BYTES + 1024 /*barriers*/ + 1024 /*align*/;
     static constexpr uint32_t TMEM_COLS = 512;
-    static constexpr uint32_t TMEM_S0 = 0, TMEM_S1 = 128, TMEM_O = 256;
-    static constexpr int THREADS = 192;
+    // TMEM columns of the score buffer and the output accumulator of query tile i
+    static __device__ __forceinline__ uint32_t tmem_s(int i) { return 128u * i; }
+    static __device__ __forceinline__ uint32_t tmem_o(int i) { return 256u + uint32_t(D) * i; }
+    static constexpr int THREADS = 320;
+    static constexpr int PRODUCER_WARP = 8, MMA_WARP = 9;
     // Rescale the output only when the running max grew by more than this (log2 units): with a
     // stale max the probabilities stay below 2^8, exact after the final division by l.
     static constexpr float RESCALE_THRESHOLD = 8.0f;
 };
 
-template <int NS>
+template <int NK, int NV>
 struct FwdBarriers {
-    uint64_t q_loaded, q_ready;
-    uint64_t k_full[NS], v_full[NS], kv_empty[NS];
-    uint64_t s_full[2], p_full[2];
-    uint64_t o_done, o_final, drain;
+    uint64_t q_loaded[2], q_ready[2];
+    uint64_t k_full[NK], k_empty[NK], v_full[NV], v_empty[NV];
+    uint64_t s_full[2], p_full[2], o_final[2];
+    uint64_t drain;
     uint32_t tmem_base;
     int abort;
 };
+
+// Key-tile range of one query tile: [jb, jb + n) of 128-key tiles with at least one visible key.
+struct TileRange {
+    int q0, jb, n;
+};
+
+__device__ __forceinline__ TileRange tile_range(int q0, int N, int causal, int window) {
+    TileRange t{q0, 0, 0};
+    if (q0 >= N) return t;
+    const int hi = causal ? min(N, q0 + 128) : N;             // exclusive
+    const int lo = window > 0 ? max(0, q0 - window + 1) : 0;  // inclusive
+    t.jb = lo / 128;
+    t.n = (hi + 127) / 128 - t.jb;
+    return t;
+}
 
 // Rotate one 128-byte-swizzled row of a Q tile in place: pairs (2i, 2i+1) by pos * theta_i, in
 // fp32 with the (cos, sin) table, rounded back to bf16 ("attention-transformers", Q "How does
@@ -101,49 +126,55 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
     using C = FwdCfg<D>;
-    constexpr int NS = C::NS;
+    constexpr int NK = C::NK, NV = C::NV;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t* sQ = smem;
-    uint8_t* sK = sQ + C::TILE_BYTES;
-    uint8_t* sV = sK + NS * C::TILE_BYTES;
-    auto* bar = reinterpret_cast<FwdBarriers<NS>*>(sV + NS * C::TILE_BYTES);
+    uint8_t* sQ = smem;                                  // QT tiles
+    uint8_t* sK = sQ + C::QT * C::TILE_BYTES;            // NK tiles
+    uint8_t* sV = sK + NK * C::TILE_BYTES;               // NV tiles
+    auto* bar = reinterpret_cast<FwdBarriers<NK, NV>*>(sV + NV * C::TILE_BYTES);
     volatile int* abort_flag = &bar->abort;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int h = blockIdx.x, b = blockIdx.y;
-    const int qt = gridDim.z - 1 - blockIdx.z;  // longest (causal) tiles first
-    const int q0 = qt * C::BM;
-    const int g = h / (p.Hq / p.Hkv);           // query head h reads K/V head h / (Hq/Hkv)
-    const int kv_hi = p.causal ? min(p.N, q0 + C::BM) : p.N;
-    const int kv_lo = p.window > 0 ? max(0, q0 - p.window + 1) : 0;
-    const int j_begin = kv_lo / C::BN;
-    const int T = (kv_hi + C::BN - 1) / C::BN - j_begin;  // >= 1
+    const int blk = gridDim.z - 1 - blockIdx.z;  // longest (causal) blocks first
+    const int g = h / (p.Hq / p.Hkv);            // query head h reads K/V head h / (Hq/Hkv)
+    const TileRange rng[2] = {tile_range(blk * 256, p.N, p.causal, p.window),
+                              tile_range(blk * 256 + 128, p.N, p.causal, p.window)};
+    // Union of the two ranges (contiguous: tile 1 starts no earlier and ends no earlier).
+    const int J0 = rng[0].jb;
+    const int T = (rng[1].n > 0 ? max(rng[0].jb + rng[0].n, rng[1].jb + rng[1].n) : rng[0].jb + rng[0].n) - J0;
+    auto active = [&](int i, int u) {
+        const int j = J0 + u;
+        return rng[i].n > 0 && j >= rng[i].jb && j < rng[i].jb + rng[i].n;
+    };
 
     if (threadIdx.x == 0) {
-        ptx::mbar_init(&bar->q_loaded, 1);
-        ptx::mbar_init(&bar->q_ready, 1);
-        for (int s = 0; s < NS; ++s) {
+        for (int i = 0; i < 2; ++i) {
+            ptx::mbar_init(&bar->q_loaded[i], 1);
+            ptx::mbar_init(&bar->q_ready[i], 1);
+            ptx::mbar_init(&bar->s_full[i], 1);
+            ptx::mbar_init(&bar->p_full[i], 128);
+            ptx::mbar_init(&bar->o_final[i], 1);
+        }
+        for (int s = 0; s < NK; ++s) {
             ptx::mbar_init(&bar->k_full[s], 1);
+            ptx::mbar_init(&bar->k_empty[s], 1);
+        }
+        for (int s = 0; s < NV; ++s) {
             ptx::mbar_init(&bar->v_full[s], 1);
-            ptx::mbar_init(&bar->kv_empty[s], 1);
+            ptx::mbar_init(&bar->v_empty[s], 1);
         }
-        for (int s = 0; s < 2; ++s) {
-            ptx::mbar_init(&bar->s_full[s], 1);
-            ptx::mbar_init(&bar->p_full[s], 128);
-        }
-        ptx::mbar_init(&bar->o_done, 1);
-        ptx::mbar_init(&bar->o_final, 1);
         ptx::mbar_init(&bar->drain, 1);
         bar->abort = 0;
         ptx::fence_mbar_init();
     }
-    if (warp == 4 && lane == 0) {
+    if (warp == C::PRODUCER_WARP && lane == 0) {
         ptx::prefetch_tensormap(&tm_q);
         ptx::prefetch_tensormap(&tm_k);
         ptx::prefetch_tensormap(&tm_v);
     }
-    if (warp == 5) {
+    if (warp == C::MMA_WARP) {
         ptx::tmem_alloc(&bar->tmem_base, C::TMEM_COLS);
         ptx::tmem_relinquish();
     }
@@ -152,34 +183,37 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     ptx::tc_fence_after();
     const uint32_t tmem = bar->tmem_base;
 
-    if (warp == 4) {
+    if (warp == C::PRODUCER_WARP) {
         // ------------------------------------------------------------------ TMA producer
         if (lane == 0) {
             const int zq = b * p.Hq + h, zk = b * p.Hkv + g;
-            ptx::mbar_arrive_expect_tx(&bar->q_loaded, C::TILE_BYTES);
+            for (int i = 0; i < 2; ++i) {
+                if (rng[i].n == 0) continue;
+                ptx::mbar_arrive_expect_tx(&bar->q_loaded[i], C::TILE_BYTES);
 #pragma unroll
-            for (int r = 0; r < C::NREG; ++r)
-                ptx::tma_load_3d(sQ + r * C::REGION_BYTES, &tm_q, &bar->q_loaded, r * 64, q0, zq);
-            int issued = 0;
+                for (int r = 0; r < C::NREG; ++r)
+                    ptx::tma_load_3d(sQ + i * C::TILE_BYTES + r * C::REGION_BYTES, &tm_q, &bar->q_loaded[i], r * 64,
+                                     rng[i].q0, zq);
+            }
+            int k_issued = 0, v_issued = 0;
             bool ok = true;
-            for (int t = 0; t < T && ok; ++t) {
-                const int s = t % NS;
-                if (t >= NS && !ptx::mbar_wait(&bar->kv_empty[s], ((t / NS) - 1) & 1, abort_flag)) {
-                    ok = false;
-                    break;
-                }
-                const int k0 = (j_begin + t) * C::BN;
-                ptx::mbar_arrive_expect_tx(&bar->k_full[s], C::TILE_BYTES);
+            for (int u = 0; u < T && ok; ++u) {
+                const int k0 = (J0 + u) * C::BN;
+                const int sk = u % NK, sv = u % NV;
+                if (u >= NK && !ptx::mbar_wait(&bar->k_empty[sk], ((u / NK) - 1) & 1, abort_flag)) { ok = false; break; }
+                ptx::mbar_arrive_expect_tx(&bar->k_full[sk], C::TILE_BYTES);
 #pragma unroll
                 for (int r = 0; r < C::NREG; ++r)
-                    ptx::tma_load_3d(sK + s * C::TILE_BYTES + r * C::REGION_BYTES, &tm_k, &bar->k_full[s], r * 64,
+                    ptx::tma_load_3d(sK + sk * C::TILE_BYTES + r * C::REGION_BYTES, &tm_k, &bar->k_full[sk], r * 64,
                                      k0, zk);
-                ptx::mbar_arrive_expect_tx(&bar->v_full[s], C::TILE_BYTES);
+                k_issued = u + 1;
+                if (u >= NV && !ptx::mbar_wait(&bar->v_empty[sv], ((u / NV) - 1) & 1, abort_flag)) { ok = false; break; }
+                ptx::mbar_arrive_expect_tx(&bar->v_full[sv], C::TILE_BYTES);
 #pragma unroll
                 for (int r = 0; r < C::NREG; ++r)
-                    ptx::tma_load_3d(sV + s * C::TILE_BYTES + r * C::REGION_BYTES, &tm_v, &bar->v_full[s], r * 64,
+                    ptx::tma_load_3d(sV + sv * C::TILE_BYTES + r * C::REGION_BYTES, &tm_v, &bar->v_full[sv], r * 64,
                                      k0, zk);
-                issued = t + 1;
+                v_issued = u + 1;
             }
             if (!ok) {
                 *abort_flag = 1;
@@ -187,53 +221,74 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
                 // Let the copies already in flight land before the CTA's shared memory is released
                 // (each wait is still bounded).
                 volatile int never = 0;
-                ptx::mbar_wait(&bar->q_loaded, 0, &never);
-                for (int t = max(0, issued - NS); t < issued; ++t) {
-                    const int s = t % NS;
-                    ptx::mbar_wait(&bar->k_full[s], (t / NS) & 1, &never);
-                    ptx::mbar_wait(&bar->v_full[s], (t / NS) & 1, &never);
-                }
+                for (int i = 0; i < 2; ++i)
+                    if (rng[i].n > 0) ptx::mbar_wait(&bar->q_loaded[i], 0, &never);
+                for (int u = max(0, k_issued - NK); u < k_issued; ++u)
+                    ptx::mbar_wait(&bar->k_full[u % NK], (u / NK) & 1, &never);
+                for (int u = max(0, v_issued - NV); u < v_issued; ++u)
+                    ptx::mbar_wait(&bar->v_full[u % NV], (u / NV) & 1, &never);
             }
         }
-    } else if (warp == 5) {
+    } else if (warp == C::MMA_WARP) {
         // ------------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             constexpr uint32_t IDESC_S = ptx::idesc_bf16_f32(128, C::BN, 0, 0);  // Q, K both K-major
             constexpr uint32_t IDESC_O = ptx::idesc_bf16_f32(128, D, 0, 1);      // P K-major, V MN-major
-            const uint32_t sq = ptx::smem_u32(sQ);
-            bool ok = ptx::mbar_wait(&bar->q_ready, 0, abort_flag);
-            bool issued_any = false;
+            bool ok = true, issued_any = false;
+            for (int i = 0; i < 2 && ok; ++i)
+                if (rng[i].n > 0) ok = ptx::mbar_wait(&bar->q_ready[i], 0, abort_flag);
             ptx::tc_fence_after();
-            for (int t = 0; ok && t <= T; ++t) {
-                if (t < T) {
-                    const int s = t % NS;
-                    if (!ptx::mbar_wait(&bar->k_full[s], (t / NS) & 1, abort_flag)) { ok = false; break; }
+            int k_waited = -1, v_waited = -1;
+            // S_i(u) = Q_i K(u)^T into score buffer i.
+            auto issue_s = [&](int i, int u) -> bool {
+                if (k_waited < u) {
+                    if (!ptx::mbar_wait(&bar->k_full[u % NK], (u / NK) & 1, abort_flag)) return false;
                     ptx::tc_fence_after();
-                    const uint32_t sk = ptx::smem_u32(sK + s * C::TILE_BYTES);
-                    const uint32_t d_s = tmem + ((t & 1) ? C::TMEM_S1 : C::TMEM_S0);
-#pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint32_t off = (kk >> 2) * C::REGION_BYTES + (kk & 3) * 32;
-                        ptx::mma_ss(d_s, ptx::sw128_desc(sq + off, 16, 1024), ptx::sw128_desc(sk + off, 16, 1024),
-                                    IDESC_S, kk > 0);
-                    }
-                    ptx::mma_commit(&bar->s_full[t & 1]);
-                    issued_any = true;
+                    k_waited = u;
                 }
-                if (t >= 1) {
-                    const int u = t - 1, su = u % NS;
-                    if (!ptx::mbar_wait(&bar->p_full[u & 1], (u >> 1) & 1, abort_flag)) { ok = false; break; }
-                    if (!ptx::mbar_wait(&bar->v_full[su], (u / NS) & 1, abort_flag)) { ok = false; break; }
-                    ptx::tc_fence_after();
-                    const uint32_t sv = ptx::smem_u32(sV + su * C::TILE_BYTES);
-                    const uint32_t a_p = tmem + ((u & 1) ? C::TMEM_S1 : C::TMEM_S0);
+                const uint32_t sq = ptx::smem_u32(sQ + i * C::TILE_BYTES);
+                const uint32_t sk = ptx::smem_u32(sK + (u % NK) * C::TILE_BYTES);
 #pragma unroll
-                    for (int kk = 0; kk < C::BN / 16; ++kk)
-                        ptx::mma_ts(tmem + C::TMEM_O, a_p + kk * 8, ptx::sw128_desc(sv + kk * 2048, C::REGION_BYTES, 1024),
-                                    IDESC_O, (u > 0 || kk > 0) ? 1u : 0u);
-                    ptx::mma_commit(&bar->kv_empty[su]);
-                    ptx::mma_commit(u == T - 1 ? &bar->o_final : &bar->o_done);
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * C::REGION_BYTES + (kk & 3) * 32;
+                    ptx::mma_ss(tmem + C::tmem_s(i), ptx::sw128_desc(sq + off, 16, 1024),
+                                ptx::sw128_desc(sk + off, 16, 1024), IDESC_S, kk > 0);
                 }
+                ptx::mma_commit(&bar->s_full[i]);
+                issued_any = true;
+                return true;
+            };
+            // O_i += P_i(u) V(u), P_i read from TMEM over the first 64 columns of score buffer i.
+            auto issue_pv = [&](int i, int u) -> bool {
+                const int c = J0 + u - rng[i].jb;  // local tile index of query tile i
+                if (v_waited < u) {
+                    if (!ptx::mbar_wait(&bar->v_full[u % NV], (u / NV) & 1, abort_flag)) return false;
+                    v_waited = u;
+                }
+                if (!ptx::mbar_wait(&bar->p_full[i], c & 1, abort_flag)) return false;
+                ptx::tc_fence_after();
+                const uint32_t sv = ptx::smem_u32(sV + (u % NV) * C::TILE_BYTES);
+#pragma unroll
+                for (int kk = 0; kk < C::BN / 16; ++kk)
+                    ptx::mma_ts(tmem + C::tmem_o(i), tmem + C::tmem_s(i) + kk * 8,
+                                ptx::sw128_desc(sv + kk * 2048, C::REGION_BYTES, 1024), IDESC_O,
+                                (c > 0 || kk > 0) ? 1u : 0u);
+                if (c == rng[i].n - 1) ptx::mma_commit(&bar->o_final[i]);
+                return true;
+            };
+            if (ok) {
+                for (int i = 0; i < 2 && ok; ++i)
+                    if (active(i, 0)) ok = issue_s(i, 0);
+                if (ok) ptx::mma_commit(&bar->k_empty[0]);
+            }
+            for (int u = 0; ok && u < T; ++u) {
+                for (int i = 0; i < 2 && ok; ++i) {
+                    if (active(i, u)) ok = issue_pv(i, u);
+                    if (ok && u + 1 < T && active(i, u + 1)) ok = issue_s(i, u + 1);
+                }
+                if (!ok) break;
+                ptx::mma_commit(&bar->v_empty[u % NV]);
+                if (u + 1 < T) ptx::mma_commit(&bar->k_empty[(u + 1) % NK]);
             }
             if (!ok) {
                 *abort_flag = 1;
@@ -247,51 +302,54 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         }
         __syncwarp();
     } else {
-        // ------------------------------------------------------------------ softmax warpgroup
-        const int r = threadIdx.x;  // row within the tile == TMEM lane
-        const int i = q0 + r;       // query position
-        const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-        bool ok = ptx::mbar_wait(&bar->q_loaded, 0, abort_flag);
-        if (ok && p.rope != nullptr && i < p.N)
-            rope_rotate_smem_row<D>(sQ, r, p.rope + static_cast<size_t>(i) * (D / 2));
-        ptx::fence_proxy_async_smem();
-        ptx::named_barrier_sync(1, 128);
-        if (threadIdx.x == 0) ptx::mbar_arrive(&bar->q_ready);
-
+        // ------------------------------------------------------------------ softmax warpgroups
+        const int wg = warp >> 2;            // query tile of this warpgroup
+        const int r = threadIdx.x & 127;     // row within the tile == TMEM lane
+        const TileRange R = rng[wg];
+        const int i_pos = R.q0 + r;          // query position
+        const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+        const uint32_t t_s = tmem + lane_base + C::tmem_s(wg);
+        const uint32_t t_o = tmem + lane_base + C::tmem_o(wg);
+        bool ok = true;
+        if (R.n > 0) {
+            ok = ptx::mbar_wait(&bar->q_loaded[wg], 0, abort_flag);
+            if (ok && p.rope != nullptr && i_pos < p.N)
+                rope_rotate_smem_row<D>(sQ + wg * C::TILE_BYTES, r, p.rope + static_cast<size_t>(i_pos) * (D / 2));
+            ptx::fence_proxy_async_smem();
+            ptx::named_barrier_sync(1 + wg, 128);
+            if (r == 0) ptx::mbar_arrive(&bar->q_ready[wg]);
+        }
+        const float sl = p.scale_log2;
         float m_used = -INFINITY, l = 0.f;
-        for (int t = 0; ok && t < T; ++t) {
-            const int j0 = (j_begin + t) * C::BN;
-            if (!ptx::mbar_wait(&bar->s_full[t & 1], (t >> 1) & 1, abort_flag)) { ok = false; break; }
+        for (int c = 0; ok && c < R.n; ++c) {
+            const int j0 = (R.jb + c) * C::BN;
+            if (!ptx::mbar_wait(&bar->s_full[wg], c & 1, abort_flag)) { ok = false; break; }
             ptx::tc_fence_after();
-            const uint32_t t_s = tmem + lane_base + ((t & 1) ? C::TMEM_S1 : C::TMEM_S0);
+            uint32_t sv[C::BN];
+            ptx::tmem_ld128(t_s, sv);
             float s[C::BN];
 #pragma unroll
-            for (int c = 0; c < C::BN / 32; ++c) {
-                uint32_t v[32];
-                ptx::tmem_ld32(t_s + c * 32, v);
-#pragma unroll
-                for (int k = 0; k < 32; ++k) s[c * 32 + k] = __uint_as_float(v[k]);
-            }
-            const bool need_mask = (j0 + C::BN > p.N) || (p.causal && j0 + C::BN - 1 > q0) ||
-                                   (p.window > 0 && j0 < q0 + C::BM - p.window);
+            for (int k = 0; k < C::BN; ++k) s[k] = __uint_as_float(sv[k]);
+            const bool need_mask = (j0 + C::BN > p.N) || (p.causal && j0 + C::BN - 1 > R.q0) ||
+                                   (p.window > 0 && j0 < R.q0 + C::BM - p.window);
             if (need_mask) {
-                const int lo = p.window > 0 ? i - p.window + 1 : -0x7fffffff;
-                const int hi = p.causal ? min(i, p.N - 1) : p.N - 1;
+                const int lo = p.window > 0 ? i_pos - p.window + 1 : -0x7fffffff;
+                const int hi = p.causal ? min(i_pos, p.N - 1) : p.N - 1;
 #pragma unroll
-                for (int c = 0; c < C::BN; ++c) {
-                    const int kj = j0 + c;
-                    if (kj < lo || kj > hi) s[c] = -INFINITY;
+                for (int k = 0; k < C::BN; ++k) {
+                    const int kj = j0 + k;
+                    if (kj < lo || kj > hi) s[k] = -INFINITY;
                 }
             }
             float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
 #pragma unroll
-            for (int c = 4; c < C::BN; c += 4) {
-                mx0 = fmaxf(mx0, s[c]);
-                mx1 = fmaxf(mx1, s[c + 1]);
-                mx2 = fmaxf(mx2, s[c + 2]);
-                mx3 = fmaxf(mx3, s[c + 3]);
+            for (int k = 4; k < C::BN; k += 8) {
+                mx0 = ptx::fmax3(mx0, s[k], s[k + 1]);
+                mx1 = ptx::fmax3(mx1, s[k + 2], s[k + 3]);
+                mx2 = ptx::fmax3(mx2, s[k + 4], s[k + 5]);
+                mx3 = ptx::fmax3(mx3, s[k + 6], s[k + 7]);
             }
-            const float m_new = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * p.scale_log2;
+            const float m_new = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl;
             float alpha = 1.f;
             bool rescale = false;
             if (m_new > m_used + C::RESCALE_THRESHOLD) {  // also the first visible key (m_used = -inf)
@@ -300,76 +358,86 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
                 rescale = true;
             }
             const float m_eff = (m_used == -INFINITY) ? 0.f : m_used;
-            float sum0 = 0.f, sum1 = 0.f, sum2 = 0.f, sum3 = 0.f;
+            const float2 sl2 = make_float2(sl, sl), nm2 = make_float2(-m_eff, -m_eff);
+            float2 acc0 = make_float2(0.f, 0.f), acc1 = acc0, acc2 = acc0, acc3 = acc0;
+            uint32_t pk[C::BN / 2];
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                uint32_t pk[32];
-#pragma unroll
-                for (int k = 0; k < 32; k += 2) {
-                    const int c = half * 64 + 2 * k;
-                    const float p0 = ptx::ex2(fmaf(s[c], p.scale_log2, -m_eff));
-                    const float p1 = ptx::ex2(fmaf(s[c + 1], p.scale_log2, -m_eff));
-                    const float p2 = ptx::ex2(fmaf(s[c + 2], p.scale_log2, -m_eff));
-                    const float p3 = ptx::ex2(fmaf(s[c + 3], p.scale_log2, -m_eff));
-                    sum0 += p0;
-                    sum1 += p1;
-                    sum2 += p2;
-                    sum3 += p3;
-                    pk[k] = ptx::pack_bf16x2(p0, p1);
-                    pk[k + 1] = ptx::pack_bf16x2(p2, p3);
-                }
-                // P (bf16 pairs) over the first 64 columns of this score buffer.
-                ptx::tmem_st32(t_s + half * 32, pk);
+            for (int k = 0; k < C::BN; k += 8) {
+                float2 x0 = ptx::ffma2(make_float2(s[k], s[k + 1]), sl2, nm2);
+                float2 x1 = ptx::ffma2(make_float2(s[k + 2], s[k + 3]), sl2, nm2);
+                float2 x2 = ptx::ffma2(make_float2(s[k + 4], s[k + 5]), sl2, nm2);
+                float2 x3 = ptx::ffma2(make_float2(s[k + 6], s[k + 7]), sl2, nm2);
+                x0 = make_float2(ptx::ex2(x0.x), ptx::ex2(x0.y));
+                x1 = make_float2(ptx::ex2(x1.x), ptx::ex2(x1.y));
+                x2 = make_float2(ptx::ex2(x2.x), ptx::ex2(x2.y));
+                x3 = make_float2(ptx::ex2(x3.x), ptx::ex2(x3.y));
+                acc0 = ptx::fadd2(acc0, x0);
+                acc1 = ptx::fadd2(acc1, x1);
+                acc2 = ptx::fadd2(acc2, x2);
+                acc3 = ptx::fadd2(acc3, x3);
+                pk[k / 2] = ptx::pack_bf16x2(x0.x, x0.y);
+                pk[k / 2 + 1] = ptx::pack_bf16x2(x1.x, x1.y);
+                pk[k / 2 + 2] = ptx::pack_bf16x2(x2.x, x2.y);
+                pk[k / 2 + 3] = ptx::pack_bf16x2(x3.x, x3.y);
             }
-            l = l * alpha + ((sum0 + sum1) + (sum2 + sum3));
-            if (t > 0 && __any_sync(0xffffffffu, rescale)) {
-                // O must hold the previous tile's product before it is rescaled.
-                if (!ptx::mbar_wait(&bar->o_done, (t - 1) & 1, abort_flag)) { ok = false; break; }
-                ptx::tc_fence_after();
+            const float2 a01 = ptx::fadd2(acc0, acc1), a23 = ptx::fadd2(acc2, acc3);
+            const float2 a = ptx::fadd2(a01, a23);
+            l = l * alpha + (a.x + a.y);
+            // P (bf16 pairs) over the first 64 columns of this tile's score buffer.
+            ptx::tmem_st64(t_s, pk);
+            if (c > 0 && __any_sync(0xffffffffu, rescale)) {
+                // The product with the previous P has completed (it was issued before this tile's
+                // scores), so O_i is stable here.
+                const float2 al2 = make_float2(alpha, alpha);
 #pragma unroll
-                for (int c = 0; c < D / 32; ++c) {
+                for (int cc = 0; cc < D / 32; ++cc) {
                     uint32_t v[32];
-                    const uint32_t t_o = tmem + lane_base + C::TMEM_O + c * 32;
-                    ptx::tmem_ld32(t_o, v);
+                    ptx::tmem_ld32(t_o + cc * 32, v);
 #pragma unroll
-                    for (int k = 0; k < 32; ++k) v[k] = __float_as_uint(__uint_as_float(v[k]) * alpha);
-                    ptx::tmem_st32(t_o, v);
+                    for (int k = 0; k < 32; k += 2) {
+                        const float2 y = ptx::fmul2(make_float2(__uint_as_float(v[k]), __uint_as_float(v[k + 1])), al2);
+                        v[k] = __float_as_uint(y.x);
+                        v[k + 1] = __float_as_uint(y.y);
+                    }
+                    ptx::tmem_st32(t_o + cc * 32, v);
                 }
             }
             ptx::tc_fence_before();
-            ptx::mbar_arrive(&bar->p_full[t & 1]);
+            ptx::mbar_arrive(&bar->p_full[wg]);
         }
-        if (ok) ok = ptx::mbar_wait(&bar->o_final, 0, abort_flag);
-        if (ok) {
-            ptx::tc_fence_after();
-            const float inv_l = l > 0.f ? 1.f / l : 0.f;
-            __nv_bfloat16* orow = p.o + ((static_cast<size_t>(b) * p.Hq + h) * p.N + i) * D;
+        if (R.n > 0) {
+            if (ok) ok = ptx::mbar_wait(&bar->o_final[wg], 0, abort_flag);
+            if (ok) {
+                ptx::tc_fence_after();
+                const float inv_l = l > 0.f ? 1.f / l : 0.f;
+                __nv_bfloat16* orow = p.o + ((static_cast<size_t>(b) * p.Hq + h) * p.N + i_pos) * D;
 #pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-                uint32_t v[32];
-                ptx::tmem_ld32(tmem + lane_base + C::TMEM_O + c * 32, v);
-                uint32_t w[16];
+                for (int cc = 0; cc < D / 32; ++cc) {
+                    uint32_t v[32];
+                    ptx::tmem_ld32(t_o + cc * 32, v);
+                    uint32_t w[16];
 #pragma unroll
-                for (int k = 0; k < 16; ++k)
-                    w[k] = ptx::pack_bf16x2(__uint_as_float(v[2 * k]) * inv_l, __uint_as_float(v[2 * k + 1]) * inv_l);
-                if (i < p.N) {
-                    uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+                    for (int k = 0; k < 16; ++k)
+                        w[k] = ptx::pack_bf16x2(__uint_as_float(v[2 * k]) * inv_l, __uint_as_float(v[2 * k + 1]) * inv_l);
+                    if (i_pos < p.N) {
+                        uint4* dst = reinterpret_cast<uint4*>(orow + cc * 32);
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) dst[k] = make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+                        for (int k = 0; k < 4; ++k) dst[k] = make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+                    }
                 }
+                if (p.lse != nullptr && i_pos < p.N)
+                    p.lse[(static_cast<size_t>(b) * p.Hq + h) * p.N + i_pos] =
+                        l > 0.f ? (m_used + ptx::lg2(l)) * kLn2 : -INFINITY;
+            } else {
+                *abort_flag = 1;
+                raise_status(kStatusTimeout);
             }
-            if (p.lse != nullptr && i < p.N)
-                p.lse[(static_cast<size_t>(b) * p.Hq + h) * p.N + i] =
-                    l > 0.f ? (m_used + ptx::lg2(l)) * kLn2 : -INFINITY;
-        } else {
-            *abort_flag = 1;
-            raise_status(kStatusTimeout);
         }
     }
 
     ptx::tc_fence_before();
     __syncthreads();
-    if (warp == 5) {
+    if (warp == C::MMA_WARP) {
         ptx::tc_fence_after();
         ptx::tmem_dealloc(tmem, C::TMEM_COLS);
     }
