@@ -196,8 +196,12 @@ attn_status launch_fwd(const void* q, const void* k, const void* v, void* o, flo
     p.causal = causal;
     p.window = window > 0 ? window : 0;
     p.scale_log2 = scale * attn::kLog2e;
+    p.nblk = (N + C::QT * C::BM - 1) / (C::QT * C::BM);
+    p.n_items = B * Hq * p.nblk;
     if ((st = ensure_smem(attn::attn_fwd_kernel<D>, C::SMEM_BYTES, dev)) != ATTN_OK) return st;
-    const dim3 grid(Hq, B, (N + C::QT * C::BM - 1) / (C::QT * C::BM));
+    int sms = 148;
+    CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+    const int grid = p.n_items < sms ? p.n_items : sms;  // persistent: one CTA per SM
     attn::attn_fwd_kernel<D><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
     CUDA_TRY(cudaGetLastError());
     return ATTN_OK;
@@ -257,7 +261,8 @@ attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float
     if (window > 0 && !causal) return fail(ATTN_ERR_INVALID_ARG, "a sliding window requires causal = 1");
     if (!std::isfinite(scale) || !std::isfinite(rope_base)) return fail(ATTN_ERR_INVALID_ARG, "scale and rope_base must be finite");
     if (D != 64 && D != 128) return fail(ATTN_ERR_UNSUPPORTED, "head dim %d not supported (64 or 128)", D);
-    if (B > 65535 || (N + 255) / 256 > 65535) return fail(ATTN_ERR_UNSUPPORTED, "B or N too large for the grid");
+    if (static_cast<long long>(B) * Hq * ((N + 255) / 256) > 0x7fffffffLL)
+        return fail(ATTN_ERR_UNSUPPORTED, "too many 256-query work items");
     if (static_cast<double>(B) * Hq * N * D * 2 >= 1099511627776.0)
         return fail(ATTN_ERR_UNSUPPORTED, "tensor larger than 1 TiB");
     if (scale <= 0.f) scale = 1.0f / std::sqrt(static_cast<float>(D));

@@ -1,8 +1,10 @@
 // fwd_sm100.cuh -- FlashAttention-style exact attention forward for sm_100a.
 //
-// One CTA computes two 128-row query tiles (256 consecutive queries) of one (batch, query head).
-// Both tiles stream the same visible 128-key tiles of the matching K/V head through shared
-// memory, so each K/V tile loaded serves 256 query rows. Per row the online softmax keeps the
+// The kernel is persistent: one CTA per SM walks a list of work items, each being two 128-row
+// query tiles (256 consecutive queries) of one (batch, query head), longest items first. Both
+// tiles stream the same visible 128-key tiles of the matching K/V head through shared memory, so
+// each K/V tile loaded serves 256 query rows; the K/V rings run on across items, and the next
+// item's queries are loaded while the current item finishes. Per row the online softmax keeps the
 // running max m, the normaliser l and the output accumulator o, rescaled as the max grows, then
 // O = o / l and the row logsumexp ("Why is attention O(n^2), how does FlashAttention help, ...",
 // "Deep dive: FlashAttention"). The n x n score matrix never leaves the SM: each 128x128 score
@@ -13,7 +15,8 @@
 //              lane r). It rotates its Q row (RoPE) once, then per key tile reads its 128 scores
 //              from TMEM with one load, masks them, updates m and l, writes P (bf16) back into
 //              TMEM over the first half of its score buffer, rescales its row of O when the max
-//              moved by more than 2^8, and finally writes O and LSE.
+//              moved by more than 2^8, and finally reads O out of TMEM (releasing it for the
+//              next item's products) and writes O and LSE.
 //   warp 8     TMA producer: the Q tiles once, then K tiles into a NK-stage ring and V tiles into
 //              a NV-stage ring.
 //   warp 9     MMA issuer (one thread) and TMEM owner.
@@ -42,6 +45,8 @@ struct FwdParams {
     int B, Hq, Hkv, N;
     int causal, window;     // window > 0 only together with causal
     float scale_log2;       // softmax scale * log2(e)
+    int nblk;               // 256-query blocks per (batch, head)
+    int n_items;            // B * Hq * nblk work items
 };
 
 template <int D>
@@ -70,9 +75,9 @@ struct FwdCfg {
 
 template <int NK, int NV>
 struct FwdBarriers {
-    uint64_t q_loaded[2], q_ready[2];
+    uint64_t q_loaded[2], q_ready[2], q_empty[2];
     uint64_t k_full[NK], k_empty[NK], v_full[NV], v_empty[NV];
-    uint64_t s_full[2], p_full[2], o_final[2];
+    uint64_t s_full[2], p_full[2], o_final[2], o_empty[2];
     uint64_t drain;
     uint32_t tmem_base;
     int abort;
@@ -95,30 +100,63 @@ __device__ __forceinline__ TileRange tile_range(int q0, int N, int causal, int w
 
 // Rotate one 128-byte-swizzled row of a Q tile in place: pairs (2i, 2i+1) by pos * theta_i, in
 // fp32 with the (cos, sin) table, rounded back to bf16 ("attention-transformers", Q "How does
-// Rotary Position Embedding (RoPE) work?").
+// Rotary Position Embedding (RoPE) work?"). The table loads of each 64-column region are issued
+// together, so their latency is paid once per region rather than once per 16-byte chunk.
 template <int D>
 __device__ __forceinline__ void rope_rotate_smem_row(uint8_t* tile, int r, const float2* __restrict__ cs_row) {
     using C = FwdCfg<D>;
 #pragma unroll
     for (int reg = 0; reg < C::NREG; ++reg) {
+        float4 cs[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c) cs[c] = __ldg(reinterpret_cast<const float4*>(cs_row + reg * 32 + 2 * c));
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
             uint4* p = reinterpret_cast<uint4*>(tile + reg * C::REGION_BYTES + r * 128 + ((c ^ (r & 7)) << 4));
             uint4 w = *p;
-            const int i0 = reg * 32 + c * 4;  // first pair index of this 16-byte chunk
-            const float4 a = __ldg(reinterpret_cast<const float4*>(cs_row + i0));
-            const float4 b = __ldg(reinterpret_cast<const float4*>(cs_row + i0 + 2));
             uint32_t* wv = reinterpret_cast<uint32_t*>(&w);
-            const float cs[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+            const float t[8] = {cs[2 * c].x, cs[2 * c].y, cs[2 * c].z, cs[2 * c].w,
+                                cs[2 * c + 1].x, cs[2 * c + 1].y, cs[2 * c + 1].z, cs[2 * c + 1].w};
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
                 const float x0 = ptx::bf16lo_to_f32(wv[k]), x1 = ptx::bf16hi_to_f32(wv[k]);
-                const float cth = cs[2 * k], sth = cs[2 * k + 1];
+                const float cth = t[2 * k], sth = t[2 * k + 1];
                 wv[k] = ptx::pack_bf16x2(fmaf(x0, cth, -x1 * sth), fmaf(x0, sth, x1 * cth));
             }
             *p = w;
         }
     }
+}
+
+// One work item: (batch b, query head h, block of 256 queries); the longest causal blocks come
+// first, and the query heads of one block are adjacent so heads sharing a K/V head run together.
+struct Item {
+    int b, h, blk;
+    TileRange rng[2];
+    int J0, T;  // union of the two key-tile ranges
+    __device__ __forceinline__ bool active(int i, int u) const {
+        const int j = J0 + u;
+        return rng[i].n > 0 && j >= rng[i].jb && j < rng[i].jb + rng[i].n;
+    }
+};
+
+// Item of round r for CTA c: rounds alternate direction over the CTAs (c, then G-1-c), which with
+// the longest-first item order balances the causal work to within a fraction of a percent.
+__device__ __forceinline__ int item_of_round(int r, int c, int G) { return r * G + ((r & 1) ? G - 1 - c : c); }
+
+__device__ __forceinline__ Item make_item(const FwdParams& p, int it) {
+    Item x;
+    const int bh = it % (p.B * p.Hq);
+    x.blk = p.nblk - 1 - it / (p.B * p.Hq);
+    x.b = bh / p.Hq;
+    x.h = bh % p.Hq;
+    x.rng[0] = tile_range(x.blk * 256, p.N, p.causal, p.window);
+    x.rng[1] = tile_range(x.blk * 256 + 128, p.N, p.causal, p.window);
+    // Tile 1 starts no earlier and ends no earlier than tile 0, so the union is contiguous.
+    x.J0 = x.rng[0].jb;
+    const int end0 = x.rng[0].jb + x.rng[0].n;
+    x.T = (x.rng[1].n > 0 ? max(end0, x.rng[1].jb + x.rng[1].n) : end0) - x.J0;
+    return x;
 }
 
 template <int D>
@@ -136,26 +174,16 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     volatile int* abort_flag = &bar->abort;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int h = blockIdx.x, b = blockIdx.y;
-    const int blk = gridDim.z - 1 - blockIdx.z;  // longest (causal) blocks first
-    const int g = h / (p.Hq / p.Hkv);            // query head h reads K/V head h / (Hq/Hkv)
-    const TileRange rng[2] = {tile_range(blk * 256, p.N, p.causal, p.window),
-                              tile_range(blk * 256 + 128, p.N, p.causal, p.window)};
-    // Union of the two ranges (contiguous: tile 1 starts no earlier and ends no earlier).
-    const int J0 = rng[0].jb;
-    const int T = (rng[1].n > 0 ? max(rng[0].jb + rng[0].n, rng[1].jb + rng[1].n) : rng[0].jb + rng[0].n) - J0;
-    auto active = [&](int i, int u) {
-        const int j = J0 + u;
-        return rng[i].n > 0 && j >= rng[i].jb && j < rng[i].jb + rng[i].n;
-    };
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < 2; ++i) {
             ptx::mbar_init(&bar->q_loaded[i], 1);
             ptx::mbar_init(&bar->q_ready[i], 1);
+            ptx::mbar_init(&bar->q_empty[i], 1);
             ptx::mbar_init(&bar->s_full[i], 1);
             ptx::mbar_init(&bar->p_full[i], 128);
             ptx::mbar_init(&bar->o_final[i], 1);
+            ptx::mbar_init(&bar->o_empty[i], 128);
         }
         for (int s = 0; s < NK; ++s) {
             ptx::mbar_init(&bar->k_full[s], 1);
@@ -186,34 +214,42 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     if (warp == C::PRODUCER_WARP) {
         // ------------------------------------------------------------------ TMA producer
         if (lane == 0) {
-            const int zq = b * p.Hq + h, zk = b * p.Hkv + g;
-            for (int i = 0; i < 2; ++i) {
-                if (rng[i].n == 0) continue;
-                ptx::mbar_arrive_expect_tx(&bar->q_loaded[i], C::TILE_BYTES);
-#pragma unroll
-                for (int r = 0; r < C::NREG; ++r)
-                    ptx::tma_load_3d(sQ + i * C::TILE_BYTES + r * C::REGION_BYTES, &tm_q, &bar->q_loaded[i], r * 64,
-                                     rng[i].q0, zq);
-            }
+            int kq[2] = {0, 0};  // items in which query tile i was loaded so far
+            int g = 0;           // key tiles streamed so far (ring position)
             int k_issued = 0, v_issued = 0;
             bool ok = true;
-            for (int u = 0; u < T && ok; ++u) {
-                const int k0 = (J0 + u) * C::BN;
-                const int sk = u % NK, sv = u % NV;
-                if (u >= NK && !ptx::mbar_wait(&bar->k_empty[sk], ((u / NK) - 1) & 1, abort_flag)) { ok = false; break; }
-                ptx::mbar_arrive_expect_tx(&bar->k_full[sk], C::TILE_BYTES);
+            for (int rnd = 0, it = blockIdx.x; ok && it < p.n_items; it = item_of_round(++rnd, blockIdx.x, gridDim.x)) {
+                const Item x = make_item(p, it);
+                const int zq = x.b * p.Hq + x.h, zk = x.b * p.Hkv + x.h / (p.Hq / p.Hkv);
+                for (int i = 0; i < 2 && ok; ++i) {
+                    if (x.rng[i].n == 0) continue;
+                    // the buffer is free once the previous item's last S_i has been computed
+                    if (kq[i] > 0 && !ptx::mbar_wait(&bar->q_empty[i], (kq[i] - 1) & 1, abort_flag)) { ok = false; break; }
+                    ptx::mbar_arrive_expect_tx(&bar->q_loaded[i], C::TILE_BYTES);
 #pragma unroll
-                for (int r = 0; r < C::NREG; ++r)
-                    ptx::tma_load_3d(sK + sk * C::TILE_BYTES + r * C::REGION_BYTES, &tm_k, &bar->k_full[sk], r * 64,
-                                     k0, zk);
-                k_issued = u + 1;
-                if (u >= NV && !ptx::mbar_wait(&bar->v_empty[sv], ((u / NV) - 1) & 1, abort_flag)) { ok = false; break; }
-                ptx::mbar_arrive_expect_tx(&bar->v_full[sv], C::TILE_BYTES);
+                    for (int r = 0; r < C::NREG; ++r)
+                        ptx::tma_load_3d(sQ + i * C::TILE_BYTES + r * C::REGION_BYTES, &tm_q, &bar->q_loaded[i],
+                                         r * 64, x.rng[i].q0, zq);
+                    ++kq[i];
+                }
+                for (int u = 0; u < x.T && ok; ++u, ++g) {
+                    const int k0 = (x.J0 + u) * C::BN;
+                    const int sk = g % NK, sv = g % NV;
+                    if (g >= NK && !ptx::mbar_wait(&bar->k_empty[sk], ((g / NK) - 1) & 1, abort_flag)) { ok = false; break; }
+                    ptx::mbar_arrive_expect_tx(&bar->k_full[sk], C::TILE_BYTES);
 #pragma unroll
-                for (int r = 0; r < C::NREG; ++r)
-                    ptx::tma_load_3d(sV + sv * C::TILE_BYTES + r * C::REGION_BYTES, &tm_v, &bar->v_full[sv], r * 64,
-                                     k0, zk);
-                v_issued = u + 1;
+                    for (int r = 0; r < C::NREG; ++r)
+                        ptx::tma_load_3d(sK + sk * C::TILE_BYTES + r * C::REGION_BYTES, &tm_k, &bar->k_full[sk],
+                                         r * 64, k0, zk);
+                    k_issued = g + 1;
+                    if (g >= NV && !ptx::mbar_wait(&bar->v_empty[sv], ((g / NV) - 1) & 1, abort_flag)) { ok = false; break; }
+                    ptx::mbar_arrive_expect_tx(&bar->v_full[sv], C::TILE_BYTES);
+#pragma unroll
+                    for (int r = 0; r < C::NREG; ++r)
+                        ptx::tma_load_3d(sV + sv * C::TILE_BYTES + r * C::REGION_BYTES, &tm_v, &bar->v_full[sv],
+                                         r * 64, k0, zk);
+                    v_issued = g + 1;
+                }
             }
             if (!ok) {
                 *abort_flag = 1;
@@ -222,7 +258,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
                 // (each wait is still bounded).
                 volatile int never = 0;
                 for (int i = 0; i < 2; ++i)
-                    if (rng[i].n > 0) ptx::mbar_wait(&bar->q_loaded[i], 0, &never);
+                    if (kq[i] > 0) ptx::mbar_wait(&bar->q_loaded[i], (kq[i] - 1) & 1, &never);
                 for (int u = max(0, k_issued - NK); u < k_issued; ++u)
                     ptx::mbar_wait(&bar->k_full[u % NK], (u / NK) & 1, &never);
                 for (int u = max(0, v_issued - NV); u < v_issued; ++u)
@@ -234,61 +270,65 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         if (lane == 0) {
             constexpr uint32_t IDESC_S = ptx::idesc_bf16_f32(128, C::BN, 0, 0);  // Q, K both K-major
             constexpr uint32_t IDESC_O = ptx::idesc_bf16_f32(128, D, 0, 1);      // P K-major, V MN-major
+            constexpr uint32_t HI = ptx::sw128_desc_hi(1024);                    // 8-row groups 1024 B apart
+            constexpr uint32_t TILE16 = C::TILE_BYTES >> 4;
+            // low descriptor words of Q tile 0, K stage 0 and V stage 0 (K-major LBO unused = 16;
+            // V is MN-major with its 64-column halves one region apart)
+            const uint32_t q_lo = ptx::sw128_desc_lo(ptx::smem_u32(sQ), 16);
+            const uint32_t k_lo = ptx::sw128_desc_lo(ptx::smem_u32(sK), 16);
+            const uint32_t v_lo = ptx::sw128_desc_lo(ptx::smem_u32(sV), C::REGION_BYTES);
             bool ok = true, issued_any = false;
-            for (int i = 0; i < 2 && ok; ++i)
-                if (rng[i].n > 0) ok = ptx::mbar_wait(&bar->q_ready[i], 0, abort_flag);
-            ptx::tc_fence_after();
-            int k_waited = -1, v_waited = -1;
-            // S_i(u) = Q_i K(u)^T into score buffer i.
-            auto issue_s = [&](int i, int u) -> bool {
-                if (k_waited < u) {
-                    if (!ptx::mbar_wait(&bar->k_full[u % NK], (u / NK) & 1, abort_flag)) return false;
-                    ptx::tc_fence_after();
-                    k_waited = u;
-                }
-                const uint32_t sq = ptx::smem_u32(sQ + i * C::TILE_BYTES);
-                const uint32_t sk = ptx::smem_u32(sK + (u % NK) * C::TILE_BYTES);
+            int kq0 = 0, kq1 = 0;  // items of query tile 0 / 1 started so far
+            int cw0 = 0, cw1 = 0;  // score tiles of query tile 0 / 1 computed so far (all items)
+            int g = 0;             // key tiles consumed so far (ring position)
+            for (int rnd = 0, it = blockIdx.x; ok && it < p.n_items; it = item_of_round(++rnd, blockIdx.x, gridDim.x)) {
+                const Item x = make_item(p, it);
+                for (int u = -1; ok && u < x.T; ++u) {
+                    // u = -1: the prologue (scores of the first key tile only)
+                    if (u >= 0) {
+                        if (!ptx::mbar_wait(&bar->v_full[(g + u) % NV], ((g + u) / NV) & 1, abort_flag)) { ok = false; break; }
+                    }
+                    for (int i = 0; i < 2; ++i) {
+                        const int kq = i ? kq1 : kq0, cw = i ? cw1 : cw0;
+                        const TileRange& R = x.rng[i];
+                        const uint32_t d_s = tmem + C::tmem_s(i), d_o = tmem + C::tmem_o(i);
+                        if (u >= 0 && x.active(i, u)) {
+                            // O_i += P_i(u) V(u); P_i in TMEM over the first 64 columns of score buffer i
+                            const int c = x.J0 + u - R.jb;
+                            if (c == 0 && kq > 0 && !ptx::mbar_wait(&bar->o_empty[i], (kq - 1) & 1, abort_flag)) { ok = false; break; }
+                            if (!ptx::mbar_wait(&bar->p_full[i], (cw + c) & 1, abort_flag)) { ok = false; break; }
+                            ptx::tc_fence_after();
+                            const uint32_t vb = v_lo + ((g + u) % NV) * TILE16;
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * C::REGION_BYTES + (kk & 3) * 32;
-                    ptx::mma_ss(tmem + C::tmem_s(i), ptx::sw128_desc(sq + off, 16, 1024),
-                                ptx::sw128_desc(sk + off, 16, 1024), IDESC_S, kk > 0);
-                }
-                ptx::mma_commit(&bar->s_full[i]);
-                issued_any = true;
-                return true;
-            };
-            // O_i += P_i(u) V(u), P_i read from TMEM over the first 64 columns of score buffer i.
-            auto issue_pv = [&](int i, int u) -> bool {
-                const int c = J0 + u - rng[i].jb;  // local tile index of query tile i
-                if (v_waited < u) {
-                    if (!ptx::mbar_wait(&bar->v_full[u % NV], (u / NV) & 1, abort_flag)) return false;
-                    v_waited = u;
-                }
-                if (!ptx::mbar_wait(&bar->p_full[i], c & 1, abort_flag)) return false;
-                ptx::tc_fence_after();
-                const uint32_t sv = ptx::smem_u32(sV + (u % NV) * C::TILE_BYTES);
+                            for (int kk = 0; kk < C::BN / 16; ++kk)
+                                ptx::mma_ts(d_o, d_s + kk * 8, ptx::desc64(vb + kk * (2048 >> 4), HI), IDESC_O,
+                                            (c > 0 || kk > 0) ? 1u : 0u);
+                            if (c == R.n - 1) ptx::mma_commit(&bar->o_final[i]);
+                        }
+                        if (u + 1 < x.T && x.active(i, u + 1)) {
+                            // S_i(u+1) = Q_i K(u+1)^T into score buffer i
+                            const int c = x.J0 + u + 1 - R.jb;
+                            if (c == 0 && !ptx::mbar_wait(&bar->q_ready[i], kq & 1, abort_flag)) { ok = false; break; }
+                            if (!ptx::mbar_wait(&bar->k_full[(g + u + 1) % NK], ((g + u + 1) / NK) & 1, abort_flag)) { ok = false; break; }
+                            ptx::tc_fence_after();
+                            const uint32_t qa = q_lo + i * TILE16, kb = k_lo + ((g + u + 1) % NK) * TILE16;
 #pragma unroll
-                for (int kk = 0; kk < C::BN / 16; ++kk)
-                    ptx::mma_ts(tmem + C::tmem_o(i), tmem + C::tmem_s(i) + kk * 8,
-                                ptx::sw128_desc(sv + kk * 2048, C::REGION_BYTES, 1024), IDESC_O,
-                                (c > 0 || kk > 0) ? 1u : 0u);
-                if (c == rng[i].n - 1) ptx::mma_commit(&bar->o_final[i]);
-                return true;
-            };
-            if (ok) {
-                for (int i = 0; i < 2 && ok; ++i)
-                    if (active(i, 0)) ok = issue_s(i, 0);
-                if (ok) ptx::mma_commit(&bar->k_empty[0]);
-            }
-            for (int u = 0; ok && u < T; ++u) {
-                for (int i = 0; i < 2 && ok; ++i) {
-                    if (active(i, u)) ok = issue_pv(i, u);
-                    if (ok && u + 1 < T && active(i, u + 1)) ok = issue_s(i, u + 1);
+                            for (int kk = 0; kk < D / 16; ++kk) {
+                                const uint32_t off = ((kk >> 2) * C::REGION_BYTES + (kk & 3) * 32) >> 4;
+                                ptx::mma_ss(d_s, ptx::desc64(qa + off, HI), ptx::desc64(kb + off, HI), IDESC_S, kk > 0);
+                            }
+                            ptx::mma_commit(&bar->s_full[i]);
+                            if (c == R.n - 1) ptx::mma_commit(&bar->q_empty[i]);  // Q_i no longer read
+                            issued_any = true;
+                        }
+                    }
+                    if (!ok) break;
+                    if (u >= 0) ptx::mma_commit(&bar->v_empty[(g + u) % NV]);
+                    if (u + 1 < x.T) ptx::mma_commit(&bar->k_empty[(g + u + 1) % NK]);
                 }
-                if (!ok) break;
-                ptx::mma_commit(&bar->v_empty[u % NV]);
-                if (u + 1 < T) ptx::mma_commit(&bar->k_empty[(u + 1) % NK]);
+                if (x.rng[0].n > 0) { ++kq0; cw0 += x.rng[0].n; }
+                if (x.rng[1].n > 0) { ++kq1; cw1 += x.rng[1].n; }
+                g += x.T;
             }
             if (!ok) {
                 *abort_flag = 1;
@@ -305,133 +345,144 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         // ------------------------------------------------------------------ softmax warpgroups
         const int wg = warp >> 2;            // query tile of this warpgroup
         const int r = threadIdx.x & 127;     // row within the tile == TMEM lane
-        const TileRange R = rng[wg];
-        const int i_pos = R.q0 + r;          // query position
         const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
         const uint32_t t_s = tmem + lane_base + C::tmem_s(wg);
         const uint32_t t_o = tmem + lane_base + C::tmem_o(wg);
+        const float sl = p.scale_log2;
         bool ok = true;
-        if (R.n > 0) {
-            ok = ptx::mbar_wait(&bar->q_loaded[wg], 0, abort_flag);
-            if (ok && p.rope != nullptr && i_pos < p.N)
+        int kq = 0, cw = 0;
+        for (int rnd = 0, it = blockIdx.x; ok && it < p.n_items; it = item_of_round(++rnd, blockIdx.x, gridDim.x)) {
+            const Item x = make_item(p, it);
+            const TileRange R = x.rng[wg];
+            if (R.n == 0) continue;
+            const int i_pos = R.q0 + r;  // query position
+            ok = ptx::mbar_wait(&bar->q_loaded[wg], kq & 1, abort_flag);
+            if (!ok) break;
+            if (p.rope != nullptr && i_pos < p.N)
                 rope_rotate_smem_row<D>(sQ + wg * C::TILE_BYTES, r, p.rope + static_cast<size_t>(i_pos) * (D / 2));
             ptx::fence_proxy_async_smem();
             ptx::named_barrier_sync(1 + wg, 128);
             if (r == 0) ptx::mbar_arrive(&bar->q_ready[wg]);
-        }
-        const float sl = p.scale_log2;
-        float m_used = -INFINITY, l = 0.f;
-        for (int c = 0; ok && c < R.n; ++c) {
-            const int j0 = (R.jb + c) * C::BN;
-            if (!ptx::mbar_wait(&bar->s_full[wg], c & 1, abort_flag)) { ok = false; break; }
-            ptx::tc_fence_after();
-            uint32_t sv[C::BN];
-            ptx::tmem_ld128(t_s, sv);
-            float s[C::BN];
+
+            float m_used = -INFINITY, l = 0.f;
+            for (int c = 0; ok && c < R.n; ++c) {
+                const int j0 = (R.jb + c) * C::BN;
+                if (!ptx::mbar_wait(&bar->s_full[wg], (cw + c) & 1, abort_flag)) { ok = false; break; }
+                ptx::tc_fence_after();
+                uint32_t sv[C::BN];
+                ptx::tmem_ld128(t_s, sv);
+                float s[C::BN];
 #pragma unroll
-            for (int k = 0; k < C::BN; ++k) s[k] = __uint_as_float(sv[k]);
-            const bool need_mask = (j0 + C::BN > p.N) || (p.causal && j0 + C::BN - 1 > R.q0) ||
-                                   (p.window > 0 && j0 < R.q0 + C::BM - p.window);
-            if (need_mask) {
-                const int lo = p.window > 0 ? i_pos - p.window + 1 : -0x7fffffff;
-                const int hi = p.causal ? min(i_pos, p.N - 1) : p.N - 1;
+                for (int k = 0; k < C::BN; ++k) s[k] = __uint_as_float(sv[k]);
+                const bool need_mask = (j0 + C::BN > p.N) || (p.causal && j0 + C::BN - 1 > R.q0) ||
+                                       (p.window > 0 && j0 < R.q0 + C::BM - p.window);
+                if (need_mask) {
+                    const int lo = p.window > 0 ? i_pos - p.window + 1 : -0x7fffffff;
+                    const int hi = p.causal ? min(i_pos, p.N - 1) : p.N - 1;
 #pragma unroll
-                for (int k = 0; k < C::BN; ++k) {
-                    const int kj = j0 + k;
-                    if (kj < lo || kj > hi) s[k] = -INFINITY;
-                }
-            }
-            float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
-#pragma unroll
-            for (int k = 4; k < C::BN; k += 8) {
-                mx0 = ptx::fmax3(mx0, s[k], s[k + 1]);
-                mx1 = ptx::fmax3(mx1, s[k + 2], s[k + 3]);
-                mx2 = ptx::fmax3(mx2, s[k + 4], s[k + 5]);
-                mx3 = ptx::fmax3(mx3, s[k + 6], s[k + 7]);
-            }
-            const float m_new = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl;
-            float alpha = 1.f;
-            bool rescale = false;
-            if (m_new > m_used + C::RESCALE_THRESHOLD) {  // also the first visible key (m_used = -inf)
-                alpha = ptx::ex2(m_used - m_new);          // 2^-inf = 0
-                m_used = m_new;
-                rescale = true;
-            }
-            const float m_eff = (m_used == -INFINITY) ? 0.f : m_used;
-            const float2 sl2 = make_float2(sl, sl), nm2 = make_float2(-m_eff, -m_eff);
-            float2 acc0 = make_float2(0.f, 0.f), acc1 = acc0, acc2 = acc0, acc3 = acc0;
-            uint32_t pk[C::BN / 2];
-#pragma unroll
-            for (int k = 0; k < C::BN; k += 8) {
-                float2 x0 = ptx::ffma2(make_float2(s[k], s[k + 1]), sl2, nm2);
-                float2 x1 = ptx::ffma2(make_float2(s[k + 2], s[k + 3]), sl2, nm2);
-                float2 x2 = ptx::ffma2(make_float2(s[k + 4], s[k + 5]), sl2, nm2);
-                float2 x3 = ptx::ffma2(make_float2(s[k + 6], s[k + 7]), sl2, nm2);
-                x0 = make_float2(ptx::ex2(x0.x), ptx::ex2(x0.y));
-                x1 = make_float2(ptx::ex2(x1.x), ptx::ex2(x1.y));
-                x2 = make_float2(ptx::ex2(x2.x), ptx::ex2(x2.y));
-                x3 = make_float2(ptx::ex2(x3.x), ptx::ex2(x3.y));
-                acc0 = ptx::fadd2(acc0, x0);
-                acc1 = ptx::fadd2(acc1, x1);
-                acc2 = ptx::fadd2(acc2, x2);
-                acc3 = ptx::fadd2(acc3, x3);
-                pk[k / 2] = ptx::pack_bf16x2(x0.x, x0.y);
-                pk[k / 2 + 1] = ptx::pack_bf16x2(x1.x, x1.y);
-                pk[k / 2 + 2] = ptx::pack_bf16x2(x2.x, x2.y);
-                pk[k / 2 + 3] = ptx::pack_bf16x2(x3.x, x3.y);
-            }
-            const float2 a01 = ptx::fadd2(acc0, acc1), a23 = ptx::fadd2(acc2, acc3);
-            const float2 a = ptx::fadd2(a01, a23);
-            l = l * alpha + (a.x + a.y);
-            // P (bf16 pairs) over the first 64 columns of this tile's score buffer.
-            ptx::tmem_st64(t_s, pk);
-            if (c > 0 && __any_sync(0xffffffffu, rescale)) {
-                // The product with the previous P has completed (it was issued before this tile's
-                // scores), so O_i is stable here.
-                const float2 al2 = make_float2(alpha, alpha);
-#pragma unroll
-                for (int cc = 0; cc < D / 32; ++cc) {
-                    uint32_t v[32];
-                    ptx::tmem_ld32(t_o + cc * 32, v);
-#pragma unroll
-                    for (int k = 0; k < 32; k += 2) {
-                        const float2 y = ptx::fmul2(make_float2(__uint_as_float(v[k]), __uint_as_float(v[k + 1])), al2);
-                        v[k] = __float_as_uint(y.x);
-                        v[k + 1] = __float_as_uint(y.y);
+                    for (int k = 0; k < C::BN; ++k) {
+                        const int kj = j0 + k;
+                        if (kj < lo || kj > hi) s[k] = -INFINITY;
                     }
-                    ptx::tmem_st32(t_o + cc * 32, v);
                 }
+                // four independent chains over s[0..7], s[8..15], ...: every element exactly once
+                float mx0 = fmaxf(s[0], s[1]), mx1 = fmaxf(s[2], s[3]), mx2 = fmaxf(s[4], s[5]),
+                      mx3 = fmaxf(s[6], s[7]);
+#pragma unroll
+                for (int k = 8; k < C::BN; k += 8) {
+                    mx0 = ptx::fmax3(mx0, s[k], s[k + 1]);
+                    mx1 = ptx::fmax3(mx1, s[k + 2], s[k + 3]);
+                    mx2 = ptx::fmax3(mx2, s[k + 4], s[k + 5]);
+                    mx3 = ptx::fmax3(mx3, s[k + 6], s[k + 7]);
+                }
+                const float m_new = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl;
+                float alpha = 1.f;
+                bool rescale = false;
+                if (m_new > m_used + C::RESCALE_THRESHOLD) {  // also the first visible key (m_used = -inf)
+                    alpha = ptx::ex2(m_used - m_new);          // 2^-inf = 0
+                    m_used = m_new;
+                    rescale = true;
+                }
+                const float m_eff = (m_used == -INFINITY) ? 0.f : m_used;
+                const float2 sl2 = make_float2(sl, sl), nm2 = make_float2(-m_eff, -m_eff);
+                float2 acc0 = make_float2(0.f, 0.f), acc1 = acc0, acc2 = acc0, acc3 = acc0;
+                uint32_t pk[C::BN / 2];
+#pragma unroll
+                for (int k = 0; k < C::BN; k += 8) {
+                    float2 x0 = ptx::ffma2(make_float2(s[k], s[k + 1]), sl2, nm2);
+                    float2 x1 = ptx::ffma2(make_float2(s[k + 2], s[k + 3]), sl2, nm2);
+                    float2 x2 = ptx::ffma2(make_float2(s[k + 4], s[k + 5]), sl2, nm2);
+                    float2 x3 = ptx::ffma2(make_float2(s[k + 6], s[k + 7]), sl2, nm2);
+                    x0 = make_float2(ptx::ex2(x0.x), ptx::ex2(x0.y));
+                    x1 = make_float2(ptx::ex2(x1.x), ptx::ex2(x1.y));
+                    x2 = make_float2(ptx::ex2(x2.x), ptx::ex2(x2.y));
+                    x3 = make_float2(ptx::ex2(x3.x), ptx::ex2(x3.y));
+                    acc0 = ptx::fadd2(acc0, x0);
+                    acc1 = ptx::fadd2(acc1, x1);
+                    acc2 = ptx::fadd2(acc2, x2);
+                    acc3 = ptx::fadd2(acc3, x3);
+                    pk[k / 2] = ptx::pack_bf16x2(x0.x, x0.y);
+                    pk[k / 2 + 1] = ptx::pack_bf16x2(x1.x, x1.y);
+                    pk[k / 2 + 2] = ptx::pack_bf16x2(x2.x, x2.y);
+                    pk[k / 2 + 3] = ptx::pack_bf16x2(x3.x, x3.y);
+                }
+                const float2 a01 = ptx::fadd2(acc0, acc1), a23 = ptx::fadd2(acc2, acc3);
+                const float2 a = ptx::fadd2(a01, a23);
+                l = l * alpha + (a.x + a.y);
+                // P (bf16 pairs) over the first 64 columns of this tile's score buffer.
+                ptx::tmem_st64(t_s, pk);
+                if (c > 0 && __any_sync(0xffffffffu, rescale)) {
+                    // The product with the previous P has completed (it was issued before this
+                    // tile's scores), so O_i is stable here.
+                    const float2 al2 = make_float2(alpha, alpha);
+#pragma unroll
+                    for (int cc = 0; cc < D / 32; ++cc) {
+                        uint32_t v[32];
+                        ptx::tmem_ld32(t_o + cc * 32, v);
+#pragma unroll
+                        for (int k = 0; k < 32; k += 2) {
+                            const float2 y =
+                                ptx::fmul2(make_float2(__uint_as_float(v[k]), __uint_as_float(v[k + 1])), al2);
+                            v[k] = __float_as_uint(y.x);
+                            v[k + 1] = __float_as_uint(y.y);
+                        }
+                        ptx::tmem_st32(t_o + cc * 32, v);
+                    }
+                }
+                ptx::tc_fence_before();
+                ptx::mbar_arrive(&bar->p_full[wg]);
+            }
+            if (!ok) break;
+            cw += R.n;
+            // ---- epilogue: O_i out of TMEM (then the next item may overwrite it), O = o / l, LSE
+            if (!ptx::mbar_wait(&bar->o_final[wg], kq & 1, abort_flag)) { ok = false; break; }
+            ptx::tc_fence_after();
+            uint32_t w[D / 2];
+            const float inv_l = l > 0.f ? 1.f / l : 0.f;
+#pragma unroll
+            for (int cc = 0; cc < D / 32; ++cc) {
+                uint32_t v[32];
+                ptx::tmem_ld32(t_o + cc * 32, v);
+#pragma unroll
+                for (int k = 0; k < 16; ++k)
+                    w[cc * 16 + k] =
+                        ptx::pack_bf16x2(__uint_as_float(v[2 * k]) * inv_l, __uint_as_float(v[2 * k + 1]) * inv_l);
             }
             ptx::tc_fence_before();
-            ptx::mbar_arrive(&bar->p_full[wg]);
-        }
-        if (R.n > 0) {
-            if (ok) ok = ptx::mbar_wait(&bar->o_final[wg], 0, abort_flag);
-            if (ok) {
-                ptx::tc_fence_after();
-                const float inv_l = l > 0.f ? 1.f / l : 0.f;
-                __nv_bfloat16* orow = p.o + ((static_cast<size_t>(b) * p.Hq + h) * p.N + i_pos) * D;
+            ptx::mbar_arrive(&bar->o_empty[wg]);
+            if (i_pos < p.N) {
+                uint4* dst = reinterpret_cast<uint4*>(p.o + ((static_cast<size_t>(x.b) * p.Hq + x.h) * p.N + i_pos) * D);
 #pragma unroll
-                for (int cc = 0; cc < D / 32; ++cc) {
-                    uint32_t v[32];
-                    ptx::tmem_ld32(t_o + cc * 32, v);
-                    uint32_t w[16];
-#pragma unroll
-                    for (int k = 0; k < 16; ++k)
-                        w[k] = ptx::pack_bf16x2(__uint_as_float(v[2 * k]) * inv_l, __uint_as_float(v[2 * k + 1]) * inv_l);
-                    if (i_pos < p.N) {
-                        uint4* dst = reinterpret_cast<uint4*>(orow + cc * 32);
-#pragma unroll
-                        for (int k = 0; k < 4; ++k) dst[k] = make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
-                    }
-                }
-                if (p.lse != nullptr && i_pos < p.N)
-                    p.lse[(static_cast<size_t>(b) * p.Hq + h) * p.N + i_pos] =
+                for (int k = 0; k < D / 8; ++k) dst[k] = make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+                if (p.lse != nullptr)
+                    p.lse[(static_cast<size_t>(x.b) * p.Hq + x.h) * p.N + i_pos] =
                         l > 0.f ? (m_used + ptx::lg2(l)) * kLn2 : -INFINITY;
-            } else {
-                *abort_flag = 1;
-                raise_status(kStatusTimeout);
             }
+            ++kq;
+        }
+        if (!ok) {
+            *abort_flag = 1;
+            raise_status(kStatusTimeout);
         }
     }
 

@@ -156,6 +156,19 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t smem_addr, uint32_t lbo_
     return d;
 }
 
+// Precomputed 128-byte-swizzle descriptors: the high word (stride byte offset, version 1,
+// swizzle mode) is fixed per operand layout; the low word is (address >> 4) | (LBO >> 4) << 16,
+// so stepping through a tile only adds (byte offset >> 4) to the low word.
+__host__ __device__ constexpr uint32_t sw128_desc_hi(uint32_t sbo_bytes) {
+    return ((sbo_bytes >> 4) & 0x3FFFu) | (1u << 14) | (2u << 29);
+}
+__device__ __forceinline__ uint32_t sw128_desc_lo(uint32_t smem_addr, uint32_t lbo_bytes) {
+    return ((smem_addr & 0x3FFFFu) >> 4) | (((lbo_bytes >> 4) & 0x3FFFu) << 16);
+}
+__device__ __forceinline__ uint64_t desc64(uint32_t lo, uint32_t hi) {
+    return (static_cast<uint64_t>(hi) << 32) | lo;
+}
+
 // 32 lanes x 32 columns of 32-bit TMEM -> registers (thread t of the warp gets lane base+t),
 // with the wait folded in so no register is read before the load has landed.
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {

@@ -70,7 +70,7 @@ typedef enum {
  *          Q "How does Rotary Position Embedding (RoPE) work?"). <=0: no rotation.
  *   scale  >0: softmax scale; <=0: 1/sqrt(D) ("Why is attention scaled by 1/sqrt(dk)?").
  * Constraints: B, Hq, Hkv, N >= 1; Hq % Hkv == 0; D in {64, 128} (else ATTN_ERR_UNSUPPORTED);
- * B <= 65535 and ceil(N/128) <= 65535. Fully masked key tiles are skipped, not computed.
+ * B * Hq * ceil(N/256) < 2^31. Fully masked key tiles are skipped, not computed.
  * Errors: ATTN_ERR_INVALID_ARG for NULL/misaligned pointers or inconsistent sizes/flags;
  * ATTN_ERR_CUDA when a runtime call or the launch fails. With RoPE, the first call for a new
  * (device, rope_base, D, N) or a new stream allocates cached device memory (cudaMalloc).

@@ -53,7 +53,7 @@ def _fwd(api, q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=None, B=1, Hq=4, Hkv=2, N=128,
     (dict(q=None), 1), (dict(o=None), 1), (dict(k=MISALIGNED), 1), (dict(lse=MISALIGNED), 1),
     (dict(B=0), 1), (dict(N=0), 1), (dict(Hq=3, Hkv=2), 1), (dict(causal=2), 1),
     (dict(causal=0, window=16), 1), (dict(scale=float("nan")), 1), (dict(rope=float("inf")), 1),
-    (dict(D=96), 2), (dict(D=256), 2), (dict(B=70000), 2), (dict(N=65536 * 128), 2),
+    (dict(D=96), 2), (dict(D=256), 2), (dict(B=65535, Hq=65535, Hkv=1), 2),
 ])
 def test_fwd_validation(api, kw, expect):
     assert _fwd(api, **kw) == expect
