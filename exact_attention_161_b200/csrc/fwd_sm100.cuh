@@ -297,7 +297,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
                             const int c = x.J0 + u - R.jb;
                             if (c == 0 && kq > 0 && !ptx::mbar_wait(&bar->o_empty[i], (kq - 1) & 1, abort_flag)) { ok = false; break; }
                             if (!ptx::mbar_wait(&bar->p_full[i], (cw + c) & 1, abort_flag)) { ok = false; break; }
-                            ptx::tc_fence_after();
+                            ptx::tc_fence_after();  // P was written to TMEM by the softmax warps
                             const uint32_t vb = v_lo + ((g + u) % NV) * TILE16;
 #pragma unroll
                             for (int kk = 0; kk < C::BN / 16; ++kk)
@@ -308,9 +308,12 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
                         if (u + 1 < x.T && x.active(i, u + 1)) {
                             // S_i(u+1) = Q_i K(u+1)^T into score buffer i
                             const int c = x.J0 + u + 1 - R.jb;
-                            if (c == 0 && !ptx::mbar_wait(&bar->q_ready[i], kq & 1, abort_flag)) { ok = false; break; }
+                            if (c == 0) {
+                                if (!ptx::mbar_wait(&bar->q_ready[i], kq & 1, abort_flag)) { ok = false; break; }
+                                ptx::tc_fence_after();
+                            }
+                            // K arrives by TMA: the barrier alone orders it before the MMA's reads
                             if (!ptx::mbar_wait(&bar->k_full[(g + u + 1) % NK], ((g + u + 1) / NK) & 1, abort_flag)) { ok = false; break; }
-                            ptx::tc_fence_after();
                             const uint32_t qa = q_lo + i * TILE16, kb = k_lo + ((g + u + 1) % NK) * TILE16;
 #pragma unroll
                             for (int kk = 0; kk < D / 16; ++kk) {
