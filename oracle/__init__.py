@@ -45,6 +45,13 @@ def _declare(lib):
     lib.oracle_round_bf16_array.restype = None
     lib.oracle_max_threads.argtypes = []
     lib.oracle_max_threads.restype = i32
+    lib.oracle_attention_f64.argtypes = [p, p, p, i32, i32, i32, i32, i32, i32, i32, f64, f64, i32, p, p]
+    lib.oracle_attention_f64.restype = i32
+    lib.oracle_attention_bwd_f64.argtypes = [p, p, p, p, i32, i32, i32, i32, i32, i32, i32, f64, f64, i32, p,
+                                             p, p, i32]
+    lib.oracle_attention_bwd_f64.restype = i32
+    lib.oracle_attention_bwd.argtypes = [p, p, p, p, i32, i32, i32, i32, i32, i32, i32, f64, f64, p, p, p, i32]
+    lib.oracle_attention_bwd.restype = i32
 
 
 def _ptr(a):
@@ -98,6 +105,61 @@ def attention(q, k, v, causal=False, window=0, rope_base=0.0, scale=None, rows=N
     if rows is None:
         return o.reshape(B, Hq, N, D), lse.reshape(B, Hq, N)
     return o, lse
+
+
+def attention_f64(q, k, v, causal=False, window=0, rope_base=0.0, scale=None, round_rotated=False, lib=None):
+    """Forward on float64 inputs (q [B,Hq,N,D], k/v [B,Hkv,N,D]); round_rotated=False keeps the
+    rotation exact. Returns (o, lse) float64."""
+    lib = lib or _lib()
+    q, k, v = (np.ascontiguousarray(x, dtype=np.float64) for x in (q, k, v))
+    B, Hq, N, D = q.shape
+    Hkv = k.shape[1]
+    if scale is None:
+        scale = 1.0 / np.sqrt(D)
+    o = np.empty_like(q)
+    lse = np.empty((B, Hq, N))
+    st = lib.oracle_attention_f64(_ptr(q), _ptr(k), _ptr(v), B, Hq, Hkv, N, D, int(causal), int(window),
+                                  float(rope_base), float(scale), int(bool(round_rotated)), _ptr(o), _ptr(lse))
+    if st != 0:
+        raise OracleError("oracle_attention_f64 failed with status %d" % st)
+    return o, lse
+
+
+def attention_bwd_f64(q, k, v, dout, causal=False, window=0, rope_base=0.0, scale=None, round_rotated=False,
+                      nthreads=0, lib=None):
+    """Gradients (dq, dk, dv) of sum(O * dout) on float64 inputs."""
+    lib = lib or _lib()
+    q, k, v, dout = (np.ascontiguousarray(x, dtype=np.float64) for x in (q, k, v, dout))
+    B, Hq, N, D = q.shape
+    Hkv = k.shape[1]
+    if scale is None:
+        scale = 1.0 / np.sqrt(D)
+    dq, dk, dv = np.empty_like(q), np.empty_like(k), np.empty_like(v)
+    st = lib.oracle_attention_bwd_f64(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), B, Hq, Hkv, N, D, int(causal),
+                                      int(window), float(rope_base), float(scale), int(bool(round_rotated)),
+                                      _ptr(dq), _ptr(dk), _ptr(dv), int(nthreads))
+    if st != 0:
+        raise OracleError("oracle_attention_bwd_f64 failed with status %d" % st)
+    return dq, dk, dv
+
+
+def attention_bwd(q, k, v, dout, causal=False, window=0, rope_base=0.0, scale=None, nthreads=0, lib=None):
+    """Gradients (dq, dk, dv) of sum(O * dout) for bf16 bit-pattern inputs (uint16), float64 out;
+    the rotated q, k are rounded to bf16 as in the forward."""
+    lib = lib or _lib()
+    q, k, v, dout = _bits(q), _bits(k), _bits(v), _bits(dout)
+    B, Hq, N, D = q.shape
+    Hkv = k.shape[1]
+    if scale is None:
+        scale = 1.0 / np.sqrt(D)
+    dq = np.empty(q.shape)
+    dk = np.empty(k.shape)
+    dv = np.empty(v.shape)
+    st = lib.oracle_attention_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), B, Hq, Hkv, N, D, int(causal), int(window),
+                                  float(rope_base), float(scale), _ptr(dq), _ptr(dk), _ptr(dv), int(nthreads))
+    if st != 0:
+        raise OracleError("oracle_attention_bwd failed with status %d" % st)
+    return dq, dk, dv
 
 
 def decode_paged(q, k_pages, v_pages, block_table, seq_lens, scale=None, nthreads=0, lib=None):

@@ -308,3 +308,205 @@ int oracle_max_threads(void) {
 void oracle_round_bf16_array(const double* x, int64_t n, uint16_t* out) {
     for (int64_t i = 0; i < n; ++i) out[i] = oracle_round_bf16(x[i]);
 }
+
+/* ============================================================================ backward
+ * Gradients of the scalar L = sum_{b,h,i,d} O[b,h,i,d] * dO[b,h,i,d] with respect to q, k, v,
+ * for the same attention as oracle_attention ("Self-Attention Complexity, FlashAttention,
+ * PagedAttention, and RoPE in Code", Part 2: the backward pass; "Why is attention O(n^2), how does
+ * FlashAttention help, ...", "Deep dive: FlashAttention": it recomputes the scores from the saved
+ * statistics instead of storing P). Per query row i, with P_i the softmax row over the visible
+ * keys (written out plainly by the chain rule):
+ *   dV_j += P_ij dO_i                         dP_ij = dO_i . v_j
+ *   dS_ij = P_ij (dP_ij - sum_k P_ik dP_ik)   dq_i  = scale * sum_j dS_ij k_j
+ *   dk_j += scale * dS_ij q_i
+ * where q, k are the rotated vectors. The rotation is linear, so the gradient of the unrotated
+ * vector is the rotated-back gradient: rotate by -angle. Rounding the rotated values to bf16 is
+ * treated as the identity in the gradient.
+ */
+
+/* Rotate a fp64 row by +angle (forward) or -angle (inverse, the transpose); optional bf16 rounding. */
+static void rope_row_f64(const double* x, int D, long pos, double base, int inverse, int round_to_bf16,
+                         double* out) {
+    if (base <= 0.0) {
+        for (int d = 0; d < D; ++d) out[d] = x[d];
+        return;
+    }
+    for (int i = 0; i < D / 2; ++i) {
+        double theta = pow(base, -2.0 * (double)i / (double)D);
+        double angle = (double)pos * theta;
+        double c = cos(angle), s = inverse ? -sin(angle) : sin(angle);
+        double y0 = x[2 * i] * c - x[2 * i + 1] * s;
+        double y1 = x[2 * i] * s + x[2 * i + 1] * c;
+        if (round_to_bf16) {
+            y0 = bf16_value(oracle_round_bf16(y0));
+            y1 = bf16_value(oracle_round_bf16(y1));
+        }
+        out[2 * i] = y0;
+        out[2 * i + 1] = y1;
+    }
+}
+
+/* Forward on fp64 inputs (every row), for the finite-difference and autograd pins. */
+int oracle_attention_f64(const double* q, const double* k, const double* v, int B, int Hq, int Hkv, int N,
+                         int D, int causal, int window, double rope_base, double scale, int round_rotated,
+                         double* o, double* lse) {
+    if (!q || !k || !v || !o || !lse) return ORACLE_ERR_ARG;
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || N <= 0 || D <= 0 || Hq % Hkv != 0) return ORACLE_ERR_ARG;
+    if (window > 0 && !causal) return ORACLE_ERR_ARG;
+    const int G = Hq / Hkv;
+    double* kk = (double*)malloc(sizeof(double) * (size_t)N * D);
+    double* s_row = (double*)malloc(sizeof(double) * (size_t)N);
+    double* qq = (double*)malloc(sizeof(double) * (size_t)D);
+    if (!kk || !s_row || !qq) {
+        free(kk); free(s_row); free(qq);
+        return ORACLE_ERR_NOMEM;
+    }
+    for (int b = 0; b < B; ++b)
+        for (int g = 0; g < Hkv; ++g) {
+            const size_t kv_off = ((size_t)b * Hkv + g) * (size_t)N * D;
+            for (int j = 0; j < N; ++j)
+                rope_row_f64(k + kv_off + (size_t)j * D, D, j, rope_base, 0, round_rotated, kk + (size_t)j * D);
+            for (int hh = 0; hh < G; ++hh) {
+                const int h = g * G + hh;
+                for (int i = 0; i < N; ++i) {
+                    const size_t row = ((size_t)b * Hq + h) * N + i;
+                    rope_row_f64(q + row * D, D, i, rope_base, 0, round_rotated, qq);
+                    attend_row(qq, kk, v + kv_off, N, D, i, causal, window, scale, s_row, o + row * D, lse + row);
+                }
+            }
+        }
+    free(kk); free(s_row); free(qq);
+    return ORACLE_OK;
+}
+
+/* Backward on fp64 inputs. dq: [B,Hq,N,D]; dk, dv: [B,Hkv,N,D]. */
+int oracle_attention_bwd_f64(const double* q, const double* k, const double* v, const double* dout, int B,
+                             int Hq, int Hkv, int N, int D, int causal, int window, double rope_base,
+                             double scale, int round_rotated, double* dq, double* dk, double* dv,
+                             int nthreads) {
+    if (!q || !k || !v || !dout || !dq || !dk || !dv) return ORACLE_ERR_ARG;
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || N <= 0 || D <= 0 || Hq % Hkv != 0) return ORACLE_ERR_ARG;
+    if (window > 0 && !causal) return ORACLE_ERR_ARG;
+    if (rope_base > 0.0 && (D % 2) != 0) return ORACLE_ERR_ARG;
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#else
+    (void)nthreads;
+#endif
+    const int G = Hq / Hkv;
+    const size_t ND = (size_t)N * D;
+    double* kk = (double*)malloc(sizeof(double) * ND);
+    double* dk_rot = (double*)malloc(sizeof(double) * ND);
+    if (!kk || !dk_rot) {
+        free(kk); free(dk_rot);
+        return ORACLE_ERR_NOMEM;
+    }
+    int status = ORACLE_OK;
+    for (int b = 0; b < B && status == ORACLE_OK; ++b)
+        for (int g = 0; g < Hkv && status == ORACLE_OK; ++g) {
+            const size_t kv_off = ((size_t)b * Hkv + g) * ND;
+            const double* vv = v + kv_off;
+            for (int j = 0; j < N; ++j)
+                rope_row_f64(k + kv_off + (size_t)j * D, D, j, rope_base, 0, round_rotated, kk + (size_t)j * D);
+            for (size_t e = 0; e < ND; ++e) dk_rot[e] = 0.0, dv[kv_off + e] = 0.0;
+            /* per-thread accumulators, summed in thread order afterwards (a fixed static schedule
+             * makes the result reproducible for a given thread count) */
+#ifdef _OPENMP
+            const int n_thr = omp_get_max_threads();
+#else
+            const int n_thr = 1;
+#endif
+            double* acc_dk = (double*)calloc((size_t)n_thr * ND, sizeof(double));
+            double* acc_dv = (double*)calloc((size_t)n_thr * ND, sizeof(double));
+            if (!acc_dk || !acc_dv) {
+                free(acc_dk); free(acc_dv);
+                status = ORACLE_ERR_NOMEM;
+                break;
+            }
+#pragma omp parallel num_threads(n_thr)
+            {
+#ifdef _OPENMP
+                const int tid = omp_get_thread_num();
+#else
+                const int tid = 0;
+#endif
+                double* s_row = (double*)malloc(sizeof(double) * (size_t)N);
+                double* dp = (double*)malloc(sizeof(double) * (size_t)N);
+                double* qq = (double*)malloc(sizeof(double) * (size_t)D);
+                double* dqr = (double*)malloc(sizeof(double) * (size_t)D);
+                double* o_row = (double*)malloc(sizeof(double) * (size_t)D);
+                double* my_dk = acc_dk + (size_t)tid * ND;
+                double* my_dv = acc_dv + (size_t)tid * ND;
+                if (!s_row || !dp || !qq || !dqr || !o_row) {
+#pragma omp atomic write
+                    status = ORACLE_ERR_NOMEM;
+                } else {
+#pragma omp for schedule(static)
+                    for (int r = 0; r < G * N; ++r) {
+                        const int h = g * G + r / N, i = r % N;
+                        const size_t row = ((size_t)b * Hq + h) * N + i;
+                        const double* dO = dout + row * D;
+                        double lse_i;
+                        rope_row_f64(q + row * D, D, i, rope_base, 0, round_rotated, qq);
+                        attend_row(qq, kk, vv, N, D, i, causal, window, scale, s_row, o_row, &lse_i);
+                        /* attend_row leaves exp(s_ij - m_i) in s_row; P_ij is that over its row sum */
+                        double lsum = 0.0;
+                        for (int j = 0; j < N; ++j) lsum += s_row[j];
+                        for (int j = 0; j < N; ++j) s_row[j] /= lsum;
+                        double dsum = 0.0;
+                        for (int j = 0; j < N; ++j) {
+                            dp[j] = 0.0;
+                            if (s_row[j] == 0.0) continue;
+                            for (int d = 0; d < D; ++d) dp[j] += dO[d] * vv[(size_t)j * D + d];
+                            dsum += s_row[j] * dp[j];
+                        }
+                        for (int d = 0; d < D; ++d) dqr[d] = 0.0;
+                        for (int j = 0; j < N; ++j) {
+                            const double p = s_row[j];
+                            if (p == 0.0) continue;
+                            const double ds = p * (dp[j] - dsum);
+                            for (int d = 0; d < D; ++d) {
+                                dqr[d] += scale * ds * kk[(size_t)j * D + d];
+                                my_dk[(size_t)j * D + d] += scale * ds * qq[d];
+                                my_dv[(size_t)j * D + d] += p * dO[d];
+                            }
+                        }
+                        rope_row_f64(dqr, D, i, rope_base, 1, 0, dq + row * D);
+                    }
+                }
+                free(s_row); free(dp); free(qq); free(dqr); free(o_row);
+            }
+            for (int t = 0; t < n_thr; ++t)
+                for (size_t e = 0; e < ND; ++e) {
+                    dk_rot[e] += acc_dk[(size_t)t * ND + e];
+                    dv[kv_off + e] += acc_dv[(size_t)t * ND + e];
+                }
+            free(acc_dk); free(acc_dv);
+            for (int j = 0; j < N; ++j)
+                rope_row_f64(dk_rot + (size_t)j * D, D, j, rope_base, 1, 0, dk + kv_off + (size_t)j * D);
+        }
+    free(kk); free(dk_rot);
+    return status;
+}
+
+/* Backward on bf16 inputs (the GPU's bits), rotated values rounded to bf16 as in the forward. */
+int oracle_attention_bwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, const uint16_t* dout, int B,
+                         int Hq, int Hkv, int N, int D, int causal, int window, double rope_base, double scale,
+                         double* dq, double* dk, double* dv, int nthreads) {
+    if (!q || !k || !v || !dout || !dq || !dk || !dv) return ORACLE_ERR_ARG;
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || N <= 0 || D <= 0 || Hq % Hkv != 0) return ORACLE_ERR_ARG;
+    const size_t nq = (size_t)B * Hq * N * D, nk = (size_t)B * Hkv * N * D;
+    double* qd = (double*)malloc(sizeof(double) * nq);
+    double* dod = (double*)malloc(sizeof(double) * nq);
+    double* kd = (double*)malloc(sizeof(double) * nk);
+    double* vd = (double*)malloc(sizeof(double) * nk);
+    int st = ORACLE_ERR_NOMEM;
+    if (qd && dod && kd && vd) {
+        for (size_t e = 0; e < nq; ++e) qd[e] = bf16_value(q[e]), dod[e] = bf16_value(dout[e]);
+        for (size_t e = 0; e < nk; ++e) kd[e] = bf16_value(k[e]), vd[e] = bf16_value(v[e]);
+        st = oracle_attention_bwd_f64(qd, kd, vd, dod, B, Hq, Hkv, N, D, causal, window, rope_base, scale, 1,
+                                      dq, dk, dv, nthreads);
+    }
+    free(qd); free(dod); free(kd); free(vd);
+    return st;
+}

@@ -375,3 +375,97 @@ ALL_CHECKS = [
     check_rows_subset, check_online_recurrence, check_decode_is_last_prefill_row,
     check_decode_library, check_decode_paging_invariance,
 ]
+
+
+# ---------------------------------------------------------------------------------- backward
+
+def _bwd_case(seed, B=1, Hq=2, Hkv=1, N=9, D=4):
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((B, Hq, N, D))
+    k = rng.standard_normal((B, Hkv, N, D))
+    v = rng.standard_normal((B, Hkv, N, D))
+    do = rng.standard_normal((B, Hq, N, D))
+    return q, k, v, do
+
+
+def check_bwd_finite_differences(lib):
+    """Every gradient entry against a central difference of L = sum(O * dO) (brute force)."""
+    for causal, window, rope in ((0, 0, 0.0), (1, 0, 0.0), (1, 3, 0.0), (1, 0, 50.0)):
+        q, k, v, do = _bwd_case(17 + window)
+        dq, dk, dv = oracle.attention_bwd_f64(q, k, v, do, causal=causal, window=window, rope_base=rope, lib=lib)
+
+        def loss(qq, kk, vv):
+            o, _ = oracle.attention_f64(qq, kk, vv, causal=causal, window=window, rope_base=rope, lib=lib)
+            return float((o * do).sum())
+
+        eps = 1e-6
+        for which, (arr, grad) in enumerate(((q, dq), (k, dk), (v, dv))):
+            for idx in np.ndindex(arr.shape):
+                a = arr.copy()
+                a[idx] += eps
+                args = [q, k, v]
+                args[which] = a
+                lp = loss(*args)
+                a[idx] -= 2 * eps
+                args[which] = a
+                lm = loss(*args)
+                assert abs((lp - lm) / (2 * eps) - grad[idx]) < 1e-7, (causal, window, rope, which, idx)
+
+
+def _torch_rope(x, base):
+    """Pairwise rotation written with torch ops, so autograd supplies the chain rule."""
+    if base <= 0:
+        return x
+    N, D = x.shape[-2], x.shape[-1]
+    pos = torch.arange(N, dtype=torch.float64)[:, None]
+    theta = base ** (-2.0 * torch.arange(D // 2, dtype=torch.float64) / D)
+    ang = pos * theta[None, :]
+    c, s = torch.cos(ang), torch.sin(ang)
+    x0, x1 = x[..., 0::2], x[..., 1::2]
+    y = torch.stack((x0 * c - x1 * s, x0 * s + x1 * c), dim=-1)
+    return y.reshape(x.shape)
+
+
+def check_bwd_torch_autograd(lib):
+    """Gradients against torch float64 autograd through SDPA (masks, GQA) and the rotation."""
+    for causal, window, rope in ((0, 0, 0.0), (1, 0, 0.0), (1, 5, 0.0), (1, 0, 1000.0)):
+        q, k, v, do = _bwd_case(23, B=2, Hq=4, Hkv=2, N=24, D=8)
+        dq, dk, dv = oracle.attention_bwd_f64(q, k, v, do, causal=causal, window=window, rope_base=rope, lib=lib)
+        qt, kt, vt = (torch.tensor(x, requires_grad=True) for x in (q, k, v))
+        mask = None
+        if window:
+            i = torch.arange(24)[:, None]
+            j = torch.arange(24)[None, :]
+            mask = (j <= i) & (j >= i - window + 1)
+        o = torch.nn.functional.scaled_dot_product_attention(
+            _torch_rope(qt, rope), _torch_rope(kt, rope), vt, attn_mask=mask, is_causal=bool(causal and not window),
+            scale=8 ** -0.5, enable_gqa=True)
+        (o * torch.tensor(do)).sum().backward()
+        assert np.abs(dq - qt.grad.numpy()).max() < 1e-10
+        assert np.abs(dk - kt.grad.numpy()).max() < 1e-10
+        assert np.abs(dv - vt.grad.numpy()).max() < 1e-10
+
+
+def check_bwd_gqa_is_sum_over_group(lib):
+    """The K/V gradient of a shared head is the sum of the gradients of its repeated copies."""
+    q, k, v, do = _bwd_case(29, Hq=4, Hkv=2, N=12, D=4)
+    dq, dk, dv = oracle.attention_bwd_f64(q, k, v, do, causal=1, rope_base=10.0, lib=lib)
+    kr, vr = np.repeat(k, 2, axis=1), np.repeat(v, 2, axis=1)
+    dq2, dk2, dv2 = oracle.attention_bwd_f64(q, kr, vr, do, causal=1, rope_base=10.0, lib=lib)
+    assert np.abs(dq - dq2).max() < 1e-12
+    assert np.abs(dk - dk2.reshape(1, 2, 2, 12, 4).sum(axis=2)).max() < 1e-12
+    assert np.abs(dv - dv2.reshape(1, 2, 2, 12, 4).sum(axis=2)).max() < 1e-12
+
+
+def check_bwd_bf16_entry(lib):
+    """The bf16 entry point is the fp64 one on the exact input values with bf16-rounded rotation."""
+    q, k, v = (synth.bits(t) for t in synth.prefill_inputs(1, 2, 1, 40, 64, 33))
+    do = _rand((1, 2, 40, 64), 34).reshape(1, 2, 40, 64)
+    g1 = oracle.attention_bwd(q, k, v, do, causal=True, rope_base=10000.0, scale=0.125, lib=lib)
+    g2 = oracle.attention_bwd_f64(_f64(q), _f64(k), _f64(v), _f64(do), causal=True, rope_base=10000.0, scale=0.125,
+                                  round_rotated=True, lib=lib)
+    assert all(np.array_equal(a, b) for a, b in zip(g1, g2))
+
+
+ALL_CHECKS += [check_bwd_finite_differences, check_bwd_torch_autograd, check_bwd_gqa_is_sum_over_group,
+               check_bwd_bf16_entry]
