@@ -297,6 +297,39 @@ def run_ours(args, rank, world, local):
     value = job_throughput(flops * K, world, prefill_sum_max / 1e3) / 1e12 if do_prefill else None
     decode_value = job_throughput(dbytes * K, world, decode_sum_max / 1e3) / 1e9 if do_decode else None
 
+    # ---- backward of the prefill workload (its own loop; not part of the step)
+    bwd = None
+    if do_prefill and args.bwd_steps > 0:
+        dout = synth.randn_bf16(tuple(q.shape), torch.Generator().manual_seed(PREFILL.seed + 1)).to(dev)
+        gq, gk, gv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        bws = torch.empty(api.bwd_workspace_size(PREFILL.B, PREFILL.Hq, PREFILL.Hkv, PREFILL.N, PREFILL.D,
+                                                 PREFILL.rope_base), dtype=torch.uint8, device=dev)
+
+        def backward():
+            api.attn_bwd(q, k, v, o, lse, dout, causal=PREFILL.causal, window=PREFILL.window,
+                         rope_base=PREFILL.rope_base, dq=gq, dk=gk, dv=gv, workspace=bws, stream=stream)
+
+        prefill()
+        for _ in range(args.warmup):
+            backward()
+        barrier(world)
+        torch.cuda.synchronize()
+        b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        b0.record(stream)
+        for _ in range(args.bwd_steps):
+            backward()
+        b1.record(stream)
+        torch.cuda.synchronize()
+        if api.device_status() != 0:
+            raise RuntimeError("device status raised during the backward loop")
+        bwd_ms = reduce_max(b0.elapsed_time(b1), world, dev) / args.bwd_steps
+        bwd_flops = flops * 5 // 2  # five products per unmasked pair (S, dP, dV, dK, dQ) vs two forward
+        bwd = {"metric": "attn bwd TFLOP/s (same workload; algorithmic FLOPs = 2.5 x forward)",
+               "value": round(job_throughput(bwd_flops, world, bwd_ms / 1e3) / 1e12, 2), "unit": "TFLOP/s",
+               "ms_per_call": round(bwd_ms, 4), "calls": args.bwd_steps,
+               "roofline": {"bound": "tensor", "achieved": round(bwd_flops / (bwd_ms / 1e3) / 1e12, 2),
+                            "unit": "TFLOP/s", "note": "five-kernel call: rotation x2, prep, dK/dV, dQ"}}
+
     # ---- end to end through the public API with pinned host buffers
     E = min(args.e2e_steps, K) if (args.e2e_steps > 0 and args.only == "all") else 0
     if E:
@@ -342,6 +375,9 @@ def run_ours(args, rank, world, local):
     tflops_launch = flops / (pre_launch_ms / 1e3) / 1e12 if do_prefill else float("nan")
     gbs_launch = dbytes / (dec_launch_ms / 1e3) / 1e9 if do_decode else float("nan")
     tensor_peak = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
+    if bwd is not None:
+        bwd["roofline"].update({"peak": tensor_peak, "frac": round(bwd["roofline"]["achieved"] / tensor_peak, 4),
+                                "peak_kind": "%s bf16 GEMM, sustained" % peaks_kind})
     line = {
         "metric": "attn fwd TFLOP/s (causal GQA prefill B2 Hq32 Hkv8 N8192 D128, RoPE 5e5) "
                   "& paged-decode KV GB/s",
@@ -384,6 +420,7 @@ def run_ours(args, rank, world, local):
         "e2e": {"value": round(e2e_value, 2) if E else None, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": (2 * do_prefill + 2 * do_decode) * K,
+        "backward": bwd,
         "device_status": status,
         "clocks": clk,
     }
@@ -461,6 +498,7 @@ def parse_args(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--e2e-steps", type=int, default=10, help="0 skips the end-to-end leg")
+    ap.add_argument("--bwd-steps", type=int, default=20, help="backward calls timed after the step loop; 0 skips")
     ap.add_argument("--only", choices=["all", "prefill", "decode"], default="all",
                     help="time one half of the step only (profiling runs); the JSON line is then partial")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle time for the CPU baseline")

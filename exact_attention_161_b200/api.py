@@ -27,6 +27,8 @@ DEVICE_TIMEOUT, DEVICE_BAD_PAGE, DEVICE_BAD_SEQLEN = 1, 2, 4
 _p, _i, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
 SIGNATURES = {
     "attn_fwd": (_i, [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _f, _f, _p]),
+    "attn_bwd_workspace_size": (_sz, [_i, _i, _i, _i, _i, _f]),
+    "attn_bwd": (_i, [_p, _p, _p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _f, _f, _p, _sz, _p]),
     "attn_decode_workspace_size": (_sz, [_i, _i, _i, _i, _i]),
     "attn_decode_paged": (_i, [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _f, _p, _p, _p, _sz, _p]),
     "attn_decode_paged_noalloc": (_i, [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _f, _p, _p, _p]),
@@ -109,6 +111,31 @@ def attn_fwd(q, k, v, causal=False, window=0, rope_base=0.0, scale=0.0, o=None, 
     _check(lib.attn_fwd(*args, B, Hq, Hkv, N, D, int(bool(causal)), int(window), float(rope_base), float(scale),
                         _stream(stream)))
     return o, lse
+
+
+def bwd_workspace_size(B, Hq, Hkv, N, D, rope_base=0.0) -> int:
+    return int(lib.attn_bwd_workspace_size(B, Hq, Hkv, N, D, float(rope_base)))
+
+
+def attn_bwd(q, k, v, o, lse, dout, causal=False, window=0, rope_base=0.0, scale=0.0, dq=None, dk=None, dv=None,
+             workspace=None, stream=None):
+    """Attention backward. q/o/dout [B,Hq,N,D], k/v [B,Hkv,N,D] bf16, lse [B,Hq,N] fp32 (from
+    attn_fwd with the same arguments). Returns (dq, dk, dv), bf16."""
+    B, Hq, N, D = q.shape
+    Hkv = k.shape[1]
+    if k.shape != (B, Hkv, N, D) or v.shape != k.shape or o.shape != q.shape or dout.shape != q.shape:
+        raise ValueError("shape mismatch")
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    if workspace is None:
+        workspace = torch.empty(bwd_workspace_size(B, Hq, Hkv, N, D, rope_base), dtype=torch.uint8, device=q.device)
+    args = [_dev_tensor(t, n, torch.bfloat16) for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"))]
+    args += [_dev_tensor(lse, "lse", torch.float32), _dev_tensor(dout, "dout", torch.bfloat16)]
+    args += [_dev_tensor(t, n, torch.bfloat16) for t, n in ((dq, "dq"), (dk, "dk"), (dv, "dv"))]
+    _check(lib.attn_bwd(*args, B, Hq, Hkv, N, D, int(bool(causal)), int(window), float(rope_base), float(scale),
+                        _dev_tensor(workspace, "workspace", torch.uint8), workspace.numel(), _stream(stream)))
+    return dq, dk, dv
 
 
 def decode_workspace_size(num_seqs, max_blocks_per_seq, page_size, Hq, D) -> int:

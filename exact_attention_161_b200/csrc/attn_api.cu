@@ -16,6 +16,7 @@
 
 #include "attn.h"
 #include "common.cuh"
+#include "bwd_sm100.cuh"
 #include "decode.cuh"
 #include "fwd_sm100.cuh"
 #include "rope.cuh"
@@ -245,6 +246,90 @@ attn_status launch_decode(const void* q, const void* k_pages, const void* v_page
     return ATTN_OK;
 }
 
+struct BwdLayout {
+    size_t vec, qrot, krot, total;  // byte offsets within the workspace
+};
+
+BwdLayout bwd_layout(int B, int Hq, int Hkv, int N, int D, bool rope) {
+    auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+    const size_t npad = static_cast<size_t>((N + 127) / 128) * 128;
+    BwdLayout L{};
+    L.vec = 0;
+    L.qrot = up(static_cast<size_t>(B) * Hq * npad * 2 * sizeof(float));
+    L.krot = L.qrot + (rope ? up(static_cast<size_t>(B) * Hq * N * D * 2) : 0);
+    L.total = L.krot + (rope ? up(static_cast<size_t>(B) * Hkv * N * D * 2) : 0);
+    return L;
+}
+
+template <int D>
+attn_status launch_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
+                       void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int N, int causal, int window,
+                       float rope_base, float scale, void* ws, cudaStream_t stream, int dev) {
+    using C = attn::BwdCfg<D>;
+    const bool rope = rope_base > 0.f;
+    const BwdLayout L = bwd_layout(B, Hq, Hkv, N, D, rope);
+    uint8_t* w = static_cast<uint8_t*>(ws);
+    attn::BwdParams p{};
+    p.o = static_cast<const __nv_bfloat16*>(o);
+    p.dout = static_cast<const __nv_bfloat16*>(dout);
+    p.lse = lse;
+    p.vec = reinterpret_cast<float*>(w + L.vec);
+    p.dq = static_cast<__nv_bfloat16*>(dq);
+    p.dk = static_cast<__nv_bfloat16*>(dk);
+    p.dv = static_cast<__nv_bfloat16*>(dv);
+    p.B = B;
+    p.Hq = Hq;
+    p.Hkv = Hkv;
+    p.N = N;
+    p.Npad = (N + 127) / 128 * 128;
+    p.causal = causal;
+    p.window = window > 0 ? window : 0;
+    p.scale = scale;
+    p.scale_log2 = scale * attn::kLog2e;
+    int sms = 148;
+    CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+    const void* q_use = q;
+    const void* k_use = k;
+    if (rope) {
+        const float2* table = nullptr;
+        attn_status st = rope_table(dev, static_cast<double>(rope_base), D, N, &table);
+        if (st != ATTN_OK) return st;
+        p.rope = table;
+        void* qr = w + L.qrot;
+        void* kr = w + L.krot;
+        const long long qrows = static_cast<long long>(B) * Hq * N, krows = static_cast<long long>(B) * Hkv * N;
+        auto grid_for = [&](long long rows) {
+            const long long want = (rows * (D / 8) + 255) / 256;
+            return static_cast<int>(want < 8LL * sms ? want : 8LL * sms);
+        };
+        attn::rope_rotate_rows_kernel<D><<<grid_for(qrows), 256, 0, stream>>>(static_cast<const uint4*>(q),
+                                                                              static_cast<uint4*>(qr), table, qrows, N);
+        CUDA_TRY(cudaGetLastError());
+        attn::rope_rotate_rows_kernel<D><<<grid_for(krows), 256, 0, stream>>>(static_cast<const uint4*>(k),
+                                                                              static_cast<uint4*>(kr), table, krows, N);
+        CUDA_TRY(cudaGetLastError());
+        q_use = qr;
+        k_use = kr;
+    }
+    const long long vec_rows = static_cast<long long>(B) * Hq * p.Npad;
+    attn::bwd_prep_kernel<D><<<static_cast<unsigned>((vec_rows * 32 + 255) / 256), 256, 0, stream>>>(p);
+    CUDA_TRY(cudaGetLastError());
+    CUtensorMap tq, tk, tv, tdo;
+    attn_status st;
+    if ((st = make_map_3d(&tq, q_use, D, N, static_cast<uint64_t>(B) * Hq, 128)) != ATTN_OK) return st;
+    if ((st = make_map_3d(&tk, k_use, D, N, static_cast<uint64_t>(B) * Hkv, 128)) != ATTN_OK) return st;
+    if ((st = make_map_3d(&tv, v, D, N, static_cast<uint64_t>(B) * Hkv, 128)) != ATTN_OK) return st;
+    if ((st = make_map_3d(&tdo, dout, D, N, static_cast<uint64_t>(B) * Hq, 128)) != ATTN_OK) return st;
+    if ((st = ensure_smem(attn::attn_bwd_dkdv_kernel<D>, C::SMEM_BYTES, dev)) != ATTN_OK) return st;
+    if ((st = ensure_smem(attn::attn_bwd_dq_kernel<D>, C::SMEM_BYTES, dev)) != ATTN_OK) return st;
+    const int ntiles = (N + 127) / 128;
+    attn::attn_bwd_dkdv_kernel<D><<<dim3(ntiles, Hkv, B), C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, p);
+    CUDA_TRY(cudaGetLastError());
+    attn::attn_bwd_dq_kernel<D><<<dim3(ntiles, Hq, B), C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, p);
+    CUDA_TRY(cudaGetLastError());
+    return ATTN_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -271,6 +356,42 @@ attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (D == 64) return launch_fwd<64>(q, k, v, o, lse, B, Hq, Hkv, N, causal, window, rope_base, scale, s, dev);
     return launch_fwd<128>(q, k, v, o, lse, B, Hq, Hkv, N, causal, window, rope_base, scale, s, dev);
+}
+
+size_t attn_bwd_workspace_size(int B, int Hq, int Hkv, int N, int D, float rope_base) {
+    if (B < 1 || Hq < 1 || Hkv < 1 || N < 1 || D < 1) return 0;
+    return bwd_layout(B, Hq, Hkv, N, D, rope_base > 0.f).total;
+}
+
+attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
+                     void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int N, int D, int causal, int window,
+                     float rope_base, float scale, void* workspace, size_t workspace_bytes, void* stream) {
+    g_last_error.clear();
+    if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv || !workspace)
+        return fail(ATTN_ERR_INVALID_ARG, "q, k, v, o, lse, dout, dq, dk, dv and workspace must be non-NULL");
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) || !aligned16(dq) ||
+        !aligned16(dk) || !aligned16(dv) || !aligned16(workspace) || (reinterpret_cast<uintptr_t>(lse) & 3u))
+        return fail(ATTN_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned (lse 4-byte)");
+    if (B < 1 || Hq < 1 || Hkv < 1 || N < 1) return fail(ATTN_ERR_INVALID_ARG, "B, Hq, Hkv, N must be >= 1");
+    if (Hq % Hkv != 0) return fail(ATTN_ERR_INVALID_ARG, "Hq (%d) must be a multiple of Hkv (%d)", Hq, Hkv);
+    if (causal != 0 && causal != 1) return fail(ATTN_ERR_INVALID_ARG, "causal must be 0 or 1");
+    if (window > 0 && !causal) return fail(ATTN_ERR_INVALID_ARG, "a sliding window requires causal = 1");
+    if (!std::isfinite(scale) || !std::isfinite(rope_base)) return fail(ATTN_ERR_INVALID_ARG, "scale and rope_base must be finite");
+    if (D != 64 && D != 128) return fail(ATTN_ERR_UNSUPPORTED, "head dim %d not supported (64 or 128)", D);
+    if (B > 65535 || Hq > 65535 || (N + 127) / 128 > 0x7fffffff / 2) return fail(ATTN_ERR_UNSUPPORTED, "grid too large");
+    if (static_cast<double>(B) * Hq * N * D * 2 >= 1099511627776.0) return fail(ATTN_ERR_UNSUPPORTED, "tensor larger than 1 TiB");
+    const size_t need = attn_bwd_workspace_size(B, Hq, Hkv, N, D, rope_base);
+    if (workspace_bytes < need)
+        return fail(ATTN_ERR_INVALID_ARG, "workspace too small: %zu < %zu bytes", workspace_bytes, need);
+    if (scale <= 0.f) scale = 1.0f / std::sqrt(static_cast<float>(D));
+    int dev = 0;
+    CUDA_TRY(cudaGetDevice(&dev));
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (D == 64)
+        return launch_bwd<64>(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, N, causal, window, rope_base, scale,
+                              workspace, s, dev);
+    return launch_bwd<128>(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, N, causal, window, rope_base, scale,
+                           workspace, s, dev);
 }
 
 size_t attn_decode_workspace_size(int num_seqs, int max_blocks_per_seq, int page_size, int Hq, int D) {

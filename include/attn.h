@@ -1,9 +1,10 @@
 /*
  * attn.h -- C ABI of libattn_b200.so: exact scaled dot-product attention on NVIDIA B200 (sm_100a).
  *
- * Two operations, both computing softmax(Q K^T * scale) V exactly (up to floating-point
- * rounding), never materialising the n x n score matrix in device memory:
+ * Operations computing softmax(Q K^T * scale) V exactly (up to floating-point rounding), never
+ * materialising the n x n score matrix in device memory:
  *   attn_fwd           prefill over whole sequences (causal / sliding-window / full, GQA, RoPE);
+ *   attn_bwd           its gradients, recomputing the scores from the saved logsumexp;
  *   attn_decode_paged  one new query token per sequence over a paged KV cache.
  *
  * Conventions shared by every entry point:
@@ -77,6 +78,36 @@ typedef enum {
  */
 attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
                      int N, int D, int causal, int window, float rope_base, float scale, void* stream);
+
+/*
+ * attn_bwd_workspace_size -- bytes of device workspace attn_bwd needs: fp32 (LSE*log2 e, D_i) per
+ * query row padded to 128-row tiles, plus, with RoPE, the rotated Q and K (bf16). 0 for invalid sizes.
+ */
+size_t attn_bwd_workspace_size(int B, int Hq, int Hkv, int N, int D, float rope_base);
+
+/*
+ * attn_bwd -- attention backward: gradients of L = sum(O * dout) with respect to q, k and v for the
+ * attention attn_fwd computes (same masks, GQA map, RoPE and scale). The scores are recomputed from
+ * q, k and the forward's row logsumexp instead of being stored ("Self-Attention Complexity,
+ * FlashAttention, PagedAttention, and RoPE in Code", Part 2: recomputation in the backward pass;
+ * "Why is attention O(n^2), how does FlashAttention help, ...", "Deep dive: FlashAttention": the
+ * backward recomputes scores from the saved m and l):
+ *   dv_j = sum_i P_ij dO_i,  dS_ij = P_ij (dO_i . v_j - dO_i . O_i),
+ *   dq_i = scale sum_j dS_ij k_j,  dk_j = scale sum_i dS_ij q_i,
+ * with q, k rotated; the gradients of the unrotated inputs are rotated back. For GQA, dk and dv of a
+ * K/V head sum over its query heads.
+ *
+ *   q, k, v, causal, window, rope_base, scale, B, Hq, Hkv, N, D   as given to attn_fwd
+ *   o      bf16 [B, Hq, N, D] and lse fp32 [B, Hq, N]: attn_fwd's outputs for these inputs
+ *   dout   bf16 [B, Hq, N, D] gradient of the loss with respect to o
+ *   dq     bf16 [B, Hq, N, D]; dk, dv bf16 [B, Hkv, N, D]: written
+ *   workspace  device scratch of at least attn_bwd_workspace_size(...) bytes, 16-byte aligned,
+ *          owned by the caller, any initial contents; overlapping calls need their own.
+ * Constraints and errors as attn_fwd (D in {64, 128}; B, Hq <= 65535).
+ */
+attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
+                     void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int N, int D, int causal, int window,
+                     float rope_base, float scale, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * attn_decode_workspace_size -- bytes of device workspace attn_decode_paged needs: fp32 partial

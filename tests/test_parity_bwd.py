@@ -1,0 +1,86 @@
+"""Backward parity (GPU only): gradients from attn_bwd against the fp64 oracle's backward.
+
+The GPU path runs its own forward (O and LSE) and then the backward, as training does; the oracle
+computes the exact gradients of sum(O * dO) from the same bf16 inputs. Tolerances (the gradients
+are stored in bf16, and P and dS pass through bf16 on the way to the tensor cores): relative RMS
+<= 5e-3 over each gradient tensor, and max-abs <= max|gradient| / 128 (four bf16 half-ulps at the
+largest gradient). Both scales have a floor (RMS 1e-3, max-abs 1e-4): with one visible key per
+row the softmax is constant, so dS = dP - D and hence dq and dk are exactly zero, and what remains is
+fp32 cancellation of two equal dot products.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from exact_attention_161_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+GRAD_REL_RMS = 5e-3
+GRAD_MAX_ABS_FRAC = 1.0 / 128
+RMS_FLOOR = 1e-3
+ABS_FLOOR = 1e-4
+
+# B, Hq, Hkv, N, D, causal, window, rope_base
+CASES = [
+    (1, 1, 1, 128, 64, 0, 0, 0.0),
+    (1, 2, 1, 200, 128, 1, 0, 10000.0),
+    (2, 2, 2, 129, 128, 0, 0, 0.0),
+    (1, 4, 2, 300, 64, 1, 0, 0.0),
+    (1, 4, 4, 500, 128, 1, 100, 10000.0),
+    (1, 8, 2, 256, 128, 1, 0, 500000.0),
+    (1, 2, 2, 17, 128, 1, 0, 10000.0),
+    (1, 2, 1, 1, 64, 1, 0, 10000.0),
+    (1, 4, 2, 640, 128, 0, 0, 10000.0),
+    (4, 16, 16, 2048, 128, 1, 0, 10000.0),  # the N=2048 MHA workload's shape
+]
+
+
+def _ids(c):
+    return "B%dHq%dHkv%dN%dD%d_c%d_w%d_r%g" % c
+
+
+def check_grad(name, got, ref):
+    x = got.float().cpu().numpy().astype(np.float64)
+    assert np.all(np.isfinite(x)), name
+    d = x - ref
+    rel_rms = np.sqrt((d ** 2).mean()) / max(np.sqrt((ref ** 2).mean()), RMS_FLOOR)
+    max_abs = np.abs(d).max()
+    assert rel_rms <= GRAD_REL_RMS, "%s rel-RMS %.3e" % (name, rel_rms)
+    assert max_abs <= GRAD_MAX_ABS_FRAC * np.abs(ref).max() + ABS_FLOOR, "%s max-abs %.3e (max ref %.3e)" % (
+        name, max_abs, np.abs(ref).max())
+
+
+@pytest.mark.parametrize("case", CASES, ids=_ids)
+def test_backward_vs_oracle(cuda_api, case):
+    B, Hq, Hkv, N, D, causal, window, rope = case
+    ci = CASES.index(case)
+    q, k, v = synth.prefill_inputs(B, Hq, Hkv, N, D, seed=300 + ci)
+    dout = synth.randn_bf16((B, Hq, N, D), torch.Generator().manual_seed(400 + ci))
+    qd, kd, vd, dod = q.cuda(), k.cuda(), v.cuda(), dout.cuda()
+    o, lse = cuda_api.attn_fwd(qd, kd, vd, causal=causal, window=window, rope_base=rope)
+    dq, dk, dv = cuda_api.attn_bwd(qd, kd, vd, o, lse, dod, causal=causal, window=window, rope_base=rope)
+    torch.cuda.synchronize()
+    assert cuda_api.device_status() == 0
+    rq, rk, rv = oracle.attention_bwd(synth.bits(q), synth.bits(k), synth.bits(v), synth.bits(dout), causal=causal,
+                                      window=window, rope_base=rope, scale=D ** -0.5)
+    check_grad("dq", dq, rq)
+    check_grad("dk", dk, rk)
+    check_grad("dv", dv, rv)
+
+
+def test_backward_gqa_equals_repeated_heads(cuda_api):
+    """dk, dv of a shared K/V head equal the sums over the copies when K/V are repeated per head."""
+    q, k, v = synth.prefill_inputs(1, 4, 2, 300, 128, seed=77)
+    dout = synth.randn_bf16((1, 4, 300, 128), torch.Generator().manual_seed(78)).cuda()
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    o, lse = cuda_api.attn_fwd(qd, kd, vd, causal=True, rope_base=10000.0)
+    dq, dk, dv = cuda_api.attn_bwd(qd, kd, vd, o, lse, dout, causal=True, rope_base=10000.0)
+    kr, vr = kd.repeat_interleave(2, dim=1), vd.repeat_interleave(2, dim=1)
+    o2, lse2 = cuda_api.attn_fwd(qd, kr, vr, causal=True, rope_base=10000.0)
+    dq2, dk2, dv2 = cuda_api.attn_bwd(qd, kr, vr, o2, lse2, dout, causal=True, rope_base=10000.0)
+    assert torch.equal(dq.view(torch.int16), dq2.view(torch.int16))
+    for a, b in ((dk, dk2), (dv, dv2)):
+        summed = b.float().reshape(1, 2, 2, 300, 128).sum(dim=2)
+        assert float((a.float() - summed).abs().max()) <= 2.0 ** -7 * float(summed.abs().max())
