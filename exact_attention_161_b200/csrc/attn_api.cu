@@ -281,7 +281,7 @@ attn_status launch_bwd(const void* q, const void* k, const void* v, const void* 
     p.Hq = Hq;
     p.Hkv = Hkv;
     p.N = N;
-    p.Npad = (N + 127) / 128 * 128;
+    p.ntiles = (N + 127) / 128;
     p.causal = causal;
     p.window = window > 0 ? window : 0;
     p.scale = scale;
@@ -311,8 +311,10 @@ attn_status launch_bwd(const void* q, const void* k, const void* v, const void* 
         q_use = qr;
         k_use = kr;
     }
-    const long long vec_rows = static_cast<long long>(B) * Hq * p.Npad;
-    attn::bwd_prep_kernel<D><<<static_cast<unsigned>((vec_rows * 32 + 255) / 256), 256, 0, stream>>>(p);
+    const long long vec_rows = static_cast<long long>(B) * Hq * p.ntiles * 128;
+    const long long prep_blocks = (vec_rows / (256 / 32 * (32 / (D / 8)))) + 1;
+    attn::bwd_prep_kernel<D><<<static_cast<unsigned>(prep_blocks < 16LL * sms ? prep_blocks : 16LL * sms), 256, 0,
+                               stream>>>(p);
     CUDA_TRY(cudaGetLastError());
     CUtensorMap tq, tk, tv, tdo;
     attn_status st;
@@ -322,10 +324,13 @@ attn_status launch_bwd(const void* q, const void* k, const void* v, const void* 
     if ((st = make_map_3d(&tdo, dout, D, N, static_cast<uint64_t>(B) * Hq, 128)) != ATTN_OK) return st;
     if ((st = ensure_smem(attn::attn_bwd_dkdv_kernel<D>, C::SMEM_BYTES, dev)) != ATTN_OK) return st;
     if ((st = ensure_smem(attn::attn_bwd_dq_kernel<D>, C::SMEM_BYTES, dev)) != ATTN_OK) return st;
-    const int ntiles = (N + 127) / 128;
-    attn::attn_bwd_dkdv_kernel<D><<<dim3(ntiles, Hkv, B), C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, p);
+    // one-dimensional grids, tile index slowest (the kernels start the longest causal tiles first)
+    const unsigned nt = static_cast<unsigned>(p.ntiles);
+    attn::attn_bwd_dkdv_kernel<D><<<nt * static_cast<unsigned>(B * Hkv), C::THREADS, C::SMEM_BYTES, stream>>>(
+        tq, tk, tv, tdo, p);
     CUDA_TRY(cudaGetLastError());
-    attn::attn_bwd_dq_kernel<D><<<dim3(ntiles, Hq, B), C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, p);
+    attn::attn_bwd_dq_kernel<D><<<nt * static_cast<unsigned>(B * Hq), C::THREADS, C::SMEM_BYTES, stream>>>(
+        tq, tk, tv, tdo, p);
     CUDA_TRY(cudaGetLastError());
     return ATTN_OK;
 }
@@ -378,7 +383,8 @@ attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o,
     if (window > 0 && !causal) return fail(ATTN_ERR_INVALID_ARG, "a sliding window requires causal = 1");
     if (!std::isfinite(scale) || !std::isfinite(rope_base)) return fail(ATTN_ERR_INVALID_ARG, "scale and rope_base must be finite");
     if (D != 64 && D != 128) return fail(ATTN_ERR_UNSUPPORTED, "head dim %d not supported (64 or 128)", D);
-    if (B > 65535 || Hq > 65535 || (N + 127) / 128 > 0x7fffffff / 2) return fail(ATTN_ERR_UNSUPPORTED, "grid too large");
+    if (static_cast<double>(B) * Hq * ((N + 127) / 128) >= 2147483648.0)
+        return fail(ATTN_ERR_UNSUPPORTED, "grid too large: B * Hq * ceil(N/128) must be < 2^31");
     if (static_cast<double>(B) * Hq * N * D * 2 >= 1099511627776.0) return fail(ATTN_ERR_UNSUPPORTED, "tensor larger than 1 TiB");
     const size_t need = attn_bwd_workspace_size(B, Hq, Hkv, N, D, rope_base);
     if (workspace_bytes < need)

@@ -15,7 +15,10 @@
 // kernel with one CTA per (128-key tile, K/V head) that walks every query head of the group and
 // every query tile that sees the keys, and a dQ kernel with one CTA per (128-query tile, query
 // head) that walks the visible key tiles. All five products per tile pair run on tcgen05 with
-// fp32 accumulators in Tensor Memory; the elementwise step runs one row per thread.
+// fp32 accumulators in Tensor Memory. Eight elementwise warps (two warpgroups, each owning 64 of
+// the 128 columns of a tile) turn scores into P and dS; the products are issued in an order that
+// lets the tensor core work on the next tile while they do (see each kernel's issue loop).
+// CTAs are numbered so that the ones with the most work start first.
 #pragma once
 #include "common.cuh"
 #include "fwd_sm100.cuh"
@@ -27,40 +30,54 @@ struct BwdParams {
     const __nv_bfloat16* o;     // [B, Hq, N, D] forward output
     const __nv_bfloat16* dout;  // [B, Hq, N, D]
     const float* lse;           // [B, Hq, N] forward logsumexp (natural log)
-    float* vec;                 // [B*Hq, Npad, 2]: (LSE * log2 e, D_i); rows >= N hold (+inf, 0)
+    float* vec;                 // [B*Hq, ntiles, 2, 128]: per 128-row tile -LSE*log2 e, then -D_i;
+                                // rows >= N hold (-inf, 0)
     __nv_bfloat16* dq;          // [B, Hq, N, D]
     __nv_bfloat16* dk;          // [B, Hkv, N, D]
     __nv_bfloat16* dv;          // [B, Hkv, N, D]
     const float2* rope;         // (cos, sin) table or nullptr
-    int B, Hq, Hkv, N, Npad;
+    int B, Hq, Hkv, N, ntiles;
     int causal, window;
     float scale, scale_log2;
 };
 
-// D_i = dO_i . O_i and LSE_i * log2(e), one warp per row; rows past N get (+inf, 0) so that their
-// recomputed probabilities are exactly 0.
+// Per query row: -D_i = -(dO_i . O_i) and -LSE_i * log2(e), stored negated so that the kernels add
+// them. D/8 lanes share a row (16-byte loads), grid-stride over all padded rows; rows past N get
+// (-inf, 0) so that their recomputed probabilities are exactly 0.
 template <int D>
 __global__ void __launch_bounds__(256) bwd_prep_kernel(const BwdParams p) {
-    const long long warp = (blockIdx.x * (long long)blockDim.x + threadIdx.x) >> 5;
-    const int lane = threadIdx.x & 31;
-    const long long rows = static_cast<long long>(p.B) * p.Hq * p.Npad;
-    if (warp >= rows) return;
-    const long long bh = warp / p.Npad;
-    const int i = static_cast<int>(warp % p.Npad);
-    float2 out = make_float2(INFINITY, 0.f);
-    if (i < p.N) {
-        const size_t off = (static_cast<size_t>(bh) * p.N + i) * D;
+    constexpr int LPR = D / 8;     // lanes per row
+    constexpr int RPW = 32 / LPR;  // rows per warp and pass
+    const int lane = threadIdx.x & 31, sub = lane / LPR, l = lane % LPR;
+    const long long npad = static_cast<long long>(p.ntiles) * 128;
+    const long long rows = static_cast<long long>(p.B) * p.Hq * npad;
+    const long long nwarps = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
+    for (long long base = (static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5)) * RPW;
+         base < rows; base += nwarps * RPW) {
+        const long long row = base + sub;
+        const long long bh = row / npad;
+        const int i = static_cast<int>(row - bh * npad);
+        const bool valid = row < rows && i < p.N;
         float acc = 0.f;
-        constexpr int PER = D / 32;  // consecutive elements per lane
-        const __nv_bfloat16* po = p.o + off + lane * PER;
-        const __nv_bfloat16* pd = p.dout + off + lane * PER;
+        if (valid) {
+            const size_t off = (static_cast<size_t>(bh) * p.N + i) * D + l * 8;
+            const uint4 a = __ldg(reinterpret_cast<const uint4*>(p.o + off));
+            const uint4 b = __ldg(reinterpret_cast<const uint4*>(p.dout + off));
+            const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
-        for (int e = 0; e < PER; ++e) acc = fmaf(__bfloat162float(po[e]), __bfloat162float(pd[e]), acc);
+            for (int e = 0; e < 4; ++e) {
+                acc = fmaf(ptx::bf16lo_to_f32(aw[e]), ptx::bf16lo_to_f32(bw[e]), acc);
+                acc = fmaf(ptx::bf16hi_to_f32(aw[e]), ptx::bf16hi_to_f32(bw[e]), acc);
+            }
+        }
 #pragma unroll
-        for (int m = 16; m >= 1; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
-        out = make_float2(p.lse[static_cast<size_t>(bh) * p.N + i] * kLog2e, acc);
+        for (int m = LPR / 2; m >= 1; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
+        if (row < rows && l == 0) {
+            float* v = p.vec + (static_cast<size_t>(bh) * p.ntiles + i / 128) * 256 + (i & 127);
+            v[0] = valid ? -p.lse[static_cast<size_t>(bh) * p.N + i] * kLog2e : -INFINITY;
+            v[128] = valid ? -acc : 0.f;
+        }
     }
-    if (lane == 0) reinterpret_cast<float2*>(p.vec)[warp] = out;
 }
 
 template <int D>
@@ -68,17 +85,19 @@ struct BwdCfg {
     static constexpr int NREG = D / 64;
     static constexpr int REGION_BYTES = 128 * 128;
     static constexpr int TILE_BYTES = 128 * D * 2;
-    static constexpr int VEC_BYTES = 128 * 8;  // (lse2, D) per row of a query tile
+    static constexpr int VEC_BYTES = 256 * 4;  // -LSE*log2 e and -D of the 128 rows of a query tile
     // fixed pair (K,V or Q,dO) + two stages of the streamed pair, with their vectors
     static constexpr int SMEM_BYTES = 6 * TILE_BYTES + 2 * VEC_BYTES + 1024 /*barriers*/ + 1024 /*align*/;
-    static constexpr int THREADS = 192;
+    static constexpr int THREADS = 320;  // warps 0-7 elementwise, 8 TMA producer, 9 MMA issuer
+    static constexpr int PRODUCER_WARP = 8, MMA_WARP = 9;
+    static constexpr int EW_THREADS = 256;
     static constexpr uint32_t TMEM_COLS = 512;
 };
 
 struct BwdBarriers {
     uint64_t fixed_loaded;
     uint64_t full[2], empty[2];
-    uint64_t s_full, p_full, acc_done, drain;
+    uint64_t s_full[2], dp_full, p_full, ds_full, acc_done, drain;
     uint32_t tmem_base;
     int abort;
 };
@@ -116,10 +135,80 @@ __device__ __forceinline__ void query_tiles_for_keys(int j0, int N, int causal, 
     if (window > 0) ie = min(nq, (j0 + 127 + window - 1) / 128 + 1);
 }
 
+// TMEM column of the k-th 16-element slice of a packed bf16 operand: each warpgroup packs its 64
+// columns of a 128-column fp32 buffer into the first 32 columns of its own half.
+__device__ __forceinline__ constexpr uint32_t packed_col(int kk) { return (kk >> 2) * 64 + (kk & 3) * 8; }
+
+// P = 2^(s * scale_log2 + nlse) for 64 consecutive fp32 scores, the (-LSE*log2 e) values given per
+// element (dK/dV: per query column, from shared memory) or as one value (dQ: per row).
+__device__ __forceinline__ void probs64_cols(const uint32_t (&sv)[64], float scale_log2, const float* nlse,
+                                             float (&pr)[64]) {
+    const float2 sc = make_float2(scale_log2, scale_log2);
+#pragma unroll
+    for (int c = 0; c < 64; c += 4) {
+        const float4 l4 = *reinterpret_cast<const float4*>(nlse + c);
+        const float2 a = ptx::ffma2(make_float2(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])), sc,
+                                    make_float2(l4.x, l4.y));
+        const float2 b = ptx::ffma2(make_float2(__uint_as_float(sv[c + 2]), __uint_as_float(sv[c + 3])), sc,
+                                    make_float2(l4.z, l4.w));
+        pr[c] = ptx::ex2(a.x);
+        pr[c + 1] = ptx::ex2(a.y);
+        pr[c + 2] = ptx::ex2(b.x);
+        pr[c + 3] = ptx::ex2(b.y);
+    }
+}
+__device__ __forceinline__ void probs64_row(const uint32_t (&sv)[64], float scale_log2, float nlse,
+                                            float (&pr)[64]) {
+    const float2 sc = make_float2(scale_log2, scale_log2), nl = make_float2(nlse, nlse);
+#pragma unroll
+    for (int c = 0; c < 64; c += 2) {
+        const float2 a = ptx::ffma2(make_float2(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])), sc, nl);
+        pr[c] = ptx::ex2(a.x);
+        pr[c + 1] = ptx::ex2(a.y);
+    }
+}
+// Zero the probabilities of columns outside [lo, hi] (column indices relative to the 64-column block).
+__device__ __forceinline__ void mask64(float (&pr)[64], int lo, int hi) {
+#pragma unroll
+    for (int c = 0; c < 64; ++c) pr[c] = (c < lo || c > hi) ? 0.f : pr[c];
+}
+// dS = P (dP - D) for 32 columns, packed to 16 bf16 pairs. nd: -D per element (pointer) or per row.
+__device__ __forceinline__ void dscores32_cols(const float* pr, const uint32_t (&dp)[32], const float* nd,
+                                               uint32_t* out) {
+#pragma unroll
+    for (int c = 0; c < 32; c += 4) {
+        const float4 d4 = *reinterpret_cast<const float4*>(nd + c);
+        const float2 a = ptx::fmul2(make_float2(pr[c], pr[c + 1]),
+                                    ptx::fadd2(make_float2(__uint_as_float(dp[c]), __uint_as_float(dp[c + 1])),
+                                               make_float2(d4.x, d4.y)));
+        const float2 b = ptx::fmul2(make_float2(pr[c + 2], pr[c + 3]),
+                                    ptx::fadd2(make_float2(__uint_as_float(dp[c + 2]), __uint_as_float(dp[c + 3])),
+                                               make_float2(d4.z, d4.w)));
+        out[c / 2] = ptx::pack_bf16x2(a.x, a.y);
+        out[c / 2 + 1] = ptx::pack_bf16x2(b.x, b.y);
+    }
+}
+__device__ __forceinline__ void dscores32_row(const float* pr, const uint32_t (&dp)[32], float nd, uint32_t* out) {
+    const float2 n2 = make_float2(nd, nd);
+#pragma unroll
+    for (int c = 0; c < 32; c += 2) {
+        const float2 a = ptx::fmul2(make_float2(pr[c], pr[c + 1]),
+                                    ptx::fadd2(make_float2(__uint_as_float(dp[c]), __uint_as_float(dp[c + 1])), n2));
+        out[c / 2] = ptx::pack_bf16x2(a.x, a.y);
+    }
+}
+
 // =============================================================================== dK, dV
-// CTA (key tile jt, K/V head g, batch b). Steps t walk (query head of the group, query tile).
-// TMEM: S^T at 0 (P^T over its first 64 columns), dP^T at 128 (dS^T over its first 64),
-// dV at 256, dK at 256 + D.
+// CTA (key tile jt, K/V head g, batch b); block numbers run over key tiles slowest, so the causal
+// key tiles with the most visible queries start first. Steps t walk (query head of the group,
+// visible query tile). TMEM: S^T at 0 (P^T packed into columns 0-31 and 64-95), dP^T at 128 (dS^T
+// packed likewise), dV at 256, dK at 256 + D.
+//
+// Issue order per step t: dV(t) once P^T(t) is written, S^T(t+1), dK(t) once dS^T(t) is written,
+// dP^T(t+1). MMAs of one thread run in issue order, so S^T(t+1) may overwrite the scores that P^T(t)
+// was packed over once dV(t) is issued, and dP^T(t+1) the dS^T(t) buffer once dK(t) is issued; the
+// elementwise warps compute P^T(t+1) while the tensor core runs dK(t) and dP^T(t+1), and dS^T(t)
+// while it runs dV(t) and S^T(t+1).
 template <int D>
 __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -132,11 +221,14 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     uint8_t* sV = sK + C::TILE_BYTES;
     uint8_t* sQ = sV + C::TILE_BYTES;          // [2] stages
     uint8_t* sDO = sQ + 2 * C::TILE_BYTES;     // [2] stages
-    float2* sVec = reinterpret_cast<float2*>(sDO + 2 * C::TILE_BYTES);  // [2][128]
+    float* sVec = reinterpret_cast<float*>(sDO + 2 * C::TILE_BYTES);  // [2][256]
     auto* bar = reinterpret_cast<BwdBarriers*>(reinterpret_cast<uint8_t*>(sVec) + 2 * C::VEC_BYTES);
     volatile int* abort_flag = &bar->abort;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int jt = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+    const int groups = p.B * p.Hkv;
+    const int jt = static_cast<int>(blockIdx.x / groups);
+    const int gb = static_cast<int>(blockIdx.x - static_cast<unsigned>(jt) * groups);
+    const int g = gb % p.Hkv, b = gb / p.Hkv;
     const int j0 = jt * 128;
     const int G = p.Hq / p.Hkv;
     int ib, ie;
@@ -149,15 +241,17 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         for (int s = 0; s < 2; ++s) {
             ptx::mbar_init(&bar->full[s], 1);
             ptx::mbar_init(&bar->empty[s], 1);
+            ptx::mbar_init(&bar->s_full[s], 1);
         }
-        ptx::mbar_init(&bar->s_full, 1);
-        ptx::mbar_init(&bar->p_full, 128);
+        ptx::mbar_init(&bar->dp_full, 1);
+        ptx::mbar_init(&bar->p_full, C::EW_THREADS);
+        ptx::mbar_init(&bar->ds_full, C::EW_THREADS);
         ptx::mbar_init(&bar->acc_done, 1);
         ptx::mbar_init(&bar->drain, 1);
         bar->abort = 0;
         ptx::fence_mbar_init();
     }
-    if (warp == 5) {
+    if (warp == C::MMA_WARP) {
         ptx::tmem_alloc(&bar->tmem_base, C::TMEM_COLS);
         ptx::tmem_relinquish();
     }
@@ -167,7 +261,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     const uint32_t tmem = bar->tmem_base;
     constexpr uint32_t T_S = 0, T_DP = 128, T_DV = 256, T_DK = 256 + D;
 
-    if (warp == 4) {
+    if (warp == C::PRODUCER_WARP) {
         // ------------------------------------------------------------------ TMA producer
         if (lane == 0 && T > 0) {
             const int zk = b * p.Hkv + g;
@@ -181,14 +275,16 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
             for (int t = 0; t < T && ok; ++t) {
                 const int s = t & 1;
                 if (t >= 2 && !ptx::mbar_wait(&bar->empty[s], ((t >> 1) - 1) & 1, abort_flag)) { ok = false; break; }
-                const int h = g * G + t / per_head, i0 = (ib + t % per_head) * 128;
+                const int h = g * G + t / per_head, qt = ib + t % per_head;
                 const int zq = b * p.Hq + h;
                 ptx::mbar_arrive_expect_tx(&bar->full[s], 2 * C::TILE_BYTES + C::VEC_BYTES);
                 for (int r = 0; r < C::NREG; ++r) {
-                    ptx::tma_load_3d(sQ + s * C::TILE_BYTES + r * C::REGION_BYTES, &tm_q, &bar->full[s], r * 64, i0, zq);
-                    ptx::tma_load_3d(sDO + s * C::TILE_BYTES + r * C::REGION_BYTES, &tm_do, &bar->full[s], r * 64, i0, zq);
+                    ptx::tma_load_3d(sQ + s * C::TILE_BYTES + r * C::REGION_BYTES, &tm_q, &bar->full[s], r * 64,
+                                     qt * 128, zq);
+                    ptx::tma_load_3d(sDO + s * C::TILE_BYTES + r * C::REGION_BYTES, &tm_do, &bar->full[s], r * 64,
+                                     qt * 128, zq);
                 }
-                ptx::bulk_load(sVec + s * 128, p.vec + (static_cast<size_t>(zq) * p.Npad + i0) * 2, C::VEC_BYTES,
+                ptx::bulk_load(sVec + s * 256, p.vec + (static_cast<size_t>(zq) * p.ntiles + qt) * 256, C::VEC_BYTES,
                                &bar->full[s]);
                 issued = t + 1;
             }
@@ -200,7 +296,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
                 for (int t = max(0, issued - 2); t < issued; ++t) ptx::mbar_wait(&bar->full[t & 1], (t >> 1) & 1, &never);
             }
         }
-    } else if (warp == 5) {
+    } else if (warp == C::MMA_WARP) {
         // ------------------------------------------------------------------ MMA issuer
         if (lane == 0 && T > 0) {
             constexpr uint32_t ID_S = ptx::idesc_bf16_f32(128, 128, 0, 0);  // K (keys) x Q^T, both K-major
@@ -213,37 +309,60 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
             const uint32_t do_lo = ptx::sw128_desc_lo(ptx::smem_u32(sDO), 16);
             const uint32_t qmn_lo = ptx::sw128_desc_lo(ptx::smem_u32(sQ), C::REGION_BYTES);
             const uint32_t domn_lo = ptx::sw128_desc_lo(ptx::smem_u32(sDO), C::REGION_BYTES);
-            bool ok = ptx::mbar_wait(&bar->fixed_loaded, 0, abort_flag);
+            // S^T = K Q^T (M = 128 keys, N = 128 queries, K = D)
+            auto issue_s = [&](int t) {
+                const uint32_t st = (t & 1) * TILE16;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = ((kk >> 2) * C::REGION_BYTES + (kk & 3) * 32) >> 4;
+                    ptx::mma_ss(tmem + T_S, ptx::desc64(k_lo + off, HI), ptx::desc64(q_lo + st + off, HI), ID_S, kk > 0);
+                }
+            };
+            // dP^T = V dO^T
+            auto issue_dp = [&](int t) {
+                const uint32_t st = (t & 1) * TILE16;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = ((kk >> 2) * C::REGION_BYTES + (kk & 3) * 32) >> 4;
+                    ptx::mma_ss(tmem + T_DP, ptx::desc64(v_lo + off, HI), ptx::desc64(do_lo + st + off, HI), ID_S, kk > 0);
+                }
+            };
+            // dV += P^T dO, dK += dS^T Q (M = 128 keys, N = D, K = 128 queries)
+            auto issue_grad = [&](int t, uint32_t acc_col, uint32_t a_col, uint32_t b_lo) {
+                const uint32_t st = (t & 1) * TILE16;
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    ptx::mma_ts(tmem + acc_col, tmem + a_col + packed_col(kk), ptx::desc64(b_lo + st + ((kk * 2048) >> 4), HI),
+                                ID_G, (t > 0 || kk > 0) ? 1u : 0u);
+            };
+            bool ok = ptx::mbar_wait(&bar->fixed_loaded, 0, abort_flag) && ptx::mbar_wait(&bar->full[0], 0, abort_flag);
             bool issued_any = false;
-            for (int t = 0; ok && t < T; ++t) {
-                const int s = t & 1;
-                if (!ptx::mbar_wait(&bar->full[s], (t >> 1) & 1, abort_flag)) { ok = false; break; }
-                // S^T = K Q^T and dP^T = V dO^T (M = 128 keys, N = 128 queries, K = D)
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = ((kk >> 2) * C::REGION_BYTES + (kk & 3) * 32) >> 4;
-                    ptx::mma_ss(tmem + T_S, ptx::desc64(k_lo + off, HI), ptx::desc64(q_lo + s * TILE16 + off, HI), ID_S, kk > 0);
-                }
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = ((kk >> 2) * C::REGION_BYTES + (kk & 3) * 32) >> 4;
-                    ptx::mma_ss(tmem + T_DP, ptx::desc64(v_lo + off, HI), ptx::desc64(do_lo + s * TILE16 + off, HI), ID_S, kk > 0);
-                }
-                ptx::mma_commit(&bar->s_full);
+            if (ok) {
+                issue_s(0);
+                ptx::mma_commit(&bar->s_full[0]);
+                issue_dp(0);
+                ptx::mma_commit(&bar->dp_full);
                 issued_any = true;
+            }
+            for (int t = 0; ok && t < T; ++t) {
                 if (!ptx::mbar_wait(&bar->p_full, t & 1, abort_flag)) { ok = false; break; }
                 ptx::tc_fence_after();
-                // dV += P^T dO and dK += dS^T Q (M = 128 keys, N = D, K = 128 queries)
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t off = (kk * 2048) >> 4;
-                    ptx::mma_ts(tmem + T_DV, tmem + T_S + kk * 8, ptx::desc64(domn_lo + s * TILE16 + off, HI), ID_G,
-                                (t > 0 || kk > 0) ? 1u : 0u);
-                    ptx::mma_ts(tmem + T_DK, tmem + T_DP + kk * 8, ptx::desc64(qmn_lo + s * TILE16 + off, HI), ID_G,
-                                (t > 0 || kk > 0) ? 1u : 0u);
+                issue_grad(t, T_DV, T_S, domn_lo);
+                if (t + 1 < T) {
+                    if (!ptx::mbar_wait(&bar->full[(t + 1) & 1], ((t + 1) >> 1) & 1, abort_flag)) { ok = false; break; }
+                    issue_s(t + 1);
+                    ptx::mma_commit(&bar->s_full[0]);
                 }
-                ptx::mma_commit(&bar->empty[s]);
-                if (t == T - 1) ptx::mma_commit(&bar->acc_done);
+                if (!ptx::mbar_wait(&bar->ds_full, t & 1, abort_flag)) { ok = false; break; }
+                ptx::tc_fence_after();
+                issue_grad(t, T_DK, T_DP, qmn_lo);
+                ptx::mma_commit(&bar->empty[t & 1]);
+                if (t + 1 < T) {
+                    issue_dp(t + 1);
+                    ptx::mma_commit(&bar->dp_full);
+                } else {
+                    ptx::mma_commit(&bar->acc_done);
+                }
             }
             if (!ok) {
                 *abort_flag = 1;
@@ -258,74 +377,72 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         __syncwarp();
     } else {
         // ------------------------------------------------------------------ elementwise warps
-        const int r = threadIdx.x;           // key row == TMEM lane
+        const int wg = warp >> 2;                  // query columns [64 wg, 64 wg + 64) of each tile
+        const int r = (warp & 3) * 32 + lane;      // key row == TMEM lane
         const int key = j0 + r;
-        const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+        const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+        const uint32_t t_s = tmem + lane_base + T_S + 64 * wg, t_dp = tmem + lane_base + T_DP + 64 * wg;
         bool ok = true;
         for (int t = 0; ok && t < T; ++t) {
             const int s = t & 1;
-            const int i0 = (ib + t % per_head) * 128;
+            const int c0 = (ib + t % per_head) * 128 + 64 * wg;  // first query of this warpgroup's columns
             if (!ptx::mbar_wait(&bar->full[s], (t >> 1) & 1, abort_flag)) { ok = false; break; }
-            if (!ptx::mbar_wait(&bar->s_full, t & 1, abort_flag)) { ok = false; break; }
+            if (!ptx::mbar_wait(&bar->s_full[0], t & 1, abort_flag)) { ok = false; break; }
             ptx::tc_fence_after();
-            const float2* vec = sVec + s * 128;
-            const bool need_mask = (p.causal && i0 < j0 + 127) || (p.window > 0 && i0 + 127 - j0 > p.window - 1);
+            const float* vec = sVec + s * 256 + 64 * wg;
+            float pr[64];
+            {
+                uint32_t sv[64];
+                ptx::tmem_ld64(t_s, sv);
+                probs64_cols(sv, p.scale_log2, vec, pr);
+            }
+            // query qpos sees this key iff qpos >= key (causal) and qpos - key < window
+            const int lo = p.causal ? key - c0 : -1;
+            const int hi = p.window > 0 ? key + p.window - 1 - c0 : 64;
+            if (lo > 0 || hi < 63) mask64(pr, lo, hi);
+            {
+                uint32_t pk[32];
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                uint32_t sv[32], dv[32], sv2[32], dv2[32];
-                ptx::tmem_ld32(tmem + lane_base + T_S + half * 64, sv);
-                ptx::tmem_ld32(tmem + lane_base + T_S + half * 64 + 32, sv2);
-                ptx::tmem_ld32(tmem + lane_base + T_DP + half * 64, dv);
-                ptx::tmem_ld32(tmem + lane_base + T_DP + half * 64 + 32, dv2);
-                uint32_t pk[32], dk[32];
-#pragma unroll
-                for (int c = 0; c < 64; c += 2) {
-                    float pr[2], ds[2];
-#pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        const int col = half * 64 + c + e;  // query column within the tile
-                        const float sraw = __uint_as_float(c + e < 32 ? sv[c + e] : sv2[c + e - 32]);
-                        const float dp = __uint_as_float(c + e < 32 ? dv[c + e] : dv2[c + e - 32]);
-                        const float2 ld = vec[col];  // (LSE * log2 e, D) of the query; +inf past N
-                        float pe = ptx::ex2(fmaf(sraw, p.scale_log2, -ld.x));
-                        if (need_mask) {
-                            const int qpos = i0 + col;
-                            const bool vis = (!p.causal || qpos >= key) && (p.window <= 0 || qpos - key < p.window);
-                            pe = vis ? pe : 0.f;
-                        }
-                        pr[e] = pe;
-                        ds[e] = pe * (dp - ld.y);
-                    }
-                    pk[c / 2] = ptx::pack_bf16x2(pr[0], pr[1]);
-                    dk[c / 2] = ptx::pack_bf16x2(ds[0], ds[1]);
-                }
-                // P^T and dS^T (bf16 pairs) over the first 64 columns of their buffers; this half's
-                // source columns were read above, the second half's lie beyond what is written now.
-                ptx::tmem_st32(tmem + lane_base + T_S + half * 32, pk);
-                ptx::tmem_st32(tmem + lane_base + T_DP + half * 32, dk);
+                for (int c = 0; c < 32; ++c) pk[c] = ptx::pack_bf16x2(pr[2 * c], pr[2 * c + 1]);
+                ptx::tmem_st32(t_s, pk);
             }
             ptx::tc_fence_before();
             ptx::mbar_arrive(&bar->p_full);
+            if (!ptx::mbar_wait(&bar->dp_full, t & 1, abort_flag)) { ok = false; break; }
+            ptx::tc_fence_after();
+            uint32_t dsk[32];
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                uint32_t dp[32];
+                ptx::tmem_ld32(t_dp + 32 * half, dp);
+                dscores32_cols(pr + 32 * half, dp, vec + 128 + 32 * half, dsk + 16 * half);
+            }
+            ptx::tmem_st32(t_dp, dsk);
+            ptx::tc_fence_before();
+            ptx::mbar_arrive(&bar->ds_full);
         }
         if (ok && T > 0) ok = ptx::mbar_wait(&bar->acc_done, 0, abort_flag);
         if (ok && T > 0) {
-            // every lane takes part in the warp-collective TMEM loads; rows past N store nothing
+            // warpgroup 0 writes dV, warpgroup 1 dK; every lane takes part in the warp-collective
+            // TMEM loads, rows past N store nothing
             ptx::tc_fence_after();
             const size_t row = (static_cast<size_t>(b) * p.Hkv + g) * p.N + min(key, p.N - 1);
 #pragma unroll 1
             for (int c = 0; c < D / 32; ++c) {
                 uint32_t v[32];
-                ptx::tmem_ld32(tmem + lane_base + T_DV + c * 32, v);
-                if (key < p.N) store_chunk_unrotated(v, 1.f, nullptr, D, key, c * 32, p.dv + row * D);
-                ptx::tmem_ld32(tmem + lane_base + T_DK + c * 32, v);
-                if (key < p.N) store_chunk_unrotated(v, p.scale, p.rope, D, key, c * 32, p.dk + row * D);
+                ptx::tmem_ld32(tmem + lane_base + (wg == 0 ? T_DV : T_DK) + c * 32, v);
+                if (key < p.N) {
+                    if (wg == 0)
+                        store_chunk_unrotated(v, 1.f, nullptr, D, key, c * 32, p.dv + row * D);
+                    else
+                        store_chunk_unrotated(v, p.scale, p.rope, D, key, c * 32, p.dk + row * D);
+                }
             }
         } else if (T == 0 && key < p.N) {
             // no query sees these keys: zero gradients
             const size_t row = (static_cast<size_t>(b) * p.Hkv + g) * p.N + key;
-            uint4* d1 = reinterpret_cast<uint4*>(p.dv + row * D);
-            uint4* d2 = reinterpret_cast<uint4*>(p.dk + row * D);
-            for (int k = 0; k < D / 8; ++k) d1[k] = d2[k] = make_uint4(0, 0, 0, 0);
+            uint4* d1 = reinterpret_cast<uint4*>((wg == 0 ? p.dv : p.dk) + row * D);
+            for (int k = 0; k < D / 8; ++k) d1[k] = make_uint4(0, 0, 0, 0);
         }
         if (!ok) {
             *abort_flag = 1;
@@ -334,15 +451,20 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     }
     ptx::tc_fence_before();
     __syncthreads();
-    if (warp == 5) {
+    if (warp == C::MMA_WARP) {
         ptx::tc_fence_after();
         ptx::tmem_dealloc(tmem, C::TMEM_COLS);
     }
 }
 
 // =============================================================================== dQ
-// CTA (query tile it, query head h, batch b). Steps walk the visible key tiles.
-// TMEM: S at 0 (dS over its first 64 columns), dP at 128, dQ at 256.
+// CTA (query tile it, query head h, batch b); block numbers run over query tiles slowest, the last
+// (causal: longest) tiles first. Steps walk the visible key tiles. TMEM: S in two buffers at 0 and
+// 128, dP at 256 (dS packed into columns 256-287 and 320-351), dQ at 384.
+//
+// Issue order per step t: S(t+1) into the other buffer, dQ(t) once dS(t) is written, dP(t+1). P
+// stays in registers, so the elementwise warps compute P(t+1) while the tensor core runs dQ(t) and
+// dP(t+1).
 template <int D>
 __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -358,8 +480,11 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     auto* bar = reinterpret_cast<BwdBarriers*>(sV + 2 * C::TILE_BYTES + 2 * C::VEC_BYTES);
     volatile int* abort_flag = &bar->abort;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int h = blockIdx.y, b = blockIdx.z;
-    const int qt = gridDim.x - 1 - blockIdx.x;  // longest (causal) tiles first
+    const int groups = p.B * p.Hq;
+    const int rank = static_cast<int>(blockIdx.x / groups);
+    const int hb = static_cast<int>(blockIdx.x - static_cast<unsigned>(rank) * groups);
+    const int h = hb % p.Hq, b = hb / p.Hq;
+    const int qt = p.ntiles - 1 - rank;
     const int q0 = qt * 128;
     const int g = h / (p.Hq / p.Hkv);
     const TileRange R = tile_range(q0, p.N, p.causal, p.window);
@@ -370,15 +495,17 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         for (int s = 0; s < 2; ++s) {
             ptx::mbar_init(&bar->full[s], 1);
             ptx::mbar_init(&bar->empty[s], 1);
+            ptx::mbar_init(&bar->s_full[s], 1);
         }
-        ptx::mbar_init(&bar->s_full, 1);
-        ptx::mbar_init(&bar->p_full, 128);
+        ptx::mbar_init(&bar->dp_full, 1);
+        ptx::mbar_init(&bar->p_full, 1);
+        ptx::mbar_init(&bar->ds_full, C::EW_THREADS);
         ptx::mbar_init(&bar->acc_done, 1);
         ptx::mbar_init(&bar->drain, 1);
         bar->abort = 0;
         ptx::fence_mbar_init();
     }
-    if (warp == 5) {
+    if (warp == C::MMA_WARP) {
         ptx::tmem_alloc(&bar->tmem_base, C::TMEM_COLS);
         ptx::tmem_relinquish();
     }
@@ -386,10 +513,10 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem = bar->tmem_base;
-    constexpr uint32_t T_S = 0, T_DP = 128, T_DQ = 256;
+    constexpr uint32_t T_S = 0, T_DP = 256, T_DQ = 384;
 
-    if (warp == 4) {
-        if (lane == 0) {
+    if (warp == C::PRODUCER_WARP) {
+        if (lane == 0 && T > 0) {
             const int zq = b * p.Hq + h, zk = b * p.Hkv + g;
             ptx::mbar_arrive_expect_tx(&bar->fixed_loaded, 2 * C::TILE_BYTES);
             for (int r = 0; r < C::NREG; ++r) {
@@ -417,8 +544,8 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
                 for (int t = max(0, issued - 2); t < issued; ++t) ptx::mbar_wait(&bar->full[t & 1], (t >> 1) & 1, &never);
             }
         }
-    } else if (warp == 5) {
-        if (lane == 0) {
+    } else if (warp == C::MMA_WARP) {
+        if (lane == 0 && T > 0) {
             constexpr uint32_t ID_S = ptx::idesc_bf16_f32(128, 128, 0, 0);  // Q K^T, dO V^T: K-major
             constexpr uint32_t ID_G = ptx::idesc_bf16_f32(128, D, 0, 1);    // dS (TMEM) x K (MN-major)
             constexpr uint32_t HI = ptx::sw128_desc_hi(1024);
@@ -428,32 +555,55 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
             const uint32_t k_lo = ptx::sw128_desc_lo(ptx::smem_u32(sK), 16);
             const uint32_t v_lo = ptx::sw128_desc_lo(ptx::smem_u32(sV), 16);
             const uint32_t kmn_lo = ptx::sw128_desc_lo(ptx::smem_u32(sK), C::REGION_BYTES);
-            bool ok = ptx::mbar_wait(&bar->fixed_loaded, 0, abort_flag);
+            // S = Q K^T into buffer t & 1 (M = 128 queries, N = 128 keys, K = D)
+            auto issue_s = [&](int t) {
+                const uint32_t st = (t & 1) * TILE16;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = ((kk >> 2) * C::REGION_BYTES + (kk & 3) * 32) >> 4;
+                    ptx::mma_ss(tmem + T_S + 128 * (t & 1), ptx::desc64(q_lo + off, HI), ptx::desc64(k_lo + st + off, HI),
+                                ID_S, kk > 0);
+                }
+            };
+            // dP = dO V^T
+            auto issue_dp = [&](int t) {
+                const uint32_t st = (t & 1) * TILE16;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = ((kk >> 2) * C::REGION_BYTES + (kk & 3) * 32) >> 4;
+                    ptx::mma_ss(tmem + T_DP, ptx::desc64(do_lo + off, HI), ptx::desc64(v_lo + st + off, HI), ID_S, kk > 0);
+                }
+            };
+            bool ok = ptx::mbar_wait(&bar->fixed_loaded, 0, abort_flag) && ptx::mbar_wait(&bar->full[0], 0, abort_flag);
             bool issued_any = false;
-            for (int t = 0; ok && t < T; ++t) {
-                const int s = t & 1;
-                if (!ptx::mbar_wait(&bar->full[s], (t >> 1) & 1, abort_flag)) { ok = false; break; }
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = ((kk >> 2) * C::REGION_BYTES + (kk & 3) * 32) >> 4;
-                    ptx::mma_ss(tmem + T_S, ptx::desc64(q_lo + off, HI), ptx::desc64(k_lo + s * TILE16 + off, HI), ID_S, kk > 0);
-                }
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = ((kk >> 2) * C::REGION_BYTES + (kk & 3) * 32) >> 4;
-                    ptx::mma_ss(tmem + T_DP, ptx::desc64(do_lo + off, HI), ptx::desc64(v_lo + s * TILE16 + off, HI), ID_S, kk > 0);
-                }
-                ptx::mma_commit(&bar->s_full);
+            if (ok) {
+                issue_s(0);
+                ptx::mma_commit(&bar->s_full[0]);
+                issue_dp(0);
+                ptx::mma_commit(&bar->dp_full);
                 issued_any = true;
-                if (!ptx::mbar_wait(&bar->p_full, t & 1, abort_flag)) { ok = false; break; }
+            }
+            for (int t = 0; ok && t < T; ++t) {
+                if (t + 1 < T) {
+                    if (!ptx::mbar_wait(&bar->full[(t + 1) & 1], ((t + 1) >> 1) & 1, abort_flag)) { ok = false; break; }
+                    issue_s(t + 1);
+                    ptx::mma_commit(&bar->s_full[(t + 1) & 1]);
+                }
+                if (!ptx::mbar_wait(&bar->ds_full, t & 1, abort_flag)) { ok = false; break; }
                 ptx::tc_fence_after();
                 // dQ += dS K (M = 128 queries, N = D, K = 128 keys)
+                const uint32_t st = (t & 1) * TILE16;
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    ptx::mma_ts(tmem + T_DQ, tmem + T_S + kk * 8, ptx::desc64(kmn_lo + s * TILE16 + ((kk * 2048) >> 4), HI),
-                                ID_G, (t > 0 || kk > 0) ? 1u : 0u);
-                ptx::mma_commit(&bar->empty[s]);
-                if (t == T - 1) ptx::mma_commit(&bar->acc_done);
+                    ptx::mma_ts(tmem + T_DQ, tmem + T_DP + packed_col(kk),
+                                ptx::desc64(kmn_lo + st + ((kk * 2048) >> 4), HI), ID_G, (t > 0 || kk > 0) ? 1u : 0u);
+                ptx::mma_commit(&bar->empty[t & 1]);
+                if (t + 1 < T) {
+                    issue_dp(t + 1);
+                    ptx::mma_commit(&bar->dp_full);
+                } else {
+                    ptx::mma_commit(&bar->acc_done);
+                }
             }
             if (!ok) {
                 *abort_flag = 1;
@@ -467,56 +617,49 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         }
         __syncwarp();
     } else {
-        const int r = threadIdx.x;  // query row == TMEM lane
+        const int wg = warp >> 2;              // key columns [64 wg, 64 wg + 64) of each tile
+        const int r = (warp & 3) * 32 + lane;  // query row == TMEM lane
         const int qpos = q0 + r;
-        const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-        float2 ld = make_float2(INFINITY, 0.f);
-        if (qpos < p.N) ld = reinterpret_cast<const float2*>(p.vec)[(static_cast<size_t>(b) * p.Hq + h) * p.Npad + qpos];
+        const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+        const uint32_t t_dp = tmem + lane_base + T_DP + 64 * wg;
+        const float* vrow = p.vec + (static_cast<size_t>(b * p.Hq + h) * p.ntiles + qt) * 256 + r;
+        const float nlse = vrow[0], nd = vrow[128];
         bool ok = true;
         for (int t = 0; ok && t < T; ++t) {
-            const int k0 = (R.jb + t) * 128;
-            if (!ptx::mbar_wait(&bar->s_full, t & 1, abort_flag)) { ok = false; break; }
+            const int c0 = (R.jb + t) * 128 + 64 * wg;  // first key of this warpgroup's columns
+            if (!ptx::mbar_wait(&bar->s_full[t & 1], (t >> 1) & 1, abort_flag)) { ok = false; break; }
             ptx::tc_fence_after();
-            const bool need_mask = (k0 + 128 > p.N) || (p.causal && k0 + 127 > q0) ||
-                                   (p.window > 0 && k0 < q0 + 128 - p.window);
-            const int lo = p.window > 0 ? qpos - p.window + 1 : -0x7fffffff;
-            const int hi = p.causal ? min(qpos, p.N - 1) : p.N - 1;
+            float pr[64];
+            {
+                uint32_t sv[64];
+                ptx::tmem_ld64(tmem + lane_base + T_S + 128 * (t & 1) + 64 * wg, sv);
+                probs64_row(sv, p.scale_log2, nlse, pr);
+            }
+            // key kpos is visible iff kpos <= qpos (causal) and qpos - kpos < window; keys past N
+            // have zero K and V rows (zero-filled loads), so their dS meets a zero K row
+            const int hi = p.causal ? qpos - c0 : 64;
+            const int lo = p.window > 0 ? qpos - p.window + 1 - c0 : -1;
+            if (lo > 0 || hi < 63) mask64(pr, lo, hi);
+            if (!ptx::mbar_wait(&bar->dp_full, t & 1, abort_flag)) { ok = false; break; }
+            ptx::tc_fence_after();
+            uint32_t dsk[32];
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
-                uint32_t sv[32], dv[32], sv2[32], dv2[32];
-                ptx::tmem_ld32(tmem + lane_base + T_S + half * 64, sv);
-                ptx::tmem_ld32(tmem + lane_base + T_S + half * 64 + 32, sv2);
-                ptx::tmem_ld32(tmem + lane_base + T_DP + half * 64, dv);
-                ptx::tmem_ld32(tmem + lane_base + T_DP + half * 64 + 32, dv2);
-                uint32_t dsk[32];
-#pragma unroll
-                for (int c = 0; c < 64; c += 2) {
-                    float ds[2];
-#pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        const int col = half * 64 + c + e;
-                        const float sraw = __uint_as_float(c + e < 32 ? sv[c + e] : sv2[c + e - 32]);
-                        const float dp = __uint_as_float(c + e < 32 ? dv[c + e] : dv2[c + e - 32]);
-                        float pe = ptx::ex2(fmaf(sraw, p.scale_log2, -ld.x));
-                        if (need_mask) {
-                            const int kj = k0 + col;
-                            pe = (kj < lo || kj > hi) ? 0.f : pe;
-                        }
-                        ds[e] = pe * (dp - ld.y);
-                    }
-                    dsk[c / 2] = ptx::pack_bf16x2(ds[0], ds[1]);
-                }
-                ptx::tmem_st32(tmem + lane_base + T_S + half * 32, dsk);
+                uint32_t dp[32];
+                ptx::tmem_ld32(t_dp + 32 * half, dp);
+                dscores32_row(pr + 32 * half, dp, nd, dsk + 16 * half);
             }
+            ptx::tmem_st32(t_dp, dsk);
             ptx::tc_fence_before();
-            ptx::mbar_arrive(&bar->p_full);
+            ptx::mbar_arrive(&bar->ds_full);
         }
         if (ok && T > 0) ok = ptx::mbar_wait(&bar->acc_done, 0, abort_flag);
         if (ok && T > 0) {
+            // each warpgroup writes half of the D columns
             ptx::tc_fence_after();
             __nv_bfloat16* dst = p.dq + ((static_cast<size_t>(b) * p.Hq + h) * p.N + min(qpos, p.N - 1)) * D;
 #pragma unroll 1
-            for (int c = 0; c < D / 32; ++c) {
+            for (int c = wg * (D / 64); c < (wg + 1) * (D / 64); ++c) {
                 uint32_t v[32];
                 ptx::tmem_ld32(tmem + lane_base + T_DQ + c * 32, v);
                 if (qpos < p.N) store_chunk_unrotated(v, p.scale, p.rope, D, qpos, c * 32, dst);
@@ -529,7 +672,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     }
     ptx::tc_fence_before();
     __syncthreads();
-    if (warp == 5) {
+    if (warp == C::MMA_WARP) {
         ptx::tc_fence_after();
         ptx::tmem_dealloc(tmem, C::TMEM_COLS);
     }

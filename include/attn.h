@@ -80,8 +80,8 @@ attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float
                      int N, int D, int causal, int window, float rope_base, float scale, void* stream);
 
 /*
- * attn_bwd_workspace_size -- bytes of device workspace attn_bwd needs: fp32 (LSE*log2 e, D_i) per
- * query row padded to 128-row tiles, plus, with RoPE, the rotated Q and K (bf16). 0 for invalid sizes.
+ * attn_bwd_workspace_size -- bytes of device workspace attn_bwd needs: fp32 (-LSE*log2 e, -D_i)
+ * per query row padded to 128-row tiles, plus, with RoPE, the rotated Q and K (bf16). 0 for invalid sizes.
  */
 size_t attn_bwd_workspace_size(int B, int Hq, int Hkv, int N, int D, float rope_base);
 
@@ -103,7 +103,7 @@ size_t attn_bwd_workspace_size(int B, int Hq, int Hkv, int N, int D, float rope_
  *   dq     bf16 [B, Hq, N, D]; dk, dv bf16 [B, Hkv, N, D]: written
  *   workspace  device scratch of at least attn_bwd_workspace_size(...) bytes, 16-byte aligned,
  *          owned by the caller, any initial contents; overlapping calls need their own.
- * Constraints and errors as attn_fwd (D in {64, 128}; B, Hq <= 65535).
+ * Constraints and errors as attn_fwd (D in {64, 128}), with B * Hq * ceil(N/128) < 2^31.
  */
 attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
                      void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int N, int D, int causal, int window,
