@@ -216,3 +216,45 @@ def contiguous_copy(cache: PagedCache) -> PagedCache:
         cursor += n
     return PagedCache(cache.q, k, v, bt, cache.seq_lens, cache.page_size, cache.Hq, cache.Hkv,
                       cache.D)
+
+
+@dataclass
+class DecodeStepInputs:
+    """A paged cache whose seq_lens already count T new tokens per sequence, with the slots of those
+    tokens poisoned (NaN) until an append fills them, plus the new tokens' q, k, v (not rotated)."""
+    cache: PagedCache
+    q: torch.Tensor      # [S, T, Hq, D] bf16
+    k_new: torch.Tensor  # [S, T, Hkv, D] bf16
+    v_new: torch.Tensor  # [S, T, Hkv, D] bf16
+
+    @property
+    def T(self) -> int:
+        return self.q.shape[1]
+
+
+def decode_step_inputs(num_seqs, T, Hq, Hkv, D, page_size, seq_lens=None, len_lo=None, len_hi=None,
+                       spare_frac=0.10, seed=0, permute: bool = True, poison: bool = True):
+    """Inputs for a decode step that appends T tokens per sequence and attends with their queries.
+    The cache is ``paged_decode_inputs`` with the same arguments; the new tokens are drawn from a
+    second seeded stream, so the cache is the same whatever T is."""
+    cache = paged_decode_inputs(num_seqs, Hq, Hkv, D, page_size, seq_lens=seq_lens, len_lo=len_lo, len_hi=len_hi,
+                                spare_frac=spare_frac, seed=seed, permute=permute, poison=poison)
+    assert int(cache.seq_lens.min()) >= T
+    g = _gen(seed + 7919)
+    q = randn_bf16((num_seqs, T, Hq, D), g)
+    k_new = randn_bf16((num_seqs, T, Hkv, D), g)
+    v_new = randn_bf16((num_seqs, T, Hkv, D), g)
+    if poison:
+        fill = torch.tensor(BF16_NAN_BITS, dtype=torch.int16).view(torch.bfloat16)
+        for s in range(num_seqs):
+            for pos in range(int(cache.seq_lens[s]) - T, int(cache.seq_lens[s])):
+                page = int(cache.block_table[s, pos // page_size])
+                cache.k_pages[page, :, pos % page_size, :] = fill
+                cache.v_pages[page, :, pos % page_size, :] = fill
+    return DecodeStepInputs(cache, q, k_new, v_new)
+
+
+def decode_step_inputs_for(cfg: DecodeConfig, T: int, permute: bool = True, poison: bool = True):
+    return decode_step_inputs(cfg.num_seqs, T, cfg.Hq, cfg.Hkv, cfg.D, cfg.page_size, len_lo=cfg.len_lo,
+                              len_hi=cfg.len_hi, spare_frac=cfg.spare_frac, seed=cfg.seed, permute=permute,
+                              poison=poison)

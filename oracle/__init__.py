@@ -39,6 +39,9 @@ def _declare(lib):
     lib.oracle_decode_paged.argtypes = [p, p, p, p, p, i32, i32, i32, i32, i32, i32, i32, f64, p, p,
                                         i32]
     lib.oracle_decode_paged.restype = i32
+    lib.oracle_decode_step.argtypes = [p, p, p, p, p, p, p, i32, i32, i32, i32, i32, i32, i32, i32, f64, f64, p,
+                                       p, i32]
+    lib.oracle_decode_step.restype = i32
     lib.oracle_rope_bf16.argtypes = [p, p, i64, i32, f64, p]
     lib.oracle_rope_bf16.restype = i32
     lib.oracle_round_bf16_array.argtypes = [p, i64, p]
@@ -187,6 +190,43 @@ def decode_paged(q, k_pages, v_pages, block_table, seq_lens, scale=None, nthread
     if st != 0:
         raise OracleError("oracle_decode_paged failed with status %d" % st)
     return o, lse
+
+
+def decode_step(q, k_new, v_new, k_pages, v_pages, block_table, seq_lens, rope_base=0.0, scale=None, nthreads=0,
+                lib=None):
+    """Decode step in fp64: append the new tokens' keys (rotated) and values to the paged cache, then
+    attend each new token's rotated query causally to the cache.
+
+    q: uint16 [S, T, Hq, D]; k_new, v_new: uint16 [S, T, Hkv, D] or both None; k_pages, v_pages:
+    uint16 [num_pages, Hkv, page_size, D] (not modified: the updated copies are returned);
+    block_table: int32 [S, max_blocks]; seq_lens: int32 [S], counting the T new tokens.
+    Returns (o [S, T, Hq, D], lse [S, T, Hq], k_pages', v_pages').
+    """
+    lib = lib or _lib()
+    q = _bits(q)
+    kp, vp = _bits(k_pages).copy(), _bits(v_pages).copy()
+    if (k_new is None) != (v_new is None):
+        raise ValueError("k_new and v_new go together")
+    kn = _bits(k_new) if k_new is not None else None
+    vn = _bits(v_new) if v_new is not None else None
+    bt = np.ascontiguousarray(block_table, dtype=np.int32)
+    sl = np.ascontiguousarray(seq_lens, dtype=np.int32)
+    S, T, Hq, D = q.shape
+    num_pages, Hkv, page_size, D2 = kp.shape
+    if D2 != D or vp.shape != kp.shape or bt.shape[0] != S or sl.shape != (S,):
+        raise ValueError("decode shape mismatch")
+    if kn is not None and (kn.shape != (S, T, Hkv, D) or vn.shape != kn.shape):
+        raise ValueError("k_new/v_new shape mismatch")
+    if scale is None:
+        scale = 1.0 / np.sqrt(D)
+    o = np.empty((S, T, Hq, D), dtype=np.float64)
+    lse = np.empty((S, T, Hq), dtype=np.float64)
+    st = lib.oracle_decode_step(_ptr(q), _ptr(kn), _ptr(vn), _ptr(kp), _ptr(vp), _ptr(bt), _ptr(sl), S, T,
+                                bt.shape[1], num_pages, page_size, Hq, Hkv, D, float(rope_base), float(scale),
+                                _ptr(o), _ptr(lse), int(nthreads))
+    if st != 0:
+        raise OracleError("oracle_decode_step failed with status %d" % st)
+    return o, lse, kp, vp
 
 
 def rope_bf16(x, pos, base, lib=None):

@@ -26,6 +26,10 @@
  *     order ("Self-Attention Complexity, FlashAttention, PagedAttention, and RoPE in Code",
  *     Part 3: fixed-size blocks and block tables) and computes the single query row at the
  *     sequence's last position over all seq_len cached tokens.
+ *   - A decode step appends the new tokens first: their keys, rotated at their positions, and
+ *     their values go into the slots the block table gives (same Part 3; the rotation of the
+ *     RoPE question above), then each new token's query, rotated at its position, attends
+ *     causally to the cache -- the last rows of causal attention over the whole sequence.
  *
  * The score row of every query is materialised in full (masked entries hold -inf), then
  * max, exp, sum, the weighted sum of V and the logsumexp are taken -- the plain definition,
@@ -286,6 +290,97 @@ int oracle_decode_paged(const uint16_t* q, const uint16_t* k_pages, const uint16
                 /* the query is the sequence's last token: position len-1, causal over the cache */
                 attend_row(qq, kk, vv, len, D, (long)len - 1, 1, 0, scale, s_row,
                            o + ((size_t)s * Hq + h) * D, lse + (size_t)s * Hq + h);
+            }
+        }
+        free(kk);
+        free(vv);
+        free(s_row);
+        free(qq);
+    }
+    return status;
+}
+
+/*
+ * Decode step over a paged cache: append, then attend. q: bf16 [S, T, Hq, D] as given (rotated
+ * here when rope_base > 0); k_new, v_new: bf16 [S, T, Hkv, D] or both NULL (the cache already
+ * holds the new tokens). seq_lens count the T new tokens, which sit at positions len-T .. len-1.
+ * k_pages, v_pages [num_pages, Hkv, page_size, D] are updated in place: the key of new token t
+ * rotated at its position and rounded to bf16, the value as given. Sequences are appended in
+ * order; slots written by two sequences are the caller's error. o: [S, T, Hq, D]; lse: [S, T, Hq].
+ */
+int oracle_decode_step(const uint16_t* q, const uint16_t* k_new, const uint16_t* v_new, uint16_t* k_pages,
+                       uint16_t* v_pages, const int32_t* block_table, const int32_t* seq_lens, int S, int T,
+                       int max_blocks, int num_pages, int page_size, int Hq, int Hkv, int D, double rope_base,
+                       double scale, double* o, double* lse, int nthreads) {
+    if (!q || !k_pages || !v_pages || !block_table || !seq_lens || !o || !lse) return ORACLE_ERR_ARG;
+    if ((k_new == NULL) != (v_new == NULL)) return ORACLE_ERR_ARG;
+    if (S <= 0 || T <= 0 || max_blocks <= 0 || num_pages <= 0 || page_size <= 0 || Hq <= 0 || Hkv <= 0 ||
+        D <= 0 || (D % 2) != 0 || Hq % Hkv != 0)
+        return ORACLE_ERR_ARG;
+    const int G = Hq / Hkv;
+    for (int s = 0; s < S; ++s) {
+        int len = seq_lens[s];
+        if (len < T || (int64_t)len > (int64_t)max_blocks * page_size) return ORACLE_ERR_INDEX;
+        int pages = (len + page_size - 1) / page_size;
+        for (int p = 0; p < pages; ++p) {
+            int32_t pg = block_table[(size_t)s * max_blocks + p];
+            if (pg < 0 || pg >= num_pages) return ORACLE_ERR_INDEX;
+        }
+    }
+    double* tmp = (double*)malloc(sizeof(double) * (size_t)D);
+    if (!tmp) return ORACLE_ERR_NOMEM;
+    if (k_new != NULL) {
+        for (int s = 0; s < S; ++s) {
+            for (int t = 0; t < T; ++t) {
+                long pos = (long)seq_lens[s] - T + t;
+                int32_t pg = block_table[(size_t)s * max_blocks + pos / page_size];
+                for (int g = 0; g < Hkv; ++g) {
+                    size_t src = (((size_t)s * T + t) * Hkv + g) * D;
+                    size_t dst = (((size_t)pg * Hkv + g) * page_size + (size_t)(pos % page_size)) * D;
+                    rope_row(k_new + src, D, pos, rope_base, tmp);
+                    for (int d = 0; d < D; ++d) {
+                        k_pages[dst + d] = oracle_round_bf16(tmp[d]);
+                        v_pages[dst + d] = v_new[src + d];
+                    }
+                }
+            }
+        }
+    }
+    free(tmp);
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#else
+    (void)nthreads;
+#endif
+    int status = ORACLE_OK;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int sg = 0; sg < S * Hkv; ++sg) {
+        int s = sg / Hkv, g = sg % Hkv;
+        int len = seq_lens[s];
+        double* kk = (double*)malloc(sizeof(double) * (size_t)len * D);
+        double* vv = (double*)malloc(sizeof(double) * (size_t)len * D);
+        double* s_row = (double*)malloc(sizeof(double) * (size_t)len);
+        double* qq = (double*)malloc(sizeof(double) * (size_t)D);
+        if (!kk || !vv || !s_row || !qq) {
+#pragma omp atomic write
+            status = ORACLE_ERR_NOMEM;
+        } else {
+            for (int t = 0; t < len; ++t) {
+                int32_t pg = block_table[(size_t)s * max_blocks + t / page_size];
+                size_t base = (((size_t)pg * Hkv + g) * page_size + (size_t)(t % page_size)) * D;
+                for (int d = 0; d < D; ++d) {
+                    kk[(size_t)t * D + d] = bf16_value(k_pages[base + d]);
+                    vv[(size_t)t * D + d] = bf16_value(v_pages[base + d]);
+                }
+            }
+            for (int t = 0; t < T; ++t) {
+                long pos = (long)len - T + t;
+                for (int hh = 0; hh < G; ++hh) {
+                    int h = g * G + hh;
+                    size_t row = ((size_t)s * T + t) * Hq + h;
+                    rope_row(q + row * D, D, pos, rope_base, qq);
+                    attend_row(qq, kk, vv, len, D, pos, 1, 0, scale, s_row, o + row * D, lse + row);
+                }
             }
         }
         free(kk);

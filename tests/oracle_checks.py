@@ -366,6 +366,129 @@ def check_decode_paging_invariance(lib):
     assert np.array_equal(o, o3) and np.array_equal(lse, lse3)
 
 
+def _step_inputs(T, seed, rope_base, lens=(4, 16, 17, 40, 33, 64)):
+    return synth.decode_step_inputs(len(lens), T, 8, 2, 64, 16, seq_lens=list(lens), spare_frac=0.5, seed=seed)
+
+
+def _step(inp, rope_base, lib, with_new=True):
+    c = inp.cache
+    return oracle.decode_step(synth.bits(inp.q), synth.bits(inp.k_new) if with_new else None,
+                              synth.bits(inp.v_new) if with_new else None, synth.bits(c.k_pages),
+                              synth.bits(c.v_pages), c.block_table.numpy(), c.seq_lens.numpy(), rope_base=rope_base,
+                              lib=lib)
+
+
+def _gather_bits(kp, vp, cache, s):
+    n = int(cache.seq_lens[s])
+    pages = cache.block_table[s, :(n + cache.page_size - 1) // cache.page_size].numpy()
+    k = kp[pages].transpose(1, 0, 2, 3).reshape(cache.Hkv, -1, cache.D)[:, :n]
+    v = vp[pages].transpose(1, 0, 2, 3).reshape(cache.Hkv, -1, cache.D)[:, :n]
+    return np.ascontiguousarray(k), np.ascontiguousarray(v)
+
+
+def check_decode_step_append_slots(lib):
+    """The append writes exactly the new tokens' slots: the key rotated at its position, the value
+    as given; every other slot keeps its bits ("Self-Attention Complexity, ...", Part 3)."""
+    T, base = 3, 10000.0
+    inp = _step_inputs(T, 11, base)
+    c = inp.cache
+    _, _, kp, vp = _step(inp, base, lib)
+    k0, v0 = synth.bits(c.k_pages).copy(), synth.bits(c.v_pages).copy()
+    touched = np.zeros(k0.shape[:1] + k0.shape[2:3], bool)  # [page, slot]
+    for s in range(c.num_seqs):
+        n = int(c.seq_lens[s])
+        for t in range(T):
+            pos = n - T + t
+            page, slot = int(c.block_table[s, pos // 16]), pos % 16
+            touched[page, slot] = True
+            for g in range(c.Hkv):
+                want_k = oracle.rope_bf16(synth.bits(inp.k_new[s, t, g])[None], np.array([pos]), base, lib=lib)[0]
+                assert np.array_equal(kp[page, g, slot], want_k)
+                assert np.array_equal(vp[page, g, slot], synth.bits(inp.v_new[s, t, g]))
+    keep = ~touched[:, None, :, None].repeat(c.Hkv, 1).repeat(c.D, 3)
+    assert np.array_equal(kp[keep], k0[keep]) and np.array_equal(vp[keep], v0[keep])
+
+
+def check_decode_step_is_last_prefill_rows(lib):
+    """T new tokens attend like the last T rows of causal prefill over the whole sequence, with q
+    rotated at positions len-T .. len-1 (the decode query sits at the end of its sequence)."""
+    T, base = 4, 500.0
+    inp = _step_inputs(T, 12, base)
+    c = inp.cache
+    o, lse, kp, vp = _step(inp, base, lib)
+    for s in range(c.num_seqs):
+        n = int(c.seq_lens[s])
+        k, v = _gather_bits(kp, vp, c, s)
+        pos = np.arange(n - T, n)
+        qs = np.zeros((1, c.Hq, n, c.D), np.uint16)
+        for h in range(c.Hq):
+            qs[0, h, n - T:] = oracle.rope_bf16(synth.bits(inp.q[s, :, h]), pos, base, lib=lib)
+        op, lsep = oracle.attention(qs, k[None], v[None], causal=True, scale=c.D ** -0.5, lib=lib)
+        assert np.array_equal(o[s], op[0, :, n - T:].transpose(1, 0, 2))
+        assert np.array_equal(lse[s], lsep[0, :, n - T:].T)
+
+
+def check_decode_step_prefill_with_rope(lib):
+    """Against prefill with RoPE applied inside: a cache holding rotated keys of a sequence plus
+    the last T tokens appended unrotated gives the last T rows of RoPE prefill on that sequence."""
+    T, base = 2, 10000.0
+    lens = (5, 17, 32)
+    inp = _step_inputs(T, 13, base, lens=lens)
+    c = inp.cache
+    k_full = [_rand((c.Hkv, n, c.D), 140 + s) for s, n in enumerate(lens)]
+    kp = synth.bits(c.k_pages).copy()
+    for s, n in enumerate(lens):
+        for j in range(n - T):
+            page, slot = int(c.block_table[s, j // 16]), j % 16
+            kp[page, :, slot] = oracle.rope_bf16(k_full[s][:, j], np.full(c.Hkv, j), base, lib=lib)
+    k_new = np.stack([k_full[s][:, n - T:].transpose(1, 0, 2) for s, n in enumerate(lens)])
+    o, lse, kp2, vp2 = oracle.decode_step(synth.bits(inp.q), np.ascontiguousarray(k_new), synth.bits(inp.v_new), kp,
+                                          synth.bits(c.v_pages), c.block_table.numpy(), c.seq_lens.numpy(),
+                                          rope_base=base, lib=lib)
+    for s, n in enumerate(lens):
+        _, v = _gather_bits(kp2, vp2, c, s)
+        qs = np.zeros((1, c.Hq, n, c.D), np.uint16)
+        qs[0, :, n - T:] = synth.bits(inp.q[s]).transpose(1, 0, 2)
+        op, lsep = oracle.attention(qs, k_full[s][None], v[None], causal=True, rope_base=base, scale=c.D ** -0.5,
+                                    lib=lib)
+        assert np.array_equal(o[s], op[0, :, n - T:].transpose(1, 0, 2))
+        assert np.array_equal(lse[s], lsep[0, :, n - T:].T)
+
+
+def check_decode_step_library(lib):
+    """torch float64 SDPA on the gathered cache, with the rotated queries and a causal mask over
+    the last T positions."""
+    T, base = 3, 10000.0
+    inp = _step_inputs(T, 15, base)
+    c = inp.cache
+    o, _, kp, vp = _step(inp, base, lib)
+    for s in range(c.num_seqs):
+        n = int(c.seq_lens[s])
+        k, v = _gather_bits(kp, vp, c, s)
+        pos = np.arange(n - T, n)
+        qr = np.stack([oracle.rope_bf16(synth.bits(inp.q[s, :, h]), pos, base, lib=lib) for h in range(c.Hq)])
+        mask = np.arange(n)[None, :] <= pos[:, None]
+        ref = _sdpa64(qr, k, v, c.D ** -0.5, mask=torch.tensor(mask), gqa=True)
+        assert np.abs(o[s] - ref.transpose(1, 0, 2)).max() < 1e-12
+
+
+def check_decode_step_reduces_to_decode(lib):
+    """One token, no append, no RoPE: the decode step is the one-token paged decode."""
+    inp = _step_inputs(1, 16, 0.0)
+    c = inp.cache
+    o, lse, _, _ = oracle.decode_step(synth.bits(inp.q), None, None, synth.bits(c.k_pages), synth.bits(c.v_pages),
+                                      c.block_table.numpy(), c.seq_lens.numpy(), lib=lib)
+    c.k_pages.view(torch.int16)[torch.isnan(c.k_pages)] = 0  # the poisoned new slots now hold tokens
+    c.v_pages.view(torch.int16)[torch.isnan(c.v_pages)] = 0
+    o1, lse1, _, _ = oracle.decode_step(synth.bits(inp.q), None, None, synth.bits(c.k_pages), synth.bits(c.v_pages),
+                                        c.block_table.numpy(), c.seq_lens.numpy(), lib=lib)
+    c1 = synth.PagedCache(inp.q[:, 0].contiguous(), c.k_pages, c.v_pages, c.block_table, c.seq_lens, c.page_size,
+                          c.Hq, c.Hkv, c.D)
+    o2, lse2 = _decode(c1, lib)
+    assert np.array_equal(o1[:, 0], o2) and np.array_equal(lse1[:, 0], lse2)
+    assert not np.all(np.isfinite(o))  # the unfilled NaN slot is read: the step does attend to it
+
+
 ALL_CHECKS = [
     check_round_bf16_golden, check_round_bf16_matches_torch, check_rope_golden,
     check_rope_matches_sinusoid, check_rope_norm_and_identity, check_rope_relative,
@@ -373,7 +496,9 @@ ALL_CHECKS = [
     check_gqa_reduces_to_mha, check_lse_library, check_probability_rows,
     check_permutation_equivariance, check_causal_row0_and_window1, check_equal_scores,
     check_rows_subset, check_online_recurrence, check_decode_is_last_prefill_row,
-    check_decode_library, check_decode_paging_invariance,
+    check_decode_library, check_decode_paging_invariance, check_decode_step_append_slots,
+    check_decode_step_is_last_prefill_rows, check_decode_step_prefill_with_rope, check_decode_step_library,
+    check_decode_step_reduces_to_decode,
 ]
 
 

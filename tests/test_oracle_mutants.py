@@ -34,6 +34,9 @@ MUTANTS = {
     "bwd_dk_unscaled": ("my_dk[(size_t)j * D + d] += scale * ds * qq[d];", "my_dk[(size_t)j * D + d] += ds * qq[d];"),
     "bwd_dq_not_rotated_back": ("rope_row_f64(dqr, D, i, rope_base, 1, 0, dq + row * D);",
                                 "rope_row_f64(dqr, D, i, rope_base, 0, 0, dq + row * D);"),
+    "step_query_position": ("long pos = (long)len - T + t;", "long pos = (long)len - T + t - (t > 0);"),
+    "step_append_slot": ("long pos = (long)seq_lens[s] - T + t;", "long pos = (long)seq_lens[s] - T + t + (t == 0);"),
+    "step_query_unrotated": ("rope_row(q + row * D, D, pos, rope_base, qq);", "rope_row(q + row * D, D, 0, rope_base, qq);"),
     "normaliser_missing": ("for (int d = 0; d < D; ++d) o[d] /= l;", "for (int d = 0; d < D; ++d) o[d] /= (l + 1e-3);"),
 }
 
