@@ -68,6 +68,17 @@ def decode_bytes(cache):
     return kv + io + tables
 
 
+def step_bytes(cache, T):
+    """Algorithmic bytes of a decode step with T new tokens per sequence: the cache read once, the
+    new keys and values read and written into their slots, T query rows in and out, LSE, tables."""
+    S, Hq, Hkv, D = cache.num_seqs, cache.Hq, cache.Hkv, cache.D
+    kv = int(cache.seq_lens.to(torch.int64).sum()) * 2 * Hkv * D * 2
+    append = S * T * Hkv * D * 2 * 2 * 2
+    io = S * T * Hq * D * 2 * 2 + S * T * Hq * 4
+    tables = S * 4 + sum(((int(n) + cache.page_size - 1) // cache.page_size) for n in cache.seq_lens) * 4
+    return kv + append + io + tables
+
+
 # ------------------------------------------------------------------------------ ranks
 def dist_env():
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -367,9 +378,52 @@ def run_ours(args, rank, world, local):
     e2e_value = job_throughput(flops * E, world, e_pre / 1e3) / 1e12 if E else None
     e2e_decode = job_throughput(dbytes * E, world, e_dec / 1e3) / 1e9 if E else None
 
+    # ---- decode step: append one or four new tokens per sequence (keys rotated, RoPE 1e4) and attend
+    # with their rotated queries, on the same cache (runs after the legs above: it writes the cache)
+    steps_out = None
+    if do_decode and args.step_calls > 0:
+        steps_out = {}
+        S, Hq, Hkv, D = DECODE.num_seqs, DECODE.Hq, DECODE.Hkv, DECODE.D
+        gen = torch.Generator().manual_seed(DECODE.seed + 7919)
+        for T in (1, 4):
+            sq = synth.randn_bf16((S, T, Hq, D), gen).to(dev)
+            kn = synth.randn_bf16((S, T, Hkv, D), gen).to(dev)
+            vn = synth.randn_bf16((S, T, Hkv, D), gen).to(dev)
+            so = torch.empty_like(sq)
+            slse = torch.empty((S, T, Hq), dtype=torch.float32, device=dev)
+            sws = torch.empty(api.decode_step_workspace_size(S, T, cache_h.max_blocks, DECODE.page_size, Hq, D),
+                              dtype=torch.uint8, device=dev)
+
+            def step_call():
+                api.attn_decode_step(sq, kp, vp, bt, sl, k_new=kn, v_new=vn, rope_base=10000.0, o=so, lse=slse,
+                                     workspace=sws, stream=stream)
+
+            for _ in range(args.warmup):
+                step_call()
+            barrier(world)
+            torch.cuda.synchronize()
+            a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a0.record(stream)
+            for _ in range(args.step_calls):
+                step_call()
+            a1.record(stream)
+            torch.cuda.synchronize()
+            if api.device_status() != 0:
+                raise RuntimeError("device status raised during the decode-step loop")
+            ms = reduce_max(a0.elapsed_time(a1), world, dev) / args.step_calls
+            sbytes = step_bytes(cache_h, T)
+            steps_out["q_len=%d" % T] = {
+                "value": round(job_throughput(sbytes, world, ms / 1e3) / 1e9, 1), "unit": "GB/s",
+                "ms_per_call": round(ms, 4), "calls": args.step_calls, "bytes_per_call": sbytes,
+                "roofline": {"bound": "hbm", "achieved": round(sbytes / (ms / 1e3) / 1e9, 1), "unit": "GB/s"}}
+
     if rank != 0:
         return None
     peaks, peaks_kind = measured_peaks()
+    if steps_out is not None:
+        for v in steps_out.values():
+            v["roofline"].update({"peak": peaks["hbm_gbs"], "frac": round(v["roofline"]["achieved"] / peaks["hbm_gbs"], 4),
+                                  "peak_kind": peaks_kind})
     pre_launch_ms = statistics.mean(prefill_ms)
     dec_launch_ms = statistics.mean(decode_ms)
     tflops_launch = flops / (pre_launch_ms / 1e3) / 1e12 if do_prefill else float("nan")
@@ -421,6 +475,9 @@ def run_ours(args, rank, world, local):
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": (2 * do_prefill + 2 * do_decode) * K,
         "backward": bwd,
+        "decode_step": None if steps_out is None else dict(
+            {"metric": "decode step KV GB/s: append q_len new tokens per sequence (keys rotated, RoPE 1e4) into "
+                       "the 64-sequence paged cache, then attend with their rotated queries"}, **steps_out),
         "device_status": status,
         "clocks": clk,
     }
@@ -499,6 +556,7 @@ def parse_args(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--e2e-steps", type=int, default=10, help="0 skips the end-to-end leg")
     ap.add_argument("--bwd-steps", type=int, default=20, help="backward calls timed after the step loop; 0 skips")
+    ap.add_argument("--step-calls", type=int, default=50, help="decode-step calls timed per q_len; 0 skips")
     ap.add_argument("--only", choices=["all", "prefill", "decode"], default="all",
                     help="time one half of the step only (profiling runs); the JSON line is then partial")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle time for the CPU baseline")

@@ -32,6 +32,9 @@ SIGNATURES = {
     "attn_decode_workspace_size": (_sz, [_i, _i, _i, _i, _i]),
     "attn_decode_paged": (_i, [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _f, _p, _p, _p, _sz, _p]),
     "attn_decode_paged_noalloc": (_i, [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _f, _p, _p, _p]),
+    "attn_decode_step_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i]),
+    "attn_decode_step": (_i, [_p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _f, _f, _p, _p, _p, _sz,
+                              _p]),
     "attn_get_device_status": (_i, [_p, ctypes.POINTER(ctypes.c_int)]),
     "attn_last_error": (ctypes.c_char_p, []),
     "attn_version": (ctypes.c_char_p, []),
@@ -167,6 +170,48 @@ def attn_decode_paged(q, k_pages, v_pages, block_table, seq_lens, scale=0.0, o=N
                                  _dev_tensor(lse, "lse", torch.float32) if lse is not None else None,
                                  _dev_tensor(workspace, "workspace", torch.uint8),
                                  workspace.numel() * workspace.element_size(), _stream(stream)))
+    return o, lse
+
+
+def decode_step_workspace_size(num_seqs, q_len, max_blocks_per_seq, page_size, Hq, D) -> int:
+    return int(lib.attn_decode_step_workspace_size(num_seqs, q_len, max_blocks_per_seq, page_size, Hq, D))
+
+
+def attn_decode_step(q, k_pages, v_pages, block_table, seq_lens, k_new=None, v_new=None, rope_base=0.0, scale=0.0,
+                     o=None, lse=None, want_lse=True, workspace=None, stream=None):
+    """Decode step with q_len new tokens per sequence: append k_new/v_new (keys rotated) into their
+    page slots, then attend with the new queries (rotated) causally over the cache.
+    q [S,q_len,Hq,D] bf16; k_new/v_new [S,q_len,Hkv,D] bf16 or None; k_pages/v_pages
+    [num_pages,Hkv,page_size,D] bf16 (updated in place); block_table [S,max_blocks] int32; seq_lens
+    [S] int32 counting the new tokens (all CUDA). Returns (o [S,q_len,Hq,D] bf16, lse [S,q_len,Hq] fp32
+    or None)."""
+    S, T, Hq, D = q.shape
+    num_pages, Hkv, page_size, D2 = k_pages.shape
+    if D2 != D or v_pages.shape != k_pages.shape:
+        raise ValueError("k_pages/v_pages must be [num_pages, Hkv, page_size, D]")
+    if (k_new is None) != (v_new is None):
+        raise ValueError("k_new and v_new go together")
+    if k_new is not None and (k_new.shape != (S, T, Hkv, D) or v_new.shape != k_new.shape):
+        raise ValueError("k_new/v_new must be [S, q_len, Hkv, D]")
+    max_blocks = block_table.shape[1]
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((S, T, Hq), dtype=torch.float32, device=q.device)
+    need = decode_step_workspace_size(S, T, max_blocks, page_size, Hq, D)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    kn = _dev_tensor(k_new, "k_new", torch.bfloat16) if k_new is not None else None
+    vn = _dev_tensor(v_new, "v_new", torch.bfloat16) if v_new is not None else None
+    _check(lib.attn_decode_step(_dev_tensor(q, "q", torch.bfloat16), kn, vn,
+                                _dev_tensor(k_pages, "k_pages", torch.bfloat16),
+                                _dev_tensor(v_pages, "v_pages", torch.bfloat16),
+                                _dev_tensor(block_table, "block_table", torch.int32),
+                                _dev_tensor(seq_lens, "seq_lens", torch.int32), S, T, max_blocks, num_pages, page_size,
+                                Hq, Hkv, D, float(rope_base), float(scale), _dev_tensor(o, "o", torch.bfloat16),
+                                _dev_tensor(lse, "lse", torch.float32) if lse is not None else None,
+                                _dev_tensor(workspace, "workspace", torch.uint8),
+                                workspace.numel() * workspace.element_size(), _stream(stream)))
     return o, lse
 
 

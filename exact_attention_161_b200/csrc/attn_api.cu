@@ -87,45 +87,63 @@ struct DevBuf {
 };
 
 std::mutex g_cache_mu;
-// (device, base, D) -> cos/sin table covering positions [0, capacity)
-std::map<std::tuple<int, double, int>, std::pair<DevBuf, int>> g_rope_tables;
+// (device, base, D, fp64?) -> cos/sin table covering positions [0, capacity)
+std::map<std::tuple<int, double, int, bool>, std::pair<DevBuf, int>> g_rope_tables;
 // (device, stream) -> rotated-key scratch
 std::map<std::pair<int, void*>, DevBuf> g_key_scratch;
 std::vector<DevBuf> g_retired;  // outgrown buffers; a launch still queued may read them
 
 // (cos, sin) of pos * base^(-2i/D) for pos < n, i < D/2: angles and trigonometry in fp64, stored
-// as fp32 pairs.
-attn_status rope_table(int dev, double base, int D, int n, const float2** out) {
+// as fp64 pairs (wide) or rounded to fp32 pairs.
+attn_status rope_table_any(int dev, double base, int D, int n, bool wide, const void** out) {
     std::lock_guard<std::mutex> lock(g_cache_mu);
-    auto key = std::make_tuple(dev, base, D);
+    auto key = std::make_tuple(dev, base, D, wide);
     auto it = g_rope_tables.find(key);
     if (it != g_rope_tables.end() && it->second.second >= n) {
-        *out = static_cast<const float2*>(it->second.first.ptr);
+        *out = it->second.first.ptr;
         return ATTN_OK;
     }
     const int cap = ((n + 1023) / 1024) * 1024;
-    std::vector<float2> host(static_cast<size_t>(cap) * (D / 2));
+    const size_t pairs = static_cast<size_t>(cap) * (D / 2);
+    std::vector<double2> host64(wide ? pairs : 0);
+    std::vector<float2> host32(wide ? 0 : pairs);
     std::vector<double> theta(D / 2);
     for (int i = 0; i < D / 2; ++i) theta[i] = std::pow(base, -2.0 * i / D);
     for (int pos = 0; pos < cap; ++pos)
         for (int i = 0; i < D / 2; ++i) {
             const double a = pos * theta[i];
-            host[static_cast<size_t>(pos) * (D / 2) + i] = make_float2(static_cast<float>(std::cos(a)),
-                                                                       static_cast<float>(std::sin(a)));
+            const size_t at = static_cast<size_t>(pos) * (D / 2) + i;
+            if (wide)
+                host64[at] = make_double2(std::cos(a), std::sin(a));
+            else
+                host32[at] = make_float2(static_cast<float>(std::cos(a)), static_cast<float>(std::sin(a)));
         }
     DevBuf buf;
     buf.dev = dev;
-    buf.bytes = host.size() * sizeof(float2);
+    buf.bytes = pairs * (wide ? sizeof(double2) : sizeof(float2));
     CUDA_TRY(cudaMalloc(&buf.ptr, buf.bytes));
-    cudaError_t e = cudaMemcpy(buf.ptr, host.data(), buf.bytes, cudaMemcpyHostToDevice);
+    cudaError_t e = cudaMemcpy(buf.ptr, wide ? static_cast<const void*>(host64.data()) : host32.data(), buf.bytes,
+                               cudaMemcpyHostToDevice);
     if (e != cudaSuccess) {
         cudaFree(buf.ptr);
         return fail(ATTN_ERR_CUDA, "rope table upload: %s", cudaGetErrorString(e));
     }
     if (it != g_rope_tables.end()) g_retired.push_back(it->second.first);
     g_rope_tables[key] = std::make_pair(buf, cap);
-    *out = static_cast<const float2*>(buf.ptr);
+    *out = buf.ptr;
     return ATTN_OK;
+}
+attn_status rope_table(int dev, double base, int D, int n, const float2** out) {
+    const void* p = nullptr;
+    attn_status st = rope_table_any(dev, base, D, n, false, &p);
+    *out = static_cast<const float2*>(p);
+    return st;
+}
+attn_status rope_table64(int dev, double base, int D, int n, const double2** out) {
+    const void* p = nullptr;
+    attn_status st = rope_table_any(dev, base, D, n, true, &p);
+    *out = static_cast<const double2*>(p);
+    return st;
 }
 
 attn_status key_scratch(int dev, void* stream, size_t bytes, void** out) {
@@ -167,6 +185,9 @@ attn_status launch_fwd(const void* q, const void* k, const void* v, void* o, flo
         const float2* table = nullptr;
         attn_status st = rope_table(dev, static_cast<double>(rope_base), D, N, &table);
         if (st != ATTN_OK) return st;
+        const double2* table64 = nullptr;
+        st = rope_table64(dev, static_cast<double>(rope_base), D, N, &table64);
+        if (st != ATTN_OK) return st;
         void* k_rot = nullptr;
         const size_t kbytes = static_cast<size_t>(B) * Hkv * N * D * 2;
         st = key_scratch(dev, stream, kbytes, &k_rot);
@@ -178,7 +199,7 @@ attn_status launch_fwd(const void* q, const void* k, const void* v, void* o, flo
         const long long want = (chunks + 255) / 256;
         const int grid = static_cast<int>(want < 8LL * sms ? want : 8LL * sms);
         attn::rope_rotate_rows_kernel<D><<<grid, 256, 0, stream>>>(static_cast<const uint4*>(k),
-                                                                   static_cast<uint4*>(k_rot), table, rows, N);
+                                                                   static_cast<uint4*>(k_rot), table64, rows, N);
         CUDA_TRY(cudaGetLastError());
         k_use = k_rot;
         p.rope = table;
@@ -211,9 +232,33 @@ attn_status launch_fwd(const void* q, const void* k, const void* v, void* o, flo
 size_t decode_chunks(int max_blocks) { return (static_cast<size_t>(max_blocks) + attn::kChunkPages - 1) / attn::kChunkPages; }
 
 template <int D>
+attn_status launch_append(const void* k_new, const void* v_new, void* k_pages, void* v_pages,
+                          const int32_t* block_table, const int32_t* seq_lens, int S, int T, int max_blocks,
+                          int num_pages, int Hkv, const double2* rope, cudaStream_t stream) {
+    attn::AppendParams a{};
+    a.k_new = static_cast<const __nv_bfloat16*>(k_new);
+    a.v_new = static_cast<const __nv_bfloat16*>(v_new);
+    a.k_pages = static_cast<__nv_bfloat16*>(k_pages);
+    a.v_pages = static_cast<__nv_bfloat16*>(v_pages);
+    a.block_table = block_table;
+    a.seq_lens = seq_lens;
+    a.rope = rope;
+    a.S = S;
+    a.T = T;
+    a.Hkv = Hkv;
+    a.max_blocks = max_blocks;
+    a.num_pages = num_pages;
+    const long long warps = static_cast<long long>(S) * T * Hkv;
+    attn::decode_append_kernel<D><<<static_cast<unsigned>((warps * 32 + 127) / 128), 128, 0, stream>>>(a);
+    CUDA_TRY(cudaGetLastError());
+    return ATTN_OK;
+}
+
+template <int D>
 attn_status launch_decode(const void* q, const void* k_pages, const void* v_pages, const int32_t* block_table,
-                          const int32_t* seq_lens, int S, int max_blocks, int num_pages, int Hq, int Hkv,
-                          float scale, void* o, float* lse, void* ws, cudaStream_t stream, int dev) {
+                          const int32_t* seq_lens, int S, int T, int max_blocks, int num_pages, int Hq, int Hkv,
+                          float scale, const double2* rope, void* o, float* lse, void* ws, cudaStream_t stream,
+                          int dev) {
     using C = attn::DecCfg<D>;
     CUtensorMap tk, tv;
     attn_status st;
@@ -228,7 +273,10 @@ attn_status launch_decode(const void* q, const void* k_pages, const void* v_page
     p.o = static_cast<__nv_bfloat16*>(o);
     p.lse = lse;
     p.ws_o = static_cast<float*>(ws);
-    p.ws_ml = p.ws_o + static_cast<size_t>(S) * Hq * max_chunks * D;
+    p.ws_ml = p.ws_o + static_cast<size_t>(S) * T * Hq * max_chunks * D;
+    p.rope = rope;
+    p.T = T;
+    p.mtiles = (Hq / Hkv * T + 15) / 16;
     p.S = S;
     p.Hq = Hq;
     p.Hkv = Hkv;
@@ -237,10 +285,18 @@ attn_status launch_decode(const void* q, const void* k_pages, const void* v_page
     p.num_pages = num_pages;
     p.max_chunks = max_chunks;
     p.scale_log2 = scale * attn::kLog2e;
-    if ((st = ensure_smem(attn::decode_split_kernel<D>, C::SMEM_BYTES, dev)) != ATTN_OK) return st;
-    attn::decode_split_kernel<D><<<dim3(max_chunks, Hkv, S), attn::kDecodeThreads, C::SMEM_BYTES, stream>>>(tk, tv, p);
+    const bool step = T > 1 || rope != nullptr;
+    if (step) {
+        if ((st = ensure_smem(attn::decode_split_kernel<D, true>, C::SMEM_BYTES, dev)) != ATTN_OK) return st;
+        attn::decode_split_kernel<D, true><<<dim3(max_chunks, Hkv * p.mtiles, S), attn::kDecodeThreads, C::SMEM_BYTES,
+                                             stream>>>(tk, tv, p);
+    } else {
+        if ((st = ensure_smem(attn::decode_split_kernel<D, false>, C::SMEM_BYTES, dev)) != ATTN_OK) return st;
+        attn::decode_split_kernel<D, false><<<dim3(max_chunks, Hkv, S), attn::kDecodeThreads, C::SMEM_BYTES, stream>>>(
+            tk, tv, p);
+    }
     CUDA_TRY(cudaGetLastError());
-    const long long warps = static_cast<long long>(S) * Hq;
+    const long long warps = static_cast<long long>(S) * T * Hq;
     attn::decode_merge_kernel<D><<<static_cast<unsigned>((warps * 32 + 127) / 128), 128, 0, stream>>>(p);
     CUDA_TRY(cudaGetLastError());
     return ATTN_OK;
@@ -294,6 +350,9 @@ attn_status launch_bwd(const void* q, const void* k, const void* v, const void* 
         const float2* table = nullptr;
         attn_status st = rope_table(dev, static_cast<double>(rope_base), D, N, &table);
         if (st != ATTN_OK) return st;
+        const double2* table64 = nullptr;
+        st = rope_table64(dev, static_cast<double>(rope_base), D, N, &table64);
+        if (st != ATTN_OK) return st;
         p.rope = table;
         void* qr = w + L.qrot;
         void* kr = w + L.krot;
@@ -303,10 +362,10 @@ attn_status launch_bwd(const void* q, const void* k, const void* v, const void* 
             return static_cast<int>(want < 8LL * sms ? want : 8LL * sms);
         };
         attn::rope_rotate_rows_kernel<D><<<grid_for(qrows), 256, 0, stream>>>(static_cast<const uint4*>(q),
-                                                                              static_cast<uint4*>(qr), table, qrows, N);
+                                                                              static_cast<uint4*>(qr), table64, qrows, N);
         CUDA_TRY(cudaGetLastError());
         attn::rope_rotate_rows_kernel<D><<<grid_for(krows), 256, 0, stream>>>(static_cast<const uint4*>(k),
-                                                                              static_cast<uint4*>(kr), table, krows, N);
+                                                                              static_cast<uint4*>(kr), table64, krows, N);
         CUDA_TRY(cudaGetLastError());
         q_use = qr;
         k_use = kr;
@@ -436,10 +495,71 @@ attn_status attn_decode_paged(const void* q, const void* k_pages, const void* v_
     CUDA_TRY(cudaGetDevice(&dev));
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (D == 64)
-        return launch_decode<64>(q, k_pages, v_pages, block_table, seq_lens, num_seqs, max_blocks_per_seq, num_pages,
-                                 Hq, Hkv, scale, o, lse, workspace, s, dev);
-    return launch_decode<128>(q, k_pages, v_pages, block_table, seq_lens, num_seqs, max_blocks_per_seq, num_pages,
-                              Hq, Hkv, scale, o, lse, workspace, s, dev);
+        return launch_decode<64>(q, k_pages, v_pages, block_table, seq_lens, num_seqs, 1, max_blocks_per_seq,
+                                 num_pages, Hq, Hkv, scale, nullptr, o, lse, workspace, s, dev);
+    return launch_decode<128>(q, k_pages, v_pages, block_table, seq_lens, num_seqs, 1, max_blocks_per_seq,
+                              num_pages, Hq, Hkv, scale, nullptr, o, lse, workspace, s, dev);
+}
+
+size_t attn_decode_step_workspace_size(int num_seqs, int q_len, int max_blocks_per_seq, int page_size, int Hq, int D) {
+    if (num_seqs < 1 || q_len < 1 || max_blocks_per_seq < 1 || page_size < 1 || Hq < 1 || D < 1) return 0;
+    const size_t rows = static_cast<size_t>(num_seqs) * q_len * Hq * decode_chunks(max_blocks_per_seq);
+    const size_t bytes = rows * (static_cast<size_t>(D) + 2) * sizeof(float);
+    return (bytes + 255) / 256 * 256;
+}
+
+attn_status attn_decode_step(const void* q, const void* k_new, const void* v_new, void* k_pages, void* v_pages,
+                             const int32_t* block_table, const int32_t* seq_lens, int num_seqs, int q_len,
+                             int max_blocks_per_seq, int num_pages, int page_size, int Hq, int Hkv, int D,
+                             float rope_base, float scale, void* o, float* lse, void* workspace,
+                             size_t workspace_bytes, void* stream) {
+    g_last_error.clear();
+    if (!q || !k_pages || !v_pages || !block_table || !seq_lens || !o || !workspace)
+        return fail(ATTN_ERR_INVALID_ARG, "q, k_pages, v_pages, block_table, seq_lens, o and workspace must be non-NULL");
+    if ((k_new == nullptr) != (v_new == nullptr))
+        return fail(ATTN_ERR_INVALID_ARG, "k_new and v_new must both be given or both be NULL");
+    if (!aligned16(q) || !aligned16(k_pages) || !aligned16(v_pages) || !aligned16(o) || !aligned16(workspace) ||
+        (k_new && (!aligned16(k_new) || !aligned16(v_new))) ||
+        (reinterpret_cast<uintptr_t>(block_table) & 3u) || (reinterpret_cast<uintptr_t>(seq_lens) & 3u) ||
+        (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+        return fail(ATTN_ERR_INVALID_ARG, "misaligned pointer (tensors 16-byte, int32/fp32 arrays 4-byte)");
+    if (num_seqs < 1 || q_len < 1 || max_blocks_per_seq < 1 || num_pages < 1 || page_size < 1 || Hq < 1 || Hkv < 1)
+        return fail(ATTN_ERR_INVALID_ARG, "sizes must be >= 1");
+    if (Hq % Hkv != 0) return fail(ATTN_ERR_INVALID_ARG, "Hq (%d) must be a multiple of Hkv (%d)", Hq, Hkv);
+    if (!std::isfinite(scale) || !std::isfinite(rope_base)) return fail(ATTN_ERR_INVALID_ARG, "scale and rope_base must be finite");
+    if (page_size != attn::kPageSize) return fail(ATTN_ERR_UNSUPPORTED, "page_size %d not supported (16)", page_size);
+    if (D != 64 && D != 128) return fail(ATTN_ERR_UNSUPPORTED, "head dim %d not supported (64 or 128)", D);
+    if (Hq / Hkv > 16) return fail(ATTN_ERR_UNSUPPORTED, "more than 16 query heads per KV head");
+    if (q_len > 64) return fail(ATTN_ERR_UNSUPPORTED, "q_len %d above 64 new tokens per sequence", q_len);
+    if (num_seqs > 65535 || static_cast<long long>(Hkv) * ((Hq / Hkv * q_len + 15) / 16) > 65535)
+        return fail(ATTN_ERR_UNSUPPORTED, "num_seqs or Hkv * row tiles too large for the grid");
+    if (static_cast<double>(num_pages) * Hkv * page_size * D * 2 >= 1099511627776.0)
+        return fail(ATTN_ERR_UNSUPPORTED, "KV pool larger than 1 TiB");
+    const size_t need = attn_decode_step_workspace_size(num_seqs, q_len, max_blocks_per_seq, page_size, Hq, D);
+    if (workspace_bytes < need)
+        return fail(ATTN_ERR_INVALID_ARG, "workspace too small: %zu < %zu bytes", workspace_bytes, need);
+    if (scale <= 0.f) scale = 1.0f / std::sqrt(static_cast<float>(D));
+    int dev = 0;
+    CUDA_TRY(cudaGetDevice(&dev));
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const double2* table = nullptr;
+    if (rope_base > 0.f) {
+        attn_status st = rope_table64(dev, static_cast<double>(rope_base), D, max_blocks_per_seq * page_size, &table);
+        if (st != ATTN_OK) return st;
+    }
+    attn_status st = ATTN_OK;
+    if (k_new != nullptr) {
+        st = D == 64 ? launch_append<64>(k_new, v_new, k_pages, v_pages, block_table, seq_lens, num_seqs, q_len,
+                                         max_blocks_per_seq, num_pages, Hkv, table, s)
+                     : launch_append<128>(k_new, v_new, k_pages, v_pages, block_table, seq_lens, num_seqs, q_len,
+                                          max_blocks_per_seq, num_pages, Hkv, table, s);
+        if (st != ATTN_OK) return st;
+    }
+    if (D == 64)
+        return launch_decode<64>(q, k_pages, v_pages, block_table, seq_lens, num_seqs, q_len, max_blocks_per_seq,
+                                 num_pages, Hq, Hkv, scale, table, o, lse, workspace, s, dev);
+    return launch_decode<128>(q, k_pages, v_pages, block_table, seq_lens, num_seqs, q_len, max_blocks_per_seq,
+                              num_pages, Hq, Hkv, scale, table, o, lse, workspace, s, dev);
 }
 
 attn_status attn_get_device_status(void* stream, int* flags_out) {

@@ -20,9 +20,17 @@
 // contiguous 16 x D blocks; a 128-byte swizzle makes the ldmatrix reads conflict-free). The G
 // query heads form the M rows of 16x8x16 bf16 tensor-core products (this path is HBM-bound,
 // so the small MMA is not the limit): S = q K^T per page, then O += P V.
+//
+// A decode step may bring T >= 1 new tokens per sequence (multi-token decode: the last T rows of
+// causal attention over the sequence). Their G*T query rows (G heads x T tokens) are cut into
+// 16-row tiles, one tile per CTA, and row (t, head) sees the cached tokens up to its position
+// len - T + t. With a RoPE table, each query row is rotated at its position as it is loaded. A
+// separate append kernel writes the new tokens' keys (rotated) and values into their page slots
+// before the split kernel reads the cache.
 #pragma once
 #include "common.cuh"
 #include "ptx.cuh"
+#include "rope.cuh"
 
 namespace attn {
 
@@ -32,15 +40,31 @@ constexpr int kDecodeWarps = 4;
 constexpr int kDecodeThreads = kDecodeWarps * 32;
 
 struct DecodeParams {
-    const __nv_bfloat16* q;      // [S, Hq, D], already rotated
+    const __nv_bfloat16* q;      // [S, T, Hq, D]; rotated here when rope != nullptr
     const int32_t* block_table;  // [S, max_blocks]
-    const int32_t* seq_lens;     // [S]
-    __nv_bfloat16* o;            // [S, Hq, D]
-    float* lse;                  // [S, Hq] or nullptr
-    float* ws_o;                 // [S, Hq, max_chunks, D] unnormalised partial outputs
-    float* ws_ml;                // [S, Hq, max_chunks, 2] partial (max in log2 units, sum)
+    const int32_t* seq_lens;     // [S], counting the T new tokens
+    __nv_bfloat16* o;            // [S, T, Hq, D]
+    float* lse;                  // [S, T, Hq] or nullptr
+    float* ws_o;                 // [S, T*Hq, max_chunks, D] unnormalised partial outputs
+    float* ws_ml;                // [S, T*Hq, max_chunks, 2] partial (max in log2 units, sum)
+    const double2* rope;         // (cos, sin) per (position, pair), fp64, or nullptr
     int S, Hq, Hkv, G, max_blocks, num_pages, max_chunks;
+    int T, mtiles;               // new tokens per sequence; 16-row tiles per KV head = ceil(G*T / 16)
     float scale_log2;
+};
+
+// Append of the T new tokens of every sequence: token t of sequence s sits at position
+// pos = len - T + t, in page block_table[s][pos / page_size], slot pos % page_size. Its key is
+// rotated at pos (when a table is given) and rounded to bf16; its value is copied.
+struct AppendParams {
+    const __nv_bfloat16* k_new;  // [S, T, Hkv, D]
+    const __nv_bfloat16* v_new;  // [S, T, Hkv, D]
+    __nv_bfloat16* k_pages;      // [num_pages, Hkv, page_size, D]
+    __nv_bfloat16* v_pages;
+    const int32_t* block_table;
+    const int32_t* seq_lens;
+    const double2* rope;
+    int S, T, Hkv, max_blocks, num_pages;
 };
 
 template <int D>
@@ -80,7 +104,9 @@ __device__ __forceinline__ uint32_t slab_off(int row, int chunk) {
     return (chunk >> 3) * (kPageSize * 128) + row * 128 + (((chunk & 7) ^ (row & 7)) << 4);
 }
 
-template <int D>
+// kStep = false: one token per sequence, q as given (the plain decode); true: the decode step's
+// general form (T tokens, per-row causal limits, optional rotation of q).
+template <int D, bool kStep>
 __global__ void __launch_bounds__(kDecodeThreads)
     decode_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                         const DecodeParams p) {
@@ -91,11 +117,13 @@ __global__ void __launch_bounds__(kDecodeThreads)
     int* abort_ptr = reinterpret_cast<int*>(full + kDecodeWarps * C::STAGES);
     volatile int* abort_flag = abort_ptr;
 
-    const int chunk = blockIdx.x, g = blockIdx.y, s = blockIdx.z;
+    const int chunk = blockIdx.x, s = blockIdx.z;
+    const int g = kStep ? blockIdx.y / p.mtiles : blockIdx.y, mt = kStep ? blockIdx.y % p.mtiles : 0;
+    const int T = kStep ? p.T : 1;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int len = p.seq_lens[s];
-    if (len < 1 || len > p.max_blocks * kPageSize) {
-        if (chunk == 0 && g == 0 && threadIdx.x == 0) raise_status(kStatusBadSeqLen);
+    if (len < T || len > p.max_blocks * kPageSize) {
+        if (chunk == 0 && blockIdx.y == 0 && threadIdx.x == 0) raise_status(kStatusBadSeqLen);
         return;
     }
     const int n_pages = (len + kPageSize - 1) / kPageSize;
@@ -145,18 +173,36 @@ __global__ void __launch_bounds__(kDecodeThreads)
         return valid;
     };
 
-    // Q fragments (A operand, rows = the G query heads of this KV head, zero-padded to 16).
+    // Q fragments (A operand). Row r of this CTA's tile is query row mt*16 + r = t*G + head of the
+    // KV head's G*T rows; rows past G*T are zero. lim: the last position the row sees (padding rows
+    // see the whole sequence, so their scores stay finite).
     const int rowA = lane >> 2, colA = 2 * (lane & 3);
     uint32_t qa[D / 16][4];
+    int lim[2];
     {
-        const __nv_bfloat16* qbase = p.q + (static_cast<size_t>(s) * p.Hq + g * p.G) * D;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-            const int d0 = kk * 16 + colA;
-            qa[kk][0] = rowA < p.G ? *reinterpret_cast<const uint32_t*>(qbase + rowA * D + d0) : 0u;
-            qa[kk][1] = rowA + 8 < p.G ? *reinterpret_cast<const uint32_t*>(qbase + (rowA + 8) * D + d0) : 0u;
-            qa[kk][2] = rowA < p.G ? *reinterpret_cast<const uint32_t*>(qbase + rowA * D + d0 + 8) : 0u;
-            qa[kk][3] = rowA + 8 < p.G ? *reinterpret_cast<const uint32_t*>(qbase + (rowA + 8) * D + d0 + 8) : 0u;
+        for (int hr = 0; hr < 2; ++hr) {
+            const int R = mt * 16 + rowA + 8 * hr;
+            const bool live = R < p.G * T;
+            const int t = kStep ? (live ? R / p.G : T - 1) : 0;
+            const int pos = len - T + t;
+            lim[hr] = pos;
+            const __nv_bfloat16* qrow =
+                p.q + ((static_cast<size_t>(s) * T + t) * p.Hq + g * p.G + (kStep ? R % p.G : R)) * D;
+            const double2* cs = kStep && p.rope != nullptr ? p.rope + static_cast<size_t>(pos) * (D / 2) : nullptr;
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    const int d0 = kk * 16 + colA + 8 * half;
+                    uint32_t w = live ? *reinterpret_cast<const uint32_t*>(qrow + d0) : 0u;
+                    if (cs != nullptr && live) {
+                        const double2 c = __ldg(cs + d0 / 2);
+                        w = rope_rotate_pair(w, c.x, c.y);
+                    }
+                    qa[kk][hr + 2 * half] = w;
+                }
+            }
         }
     }
 
@@ -202,13 +248,15 @@ __global__ void __launch_bounds__(kDecodeThreads)
             float mx[2];
 #pragma unroll
             for (int hr = 0; hr < 2; ++hr) {
+                // last slot of this page the row sees (one token: the page's last valid slot)
+                const int last = kStep ? lim[hr] - pg * kPageSize : valid - 1;
 #pragma unroll
                 for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
                     for (int e = 0; e < 2; ++e) {
                         const int tok = nt * 8 + colA + e;
                         float v = sc[nt][2 * hr + e];
-                        v = tok < valid ? v : -INFINITY;  // select: NaN-poisoned slots never leak
+                        v = tok <= last ? v : -INFINITY;  // select: NaN-poisoned slots never leak
                         sc[nt][2 * hr + e] = v;
                     }
                 float t = fmaxf(fmaxf(sc[0][2 * hr], sc[0][2 * hr + 1]), fmaxf(sc[1][2 * hr], sc[1][2 * hr + 1]));
@@ -220,14 +268,17 @@ __global__ void __launch_bounds__(kDecodeThreads)
             uint32_t pa[4];
 #pragma unroll
             for (int hr = 0; hr < 2; ++hr) {
-                const float m_new = fmaxf(m[hr], mx[hr]);  // finite: every page has >= 1 valid token
-                alpha[hr] = ptx::ex2(m[hr] - m_new);
+                // -inf while the row has seen none of this warp's tokens (a later token of a
+                // multi-token step): exponents then use 0, giving p = 0 and alpha = 0
+                const float m_new = fmaxf(m[hr], mx[hr]);
+                const float m_use = (kStep && m_new == -INFINITY) ? 0.f : m_new;
+                alpha[hr] = ptx::ex2(m[hr] - m_use);
                 m[hr] = m_new;
                 float ps[4];
 #pragma unroll
                 for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-                    for (int e = 0; e < 2; ++e) ps[nt * 2 + e] = ptx::ex2(fmaf(sc[nt][2 * hr + e], p.scale_log2, -m_new));
+                    for (int e = 0; e < 2; ++e) ps[nt * 2 + e] = ptx::ex2(fmaf(sc[nt][2 * hr + e], p.scale_log2, -m_use));
                 l[hr] = l[hr] * alpha[hr] + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
                 pa[hr] = ptx::pack_bf16x2(ps[0], ps[1]);       // tokens colA, colA+1
                 pa[2 + hr] = ptx::pack_bf16x2(ps[2], ps[3]);   // tokens 8+colA, 8+colA+1
@@ -299,7 +350,8 @@ __global__ void __launch_bounds__(kDecodeThreads)
     }
     __syncthreads();
     if (!ok) return;
-    for (int idx = threadIdx.x; idx < p.G * D; idx += kDecodeThreads) {
+    const int rows_here = kStep ? min(16, p.G * T - mt * 16) : p.G;
+    for (int idx = threadIdx.x; idx < rows_here * D; idx += kDecodeThreads) {
         const int row = idx / D, d = idx % D;
         float M = -INFINITY;
 #pragma unroll
@@ -312,7 +364,9 @@ __global__ void __launch_bounds__(kDecodeThreads)
             acc += sw * co[(w * 16 + row) * D + d];
             lacc += sw * cl[w * 16 + row];
         }
-        const size_t prow = (static_cast<size_t>(s) * p.Hq + g * p.G + row) * p.max_chunks + chunk;
+        const int R = mt * 16 + row, t = kStep ? R / p.G : 0;
+        const size_t out_row = (static_cast<size_t>(s) * T + t) * p.Hq + g * p.G + (kStep ? R % p.G : R);
+        const size_t prow = out_row * p.max_chunks + chunk;
         p.ws_o[prow * D + d] = acc;
         if (d == 0) {
             p.ws_ml[prow * 2] = M;
@@ -321,24 +375,27 @@ __global__ void __launch_bounds__(kDecodeThreads)
     }
 }
 
-// Merge the chunk partials of every (sequence, head) in ascending chunk order:
+// Merge the chunk partials of every (sequence, token, head) row in ascending chunk order:
 // M = max m_c, L = sum 2^(m_c - M) l_c, O = sum 2^(m_c - M) o_c / L, LSE = (M + log2 L) ln 2.
+// Chunks a row sees none of carry m_c = -inf and weigh 0.
 template <int D>
 __global__ void __launch_bounds__(128) decode_merge_kernel(const DecodeParams p) {
-    const int warp_global = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const long long warp_global = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
-    if (warp_global >= p.S * p.Hq) return;
-    const int s = warp_global / p.Hq, h = warp_global % p.Hq;
+    const long long rows_per_seq = static_cast<long long>(p.T) * p.Hq;
+    if (warp_global >= p.S * rows_per_seq) return;
+    const int s = static_cast<int>(warp_global / rows_per_seq);
+    const size_t out_row = static_cast<size_t>(warp_global);
     const int len = p.seq_lens[s];
     constexpr int PER = D / 32;
-    __nv_bfloat16* orow = p.o + (static_cast<size_t>(s) * p.Hq + h) * D;
-    if (len < 1 || len > p.max_blocks * kPageSize) {  // flagged by the split kernel
+    __nv_bfloat16* orow = p.o + out_row * D;
+    if (len < p.T || len > p.max_blocks * kPageSize) {  // flagged by the split kernel
         for (int e = 0; e < PER; ++e) orow[lane * PER + e] = __float2bfloat16(__int_as_float(0x7fc00000));
-        if (p.lse != nullptr && lane == 0) p.lse[static_cast<size_t>(s) * p.Hq + h] = __int_as_float(0x7fc00000);
+        if (p.lse != nullptr && lane == 0) p.lse[out_row] = __int_as_float(0x7fc00000);
         return;
     }
     const int n_chunks = (len + kChunkPages * kPageSize - 1) / (kChunkPages * kPageSize);
-    const size_t base = (static_cast<size_t>(s) * p.Hq + h) * p.max_chunks;
+    const size_t base = out_row * p.max_chunks;
     float M = -INFINITY;
     for (int c = 0; c < n_chunks; ++c) M = fmaxf(M, p.ws_ml[(base + c) * 2]);
     float acc[PER];
@@ -356,8 +413,48 @@ __global__ void __launch_bounds__(128) decode_merge_kernel(const DecodeParams p)
     const float inv = L > 0.f ? 1.f / L : 0.f;
 #pragma unroll
     for (int e = 0; e < PER; ++e) orow[lane * PER + e] = __float2bfloat16_rn(acc[e] * inv);
-    if (p.lse != nullptr && lane == 0)
-        p.lse[static_cast<size_t>(s) * p.Hq + h] = L > 0.f ? (M + ptx::lg2(L)) * kLn2 : -INFINITY;
+    if (p.lse != nullptr && lane == 0) p.lse[out_row] = L > 0.f ? (M + ptx::lg2(L)) * kLn2 : -INFINITY;
+}
+
+// One warp per (sequence, new token, KV head): each lane moves D/64 bf16 pairs of the key (rotated
+// at the token's position when a table is given) and of the value into the token's page slot. An
+// invalid length or block-table entry raises a status bit and writes nothing.
+template <int D>
+__global__ void __launch_bounds__(128) decode_append_kernel(const AppendParams a) {
+    const long long w = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (w >= static_cast<long long>(a.S) * a.T * a.Hkv) return;
+    const int g = static_cast<int>(w % a.Hkv);
+    const long long st = w / a.Hkv;
+    const int t = static_cast<int>(st % a.T), s = static_cast<int>(st / a.T);
+    const int len = a.seq_lens[s];
+    if (len < a.T || len > a.max_blocks * kPageSize) {
+        if (lane == 0) raise_status(kStatusBadSeqLen);
+        return;
+    }
+    const int pos = len - a.T + t;
+    const int page = a.block_table[static_cast<size_t>(s) * a.max_blocks + pos / kPageSize];
+    if (page < 0 || page >= a.num_pages) {
+        if (lane == 0) raise_status(kStatusBadPage);
+        return;
+    }
+    const size_t src = static_cast<size_t>(w) * D;
+    const size_t dst = ((static_cast<size_t>(page) * a.Hkv + g) * kPageSize + pos % kPageSize) * D;
+    const uint32_t* ks = reinterpret_cast<const uint32_t*>(a.k_new + src);
+    const uint32_t* vs = reinterpret_cast<const uint32_t*>(a.v_new + src);
+    uint32_t* kd = reinterpret_cast<uint32_t*>(a.k_pages + dst);
+    uint32_t* vd = reinterpret_cast<uint32_t*>(a.v_pages + dst);
+    const double2* cs = a.rope != nullptr ? a.rope + static_cast<size_t>(pos) * (D / 2) : nullptr;
+#pragma unroll
+    for (int i = lane; i < D / 2; i += 32) {
+        uint32_t kw = ks[i];
+        if (cs != nullptr) {
+            const double2 c = __ldg(cs + i);
+            kw = rope_rotate_pair(kw, c.x, c.y);
+        }
+        kd[i] = kw;
+        vd[i] = vs[i];
+    }
 }
 
 }  // namespace attn

@@ -14,12 +14,26 @@
 
 namespace attn {
 
-// k, k_rot: [rows, D] bf16 with row r at position r % N; cs: [>= N, D/2] (cos, sin) float2.
+// One interleaved pair (x0 in the low half, x1 in the high half of a bf16x2 word) rotated by the
+// angle whose (cos, sin) is given: x0 cos - x1 sin and x0 sin + x1 cos, each product and the sum
+// rounded once in fp64 (no fused multiply-add), then rounded to bf16 (nearest even). With the
+// fp64 cos/sin of the host-built table this is the rotation rounded exactly as an fp64 reference
+// computes it, so rotated operands carry no fp32 rotation error.
+__device__ __forceinline__ uint32_t rope_rotate_pair(uint32_t w, double cth, double sth) {
+    const double x0 = static_cast<double>(ptx::bf16lo_to_f32(w)), x1 = static_cast<double>(ptx::bf16hi_to_f32(w));
+    const double y0 = __dsub_rn(__dmul_rn(x0, cth), __dmul_rn(x1, sth));
+    const double y1 = __dadd_rn(__dmul_rn(x0, sth), __dmul_rn(x1, cth));
+    const uint32_t lo = __bfloat16_as_ushort(__double2bfloat16(y0));
+    const uint32_t hi = __bfloat16_as_ushort(__double2bfloat16(y1));
+    return lo | (hi << 16);
+}
+
+// k, k_rot: [rows, D] bf16 with row r at position r % N; cs: [>= N, D/2] (cos, sin) in fp64.
 // Each thread handles 16-byte chunks (4 pairs); consecutive threads take consecutive chunks, so
 // loads and stores are fully coalesced.
 template <int D>
 __global__ void __launch_bounds__(256) rope_rotate_rows_kernel(const uint4* __restrict__ k, uint4* __restrict__ k_rot,
-                                                               const float2* __restrict__ cs, long long rows, int N) {
+                                                               const double2* __restrict__ cs, long long rows, int N) {
     constexpr int CHUNKS = D / 8;
     const long long total = rows * CHUNKS;
     for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
@@ -28,15 +42,12 @@ __global__ void __launch_bounds__(256) rope_rotate_rows_kernel(const uint4* __re
         const int c = static_cast<int>(idx % CHUNKS);
         const int pos = static_cast<int>(row % N);
         uint4 w = __ldg(k + idx);
-        const float4* t = reinterpret_cast<const float4*>(cs + static_cast<size_t>(pos) * (D / 2) + c * 4);
-        const float4 a = __ldg(t), b = __ldg(t + 1);
-        const float csv[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+        const double2* t = cs + static_cast<size_t>(pos) * (D / 2) + c * 4;
         uint32_t* wv = reinterpret_cast<uint32_t*>(&w);
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-            const float x0 = ptx::bf16lo_to_f32(wv[e]), x1 = ptx::bf16hi_to_f32(wv[e]);
-            const float cth = csv[2 * e], sth = csv[2 * e + 1];
-            wv[e] = ptx::pack_bf16x2(fmaf(x0, cth, -x1 * sth), fmaf(x0, sth, x1 * cth));
+            const double2 a = __ldg(t + e);
+            wv[e] = rope_rotate_pair(wv[e], a.x, a.y);
         }
         k_rot[idx] = w;
     }

@@ -152,6 +152,53 @@ attn_status attn_decode_paged(const void* q, const void* k_pages, const void* v_
                               void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * attn_decode_step_workspace_size -- bytes of device workspace attn_decode_step needs: fp32 partial
+ * outputs and (max, sum) per (sequence, new token, query head, 512-token chunk), rounded up to
+ * 256 bytes. 0 for invalid sizes.
+ */
+size_t attn_decode_step_workspace_size(int num_seqs, int q_len, int max_blocks_per_seq, int page_size, int Hq, int D);
+
+/*
+ * attn_decode_step -- a decode step that brings q_len new tokens per sequence: it appends their
+ * keys and values to the paged cache, then attends with their queries.
+ *
+ * The new tokens of sequence s sit at positions seq_lens[s]-q_len .. seq_lens[s]-1 (seq_lens
+ * count them). With rope_base > 0, every new query and key is rotated at its position, on
+ * interleaved pairs (2i, 2i+1) by pos * rope_base^(-2i/D) ("attention-transformers", Q "How does
+ * Rotary Position Embedding (RoPE) work?"), in fp32 and rounded to bf16; values are never rotated.
+ * 1. Append (when k_new is given): new token t's rotated key and its value go to page
+ *    block_table[s][pos / page_size], slot pos % page_size ("Self-Attention Complexity,
+ *    FlashAttention, PagedAttention, and RoPE in Code", Part 3: the cache grows one block-table
+ *    slot at a time). k_new == NULL: the cache already holds the new tokens.
+ * 2. Attend: new token t's queries attend causally to cached tokens 0..pos -- the last q_len rows of
+ *    causal attention over the sequence (multi-token decode; q_len = 1 is one-token decode), with
+ *    the split-and-merge of attn_decode_paged.
+ *
+ *   q            bf16 [num_seqs, q_len, Hq, D] device, not rotated (rotated here if rope_base > 0)
+ *   k_new, v_new bf16 [num_seqs, q_len, Hkv, D] device, or both NULL; k_new not rotated
+ *   k_pages,
+ *   v_pages      bf16 [num_pages, Hkv, page_size, D] device; the new tokens' slots are written.
+ *                Slots written by two sequences in one call are the caller's error.
+ *   block_table, seq_lens   as attn_decode_paged, with seq_lens[s] in [q_len, max_blocks_per_seq * page_size]
+ *   rope_base    > 0: RoPE base; <= 0: no rotation (q and k_new are used as given)
+ *   o            bf16 [num_seqs, q_len, Hq, D] device, written
+ *   lse          fp32 [num_seqs, q_len, Hq] device, written (natural log), or NULL
+ *   workspace    device scratch of at least attn_decode_step_workspace_size(...) bytes, 16-byte
+ *                aligned, owned by the caller; overwritten; overlapping calls need their own.
+ *   scale        >0 softmax scale, <=0: 1/sqrt(D)
+ * Constraints as attn_decode_paged, plus 1 <= q_len <= 64 (else ATTN_ERR_UNSUPPORTED above 64) and
+ * Hkv * ceil(q_len * Hq / Hkv / 16) <= 65535. Bad block-table entries or lengths set device status
+ * bits (see attn_get_device_status); the tokens concerned are not written.
+ * The RoPE table covers positions up to max_blocks_per_seq * page_size and is cached per (device,
+ * base, D); its first build synchronises the device.
+ */
+attn_status attn_decode_step(const void* q, const void* k_new, const void* v_new, void* k_pages, void* v_pages,
+                             const int32_t* block_table, const int32_t* seq_lens, int num_seqs, int q_len,
+                             int max_blocks_per_seq, int num_pages, int page_size, int Hq, int Hkv, int D,
+                             float rope_base, float scale, void* o, float* lse, void* workspace,
+                             size_t workspace_bytes, void* stream);
+
+/*
  * attn_decode_paged_noalloc -- attn_decode_paged for callers that cannot allocate device memory.
  * The pages have no counterpart to this entry point; it exists for callers that cannot call
  * cudaMalloc when they call in -- for example a plugin inside a framework that owns the device's

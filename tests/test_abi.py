@@ -84,5 +84,26 @@ def test_workspace_size(api):
     assert api.decode_workspace_size(0, 1, 16, 1, 64) == 0
 
 
+def _step(api, q_len=2, Hq=8, Hkv=2, D=128, k_new=FAKE, v_new=FAKE, ws_bytes=None, rope=0.0):
+    if ws_bytes is None:
+        ws_bytes = api.decode_step_workspace_size(2, q_len, 8, 16, Hq, D)
+    return api.lib.attn_decode_step(FAKE, k_new, v_new, FAKE, FAKE, FAKE, FAKE, 2, q_len, 8, 16, 16, Hq, Hkv, D,
+                                    rope, 0.0, FAKE, None, FAKE, ws_bytes, None)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(q_len=0), 1), (dict(k_new=None), 1), (dict(v_new=MISALIGNED), 1), (dict(ws_bytes=16), 1),
+    (dict(rope=float("nan")), 1), (dict(q_len=65), 2), (dict(D=96), 2), (dict(Hq=34, Hkv=2), 2),
+])
+def test_decode_step_validation(api, kw, expect):
+    assert _step(api, **kw) == expect
+
+
+def test_decode_step_workspace_size(api):
+    assert api.decode_step_workspace_size(64, 4, 1024, 16, 32, 128) == 64 * 4 * 32 * 32 * 130 * 4
+    assert api.decode_step_workspace_size(64, 1, 1024, 16, 32, 128) == api.decode_workspace_size(64, 1024, 16, 32, 128)
+    assert api.decode_step_workspace_size(1, 0, 1, 16, 1, 64) == 0
+
+
 def test_device_status_needs_out_pointer(api):
     assert api.lib.attn_get_device_status(None, None) == 1
