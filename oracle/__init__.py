@@ -42,6 +42,11 @@ def _declare(lib):
     lib.oracle_decode_step.argtypes = [p, p, p, p, p, p, p, i32, i32, i32, i32, i32, i32, i32, i32, f64, f64, p,
                                        p, i32]
     lib.oracle_decode_step.restype = i32
+    lib.oracle_rope_bf16_ex.argtypes = [p, p, i64, i32, f64, i32, f64, f64, p]
+    lib.oracle_rope_bf16_ex.restype = i32
+    lib.oracle_attention_pos.argtypes = [p, p, p, i32, i32, i32, i32, i32, i32, i32, f64, i32, f64, f64, p, f64, p,
+                                         i64, p, p, i32]
+    lib.oracle_attention_pos.restype = i32
     lib.oracle_rope_bf16.argtypes = [p, p, i64, i32, f64, p]
     lib.oracle_rope_bf16.restype = i32
     lib.oracle_round_bf16_array.argtypes = [p, i64, p]
@@ -227,6 +232,57 @@ def decode_step(q, k_new, v_new, k_pages, v_pages, block_table, seq_lens, rope_b
     if st != 0:
         raise OracleError("oracle_decode_step failed with status %d" % st)
     return o, lse, kp, vp
+
+
+def attention_pos(q, k, v, causal=False, window=0, rope_base=0.0, rope_half_split=False, rope_pos_scale=1.0,
+                  rope_ntk_factor=1.0, alibi_slopes=None, scale=None, rows=None, nthreads=0, lib=None):
+    """Exact attention in fp64 with position variants: half-split RoPE pairing, Position
+    Interpolation (positions divided by rope_pos_scale), NTK-aware base scaling (base times
+    rope_ntk_factor^(D/(D-2))), and ALiBi (alibi_slopes: per-query-head slopes m_h, logits minus
+    m_h (i - j)). Shapes and returns as ``attention``."""
+    lib = lib or _lib()
+    q, k, v = _bits(q), _bits(k), _bits(v)
+    B, Hq, N, D = q.shape
+    Hkv = k.shape[1]
+    if k.shape != (B, Hkv, N, D) or v.shape != k.shape:
+        raise ValueError("k/v shape mismatch")
+    if scale is None:
+        scale = 1.0 / np.sqrt(D)
+    slopes = None if alibi_slopes is None else np.ascontiguousarray(alibi_slopes, dtype=np.float64)
+    if slopes is not None and slopes.shape != (Hq,):
+        raise ValueError("alibi_slopes must have Hq entries")
+    if rows is None:
+        n = B * Hq * N
+        rws = None
+    else:
+        rws = np.ascontiguousarray(rows, dtype=np.int64)
+        n = rws.shape[0]
+    o = np.empty((n, D), dtype=np.float64)
+    lse = np.empty((n,), dtype=np.float64)
+    st = lib.oracle_attention_pos(_ptr(q), _ptr(k), _ptr(v), B, Hq, Hkv, N, D, int(causal), int(window),
+                                  float(rope_base), int(bool(rope_half_split)), float(rope_pos_scale),
+                                  float(rope_ntk_factor), _ptr(slopes), float(scale), _ptr(rws), n, _ptr(o), _ptr(lse),
+                                  int(nthreads))
+    if st != 0:
+        raise OracleError("oracle_attention_pos failed with status %d" % st)
+    if rows is None:
+        return o.reshape(B, Hq, N, D), lse.reshape(B, Hq, N)
+    return o, lse
+
+
+def rope_bf16_ex(x, pos, base, half_split=False, pos_scale=1.0, ntk_factor=1.0, lib=None):
+    """``rope_bf16`` with a choice of pairing ((2i, 2i+1) or (i, i + D/2)), Position Interpolation
+    and NTK-aware base scaling."""
+    lib = lib or _lib()
+    x = _bits(x)
+    n, D = x.shape
+    pos = np.ascontiguousarray(pos, dtype=np.int64)
+    out = np.empty_like(x)
+    st = lib.oracle_rope_bf16_ex(_ptr(x), _ptr(pos), n, D, float(base), int(bool(half_split)), float(pos_scale),
+                                 float(ntk_factor), _ptr(out))
+    if st != 0:
+        raise OracleError("oracle_rope_bf16_ex failed with status %d" % st)
+    return out
 
 
 def rope_bf16(x, pos, base, lib=None):

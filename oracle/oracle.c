@@ -26,6 +26,13 @@
  *     order ("Self-Attention Complexity, FlashAttention, PagedAttention, and RoPE in Code",
  *     Part 3: fixed-size blocks and block tables) and computes the single query row at the
  *     sequence's last position over all seq_len cached tokens.
+ *   - Position variants of the prefill: half-split RoPE pairs (i, i + D/2) instead of (2i, 2i+1)
+ *     (the pages' "each 2D subspace" allows either pairing); Position Interpolation divides
+ *     positions by a factor; NTK-aware scaling multiplies the base by factor^(D/(D-2)), which
+ *     leaves the highest frequency unchanged and divides the lowest by the factor
+ *     ("attention-transformers", Q "What are NTK-aware RoPE scaling and YaRN?"); ALiBi subtracts
+ *     m_h (i - j) from the logit of query i and key j, with a per-head slope m_h
+ *     ("attention-transformers", Q "How does ALiBi encode position?").
  *   - A decode step appends the new tokens first: their keys, rotated at their positions, and
  *     their values go into the slots the block table gives (same Part 3; the rotation of the
  *     RoPE question above), then each new token's query, rotated at its position, attends
@@ -100,6 +107,42 @@ static void rope_row(const uint16_t* x, int D, long pos, double base, double* ou
 }
 
 /* Exposed for the pins: rotate n_rows rows of length D; row r sits at position pos[r]. */
+/* RoPE with a choice of pairing and scaling: pairs (2i, 2i+1) (half_split = 0) or (i, i + D/2)
+ * (half_split = 1); the angle of pair i at position pos is (pos / pos_scale) * b^(-2i/D) with
+ * b = base * ntk_factor^(D/(D-2)). Rotated values are rounded to bf16. */
+static void rope_row_ex(const uint16_t* x, int D, long pos, double base, int half_split, double pos_scale,
+                        double ntk_factor, double* out) {
+    if (base <= 0.0) {
+        for (int d = 0; d < D; ++d) out[d] = bf16_value(x[d]);
+        return;
+    }
+    const double b = base * pow(ntk_factor, (double)D / (double)(D - 2));
+    for (int i = 0; i < D / 2; ++i) {
+        const double theta = pow(b, -2.0 * (double)i / (double)D);
+        const double angle = ((double)pos / pos_scale) * theta;
+        const double c = cos(angle), sn = sin(angle);
+        const int a0 = half_split ? i : 2 * i;
+        const int a1 = half_split ? i + D / 2 : 2 * i + 1;
+        const double x0 = bf16_value(x[a0]), x1 = bf16_value(x[a1]);
+        out[a0] = bf16_value(oracle_round_bf16(x0 * c - x1 * sn));
+        out[a1] = bf16_value(oracle_round_bf16(x0 * sn + x1 * c));
+    }
+}
+
+int oracle_rope_bf16_ex(const uint16_t* x, const int64_t* pos, int64_t n_rows, int D, double base, int half_split,
+                        double pos_scale, double ntk_factor, uint16_t* out) {
+    if (!x || !pos || !out || D <= 0 || (D % 2) != 0 || n_rows < 0 || !(pos_scale > 0.0) || !(ntk_factor > 0.0))
+        return ORACLE_ERR_ARG;
+    double* tmp = (double*)malloc(sizeof(double) * (size_t)D);
+    if (!tmp) return ORACLE_ERR_NOMEM;
+    for (int64_t r = 0; r < n_rows; ++r) {
+        rope_row_ex(x + r * D, D, (long)pos[r], base, half_split, pos_scale, ntk_factor, tmp);
+        for (int d = 0; d < D; ++d) out[r * D + d] = oracle_round_bf16(tmp[d]);
+    }
+    free(tmp);
+    return ORACLE_OK;
+}
+
 int oracle_rope_bf16(const uint16_t* x, const int64_t* pos, int64_t n_rows, int D, double base,
                      uint16_t* out) {
     if (!x || !pos || !out || D <= 0 || (D % 2) != 0 || n_rows < 0) return ORACLE_ERR_ARG;
@@ -116,8 +159,8 @@ int oracle_rope_bf16(const uint16_t* x, const int64_t* pos, int64_t n_rows, int 
 /* One query row against keys/values already converted to doubles.
  * q[D]; kk, vv: [N, D]; writes o[D] and *lse. Masked keys get score -inf. */
 static void attend_row(const double* q, const double* kk, const double* vv, int N, int D,
-                       long i, int causal, int window, double scale, double* s_row, double* o,
-                       double* lse) {
+                       long i, int causal, int window, double scale, double alibi_slope, double* s_row,
+                       double* o, double* lse) {
     for (int j = 0; j < N; ++j) {
         int visible = 1;
         if (causal && j > i) visible = 0;
@@ -129,6 +172,7 @@ static void attend_row(const double* q, const double* kk, const double* vv, int 
         double acc = 0.0;
         for (int d = 0; d < D; ++d) acc += q[d] * kk[(size_t)j * D + d];
         s_row[j] = acc * scale;
+        if (alibi_slope != 0.0) s_row[j] -= alibi_slope * (double)(i - j);
     }
     double m = -INFINITY;
     for (int j = 0; j < N; ++j)
@@ -159,11 +203,17 @@ static void attend_row(const double* q, const double* kk, const double* vv, int 
  * rows: NULL for every row, else n_rows flat row ids ((b*Hq + h)*N + i).
  * o: [n_rows, D] (or [B*Hq*N, D]); lse: [n_rows] (or [B*Hq*N]). Query i sits at position i.
  */
-int oracle_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, int B, int Hq,
-                     int Hkv, int N, int D, int causal, int window, double rope_base,
-                     double scale, const int64_t* rows, int64_t n_rows, double* o, double* lse,
-                     int nthreads) {
+/*
+ * Prefill attention with position variants: rope_half_split, rope_pos_scale, rope_ntk_factor as in
+ * rope_row_ex (0, 1, 1: the plain interleaved RoPE), alibi_slopes: NULL or [Hq] slopes m_h.
+ */
+int oracle_attention_pos(const uint16_t* q, const uint16_t* k, const uint16_t* v, int B, int Hq, int Hkv, int N,
+                         int D, int causal, int window, double rope_base, int rope_half_split, double rope_pos_scale,
+                         double rope_ntk_factor, const double* alibi_slopes, double scale, const int64_t* rows,
+                         int64_t n_rows, double* o, double* lse, int nthreads) {
     if (!q || !k || !v || !o || !lse) return ORACLE_ERR_ARG;
+    if (!(rope_pos_scale > 0.0) || !(rope_ntk_factor > 0.0)) return ORACLE_ERR_ARG;
+    const int plain_rope = !rope_half_split && rope_pos_scale == 1.0 && rope_ntk_factor == 1.0;
     if (B <= 0 || Hq <= 0 || Hkv <= 0 || N <= 0 || D <= 0 || Hq % Hkv != 0) return ORACLE_ERR_ARG;
     if (window > 0 && !causal) return ORACLE_ERR_ARG;
     if (rope_base > 0.0 && (D % 2) != 0) return ORACLE_ERR_ARG;
@@ -200,7 +250,11 @@ int oracle_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, in
             const size_t kv_off = ((size_t)b * Hkv + g) * (size_t)N * D;
 #pragma omp parallel for schedule(static)
             for (int j = 0; j < N; ++j) {
-                rope_row(k + kv_off + (size_t)j * D, D, j, rope_base, kk + (size_t)j * D);
+                if (plain_rope)
+                    rope_row(k + kv_off + (size_t)j * D, D, j, rope_base, kk + (size_t)j * D);
+                else
+                    rope_row_ex(k + kv_off + (size_t)j * D, D, j, rope_base, rope_half_split, rope_pos_scale,
+                                rope_ntk_factor, kk + (size_t)j * D);
                 for (int d = 0; d < D; ++d) vv[(size_t)j * D + d] = bf16_value(v[kv_off + (size_t)j * D + d]);
             }
 #pragma omp parallel
@@ -218,9 +272,13 @@ int oracle_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, in
                         int rh = (int)((id / N) % Hq);
                         long i = (long)(id % N);
                         if (rb != b || rh / G != g) continue;
-                        rope_row(q + (size_t)id * D, D, i, rope_base, qq);
-                        attend_row(qq, kk, vv, N, D, i, causal, window, scale, s_row,
-                                   o + (size_t)r * D, lse + r);
+                        if (plain_rope)
+                            rope_row(q + (size_t)id * D, D, i, rope_base, qq);
+                        else
+                            rope_row_ex(q + (size_t)id * D, D, i, rope_base, rope_half_split, rope_pos_scale,
+                                        rope_ntk_factor, qq);
+                        attend_row(qq, kk, vv, N, D, i, causal, window, scale,
+                                   alibi_slopes ? alibi_slopes[rh] : 0.0, s_row, o + (size_t)r * D, lse + r);
                     }
                 }
                 free(s_row);
@@ -231,6 +289,14 @@ int oracle_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, in
     free(kk);
     free(vv);
     return status;
+}
+
+int oracle_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, int B, int Hq,
+                     int Hkv, int N, int D, int causal, int window, double rope_base,
+                     double scale, const int64_t* rows, int64_t n_rows, double* o, double* lse,
+                     int nthreads) {
+    return oracle_attention_pos(q, k, v, B, Hq, Hkv, N, D, causal, window, rope_base, 0, 1.0, 1.0, NULL, scale,
+                                rows, n_rows, o, lse, nthreads);
 }
 
 /*
@@ -288,7 +354,7 @@ int oracle_decode_paged(const uint16_t* q, const uint16_t* k_pages, const uint16
                 int h = g * G + hh;
                 for (int d = 0; d < D; ++d) qq[d] = bf16_value(q[((size_t)s * Hq + h) * D + d]);
                 /* the query is the sequence's last token: position len-1, causal over the cache */
-                attend_row(qq, kk, vv, len, D, (long)len - 1, 1, 0, scale, s_row,
+                attend_row(qq, kk, vv, len, D, (long)len - 1, 1, 0, scale, 0.0, s_row,
                            o + ((size_t)s * Hq + h) * D, lse + (size_t)s * Hq + h);
             }
         }
@@ -379,7 +445,7 @@ int oracle_decode_step(const uint16_t* q, const uint16_t* k_new, const uint16_t*
                     int h = g * G + hh;
                     size_t row = ((size_t)s * T + t) * Hq + h;
                     rope_row(q + row * D, D, pos, rope_base, qq);
-                    attend_row(qq, kk, vv, len, D, pos, 1, 0, scale, s_row, o + row * D, lse + row);
+                    attend_row(qq, kk, vv, len, D, pos, 1, 0, scale, 0.0, s_row, o + row * D, lse + row);
                 }
             }
         }
@@ -466,7 +532,7 @@ int oracle_attention_f64(const double* q, const double* k, const double* v, int 
                 for (int i = 0; i < N; ++i) {
                     const size_t row = ((size_t)b * Hq + h) * N + i;
                     rope_row_f64(q + row * D, D, i, rope_base, 0, round_rotated, qq);
-                    attend_row(qq, kk, v + kv_off, N, D, i, causal, window, scale, s_row, o + row * D, lse + row);
+                    attend_row(qq, kk, v + kv_off, N, D, i, causal, window, scale, 0.0, s_row, o + row * D, lse + row);
                 }
             }
         }
@@ -543,7 +609,7 @@ int oracle_attention_bwd_f64(const double* q, const double* k, const double* v, 
                         const double* dO = dout + row * D;
                         double lse_i;
                         rope_row_f64(q + row * D, D, i, rope_base, 0, round_rotated, qq);
-                        attend_row(qq, kk, vv, N, D, i, causal, window, scale, s_row, o_row, &lse_i);
+                        attend_row(qq, kk, vv, N, D, i, causal, window, scale, 0.0, s_row, o_row, &lse_i);
                         /* attend_row leaves exp(s_ij - m_i) in s_row; P_ij is that over its row sum */
                         double lsum = 0.0;
                         for (int j = 0; j < N; ++j) lsum += s_row[j];

@@ -489,6 +489,100 @@ def check_decode_step_reduces_to_decode(lib):
     assert not np.all(np.isfinite(o))  # the unfilled NaN slot is read: the step does attend to it
 
 
+# ---------------------------------------------------------------------------------- position variants
+
+def check_rope_half_split_library(lib):
+    """Half-split pairing against the rotate-half formulation written with torch in float64:
+    x * [cos, cos] + rotate_half(x) * [sin, sin], rotate_half(x) = [-x2, x1]; then the pinned
+    bf16 rounding."""
+    D, base = 16, 10000.0
+    x = _rand((9, D), 41)
+    pos = np.array([0, 1, 2, 5, 17, 100, 999, 4096, 32767])
+    got = oracle.rope_bf16_ex(x, pos, base, half_split=True, lib=lib)
+    xt = torch.from_numpy(_f64(x))
+    theta = base ** (-2.0 * torch.arange(D // 2, dtype=torch.float64) / D)
+    ang = torch.from_numpy(pos.astype(np.float64))[:, None] * theta[None, :]
+    cos, sin = torch.cat([ang.cos(), ang.cos()], 1), torch.cat([ang.sin(), ang.sin()], 1)
+    rot = torch.cat([-xt[:, D // 2:], xt[:, :D // 2]], 1)
+    ref = oracle.round_bf16((xt * cos + rot * sin).numpy(), lib=lib)
+    assert np.array_equal(got, ref)
+    assert not np.array_equal(got, oracle.rope_bf16(x, pos, base, lib=lib))  # the pairing matters
+
+
+def check_rope_position_interpolation(lib):
+    """Position Interpolation divides positions: factor f at position f*k equals plain RoPE at k."""
+    x = _rand((6, 32), 42)
+    for f in (2.0, 4.0):
+        k = np.array([0, 1, 3, 10, 250, 4000])
+        got = oracle.rope_bf16_ex(x, (k * f).astype(np.int64), 10000.0, pos_scale=f, lib=lib)
+        assert np.array_equal(got, oracle.rope_bf16(x, k, 10000.0, lib=lib))
+
+
+def check_rope_ntk_frequencies(lib):
+    """NTK-aware scaling keeps the highest frequency (pair 0) and divides the lowest (pair D/2-1) by
+    the factor: pair 0 matches plain RoPE at any position, and the last pair at position f*p matches
+    plain RoPE at p (within one bf16 step: the two angles agree only up to fp64 rounding)."""
+    D, f = 32, 4.0
+    x = _rand((7, D), 43)
+    p = np.array([1, 2, 7, 33, 500, 1000, 3000])
+    ntk = oracle.rope_bf16_ex(x, p * 4, 10000.0, ntk_factor=f, lib=lib)
+    plain_same_pos = oracle.rope_bf16(x, p * 4, 10000.0, lib=lib)
+    assert np.array_equal(ntk[:, :2], plain_same_pos[:, :2])
+    plain = oracle.rope_bf16(x, p, 10000.0, lib=lib)
+    a, b = _f64(ntk[:, -2:]), _f64(plain[:, -2:])
+    assert np.all(np.abs(a - b) <= np.abs(b) * 2.0 ** -7 + 1e-12)
+    assert not np.array_equal(ntk[:, 2:-2], plain_same_pos[:, 2:-2])  # middle frequencies move
+
+
+def check_alibi_closed_form(lib):
+    """q = 0 leaves only the bias: row i weighs key j <= i by e^(-m (i - j)), so with V = identity
+    O_i[j] is that weight normalised and LSE_i = ln((1 - e^(-m (i+1))) / (1 - e^(-m)))."""
+    N, D, m = 12, 16, 0.375
+    q = np.zeros((1, 1, N, D), np.uint16)
+    k = _rand((1, 1, N, D), 44)
+    v = _to_bits(np.eye(N, D)[None, None])
+    o, lse = oracle.attention_pos(q, k, v, causal=True, alibi_slopes=[m], lib=lib)
+    for i in range(N):
+        w = np.exp(-m * (i - np.arange(i + 1)))
+        assert np.abs(o[0, 0, i, :i + 1] - w / w.sum()).max() < 1e-14
+        assert np.abs(o[0, 0, i, i + 1:]).max() == 0.0
+        assert abs(lse[0, 0, i] - math.log((1 - math.exp(-m * (i + 1))) / (1 - math.exp(-m)))) < 1e-13
+
+
+def check_alibi_library(lib):
+    """ALiBi with GQA and RoPE against torch float64 SDPA given the bias -m_h (i - j) as a float mask."""
+    B, Hq, Hkv, N, D = 1, 4, 2, 20, 8
+    q, k, v = _rand((B, Hq, N, D), 45), _rand((B, Hkv, N, D), 46), _rand((B, Hkv, N, D), 47)
+    slopes = np.array([0.5, 0.25, 0.125, 0.0625])
+    base = 100.0
+    o, _ = oracle.attention_pos(q, k, v, causal=True, rope_base=base, alibi_slopes=slopes, lib=lib)
+    pos = np.arange(N)
+    qr = np.stack([oracle.rope_bf16(q[0, h], pos, base, lib=lib) for h in range(Hq)])[None]
+    kr = np.stack([oracle.rope_bf16(k[0, g], pos, base, lib=lib) for g in range(Hkv)])[None]
+    i, j = np.meshgrid(pos, pos, indexing="ij")
+    bias = np.where(j <= i, -slopes[:, None, None] * (i - j)[None], -np.inf)[None]
+    ref = _sdpa64(qr, kr, v, D ** -0.5, mask=torch.from_numpy(bias), gqa=True)
+    assert np.abs(o - ref).max() < 1e-12
+
+
+def check_position_variants_combined(lib):
+    """Half-split pairing, both scalings and ALiBi together reduce to the plain oracle when the
+    variants are neutral, and the half-split result equals interleaved RoPE on dimensions
+    permuted so that (i, i + D/2) become (2i, 2i+1) -- a score is unchanged by permuting the
+    dimensions of q and k alike."""
+    B, Hq, Hkv, N, D = 1, 2, 1, 24, 16
+    q, k, v = _rand((B, Hq, N, D), 48), _rand((B, Hkv, N, D), 49), _rand((B, Hkv, N, D), 50)
+    o1, l1 = oracle.attention_pos(q, k, v, causal=True, rope_base=500.0, lib=lib)
+    o2, l2 = oracle.attention(q, k, v, causal=True, rope_base=500.0, lib=lib)
+    assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
+    perm = np.stack([np.arange(D // 2), np.arange(D // 2) + D // 2], 1).reshape(-1)
+    oh, lh = oracle.attention_pos(q, k, v, causal=True, rope_base=500.0, rope_half_split=True, rope_pos_scale=2.0,
+                                  rope_ntk_factor=3.0, lib=lib)
+    op, lp = oracle.attention_pos(np.ascontiguousarray(q[..., perm]), np.ascontiguousarray(k[..., perm]), v,
+                                  causal=True, rope_base=500.0, rope_pos_scale=2.0, rope_ntk_factor=3.0, lib=lib)
+    assert np.abs(oh - op).max() < 1e-12 and np.abs(lh - lp).max() < 1e-12
+
+
 ALL_CHECKS = [
     check_round_bf16_golden, check_round_bf16_matches_torch, check_rope_golden,
     check_rope_matches_sinusoid, check_rope_norm_and_identity, check_rope_relative,
@@ -498,7 +592,8 @@ ALL_CHECKS = [
     check_rows_subset, check_online_recurrence, check_decode_is_last_prefill_row,
     check_decode_library, check_decode_paging_invariance, check_decode_step_append_slots,
     check_decode_step_is_last_prefill_rows, check_decode_step_prefill_with_rope, check_decode_step_library,
-    check_decode_step_reduces_to_decode,
+    check_decode_step_reduces_to_decode, check_rope_half_split_library, check_rope_position_interpolation,
+    check_rope_ntk_frequencies, check_alibi_closed_form, check_alibi_library, check_position_variants_combined,
 ]
 
 

@@ -28,8 +28,8 @@ MUTANTS = {
     "gqa_interleaved_heads": ("if (rb != b || rh / G != g) continue;", "if (rb != b || rh % Hkv != g) continue;"),
     "round_truncates": ("double r = nearbyint(ldexp(ax, -qexp));", "double r = floor(ldexp(ax, -qexp));"),
     "decode_slot_index": ("(size_t)(t % page_size)) * D;", "(size_t)((t + 1) % page_size)) * D;"),
-    "decode_query_position": ("attend_row(qq, kk, vv, len, D, (long)len - 1, 1, 0, scale, s_row,",
-                              "attend_row(qq, kk, vv, len, D, (long)len - 2, 1, 0, scale, s_row,"),
+    "decode_query_position": ("attend_row(qq, kk, vv, len, D, (long)len - 1, 1, 0, scale, 0.0, s_row,",
+                              "attend_row(qq, kk, vv, len, D, (long)len - 2, 1, 0, scale, 0.0, s_row,"),
     "bwd_no_row_correction": ("const double ds = p * (dp[j] - dsum);", "const double ds = p * dp[j];"),
     "bwd_dk_unscaled": ("my_dk[(size_t)j * D + d] += scale * ds * qq[d];", "my_dk[(size_t)j * D + d] += ds * qq[d];"),
     "bwd_dq_not_rotated_back": ("rope_row_f64(dqr, D, i, rope_base, 1, 0, dq + row * D);",
@@ -37,6 +37,12 @@ MUTANTS = {
     "step_query_position": ("long pos = (long)len - T + t;", "long pos = (long)len - T + t - (t > 0);"),
     "step_append_slot": ("long pos = (long)seq_lens[s] - T + t;", "long pos = (long)seq_lens[s] - T + t + (t == 0);"),
     "step_query_unrotated": ("rope_row(q + row * D, D, pos, rope_base, qq);", "rope_row(q + row * D, D, 0, rope_base, qq);"),
+    "alibi_sign": ("s_row[j] -= alibi_slope * (double)(i - j);", "s_row[j] += alibi_slope * (double)(i - j);"),
+    "half_split_partner": ("const int a1 = half_split ? i + D / 2 : 2 * i + 1;",
+                           "const int a1 = half_split ? D - 1 - i : 2 * i + 1;"),
+    "pi_multiplies": ("const double angle = ((double)pos / pos_scale) * theta;",
+                      "const double angle = ((double)pos * pos_scale) * theta;"),
+    "ntk_exponent": ("pow(ntk_factor, (double)D / (double)(D - 2))", "pow(ntk_factor, 1.0)"),
     "normaliser_missing": ("for (int d = 0; d < D; ++d) o[d] /= l;", "for (int d = 0; d < D; ++d) o[d] /= (l + 1e-3);"),
 }
 
