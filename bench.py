@@ -341,6 +341,35 @@ def run_ours(args, rank, world, local):
                "roofline": {"bound": "tensor", "achieved": round(bwd_flops / (bwd_ms / 1e3) / 1e12, 2),
                             "unit": "TFLOP/s", "note": "five-kernel call: rotation x2, prep, dK/dV, dQ"}}
 
+    # ---- position variants of the prefill workload (own loops; not part of the step)
+    variants = None
+    if do_prefill and args.variant_calls > 0:
+        variants = {}
+        slopes = synth.alibi_slopes(PREFILL.Hq).to(dev)
+        for name, kw in (("alibi", dict(alibi_slopes=slopes)),
+                         ("half_split_rope_ntk4", dict(rope_half_split=True, rope_ntk_factor=4.0))):
+            def variant_call():
+                api.attn_fwd_pos(q, k, v, causal=PREFILL.causal, window=PREFILL.window, rope_base=PREFILL.rope_base,
+                                 o=o, lse=lse, stream=stream, **kw)
+
+            for _ in range(args.warmup):
+                variant_call()
+            barrier(world)
+            torch.cuda.synchronize()
+            v0, v1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            v0.record(stream)
+            for _ in range(args.variant_calls):
+                variant_call()
+            v1.record(stream)
+            torch.cuda.synchronize()
+            if api.device_status() != 0:
+                raise RuntimeError("device status raised during the %s loop" % name)
+            vms = reduce_max(v0.elapsed_time(v1), world, dev) / args.variant_calls
+            variants[name] = {"value": round(job_throughput(flops, world, vms / 1e3) / 1e12, 2), "unit": "TFLOP/s",
+                              "ms_per_call": round(vms, 4), "calls": args.variant_calls,
+                              "roofline": {"bound": "tensor", "achieved": round(flops / (vms / 1e3) / 1e12, 2),
+                                           "unit": "TFLOP/s"}}
+
     # ---- end to end through the public API with pinned host buffers
     E = min(args.e2e_steps, K) if (args.e2e_steps > 0 and args.only == "all") else 0
     if E:
@@ -432,6 +461,10 @@ def run_ours(args, rank, world, local):
     if bwd is not None:
         bwd["roofline"].update({"peak": tensor_peak, "frac": round(bwd["roofline"]["achieved"] / tensor_peak, 4),
                                 "peak_kind": "%s bf16 GEMM, sustained" % peaks_kind})
+    if variants is not None:
+        for vv in variants.values():
+            vv["roofline"].update({"peak": tensor_peak, "frac": round(vv["roofline"]["achieved"] / tensor_peak, 4),
+                                   "peak_kind": "%s bf16 GEMM, sustained" % peaks_kind})
     line = {
         "metric": "attn fwd TFLOP/s (causal GQA prefill B2 Hq32 Hkv8 N8192 D128, RoPE 5e5) "
                   "& paged-decode KV GB/s",
@@ -475,6 +508,9 @@ def run_ours(args, rank, world, local):
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": (2 * do_prefill + 2 * do_decode) * K,
         "backward": bwd,
+        "position_variants": None if variants is None else dict(
+            {"metric": "attn fwd TFLOP/s of the same prefill workload with ALiBi (slopes 2^(-8h/H)), and with "
+                       "half-split RoPE pairing plus NTK-aware base scaling x4"}, **variants),
         "decode_step": None if steps_out is None else dict(
             {"metric": "decode step KV GB/s: append q_len new tokens per sequence (keys rotated, RoPE 1e4) into "
                        "the 64-sequence paged cache, then attend with their rotated queries"}, **steps_out),
@@ -557,6 +593,7 @@ def parse_args(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=10, help="0 skips the end-to-end leg")
     ap.add_argument("--bwd-steps", type=int, default=20, help="backward calls timed after the step loop; 0 skips")
     ap.add_argument("--step-calls", type=int, default=50, help="decode-step calls timed per q_len; 0 skips")
+    ap.add_argument("--variant-calls", type=int, default=20, help="position-variant prefill calls timed each; 0 skips")
     ap.add_argument("--only", choices=["all", "prefill", "decode"], default="all",
                     help="time one half of the step only (profiling runs); the JSON line is then partial")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle time for the CPU baseline")

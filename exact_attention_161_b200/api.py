@@ -27,6 +27,7 @@ DEVICE_TIMEOUT, DEVICE_BAD_PAGE, DEVICE_BAD_SEQLEN = 1, 2, 4
 _p, _i, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
 SIGNATURES = {
     "attn_fwd": (_i, [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _f, _f, _p]),
+    "attn_fwd_pos": (_i, [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _f, _i, _f, _f, _p, _f, _p]),
     "attn_bwd_workspace_size": (_sz, [_i, _i, _i, _i, _i, _f]),
     "attn_bwd": (_i, [_p, _p, _p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _f, _f, _p, _sz, _p]),
     "attn_decode_workspace_size": (_sz, [_i, _i, _i, _i, _i]),
@@ -113,6 +114,31 @@ def attn_fwd(q, k, v, causal=False, window=0, rope_base=0.0, scale=0.0, o=None, 
             _dev_tensor(lse, "lse", torch.float32) if lse is not None else None]
     _check(lib.attn_fwd(*args, B, Hq, Hkv, N, D, int(bool(causal)), int(window), float(rope_base), float(scale),
                         _stream(stream)))
+    return o, lse
+
+
+def attn_fwd_pos(q, k, v, causal=False, window=0, rope_base=0.0, rope_half_split=False, rope_pos_scale=1.0,
+                 rope_ntk_factor=1.0, alibi_slopes=None, scale=0.0, o=None, lse=None, want_lse=True, stream=None):
+    """attn_fwd with position variants: half-split RoPE pairing, Position Interpolation
+    (rope_pos_scale), NTK-aware base scaling (rope_ntk_factor) and ALiBi (alibi_slopes: fp32 [Hq]
+    CUDA tensor of per-head slopes, causal only). Returns (o, lse) as attn_fwd."""
+    B, Hq, N, D = q.shape
+    Hkv = k.shape[1]
+    if k.shape != (B, Hkv, N, D) or v.shape != k.shape:
+        raise ValueError("k and v must be [B, Hkv, N, D] with q [B, Hq, N, D]")
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device)
+    if alibi_slopes is not None and tuple(alibi_slopes.shape) != (Hq,):
+        raise ValueError("alibi_slopes must be [Hq]")
+    _check(lib.attn_fwd_pos(_dev_tensor(q, "q", torch.bfloat16), _dev_tensor(k, "k", torch.bfloat16),
+                            _dev_tensor(v, "v", torch.bfloat16), _dev_tensor(o, "o", torch.bfloat16),
+                            _dev_tensor(lse, "lse", torch.float32) if lse is not None else None, B, Hq, Hkv, N, D,
+                            int(causal), int(window), float(rope_base), int(bool(rope_half_split)),
+                            float(rope_pos_scale), float(rope_ntk_factor),
+                            _dev_tensor(alibi_slopes, "alibi_slopes", torch.float32) if alibi_slopes is not None
+                            else None, float(scale), _stream(stream)))
     return o, lse
 
 

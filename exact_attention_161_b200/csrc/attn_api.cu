@@ -87,17 +87,19 @@ struct DevBuf {
 };
 
 std::mutex g_cache_mu;
-// (device, base, D, fp64?) -> cos/sin table covering positions [0, capacity)
-std::map<std::tuple<int, double, int, bool>, std::pair<DevBuf, int>> g_rope_tables;
+// (device, base, D, position scale, NTK factor, fp64?) -> cos/sin table covering positions [0, capacity)
+std::map<std::tuple<int, double, int, double, double, bool>, std::pair<DevBuf, int>> g_rope_tables;
 // (device, stream) -> rotated-key scratch
 std::map<std::pair<int, void*>, DevBuf> g_key_scratch;
 std::vector<DevBuf> g_retired;  // outgrown buffers; a launch still queued may read them
 
-// (cos, sin) of pos * base^(-2i/D) for pos < n, i < D/2: angles and trigonometry in fp64, stored
-// as fp64 pairs (wide) or rounded to fp32 pairs.
-attn_status rope_table_any(int dev, double base, int D, int n, bool wide, const void** out) {
+// (cos, sin) of (pos / pos_scale) * b^(-2i/D), b = base * ntk^(D/(D-2)), for pos < n, i < D/2:
+// angles and trigonometry in fp64 (Position Interpolation divides the positions; NTK-aware scaling
+// raises the base), stored as fp64 pairs (wide) or rounded to fp32 pairs.
+attn_status rope_table_any(int dev, double base, int D, int n, double pos_scale, double ntk, bool wide,
+                           const void** out) {
     std::lock_guard<std::mutex> lock(g_cache_mu);
-    auto key = std::make_tuple(dev, base, D, wide);
+    auto key = std::make_tuple(dev, base, D, pos_scale, ntk, wide);
     auto it = g_rope_tables.find(key);
     if (it != g_rope_tables.end() && it->second.second >= n) {
         *out = it->second.first.ptr;
@@ -108,10 +110,11 @@ attn_status rope_table_any(int dev, double base, int D, int n, bool wide, const 
     std::vector<double2> host64(wide ? pairs : 0);
     std::vector<float2> host32(wide ? 0 : pairs);
     std::vector<double> theta(D / 2);
-    for (int i = 0; i < D / 2; ++i) theta[i] = std::pow(base, -2.0 * i / D);
+    const double b = base * std::pow(ntk, static_cast<double>(D) / static_cast<double>(D - 2));
+    for (int i = 0; i < D / 2; ++i) theta[i] = std::pow(b, -2.0 * static_cast<double>(i) / static_cast<double>(D));
     for (int pos = 0; pos < cap; ++pos)
         for (int i = 0; i < D / 2; ++i) {
-            const double a = pos * theta[i];
+            const double a = (static_cast<double>(pos) / pos_scale) * theta[i];
             const size_t at = static_cast<size_t>(pos) * (D / 2) + i;
             if (wide)
                 host64[at] = make_double2(std::cos(a), std::sin(a));
@@ -133,15 +136,17 @@ attn_status rope_table_any(int dev, double base, int D, int n, bool wide, const 
     *out = buf.ptr;
     return ATTN_OK;
 }
-attn_status rope_table(int dev, double base, int D, int n, const float2** out) {
+attn_status rope_table(int dev, double base, int D, int n, const float2** out, double pos_scale = 1.0,
+                       double ntk = 1.0) {
     const void* p = nullptr;
-    attn_status st = rope_table_any(dev, base, D, n, false, &p);
+    attn_status st = rope_table_any(dev, base, D, n, pos_scale, ntk, false, &p);
     *out = static_cast<const float2*>(p);
     return st;
 }
-attn_status rope_table64(int dev, double base, int D, int n, const double2** out) {
+attn_status rope_table64(int dev, double base, int D, int n, const double2** out, double pos_scale = 1.0,
+                         double ntk = 1.0) {
     const void* p = nullptr;
-    attn_status st = rope_table_any(dev, base, D, n, true, &p);
+    attn_status st = rope_table_any(dev, base, D, n, pos_scale, ntk, true, &p);
     *out = static_cast<const double2*>(p);
     return st;
 }
@@ -175,35 +180,48 @@ attn_status ensure_smem(K kernel, int bytes, int dev) {
     return ATTN_OK;
 }
 
+struct PosVariant {
+    int half_split = 0;
+    double pos_scale = 1.0, ntk = 1.0;
+    const float* alibi = nullptr;
+};
+
 template <int D>
 attn_status launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
-                       int N, int causal, int window, float rope_base, float scale, cudaStream_t stream, int dev) {
+                       int N, int causal, int window, float rope_base, float scale, cudaStream_t stream, int dev,
+                       const PosVariant& pv = PosVariant()) {
     using C = attn::FwdCfg<D>;
     const void* k_use = k;
     attn::FwdParams p{};
     if (rope_base > 0.f) {
         const float2* table = nullptr;
-        attn_status st = rope_table(dev, static_cast<double>(rope_base), D, N, &table);
+        attn_status st = rope_table(dev, static_cast<double>(rope_base), D, N, &table, pv.pos_scale, pv.ntk);
         if (st != ATTN_OK) return st;
         const double2* table64 = nullptr;
-        st = rope_table64(dev, static_cast<double>(rope_base), D, N, &table64);
+        st = rope_table64(dev, static_cast<double>(rope_base), D, N, &table64, pv.pos_scale, pv.ntk);
         if (st != ATTN_OK) return st;
         void* k_rot = nullptr;
         const size_t kbytes = static_cast<size_t>(B) * Hkv * N * D * 2;
         st = key_scratch(dev, stream, kbytes, &k_rot);
         if (st != ATTN_OK) return st;
         const long long rows = static_cast<long long>(B) * Hkv * N;
-        const long long chunks = rows * (D / 8);
+        const long long chunks = static_cast<long long>(N) * (D / 8);  // one thread per (position, chunk)
         int sms = 148;
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
         const long long want = (chunks + 255) / 256;
         const int grid = static_cast<int>(want < 8LL * sms ? want : 8LL * sms);
-        attn::rope_rotate_rows_kernel<D><<<grid, 256, 0, stream>>>(static_cast<const uint4*>(k),
-                                                                   static_cast<uint4*>(k_rot), table64, rows, N);
+        if (pv.half_split)
+            attn::rope_rotate_rows_kernel<D, true><<<grid, 256, 0, stream>>>(static_cast<const uint4*>(k),
+                                                                             static_cast<uint4*>(k_rot), table64, rows, N);
+        else
+            attn::rope_rotate_rows_kernel<D><<<grid, 256, 0, stream>>>(static_cast<const uint4*>(k),
+                                                                       static_cast<uint4*>(k_rot), table64, rows, N);
         CUDA_TRY(cudaGetLastError());
         k_use = k_rot;
         p.rope = table;
+        p.rope_half = pv.half_split;
     }
+    p.alibi = pv.alibi;
     CUtensorMap tq, tk, tv;
     attn_status st;
     if ((st = make_map_3d(&tq, q, D, N, static_cast<uint64_t>(B) * Hq, 128)) != ATTN_OK) return st;
@@ -220,11 +238,16 @@ attn_status launch_fwd(const void* q, const void* k, const void* v, void* o, flo
     p.scale_log2 = scale * attn::kLog2e;
     p.nblk = (N + C::QT * C::BM - 1) / (C::QT * C::BM);
     p.n_items = B * Hq * p.nblk;
-    if ((st = ensure_smem(attn::attn_fwd_kernel<D>, C::SMEM_BYTES, dev)) != ATTN_OK) return st;
     int sms = 148;
     CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
     const int grid = p.n_items < sms ? p.n_items : sms;  // persistent: one CTA per SM
-    attn::attn_fwd_kernel<D><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+    if (pv.alibi != nullptr) {
+        if ((st = ensure_smem(attn::attn_fwd_kernel<D, true>, C::SMEM_BYTES, dev)) != ATTN_OK) return st;
+        attn::attn_fwd_kernel<D, true><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+    } else {
+        if ((st = ensure_smem(attn::attn_fwd_kernel<D, false>, C::SMEM_BYTES, dev)) != ATTN_OK) return st;
+        attn::attn_fwd_kernel<D, false><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+    }
     CUDA_TRY(cudaGetLastError());
     return ATTN_OK;
 }
@@ -232,10 +255,13 @@ attn_status launch_fwd(const void* q, const void* k, const void* v, void* o, flo
 size_t decode_chunks(int max_blocks) { return (static_cast<size_t>(max_blocks) + attn::kChunkPages - 1) / attn::kChunkPages; }
 
 template <int D>
-attn_status launch_append(const void* k_new, const void* v_new, void* k_pages, void* v_pages,
-                          const int32_t* block_table, const int32_t* seq_lens, int S, int T, int max_blocks,
-                          int num_pages, int Hkv, const double2* rope, cudaStream_t stream) {
-    attn::AppendParams a{};
+attn_status launch_step_prep(const void* q, void* q_rot, const void* k_new, const void* v_new, void* k_pages,
+                             void* v_pages, const int32_t* block_table, const int32_t* seq_lens, int S, int T,
+                             int max_blocks, int num_pages, int Hq, int Hkv, const double2* rope,
+                             cudaStream_t stream) {
+    attn::StepPrepParams a{};
+    a.q = static_cast<const __nv_bfloat16*>(q);
+    a.q_rot = static_cast<__nv_bfloat16*>(q_rot);
     a.k_new = static_cast<const __nv_bfloat16*>(k_new);
     a.v_new = static_cast<const __nv_bfloat16*>(v_new);
     a.k_pages = static_cast<__nv_bfloat16*>(k_pages);
@@ -245,11 +271,13 @@ attn_status launch_append(const void* k_new, const void* v_new, void* k_pages, v
     a.rope = rope;
     a.S = S;
     a.T = T;
+    a.Hq = Hq;
     a.Hkv = Hkv;
     a.max_blocks = max_blocks;
     a.num_pages = num_pages;
-    const long long warps = static_cast<long long>(S) * T * Hkv;
-    attn::decode_append_kernel<D><<<static_cast<unsigned>((warps * 32 + 127) / 128), 128, 0, stream>>>(a);
+    const long long warps = static_cast<long long>(S) * T * ((q_rot ? Hq : 0) + (k_new ? Hkv : 0));
+    if (warps == 0) return ATTN_OK;
+    attn::decode_step_prep_kernel<D><<<static_cast<unsigned>((warps * 32 + 127) / 128), 128, 0, stream>>>(a);
     CUDA_TRY(cudaGetLastError());
     return ATTN_OK;
 }
@@ -257,8 +285,7 @@ attn_status launch_append(const void* k_new, const void* v_new, void* k_pages, v
 template <int D>
 attn_status launch_decode(const void* q, const void* k_pages, const void* v_pages, const int32_t* block_table,
                           const int32_t* seq_lens, int S, int T, int max_blocks, int num_pages, int Hq, int Hkv,
-                          float scale, const double2* rope, void* o, float* lse, void* ws, cudaStream_t stream,
-                          int dev) {
+                          float scale, void* o, float* lse, void* ws, cudaStream_t stream, int dev) {
     using C = attn::DecCfg<D>;
     CUtensorMap tk, tv;
     attn_status st;
@@ -274,7 +301,6 @@ attn_status launch_decode(const void* q, const void* k_pages, const void* v_page
     p.lse = lse;
     p.ws_o = static_cast<float*>(ws);
     p.ws_ml = p.ws_o + static_cast<size_t>(S) * T * Hq * max_chunks * D;
-    p.rope = rope;
     p.T = T;
     p.mtiles = (Hq / Hkv * T + 15) / 16;
     p.S = S;
@@ -285,7 +311,7 @@ attn_status launch_decode(const void* q, const void* k_pages, const void* v_page
     p.num_pages = num_pages;
     p.max_chunks = max_chunks;
     p.scale_log2 = scale * attn::kLog2e;
-    const bool step = T > 1 || rope != nullptr;
+    const bool step = T > 1;
     if (step) {
         if ((st = ensure_smem(attn::decode_split_kernel<D, true>, C::SMEM_BYTES, dev)) != ATTN_OK) return st;
         attn::decode_split_kernel<D, true><<<dim3(max_chunks, Hkv * p.mtiles, S), attn::kDecodeThreads, C::SMEM_BYTES,
@@ -357,8 +383,8 @@ attn_status launch_bwd(const void* q, const void* k, const void* v, const void* 
         void* qr = w + L.qrot;
         void* kr = w + L.krot;
         const long long qrows = static_cast<long long>(B) * Hq * N, krows = static_cast<long long>(B) * Hkv * N;
-        auto grid_for = [&](long long rows) {
-            const long long want = (rows * (D / 8) + 255) / 256;
+        auto grid_for = [&](long long) {  // one thread per (position, chunk); rows loop inside
+            const long long want = (static_cast<long long>(N) * (D / 8) + 255) / 256;
             return static_cast<int>(want < 8LL * sms ? want : 8LL * sms);
         };
         attn::rope_rotate_rows_kernel<D><<<grid_for(qrows), 256, 0, stream>>>(static_cast<const uint4*>(q),
@@ -398,17 +424,25 @@ attn_status launch_bwd(const void* q, const void* k, const void* v, const void* 
 
 extern "C" {
 
-attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
-                     int N, int D, int causal, int window, float rope_base, float scale, void* stream) {
+attn_status attn_fwd_pos(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                         int N, int D, int causal, int window, float rope_base, int rope_half_split,
+                         float rope_pos_scale, float rope_ntk_factor, const float* alibi_slopes, float scale,
+                         void* stream) {
     g_last_error.clear();
     if (!q || !k || !v || !o) return fail(ATTN_ERR_INVALID_ARG, "q, k, v and o must be non-NULL");
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || (lse && !aligned16(lse)))
         return fail(ATTN_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+    if (alibi_slopes && (reinterpret_cast<uintptr_t>(alibi_slopes) & 3u))
+        return fail(ATTN_ERR_INVALID_ARG, "alibi_slopes must be 4-byte aligned");
     if (B < 1 || Hq < 1 || Hkv < 1 || N < 1) return fail(ATTN_ERR_INVALID_ARG, "B, Hq, Hkv, N must be >= 1");
     if (Hq % Hkv != 0) return fail(ATTN_ERR_INVALID_ARG, "Hq (%d) must be a multiple of Hkv (%d)", Hq, Hkv);
     if (causal != 0 && causal != 1) return fail(ATTN_ERR_INVALID_ARG, "causal must be 0 or 1");
     if (window > 0 && !causal) return fail(ATTN_ERR_INVALID_ARG, "a sliding window requires causal = 1");
+    if (alibi_slopes && !causal) return fail(ATTN_ERR_INVALID_ARG, "ALiBi requires causal = 1");
+    if (rope_half_split != 0 && rope_half_split != 1) return fail(ATTN_ERR_INVALID_ARG, "rope_half_split must be 0 or 1");
     if (!std::isfinite(scale) || !std::isfinite(rope_base)) return fail(ATTN_ERR_INVALID_ARG, "scale and rope_base must be finite");
+    if (!(std::isfinite(rope_pos_scale) && rope_pos_scale > 0.f) || !(std::isfinite(rope_ntk_factor) && rope_ntk_factor > 0.f))
+        return fail(ATTN_ERR_INVALID_ARG, "rope_pos_scale and rope_ntk_factor must be finite and > 0");
     if (D != 64 && D != 128) return fail(ATTN_ERR_UNSUPPORTED, "head dim %d not supported (64 or 128)", D);
     if (static_cast<long long>(B) * Hq * ((N + 255) / 256) > 0x7fffffffLL)
         return fail(ATTN_ERR_UNSUPPORTED, "too many 256-query work items");
@@ -418,8 +452,19 @@ attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float
     int dev = 0;
     CUDA_TRY(cudaGetDevice(&dev));
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (D == 64) return launch_fwd<64>(q, k, v, o, lse, B, Hq, Hkv, N, causal, window, rope_base, scale, s, dev);
-    return launch_fwd<128>(q, k, v, o, lse, B, Hq, Hkv, N, causal, window, rope_base, scale, s, dev);
+    PosVariant pv;
+    pv.half_split = rope_half_split;
+    pv.pos_scale = rope_pos_scale;
+    pv.ntk = rope_ntk_factor;
+    pv.alibi = alibi_slopes;
+    if (D == 64) return launch_fwd<64>(q, k, v, o, lse, B, Hq, Hkv, N, causal, window, rope_base, scale, s, dev, pv);
+    return launch_fwd<128>(q, k, v, o, lse, B, Hq, Hkv, N, causal, window, rope_base, scale, s, dev, pv);
+}
+
+attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                     int N, int D, int causal, int window, float rope_base, float scale, void* stream) {
+    return attn_fwd_pos(q, k, v, o, lse, B, Hq, Hkv, N, D, causal, window, rope_base, 0, 1.f, 1.f, nullptr, scale,
+                        stream);
 }
 
 size_t attn_bwd_workspace_size(int B, int Hq, int Hkv, int N, int D, float rope_base) {
@@ -496,16 +541,22 @@ attn_status attn_decode_paged(const void* q, const void* k_pages, const void* v_
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (D == 64)
         return launch_decode<64>(q, k_pages, v_pages, block_table, seq_lens, num_seqs, 1, max_blocks_per_seq,
-                                 num_pages, Hq, Hkv, scale, nullptr, o, lse, workspace, s, dev);
+                                 num_pages, Hq, Hkv, scale, o, lse, workspace, s, dev);
     return launch_decode<128>(q, k_pages, v_pages, block_table, seq_lens, num_seqs, 1, max_blocks_per_seq,
-                              num_pages, Hq, Hkv, scale, nullptr, o, lse, workspace, s, dev);
+                              num_pages, Hq, Hkv, scale, o, lse, workspace, s, dev);
+}
+
+// Partial states of the split (as attn_decode_workspace_size, per new token), then the rotated
+// queries (bf16).
+size_t step_partials_bytes(int num_seqs, int q_len, int max_blocks_per_seq, int Hq, int D) {
+    const size_t rows = static_cast<size_t>(num_seqs) * q_len * Hq * decode_chunks(max_blocks_per_seq);
+    return (rows * (static_cast<size_t>(D) + 2) * sizeof(float) + 255) / 256 * 256;
 }
 
 size_t attn_decode_step_workspace_size(int num_seqs, int q_len, int max_blocks_per_seq, int page_size, int Hq, int D) {
     if (num_seqs < 1 || q_len < 1 || max_blocks_per_seq < 1 || page_size < 1 || Hq < 1 || D < 1) return 0;
-    const size_t rows = static_cast<size_t>(num_seqs) * q_len * Hq * decode_chunks(max_blocks_per_seq);
-    const size_t bytes = rows * (static_cast<size_t>(D) + 2) * sizeof(float);
-    return (bytes + 255) / 256 * 256;
+    const size_t qrot = (static_cast<size_t>(num_seqs) * q_len * Hq * D * 2 + 255) / 256 * 256;
+    return step_partials_bytes(num_seqs, q_len, max_blocks_per_seq, Hq, D) + qrot;
 }
 
 attn_status attn_decode_step(const void* q, const void* k_new, const void* v_new, void* k_pages, void* v_pages,
@@ -547,19 +598,21 @@ attn_status attn_decode_step(const void* q, const void* k_new, const void* v_new
         attn_status st = rope_table64(dev, static_cast<double>(rope_base), D, max_blocks_per_seq * page_size, &table);
         if (st != ATTN_OK) return st;
     }
-    attn_status st = ATTN_OK;
-    if (k_new != nullptr) {
-        st = D == 64 ? launch_append<64>(k_new, v_new, k_pages, v_pages, block_table, seq_lens, num_seqs, q_len,
-                                         max_blocks_per_seq, num_pages, Hkv, table, s)
-                     : launch_append<128>(k_new, v_new, k_pages, v_pages, block_table, seq_lens, num_seqs, q_len,
-                                          max_blocks_per_seq, num_pages, Hkv, table, s);
-        if (st != ATTN_OK) return st;
-    }
+    // rotated queries live after the partial states
+    void* q_rot = table != nullptr ? static_cast<uint8_t*>(workspace) +
+                                         step_partials_bytes(num_seqs, q_len, max_blocks_per_seq, Hq, D)
+                                   : nullptr;
+    attn_status st = D == 64 ? launch_step_prep<64>(q, q_rot, k_new, v_new, k_pages, v_pages, block_table, seq_lens,
+                                                     num_seqs, q_len, max_blocks_per_seq, num_pages, Hq, Hkv, table, s)
+                             : launch_step_prep<128>(q, q_rot, k_new, v_new, k_pages, v_pages, block_table, seq_lens,
+                                                      num_seqs, q_len, max_blocks_per_seq, num_pages, Hq, Hkv, table, s);
+    if (st != ATTN_OK) return st;
+    const void* q_use = q_rot != nullptr ? q_rot : q;
     if (D == 64)
-        return launch_decode<64>(q, k_pages, v_pages, block_table, seq_lens, num_seqs, q_len, max_blocks_per_seq,
-                                 num_pages, Hq, Hkv, scale, table, o, lse, workspace, s, dev);
-    return launch_decode<128>(q, k_pages, v_pages, block_table, seq_lens, num_seqs, q_len, max_blocks_per_seq,
-                              num_pages, Hq, Hkv, scale, table, o, lse, workspace, s, dev);
+        return launch_decode<64>(q_use, k_pages, v_pages, block_table, seq_lens, num_seqs, q_len, max_blocks_per_seq,
+                                 num_pages, Hq, Hkv, scale, o, lse, workspace, s, dev);
+    return launch_decode<128>(q_use, k_pages, v_pages, block_table, seq_lens, num_seqs, q_len, max_blocks_per_seq,
+                              num_pages, Hq, Hkv, scale, o, lse, workspace, s, dev);
 }
 
 attn_status attn_get_device_status(void* stream, int* flags_out) {

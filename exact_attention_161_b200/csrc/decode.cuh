@@ -24,9 +24,9 @@
 // A decode step may bring T >= 1 new tokens per sequence (multi-token decode: the last T rows of
 // causal attention over the sequence). Their G*T query rows (G heads x T tokens) are cut into
 // 16-row tiles, one tile per CTA, and row (t, head) sees the cached tokens up to its position
-// len - T + t. With a RoPE table, each query row is rotated at its position as it is loaded. A
-// separate append kernel writes the new tokens' keys (rotated) and values into their page slots
-// before the split kernel reads the cache.
+// len - T + t. A prep kernel runs first: it rotates each new query row once at its position (into
+// the workspace) and writes the new tokens' keys (rotated) and values into their page slots, so
+// the split kernel reads a cache that already holds them and queries that are already rotated.
 #pragma once
 #include "common.cuh"
 #include "ptx.cuh"
@@ -40,31 +40,33 @@ constexpr int kDecodeWarps = 4;
 constexpr int kDecodeThreads = kDecodeWarps * 32;
 
 struct DecodeParams {
-    const __nv_bfloat16* q;      // [S, T, Hq, D]; rotated here when rope != nullptr
+    const __nv_bfloat16* q;      // [S, T, Hq, D], rotated
     const int32_t* block_table;  // [S, max_blocks]
     const int32_t* seq_lens;     // [S], counting the T new tokens
     __nv_bfloat16* o;            // [S, T, Hq, D]
     float* lse;                  // [S, T, Hq] or nullptr
     float* ws_o;                 // [S, T*Hq, max_chunks, D] unnormalised partial outputs
     float* ws_ml;                // [S, T*Hq, max_chunks, 2] partial (max in log2 units, sum)
-    const double2* rope;         // (cos, sin) per (position, pair), fp64, or nullptr
     int S, Hq, Hkv, G, max_blocks, num_pages, max_chunks;
     int T, mtiles;               // new tokens per sequence; 16-row tiles per KV head = ceil(G*T / 16)
     float scale_log2;
 };
 
-// Append of the T new tokens of every sequence: token t of sequence s sits at position
-// pos = len - T + t, in page block_table[s][pos / page_size], slot pos % page_size. Its key is
-// rotated at pos (when a table is given) and rounded to bf16; its value is copied.
-struct AppendParams {
-    const __nv_bfloat16* k_new;  // [S, T, Hkv, D]
+// Prep of a decode step: token t of sequence s sits at position pos = len - T + t. Its query rows
+// are rotated at pos into q_rot (when a table is given), and its key (rotated at pos, rounded to
+// bf16) and value are written to page block_table[s][pos / page_size], slot pos % page_size (when
+// k_new is given).
+struct StepPrepParams {
+    const __nv_bfloat16* q;      // [S, T, Hq, D]
+    __nv_bfloat16* q_rot;        // [S, T, Hq, D] or nullptr (no rotation)
+    const __nv_bfloat16* k_new;  // [S, T, Hkv, D] or nullptr (no append)
     const __nv_bfloat16* v_new;  // [S, T, Hkv, D]
     __nv_bfloat16* k_pages;      // [num_pages, Hkv, page_size, D]
     __nv_bfloat16* v_pages;
     const int32_t* block_table;
     const int32_t* seq_lens;
     const double2* rope;
-    int S, T, Hkv, max_blocks, num_pages;
+    int S, T, Hq, Hkv, max_blocks, num_pages;
 };
 
 template <int D>
@@ -189,18 +191,12 @@ __global__ void __launch_bounds__(kDecodeThreads)
             lim[hr] = pos;
             const __nv_bfloat16* qrow =
                 p.q + ((static_cast<size_t>(s) * T + t) * p.Hq + g * p.G + (kStep ? R % p.G : R)) * D;
-            const double2* cs = kStep && p.rope != nullptr ? p.rope + static_cast<size_t>(pos) * (D / 2) : nullptr;
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
                     const int d0 = kk * 16 + colA + 8 * half;
-                    uint32_t w = live ? *reinterpret_cast<const uint32_t*>(qrow + d0) : 0u;
-                    if (cs != nullptr && live) {
-                        const double2 c = __ldg(cs + d0 / 2);
-                        w = rope_rotate_pair(w, c.x, c.y);
-                    }
-                    qa[kk][hr + 2 * half] = w;
+                    qa[kk][hr + 2 * half] = live ? *reinterpret_cast<const uint32_t*>(qrow + d0) : 0u;
                 }
             }
         }
@@ -416,16 +412,21 @@ __global__ void __launch_bounds__(128) decode_merge_kernel(const DecodeParams p)
     if (p.lse != nullptr && lane == 0) p.lse[out_row] = L > 0.f ? (M + ptx::lg2(L)) * kLn2 : -INFINITY;
 }
 
-// One warp per (sequence, new token, KV head): each lane moves D/64 bf16 pairs of the key (rotated
-// at the token's position when a table is given) and of the value into the token's page slot. An
-// invalid length or block-table entry raises a status bit and writes nothing.
+// One warp per row: the first S*T*Hq warps rotate a new query row (when q_rot is given), the next
+// S*T*Hkv warps append a new token's key and value for one KV head (when k_new is given). Each
+// lane handles D/64 bf16 pairs. An invalid length or block-table entry raises a status bit and
+// the row is left alone.
 template <int D>
-__global__ void __launch_bounds__(128) decode_append_kernel(const AppendParams a) {
+__global__ void __launch_bounds__(128) decode_step_prep_kernel(const StepPrepParams a) {
     const long long w = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
-    if (w >= static_cast<long long>(a.S) * a.T * a.Hkv) return;
-    const int g = static_cast<int>(w % a.Hkv);
-    const long long st = w / a.Hkv;
+    const long long q_rows = a.q_rot != nullptr ? static_cast<long long>(a.S) * a.T * a.Hq : 0;
+    const long long kv_rows = a.k_new != nullptr ? static_cast<long long>(a.S) * a.T * a.Hkv : 0;
+    if (w >= q_rows + kv_rows) return;
+    const bool is_q = w < q_rows;
+    const long long r = is_q ? w : w - q_rows;
+    const int H = is_q ? a.Hq : a.Hkv;
+    const long long st = r / H;
     const int t = static_cast<int>(st % a.T), s = static_cast<int>(st / a.T);
     const int len = a.seq_lens[s];
     if (len < a.T || len > a.max_blocks * kPageSize) {
@@ -433,18 +434,29 @@ __global__ void __launch_bounds__(128) decode_append_kernel(const AppendParams a
         return;
     }
     const int pos = len - a.T + t;
+    const double2* cs = a.rope != nullptr ? a.rope + static_cast<size_t>(pos) * (D / 2) : nullptr;
+    if (is_q) {
+        const uint32_t* src = reinterpret_cast<const uint32_t*>(a.q + static_cast<size_t>(r) * D);
+        uint32_t* dst = reinterpret_cast<uint32_t*>(a.q_rot + static_cast<size_t>(r) * D);
+#pragma unroll
+        for (int i = lane; i < D / 2; i += 32) {
+            const double2 c = __ldg(cs + i);
+            dst[i] = rope_rotate_pair(src[i], c.x, c.y);
+        }
+        return;
+    }
+    const int g = static_cast<int>(r % a.Hkv);
     const int page = a.block_table[static_cast<size_t>(s) * a.max_blocks + pos / kPageSize];
     if (page < 0 || page >= a.num_pages) {
         if (lane == 0) raise_status(kStatusBadPage);
         return;
     }
-    const size_t src = static_cast<size_t>(w) * D;
+    const size_t src = static_cast<size_t>(r) * D;
     const size_t dst = ((static_cast<size_t>(page) * a.Hkv + g) * kPageSize + pos % kPageSize) * D;
     const uint32_t* ks = reinterpret_cast<const uint32_t*>(a.k_new + src);
     const uint32_t* vs = reinterpret_cast<const uint32_t*>(a.v_new + src);
     uint32_t* kd = reinterpret_cast<uint32_t*>(a.k_pages + dst);
     uint32_t* vd = reinterpret_cast<uint32_t*>(a.v_pages + dst);
-    const double2* cs = a.rope != nullptr ? a.rope + static_cast<size_t>(pos) * (D / 2) : nullptr;
 #pragma unroll
     for (int i = lane; i < D / 2; i += 32) {
         uint32_t kw = ks[i];

@@ -41,7 +41,9 @@ namespace attn {
 struct FwdParams {
     __nv_bfloat16* o;       // [B, Hq, N, D]
     float* lse;             // [B, Hq, N] natural-log row logsumexp, or nullptr
-    const float2* rope;     // [>= N, D/2] (cos, sin) of pos * base^(-2i/D), or nullptr (no RoPE)
+    const float2* rope;     // [>= N, D/2] (cos, sin) of pair i at pos, or nullptr (no RoPE)
+    const float* alibi;     // [Hq] ALiBi slopes m_h (logit minus m_h (i - j)), read when kAlibi
+    int rope_half;          // 1: half-split pairing (i, i + D/2); the key pass permutes to match
     int B, Hq, Hkv, N;
     int causal, window;     // window > 0 only together with causal
     float scale_log2;       // softmax scale * log2(e)
@@ -128,6 +130,41 @@ __device__ __forceinline__ void rope_rotate_smem_row(uint8_t* tile, int r, const
     }
 }
 
+// Half-split pairing: the row's pairs (i, i + D/2) are rotated and written back interleaved, at
+// (2i, 2i+1). The key rotation pass applies the same permutation, and a score q.k is unchanged when
+// the dimensions of q and k are permuted alike, so the rest of the kernel is the interleaved one.
+// The whole row is read into registers before anything is written back.
+template <int D>
+__device__ __forceinline__ void rope_rotate_smem_row_half(uint8_t* tile, int r, const float2* __restrict__ cs_row) {
+    using C = FwdCfg<D>;
+    uint32_t w[D / 2];
+#pragma unroll
+    for (int reg = 0; reg < C::NREG; ++reg)
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            const uint4 v = *reinterpret_cast<const uint4*>(tile + reg * C::REGION_BYTES + r * 128 + ((c ^ (r & 7)) << 4));
+            w[reg * 32 + c * 4 + 0] = v.x;
+            w[reg * 32 + c * 4 + 1] = v.y;
+            w[reg * 32 + c * 4 + 2] = v.z;
+            w[reg * 32 + c * 4 + 3] = v.w;
+        }
+#pragma unroll
+    for (int oc = 0; oc < D / 8; ++oc) {  // output chunk: pairs 4 oc .. 4 oc + 3
+        uint32_t ow[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int pi = oc * 4 + k;
+            const uint32_t a = w[pi / 2], b = w[pi / 2 + D / 4];
+            const float x0 = (pi & 1) ? ptx::bf16hi_to_f32(a) : ptx::bf16lo_to_f32(a);
+            const float x1 = (pi & 1) ? ptx::bf16hi_to_f32(b) : ptx::bf16lo_to_f32(b);
+            const float2 t = __ldg(cs_row + pi);
+            ow[k] = ptx::pack_bf16x2(fmaf(x0, t.x, -x1 * t.y), fmaf(x0, t.y, x1 * t.x));
+        }
+        *reinterpret_cast<uint4*>(tile + (oc / 8) * C::REGION_BYTES + r * 128 + (((oc % 8) ^ (r & 7)) << 4)) =
+            make_uint4(ow[0], ow[1], ow[2], ow[3]);
+    }
+}
+
 // One work item: (batch b, query head h, block of 256 queries); the longest causal blocks come
 // first, and the query heads of one block are adjacent so heads sharing a K/V head run together.
 struct Item {
@@ -159,7 +196,7 @@ __device__ __forceinline__ Item make_item(const FwdParams& p, int it) {
     return x;
 }
 
-template <int D>
+template <int D, bool kAlibi>
 __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
@@ -361,8 +398,14 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
             const int i_pos = R.q0 + r;  // query position
             ok = ptx::mbar_wait(&bar->q_loaded[wg], kq & 1, abort_flag);
             if (!ok) break;
-            if (p.rope != nullptr && i_pos < p.N)
-                rope_rotate_smem_row<D>(sQ + wg * C::TILE_BYTES, r, p.rope + static_cast<size_t>(i_pos) * (D / 2));
+            if (p.rope != nullptr && i_pos < p.N) {
+                if (p.rope_half)
+                    rope_rotate_smem_row_half<D>(sQ + wg * C::TILE_BYTES, r, p.rope + static_cast<size_t>(i_pos) * (D / 2));
+                else
+                    rope_rotate_smem_row<D>(sQ + wg * C::TILE_BYTES, r, p.rope + static_cast<size_t>(i_pos) * (D / 2));
+            }
+            // ALiBi: this head's slope in log2 units
+            const float slope2 = kAlibi ? p.alibi[x.h] * kLog2e : 0.f;
             ptx::fence_proxy_async_smem();
             ptx::named_barrier_sync(1 + wg, 128);
             if (r == 0) ptx::mbar_arrive(&bar->q_ready[wg]);
@@ -388,6 +431,20 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
                         if (kj < lo || kj > hi) s[k] = -INFINITY;
                     }
                 }
+                if constexpr (kAlibi) {
+                    // logits in log2 units with the bias -m (i - j) folded in: s*scale_log2 +
+                    // slope2 * (j - i); masked entries stay -inf
+                    const float2 sl2 = make_float2(sl, sl), sp2 = make_float2(slope2, slope2);
+                    const float b0 = slope2 * static_cast<float>(j0 - i_pos);
+                    const float2 bb = make_float2(b0, b0);
+#pragma unroll
+                    for (int k = 0; k < C::BN; k += 2) {
+                        const float2 bias = ptx::ffma2(sp2, make_float2(static_cast<float>(k), static_cast<float>(k + 1)), bb);
+                        const float2 y = ptx::ffma2(make_float2(s[k], s[k + 1]), sl2, bias);
+                        s[k] = y.x;
+                        s[k + 1] = y.y;
+                    }
+                }
                 // four independent chains over s[0..7], s[8..15], ...: every element exactly once
                 float mx0 = fmaxf(s[0], s[1]), mx1 = fmaxf(s[2], s[3]), mx2 = fmaxf(s[4], s[5]),
                       mx3 = fmaxf(s[6], s[7]);
@@ -398,7 +455,8 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
                     mx2 = ptx::fmax3(mx2, s[k + 4], s[k + 5]);
                     mx3 = ptx::fmax3(mx3, s[k + 6], s[k + 7]);
                 }
-                const float m_new = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl;
+                const float slx = kAlibi ? 1.f : sl;  // ALiBi logits are already scaled
+                const float m_new = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * slx;
                 float alpha = 1.f;
                 bool rescale = false;
                 if (m_new > m_used + C::RESCALE_THRESHOLD) {  // also the first visible key (m_used = -inf)
@@ -407,7 +465,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
                     rescale = true;
                 }
                 const float m_eff = (m_used == -INFINITY) ? 0.f : m_used;
-                const float2 sl2 = make_float2(sl, sl), nm2 = make_float2(-m_eff, -m_eff);
+                const float2 sl2 = make_float2(slx, slx), nm2 = make_float2(-m_eff, -m_eff);
                 float2 acc0 = make_float2(0.f, 0.f), acc1 = acc0, acc2 = acc0, acc3 = acc0;
                 uint32_t pk[C::BN / 2];
 #pragma unroll

@@ -28,28 +28,50 @@ __device__ __forceinline__ uint32_t rope_rotate_pair(uint32_t w, double cth, dou
     return lo | (hi << 16);
 }
 
-// k, k_rot: [rows, D] bf16 with row r at position r % N; cs: [>= N, D/2] (cos, sin) in fp64.
-// Each thread handles 16-byte chunks (4 pairs); consecutive threads take consecutive chunks, so
-// loads and stores are fully coalesced.
-template <int D>
+// k, k_rot: [rows, D] bf16 with row r at position r % N (rows = BH * N); cs: [>= N, D/2] (cos, sin)
+// in fp64. A thread takes one 16-byte output chunk (4 pairs) of one position, loads that chunk's 4
+// table entries once and applies them to the chunk in every one of the BH rows at the position;
+// consecutive threads take consecutive chunks, so each row's loads and stores are coalesced.
+// kHalf: the pairs are (i, i + D/2) and the rotated pair i is written interleaved at (2i, 2i+1) --
+// the dimensions are permuted so that the attention kernel, which rotates its queries the same
+// way, can treat both pairings alike.
+template <int D, bool kHalf = false>
 __global__ void __launch_bounds__(256) rope_rotate_rows_kernel(const uint4* __restrict__ k, uint4* __restrict__ k_rot,
                                                                const double2* __restrict__ cs, long long rows, int N) {
     constexpr int CHUNKS = D / 8;
-    const long long total = rows * CHUNKS;
+    const long long bh_count = rows / N;
+    const long long total = static_cast<long long>(N) * CHUNKS;
     for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
          idx += (long long)gridDim.x * blockDim.x) {
-        const long long row = idx / CHUNKS;
+        const int pos = static_cast<int>(idx / CHUNKS);
         const int c = static_cast<int>(idx % CHUNKS);
-        const int pos = static_cast<int>(row % N);
-        uint4 w = __ldg(k + idx);
-        const double2* t = cs + static_cast<size_t>(pos) * (D / 2) + c * 4;
-        uint32_t* wv = reinterpret_cast<uint32_t*>(&w);
+        double2 t[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const double2 a = __ldg(t + e);
-            wv[e] = rope_rotate_pair(wv[e], a.x, a.y);
+        for (int e = 0; e < 4; ++e) t[e] = __ldg(cs + static_cast<size_t>(pos) * (D / 2) + c * 4 + e);
+#pragma unroll 4
+        for (long long bh = 0; bh < bh_count; ++bh) {
+            const long long row = bh * N + pos;
+            uint4 w;
+            if constexpr (kHalf) {
+                // pairs 4c .. 4c+3: first members at elements 4c.., second members at D/2 + 4c..
+                const uint2* src = reinterpret_cast<const uint2*>(k + row * CHUNKS);
+                const uint2 a = __ldg(src + c), b = __ldg(src + c + D / 8);
+                const uint32_t av[2] = {a.x, a.y}, bv[2] = {b.x, b.y};
+                uint32_t* wv = reinterpret_cast<uint32_t*>(&w);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const uint32_t lo = (e & 1) ? (av[e / 2] >> 16) : (av[e / 2] & 0xFFFFu);
+                    const uint32_t hi = (e & 1) ? (bv[e / 2] >> 16) : (bv[e / 2] & 0xFFFFu);
+                    wv[e] = lo | (hi << 16);
+                }
+            } else {
+                w = __ldg(k + row * CHUNKS + c);
+            }
+            uint32_t* wv = reinterpret_cast<uint32_t*>(&w);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) wv[e] = rope_rotate_pair(wv[e], t[e].x, t[e].y);
+            k_rot[row * CHUNKS + c] = w;
         }
-        k_rot[idx] = w;
     }
 }
 

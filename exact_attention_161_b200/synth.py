@@ -258,3 +258,10 @@ def decode_step_inputs_for(cfg: DecodeConfig, T: int, permute: bool = True, pois
     return decode_step_inputs(cfg.num_seqs, T, cfg.Hq, cfg.Hkv, cfg.D, cfg.page_size, len_lo=cfg.len_lo,
                               len_hi=cfg.len_hi, spare_frac=cfg.spare_frac, seed=cfg.seed, permute=permute,
                               poison=poison)
+
+
+def alibi_slopes(H: int) -> torch.Tensor:
+    """Per-head ALiBi slopes, the geometric sequence m_h = 2^(-8h/H), h = 1..H, of the ALiBi paper
+    (Press et al., 2021; the pages name the method and say only that each head has a fixed slope).
+    fp32 [H]; every value is a power of two, so both implementations see it exactly."""
+    return torch.tensor([2.0 ** (-8.0 * h / H) for h in range(1, H + 1)], dtype=torch.float32)

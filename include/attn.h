@@ -80,6 +80,29 @@ attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float
                      int N, int D, int causal, int window, float rope_base, float scale, void* stream);
 
 /*
+ * attn_fwd_pos -- attn_fwd with the position-encoding variants ("attention-transformers": Q "How
+ * does Rotary Position Embedding (RoPE) work?", Q "What are NTK-aware RoPE scaling and YaRN?",
+ * Q "How does ALiBi encode position?"):
+ *   rope_half_split  0: RoPE pairs (2i, 2i+1) as attn_fwd; 1: pairs (i, i + D/2) (the rotate-half
+ *                    layout). The output is the same attention either way; only which
+ *                    dimensions form a pair changes.
+ *   rope_pos_scale   Position Interpolation: pair i of position pos is rotated by
+ *                    (pos / rope_pos_scale) * b^(-2i/D); 1 = off. Finite, > 0.
+ *   rope_ntk_factor  NTK-aware scaling: b = rope_base * rope_ntk_factor^(D/(D-2)), which leaves the
+ *                    highest frequency as is and divides the lowest by the factor; 1 = off.
+ *                    Finite, > 0. Both scalings change only the cos/sin table.
+ *   alibi_slopes     device fp32 [Hq], 4-byte aligned, or NULL: ALiBi subtracts
+ *                    alibi_slopes[h] * (i - j) from the scaled logit of query i and key j of head
+ *                    h (then the softmax as usual; LSE includes the bias). Requires causal = 1.
+ * Other arguments, constraints and errors as attn_fwd; attn_fwd is attn_fwd_pos with (0, 1, 1,
+ * NULL). The scalings and pairing apply only when rope_base > 0.
+ */
+attn_status attn_fwd_pos(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                         int N, int D, int causal, int window, float rope_base, int rope_half_split,
+                         float rope_pos_scale, float rope_ntk_factor, const float* alibi_slopes, float scale,
+                         void* stream);
+
+/*
  * attn_bwd_workspace_size -- bytes of device workspace attn_bwd needs: fp32 (-LSE*log2 e, -D_i)
  * per query row padded to 128-row tiles, plus, with RoPE, the rotated Q and K (bf16). 0 for invalid sizes.
  */

@@ -60,6 +60,19 @@ def test_fwd_validation(api, kw, expect):
     assert api.last_error() != ""
 
 
+def _fwd_pos(api, causal=1, half=0, ps=1.0, ntk=1.0, alibi=None, rope=10000.0):
+    return api.lib.attn_fwd_pos(FAKE, FAKE, FAKE, FAKE, None, 1, 4, 2, 128, 128, causal, 0, rope, half, ps, ntk, alibi,
+                                0.0, None)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(half=2), 1), (dict(ps=0.0), 1), (dict(ps=float("inf")), 1), (dict(ntk=-1.0), 1),
+    (dict(causal=0, alibi=FAKE), 1), (dict(alibi=ctypes.c_void_p(0x10002)), 1),
+])
+def test_fwd_pos_validation(api, kw, expect):
+    assert _fwd_pos(api, **kw) == expect
+
+
 def _dec(api, num_seqs=2, max_blocks=8, num_pages=16, page_size=16, Hq=8, Hkv=2, D=128, ws_bytes=None,
          ws=FAKE, q=FAKE, bt=FAKE):
     if ws_bytes is None:
@@ -100,8 +113,10 @@ def test_decode_step_validation(api, kw, expect):
 
 
 def test_decode_step_workspace_size(api):
-    assert api.decode_step_workspace_size(64, 4, 1024, 16, 32, 128) == 64 * 4 * 32 * 32 * 130 * 4
-    assert api.decode_step_workspace_size(64, 1, 1024, 16, 32, 128) == api.decode_workspace_size(64, 1024, 16, 32, 128)
+    # the split's partial states per (sequence, new token, head, chunk), then the rotated queries
+    assert api.decode_step_workspace_size(64, 4, 1024, 16, 32, 128) == 64 * 4 * 32 * 32 * 130 * 4 + 64 * 4 * 32 * 128 * 2
+    assert api.decode_step_workspace_size(64, 1, 1024, 16, 32, 128) == (
+        api.decode_workspace_size(64, 1024, 16, 32, 128) + 64 * 32 * 128 * 2)
     assert api.decode_step_workspace_size(1, 0, 1, 16, 1, 64) == 0
 
 

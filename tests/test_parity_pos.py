@@ -1,0 +1,89 @@
+"""Position-variant parity (GPU only): half-split RoPE pairing, Position Interpolation, NTK-aware
+base scaling and ALiBi in the prefill kernel, against the fp64 oracle's attention_pos."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from exact_attention_161_b200 import synth
+from parity import assert_close, bits, f64, sample_rows
+
+pytestmark = pytest.mark.gpu
+
+# B, Hq, Hkv, N, D, causal, window, rope_base, half_split, pos_scale, ntk, alibi
+CASES = [
+    (1, 4, 2, 300, 128, 1, 0, 10000.0, True, 1.0, 1.0, False),
+    (1, 2, 2, 257, 64, 0, 0, 10000.0, True, 1.0, 1.0, False),
+    (1, 4, 1, 640, 128, 1, 0, 10000.0, False, 4.0, 1.0, False),
+    (1, 4, 1, 640, 128, 1, 0, 10000.0, False, 1.0, 8.0, False),
+    (1, 2, 2, 513, 64, 1, 100, 500000.0, True, 2.0, 4.0, False),
+    (1, 8, 2, 300, 128, 1, 0, 0.0, False, 1.0, 1.0, True),
+    (1, 8, 8, 1000, 128, 1, 0, 10000.0, False, 1.0, 1.0, True),
+    (2, 4, 2, 129, 64, 1, 64, 10000.0, True, 4.0, 2.0, True),
+    (1, 32, 8, 1024, 128, 1, 0, 500000.0, True, 1.0, 4.0, True),
+]
+
+
+def _ids(c):
+    return "B%dHq%dHkv%dN%dD%d_c%d_w%d_r%g_half%d_pi%g_ntk%g_alibi%d" % c
+
+
+def _gpu(api, q, k, v, case):
+    B, Hq, Hkv, N, D, causal, window, rope, half, ps, ntk, alibi = case
+    slopes = synth.alibi_slopes(Hq).cuda() if alibi else None
+    o, lse = api.attn_fwd_pos(q.cuda(), k.cuda(), v.cuda(), causal=causal, window=window, rope_base=rope,
+                              rope_half_split=half, rope_pos_scale=ps, rope_ntk_factor=ntk, alibi_slopes=slopes)
+    torch.cuda.synchronize()
+    return o, lse
+
+
+def _oracle(q, k, v, case, rows=None):
+    B, Hq, Hkv, N, D, causal, window, rope, half, ps, ntk, alibi = case
+    slopes = synth.alibi_slopes(Hq).double().numpy() if alibi else None
+    return oracle.attention_pos(bits(q), bits(k), bits(v), causal=causal, window=window, rope_base=rope,
+                                rope_half_split=half, rope_pos_scale=ps, rope_ntk_factor=ntk, alibi_slopes=slopes,
+                                rows=rows)
+
+
+@pytest.mark.parametrize("case", CASES, ids=_ids)
+def test_variant_vs_oracle(cuda_api, case):
+    B, Hq, Hkv, N, D = case[:5]
+    q, k, v = synth.prefill_inputs(B, Hq, Hkv, N, D, seed=500 + CASES.index(case))
+    o, lse = _gpu(cuda_api, q, k, v, case)
+    assert cuda_api.device_status() == 0
+    o_ref, lse_ref = _oracle(q, k, v, case)
+    assert_close(f64(o), f64(lse), o_ref, lse_ref, _ids(case))
+
+
+def test_neutral_variants_are_attn_fwd(cuda_api):
+    """Interleaved pairing, both factors 1 and no ALiBi: the same bits as attn_fwd."""
+    q, k, v = synth.prefill_inputs(1, 8, 2, 500, 128, seed=520)
+    o1, l1 = cuda_api.attn_fwd(q.cuda(), k.cuda(), v.cuda(), causal=True, rope_base=10000.0)
+    o2, l2 = _gpu(cuda_api, q, k, v, (1, 8, 2, 500, 128, 1, 0, 10000.0, False, 1.0, 1.0, False))
+    assert torch.equal(o1.view(torch.int16), o2.view(torch.int16)) and torch.equal(l1, l2)
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_half_split_is_interleaved_on_permuted_dims(cuda_api, D):
+    """Half-split RoPE equals interleaved RoPE on q and k whose dimensions are permuted so that
+    (i, i + D/2) become (2i, 2i+1): the same bits, since both rotate the same numbers the same way."""
+    q, k, v = synth.prefill_inputs(1, 4, 2, 400, D, seed=521)
+    perm = torch.stack([torch.arange(D // 2), torch.arange(D // 2) + D // 2], 1).reshape(-1)
+    o1, l1 = _gpu(cuda_api, q, k, v, (1, 4, 2, 400, D, 1, 0, 10000.0, True, 1.0, 1.0, False))
+    qp, kp = q[..., perm].contiguous(), k[..., perm].contiguous()
+    o2, l2 = _gpu(cuda_api, qp, kp, v, (1, 4, 2, 400, D, 1, 0, 10000.0, False, 1.0, 1.0, False))
+    assert torch.equal(o1.view(torch.int16), o2.view(torch.int16)) and torch.equal(l1, l2)
+
+
+def test_alibi_full_size_sampled(cuda_api):
+    """ALiBi (with half-split RoPE and NTK scaling) on the GQA causal N=8192 workload, sampled rows."""
+    cfg = synth.GQA_CAUSAL_N8192
+    q, k, v = synth.prefill_inputs_for(cfg)
+    case = (cfg.B, cfg.Hq, cfg.Hkv, cfg.N, cfg.D, 1, 0, cfg.rope_base, True, 1.0, 4.0, True)
+    o, lse = _gpu(cuda_api, q, k, v, case)
+    assert cuda_api.device_status() == 0
+    rows = sample_rows(cfg.B, cfg.Hq, cfg.N, per_head=6, seed=3)
+    o_ref, lse_ref = _oracle(q, k, v, case, rows=rows)
+    og = f64(o).reshape(-1, cfg.D)[rows]
+    lg = f64(lse).reshape(-1)[rows]
+    assert_close(og, lg, o_ref, lse_ref, "alibi full size")
