@@ -431,32 +431,40 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
                         if (kj < lo || kj > hi) s[k] = -INFINITY;
                     }
                 }
+                // Row max. Plain: the max of the scores, scaled. ALiBi: an upper bound of the biased
+                // logits s*scale_log2 + slope2*(j - i), from the max score of each 16-column group plus
+                // the group's largest bias; it exceeds the true max by at most 15 slope steps, which
+                // keeps P far from underflow, and the online softmax and the LSE are exact for any
+                // upper bound. The bias then enters only the exponent argument below.
+                float m_new;
+                const float b0 = kAlibi ? slope2 * static_cast<float>(j0 - i_pos) : 0.f;
                 if constexpr (kAlibi) {
-                    // logits in log2 units with the bias -m (i - j) folded in: s*scale_log2 +
-                    // slope2 * (j - i); masked entries stay -inf
-                    const float2 sl2 = make_float2(sl, sl), sp2 = make_float2(slope2, slope2);
-                    const float b0 = slope2 * static_cast<float>(j0 - i_pos);
-                    const float2 bb = make_float2(b0, b0);
+                    const int kend = slope2 >= 0.f ? 15 : 0;
+                    float bound = -INFINITY;
 #pragma unroll
-                    for (int k = 0; k < C::BN; k += 2) {
-                        const float2 bias = ptx::ffma2(sp2, make_float2(static_cast<float>(k), static_cast<float>(k + 1)), bb);
-                        const float2 y = ptx::ffma2(make_float2(s[k], s[k + 1]), sl2, bias);
-                        s[k] = y.x;
-                        s[k + 1] = y.y;
+                    for (int g = 0; g < C::BN / 16; ++g) {
+                        float a = fmaxf(s[16 * g], s[16 * g + 1]), b = fmaxf(s[16 * g + 2], s[16 * g + 3]);
+#pragma unroll
+                        for (int k = 16 * g + 4; k < 16 * g + 16; k += 4) {
+                            a = ptx::fmax3(a, s[k], s[k + 1]);
+                            b = ptx::fmax3(b, s[k + 2], s[k + 3]);
+                        }
+                        bound = fmaxf(bound, fmaf(fmaxf(a, b), sl, fmaf(slope2, static_cast<float>(16 * g + kend), b0)));
                     }
-                }
-                // four independent chains over s[0..7], s[8..15], ...: every element exactly once
-                float mx0 = fmaxf(s[0], s[1]), mx1 = fmaxf(s[2], s[3]), mx2 = fmaxf(s[4], s[5]),
-                      mx3 = fmaxf(s[6], s[7]);
+                    m_new = bound;
+                } else {
+                    // four independent chains over s[0..7], s[8..15], ...: every element exactly once
+                    float mx0 = fmaxf(s[0], s[1]), mx1 = fmaxf(s[2], s[3]), mx2 = fmaxf(s[4], s[5]),
+                          mx3 = fmaxf(s[6], s[7]);
 #pragma unroll
-                for (int k = 8; k < C::BN; k += 8) {
-                    mx0 = ptx::fmax3(mx0, s[k], s[k + 1]);
-                    mx1 = ptx::fmax3(mx1, s[k + 2], s[k + 3]);
-                    mx2 = ptx::fmax3(mx2, s[k + 4], s[k + 5]);
-                    mx3 = ptx::fmax3(mx3, s[k + 6], s[k + 7]);
+                    for (int k = 8; k < C::BN; k += 8) {
+                        mx0 = ptx::fmax3(mx0, s[k], s[k + 1]);
+                        mx1 = ptx::fmax3(mx1, s[k + 2], s[k + 3]);
+                        mx2 = ptx::fmax3(mx2, s[k + 4], s[k + 5]);
+                        mx3 = ptx::fmax3(mx3, s[k + 6], s[k + 7]);
+                    }
+                    m_new = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl;
                 }
-                const float slx = kAlibi ? 1.f : sl;  // ALiBi logits are already scaled
-                const float m_new = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * slx;
                 float alpha = 1.f;
                 bool rescale = false;
                 if (m_new > m_used + C::RESCALE_THRESHOLD) {  // also the first visible key (m_used = -inf)
@@ -465,15 +473,21 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
                     rescale = true;
                 }
                 const float m_eff = (m_used == -INFINITY) ? 0.f : m_used;
-                const float2 sl2 = make_float2(slx, slx), nm2 = make_float2(-m_eff, -m_eff);
+                const float2 sl2 = make_float2(sl, sl), nm2 = make_float2(-m_eff, -m_eff);
+                // ALiBi: per pair, the addend is slope2*(k, k+1) + b0 - m instead of -m
+                const float2 sp2 = make_float2(slope2, slope2), bm2 = make_float2(b0 - m_eff, b0 - m_eff);
+                auto addend = [&](int k) {
+                    return kAlibi ? ptx::ffma2(sp2, make_float2(static_cast<float>(k), static_cast<float>(k + 1)), bm2)
+                                  : nm2;
+                };
                 float2 acc0 = make_float2(0.f, 0.f), acc1 = acc0, acc2 = acc0, acc3 = acc0;
                 uint32_t pk[C::BN / 2];
 #pragma unroll
                 for (int k = 0; k < C::BN; k += 8) {
-                    float2 x0 = ptx::ffma2(make_float2(s[k], s[k + 1]), sl2, nm2);
-                    float2 x1 = ptx::ffma2(make_float2(s[k + 2], s[k + 3]), sl2, nm2);
-                    float2 x2 = ptx::ffma2(make_float2(s[k + 4], s[k + 5]), sl2, nm2);
-                    float2 x3 = ptx::ffma2(make_float2(s[k + 6], s[k + 7]), sl2, nm2);
+                    float2 x0 = ptx::ffma2(make_float2(s[k], s[k + 1]), sl2, addend(k));
+                    float2 x1 = ptx::ffma2(make_float2(s[k + 2], s[k + 3]), sl2, addend(k + 2));
+                    float2 x2 = ptx::ffma2(make_float2(s[k + 4], s[k + 5]), sl2, addend(k + 4));
+                    float2 x3 = ptx::ffma2(make_float2(s[k + 6], s[k + 7]), sl2, addend(k + 6));
                     x0 = make_float2(ptx::ex2(x0.x), ptx::ex2(x0.y));
                     x1 = make_float2(ptx::ex2(x1.x), ptx::ex2(x1.y));
                     x2 = make_float2(ptx::ex2(x2.x), ptx::ex2(x2.y));
