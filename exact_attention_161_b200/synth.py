@@ -9,6 +9,7 @@ Every tensor is drawn on the CPU from ``torch.Generator('cpu').manual_seed(seed)
 does). The pages draw Q/K/V i.i.d. N(0, 1), which gives q.k/sqrt(d) unit variance
 ("attention-transformers", Q "Why is attention scaled by 1/sqrt(dk)?").
 """
+import math
 from dataclasses import dataclass
 from typing import Optional
 
@@ -265,3 +266,37 @@ def alibi_slopes(H: int) -> torch.Tensor:
     (Press et al., 2021; the pages name the method and say only that each head has a fixed slope).
     fp32 [H]; every value is a power of two, so both implementations see it exactly."""
     return torch.tensor([2.0 ** (-8.0 * h / H) for h in range(1, H + 1)], dtype=torch.float32)
+
+
+@dataclass
+class Fp8Inputs:
+    """FP8 e4m3 Q/K/V (bit patterns, uint8) with per-tensor scales: the value of an element is its
+    e4m3 value times the tensor's descale."""
+    q8: torch.Tensor
+    k8: torch.Tensor
+    v8: torch.Tensor
+    descale_q: float
+    descale_k: float
+    descale_v: float
+
+
+E4M3_MAX = 448.0
+
+
+def fp8_inputs(B, Hq, Hkv, N, D, seed) -> Fp8Inputs:
+    """N(0,1) fp32 draws quantised to e4m3 per tensor: descale = max|x| / 448 rounded up to a power of
+    two (so the scaling is exact), then x / descale rounded to e4m3 by torch (nearest even; no value
+    exceeds 448)."""
+    g = _gen(seed)
+    out = []
+    for shape in ((B, Hq, N, D), (B, Hkv, N, D), (B, Hkv, N, D)):
+        x = torch.randn(shape, generator=g, dtype=torch.float32)
+        amax = float(x.abs().max())
+        descale = 2.0 ** math.ceil(math.log2(amax / E4M3_MAX))
+        x8 = (x / descale).to(torch.float8_e4m3fn).view(torch.uint8)
+        out.append((x8, descale))
+    return Fp8Inputs(out[0][0], out[1][0], out[2][0], out[0][1], out[1][1], out[2][1])
+
+
+def fp8_inputs_for(cfg: PrefillConfig) -> Fp8Inputs:
+    return fp8_inputs(cfg.B, cfg.Hq, cfg.Hkv, cfg.N, cfg.D, cfg.seed + 2000)

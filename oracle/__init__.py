@@ -47,6 +47,8 @@ def _declare(lib):
     lib.oracle_attention_pos.argtypes = [p, p, p, i32, i32, i32, i32, i32, i32, i32, f64, i32, f64, f64, p, f64, p,
                                          i64, p, p, i32]
     lib.oracle_attention_pos.restype = i32
+    lib.oracle_e4m3_to_f64.argtypes = [p, i64, p]
+    lib.oracle_e4m3_to_f64.restype = None
     lib.oracle_rope_bf16.argtypes = [p, p, i64, i32, f64, p]
     lib.oracle_rope_bf16.restype = i32
     lib.oracle_round_bf16_array.argtypes = [p, i64, p]
@@ -283,6 +285,39 @@ def rope_bf16_ex(x, pos, base, half_split=False, pos_scale=1.0, ntk_factor=1.0, 
     if st != 0:
         raise OracleError("oracle_rope_bf16_ex failed with status %d" % st)
     return out
+
+
+def e4m3_to_f64(x, lib=None):
+    """FP8 e4m3 bit patterns (numpy uint8) -> exact float64 values."""
+    lib = lib or _lib()
+    x = np.ascontiguousarray(x)
+    if x.dtype != np.uint8:
+        raise TypeError("e4m3 inputs are bit patterns (numpy.uint8), got %s" % x.dtype)
+    out = np.empty(x.shape, dtype=np.float64)
+    lib.oracle_e4m3_to_f64(_ptr(x), x.size, _ptr(out))
+    return out
+
+
+def attention_fp8(q8, k8, v8, descale_q, descale_k, descale_v, causal=False, window=0, scale=None, rows=None,
+                  nthreads=0, lib=None):
+    """Exact attention on FP8 e4m3 inputs: q = q8 * descale_q, k = k8 * descale_k, v = v8 * descale_v
+    (per-tensor scales), in fp64. Every e4m3 value is exactly a bf16 value, so the bf16-input
+    attention runs on the converted bits with the score scale times descale_q * descale_k, and the
+    output is multiplied by descale_v. Shapes and returns as ``attention``."""
+    lib = lib or _lib()
+    conv = []
+    for x in (q8, k8, v8):
+        val = e4m3_to_f64(x, lib=lib)
+        b = round_bf16(val, lib=lib)
+        if not np.array_equal(bf16_bits_to_f64(b), val):
+            raise OracleError("e4m3 value not exact in bf16 (NaN input?)")
+        conv.append(b)
+    D = q8.shape[-1]
+    if scale is None:
+        scale = 1.0 / np.sqrt(D)
+    o, lse = attention(conv[0], conv[1], conv[2], causal=causal, window=window, rope_base=0.0,
+                       scale=float(scale) * float(descale_q) * float(descale_k), rows=rows, nthreads=nthreads, lib=lib)
+    return o * float(descale_v), lse
 
 
 def rope_bf16(x, pos, base, lib=None):

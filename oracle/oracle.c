@@ -457,6 +457,26 @@ int oracle_decode_step(const uint16_t* q, const uint16_t* k_new, const uint16_t*
     return status;
 }
 
+/*
+ * FP8 e4m3 (the "fn" encoding: 1 sign bit, 4 exponent bits with bias 7, 3 mantissa bits, no
+ * infinities, S.1111.111 is NaN) to its exact value: exponent field 0 gives the subnormals
+ * m * 2^-9, otherwise (1 + m/8) * 2^(e-7). FP8 attention of the pages ("Why is attention O(n^2),
+ * ...": newer hardware, FP8) is exact attention on these values times their per-tensor scales.
+ */
+void oracle_e4m3_to_f64(const uint8_t* x, int64_t n, double* out) {
+    for (int64_t i = 0; i < n; ++i) {
+        const int sign = x[i] >> 7, e = (x[i] >> 3) & 15, m = x[i] & 7;
+        double v;
+        if (e == 15 && m == 7)
+            v = NAN;
+        else if (e == 0)
+            v = ldexp((double)m, -9);
+        else
+            v = ldexp(1.0 + (double)m / 8.0, e - 7);
+        out[i] = sign ? -v : v;
+    }
+}
+
 int oracle_max_threads(void) {
 #ifdef _OPENMP
     return omp_get_max_threads();

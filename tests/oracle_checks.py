@@ -583,6 +583,48 @@ def check_position_variants_combined(lib):
     assert np.abs(oh - op).max() < 1e-12 and np.abs(lh - lp).max() < 1e-12
 
 
+# ---------------------------------------------------------------------------------- FP8
+
+def check_e4m3_golden_and_library(lib):
+    """e4m3 decoding: values worked by hand from the encoding (bias 7, 3 mantissa bits, subnormals
+    m * 2^-9, S.1111.111 = NaN), and torch's float8_e4m3fn conversion on all 256 codes."""
+    hand = {0x00: 0.0, 0x01: 2.0 ** -9, 0x07: 7 * 2.0 ** -9, 0x08: 2.0 ** -6, 0x38: 1.0, 0x39: 1.125,
+            0x3F: 1.875, 0x40: 2.0, 0x7E: 448.0, 0xFE: -448.0, 0xB8: -1.0, 0x80: -0.0}
+    codes = np.array(sorted(hand), np.uint8)
+    got = oracle.e4m3_to_f64(codes, lib=lib)
+    assert np.array_equal(got, np.array([hand[c] for c in sorted(hand)]))
+    assert np.isnan(oracle.e4m3_to_f64(np.array([0x7F, 0xFF], np.uint8), lib=lib)).all()
+    allc = np.arange(256, dtype=np.uint8)
+    ref = torch.from_numpy(allc).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    mine = oracle.e4m3_to_f64(allc, lib=lib)
+    ok = np.isnan(ref) & np.isnan(mine) | (ref == mine)
+    assert ok.all()
+
+
+def check_fp8_attention_library(lib):
+    """FP8 attention = torch float64 SDPA on the dequantised tensors (values times descales)."""
+    f = synth.fp8_inputs(1, 4, 2, 40, 16, 60)
+    o, lse = oracle.attention_fp8(f.q8.numpy(), f.k8.numpy(), f.v8.numpy(), f.descale_q, f.descale_k, f.descale_v,
+                                  causal=True, lib=lib)
+    deq = [torch.from_numpy(oracle.e4m3_to_f64(x.numpy(), lib=lib) * d)
+           for x, d in ((f.q8, f.descale_q), (f.k8, f.descale_k), (f.v8, f.descale_v))]
+    ref = torch.nn.functional.scaled_dot_product_attention(*deq, is_causal=True, scale=16 ** -0.5, enable_gqa=True)
+    assert np.abs(o - ref.numpy()).max() < 1e-12
+    s = torch.einsum("bhid,bhjd->bhij", deq[0], deq[1].repeat_interleave(2, dim=1)) * 16 ** -0.5
+    s = s.masked_fill(torch.ones(40, 40, dtype=torch.bool).triu(1), float("-inf"))
+    assert np.abs(lse - torch.logsumexp(s, -1).numpy()).max() < 1e-12
+
+
+def check_fp8_descales(lib):
+    """The value scale of V scales O exactly (powers of two); the scores depend on descale_q *
+    descale_k only."""
+    f = synth.fp8_inputs(1, 2, 1, 24, 16, 61)
+    args = (f.q8.numpy(), f.k8.numpy(), f.v8.numpy())
+    o1, l1 = oracle.attention_fp8(*args, 0.5, 0.25, 1.0, causal=True, lib=lib)
+    o2, l2 = oracle.attention_fp8(*args, 0.25, 0.5, 4.0, causal=True, lib=lib)
+    assert np.array_equal(o1 * 4.0, o2) and np.array_equal(l1, l2)
+
+
 ALL_CHECKS = [
     check_round_bf16_golden, check_round_bf16_matches_torch, check_rope_golden,
     check_rope_matches_sinusoid, check_rope_norm_and_identity, check_rope_relative,
@@ -594,6 +636,7 @@ ALL_CHECKS = [
     check_decode_step_is_last_prefill_rows, check_decode_step_prefill_with_rope, check_decode_step_library,
     check_decode_step_reduces_to_decode, check_rope_half_split_library, check_rope_position_interpolation,
     check_rope_ntk_frequencies, check_alibi_closed_form, check_alibi_library, check_position_variants_combined,
+    check_e4m3_golden_and_library, check_fp8_attention_library, check_fp8_descales,
 ]
 
 

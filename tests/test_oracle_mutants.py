@@ -43,6 +43,8 @@ MUTANTS = {
     "pi_multiplies": ("const double angle = ((double)pos / pos_scale) * theta;",
                       "const double angle = ((double)pos * pos_scale) * theta;"),
     "ntk_exponent": ("pow(ntk_factor, (double)D / (double)(D - 2))", "pow(ntk_factor, 1.0)"),
+    "e4m3_bias": ("v = ldexp(1.0 + (double)m / 8.0, e - 7);", "v = ldexp(1.0 + (double)m / 8.0, e - 8);"),
+    "e4m3_subnormal": ("v = ldexp((double)m, -9);", "v = ldexp((double)m, -10);"),
     "normaliser_missing": ("for (int d = 0; d < D; ++d) o[d] /= l;", "for (int d = 0; d < D; ++d) o[d] /= (l + 1e-3);"),
 }
 
