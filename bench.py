@@ -41,7 +41,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 DATASHEET_BF16_TFLOPS = 2250.0
 DATASHEET_HBM_GBS = 8000.0
 KERNEL_SOURCES = ["exact_attention_161_b200/csrc/fwd_sm100.cuh", "exact_attention_161_b200/csrc/decode.cuh",
-                  "exact_attention_161_b200/csrc/ptx.cuh", "exact_attention_161_b200/csrc/rope.cuh",
+                  "exact_attention_161_b200/csrc/bwd_sm100.cuh", "exact_attention_161_b200/csrc/ptx.cuh",
+                  "exact_attention_161_b200/csrc/rope.cuh", "exact_attention_161_b200/csrc/common.cuh",
                   "exact_attention_161_b200/csrc/attn_api.cu"]
 
 
@@ -370,6 +371,34 @@ def run_ours(args, rank, world, local):
                               "roofline": {"bound": "tensor", "achieved": round(flops / (vms / 1e3) / 1e12, 2),
                                            "unit": "TFLOP/s"}}
 
+    # ---- FP8 e4m3 prefill of the same shape (inputs quantised per tensor; no RoPE on this path)
+    fp8 = None
+    if do_prefill and args.fp8_calls > 0:
+        f8 = synth.fp8_inputs_for(PREFILL)
+        q8, k8, v8 = f8.q8.to(dev), f8.k8.to(dev), f8.v8.to(dev)
+
+        def fp8_call():
+            api.attn_fwd_fp8(q8, k8, v8, f8.descale_q, f8.descale_k, f8.descale_v, causal=PREFILL.causal,
+                             window=PREFILL.window, o=o, lse=lse, stream=stream)
+
+        for _ in range(args.warmup):
+            fp8_call()
+        barrier(world)
+        torch.cuda.synchronize()
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for _ in range(args.fp8_calls):
+            fp8_call()
+        f1.record(stream)
+        torch.cuda.synchronize()
+        if api.device_status() != 0:
+            raise RuntimeError("device status raised during the FP8 loop")
+        fms = reduce_max(f0.elapsed_time(f1), world, dev) / args.fp8_calls
+        fp8 = {"metric": "attn fwd TFLOP/s, e4m3 Q/K/V (per-tensor scales), same shape and mask, no RoPE",
+               "value": round(job_throughput(flops, world, fms / 1e3) / 1e12, 2), "unit": "TFLOP/s", "dtype": "e4m3",
+               "ms_per_call": round(fms, 4), "calls": args.fp8_calls,
+               "roofline": {"bound": "tensor", "achieved": round(flops / (fms / 1e3) / 1e12, 2), "unit": "TFLOP/s"}}
+
     # ---- end to end through the public API with pinned host buffers
     E = min(args.e2e_steps, K) if (args.e2e_steps > 0 and args.only == "all") else 0
     if E:
@@ -450,9 +479,10 @@ def run_ours(args, rank, world, local):
         return None
     peaks, peaks_kind = measured_peaks()
     if steps_out is not None:
-        for v in steps_out.values():
+        for key, v in steps_out.items():
             v["roofline"].update({"peak": peaks["hbm_gbs"], "frac": round(v["roofline"]["achieved"] / peaks["hbm_gbs"], 4),
-                                  "peak_kind": peaks_kind})
+                                  "peak_kind": peaks_kind,
+                                  "traffic": profiled_traffic("decode_split" if key == "q_len=1" else "decode_step_split_q4")})
     pre_launch_ms = statistics.mean(prefill_ms)
     dec_launch_ms = statistics.mean(decode_ms)
     tflops_launch = flops / (pre_launch_ms / 1e3) / 1e12 if do_prefill else float("nan")
@@ -460,7 +490,13 @@ def run_ours(args, rank, world, local):
     tensor_peak = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
     if bwd is not None:
         bwd["roofline"].update({"peak": tensor_peak, "frac": round(bwd["roofline"]["achieved"] / tensor_peak, 4),
-                                "peak_kind": "%s bf16 GEMM, sustained" % peaks_kind})
+                                "peak_kind": "%s bf16 GEMM, sustained" % peaks_kind,
+                                "traffic": profiled_traffic("attn_bwd_dkdv"),
+                                "traffic_kernel": "attn_bwd_dkdv_kernel<128> (the larger of the two backward kernels)"})
+    if fp8 is not None:
+        fp8_peak = 2.0 * tensor_peak
+        fp8["roofline"].update({"peak": fp8_peak, "frac": round(fp8["roofline"]["achieved"] / fp8_peak, 4),
+                                "peak_kind": "2 x %s bf16 GEMM sustained (nominal fp8:bf16 ratio 4.5:2.25)" % peaks_kind})
     if variants is not None:
         for vv in variants.values():
             vv["roofline"].update({"peak": tensor_peak, "frac": round(vv["roofline"]["achieved"] / tensor_peak, 4),
@@ -508,6 +544,7 @@ def run_ours(args, rank, world, local):
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": (2 * do_prefill + 2 * do_decode) * K,
         "backward": bwd,
+        "fp8": fp8,
         "position_variants": None if variants is None else dict(
             {"metric": "attn fwd TFLOP/s of the same prefill workload with ALiBi (slopes 2^(-8h/H)), and with "
                        "half-split RoPE pairing plus NTK-aware base scaling x4"}, **variants),
@@ -594,6 +631,7 @@ def parse_args(argv=None):
     ap.add_argument("--bwd-steps", type=int, default=20, help="backward calls timed after the step loop; 0 skips")
     ap.add_argument("--step-calls", type=int, default=50, help="decode-step calls timed per q_len; 0 skips")
     ap.add_argument("--variant-calls", type=int, default=20, help="position-variant prefill calls timed each; 0 skips")
+    ap.add_argument("--fp8-calls", type=int, default=20, help="FP8 prefill calls timed; 0 skips")
     ap.add_argument("--only", choices=["all", "prefill", "decode"], default="all",
                     help="time one half of the step only (profiling runs); the JSON line is then partial")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle time for the CPU baseline")

@@ -28,6 +28,7 @@ _p, _i, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
 SIGNATURES = {
     "attn_fwd": (_i, [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _f, _f, _p]),
     "attn_fwd_pos": (_i, [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _f, _i, _f, _f, _p, _f, _p]),
+    "attn_fwd_fp8": (_i, [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _f, _f, _f, _f, _p]),
     "attn_bwd_workspace_size": (_sz, [_i, _i, _i, _i, _i, _f]),
     "attn_bwd": (_i, [_p, _p, _p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _f, _f, _p, _sz, _p]),
     "attn_decode_workspace_size": (_sz, [_i, _i, _i, _i, _i]),
@@ -139,6 +140,26 @@ def attn_fwd_pos(q, k, v, causal=False, window=0, rope_base=0.0, rope_half_split
                             float(rope_pos_scale), float(rope_ntk_factor),
                             _dev_tensor(alibi_slopes, "alibi_slopes", torch.float32) if alibi_slopes is not None
                             else None, float(scale), _stream(stream)))
+    return o, lse
+
+
+def attn_fwd_fp8(q8, k8, v8, descale_q, descale_k, descale_v, causal=False, window=0, scale=0.0, o=None, lse=None,
+                 want_lse=True, stream=None):
+    """FP8 attention forward. q8 [B,Hq,N,128], k8/v8 [B,Hkv,N,128]: e4m3 bit patterns as uint8 CUDA
+    tensors, with per-tensor descales. Returns (o [B,Hq,N,128] bf16, lse [B,Hq,N] fp32 or None)."""
+    B, Hq, N, D = q8.shape
+    Hkv = k8.shape[1]
+    if k8.shape != (B, Hkv, N, D) or v8.shape != k8.shape:
+        raise ValueError("k8 and v8 must be [B, Hkv, N, D] with q8 [B, Hq, N, D]")
+    if o is None:
+        o = torch.empty((B, Hq, N, D), dtype=torch.bfloat16, device=q8.device)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q8.device)
+    _check(lib.attn_fwd_fp8(_dev_tensor(q8, "q8", torch.uint8), _dev_tensor(k8, "k8", torch.uint8),
+                            _dev_tensor(v8, "v8", torch.uint8), _dev_tensor(o, "o", torch.bfloat16),
+                            _dev_tensor(lse, "lse", torch.float32) if lse is not None else None, B, Hq, Hkv, N, D,
+                            int(causal), int(window), float(descale_q), float(descale_k), float(descale_v),
+                            float(scale), _stream(stream)))
     return o, lse
 
 

@@ -63,16 +63,18 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// A rank-3 bf16 tensor map: dims {d0 (contiguous), d1, d2}, box {64, box1, 1}, 128-byte swizzle,
-// out-of-bounds elements read as zero.
-attn_status make_map_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t box1) {
+// A rank-3 tensor map of bf16 (elem = 2) or 8-bit (elem = 1) elements: dims {d0 (contiguous), d1,
+// d2}, box {128 bytes of d0, box1, 1}, 128-byte swizzle, out-of-bounds elements read as zero.
+attn_status make_map_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t box1,
+                        int elem = 2) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return fail(ATTN_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable (no CUDA driver?)");
     const cuuint64_t dims[3] = {d0, d1, d2};
-    const cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
-    const cuuint32_t box[3] = {64, box1, 1};
+    const cuuint64_t strides[2] = {d0 * elem, d0 * d1 * elem};
+    const cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / elem), box1, 1};
     const cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+    CUresult r = fn(map, elem == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                    const_cast<void*>(base), dims, strides, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(ATTN_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
@@ -222,6 +224,7 @@ attn_status launch_fwd(const void* q, const void* k, const void* v, void* o, flo
         p.rope_half = pv.half_split;
     }
     p.alibi = pv.alibi;
+    p.o_scale = 1.f;
     CUtensorMap tq, tk, tv;
     attn_status st;
     if ((st = make_map_3d(&tq, q, D, N, static_cast<uint64_t>(B) * Hq, 128)) != ATTN_OK) return st;
@@ -253,6 +256,38 @@ attn_status launch_fwd(const void* q, const void* k, const void* v, void* o, flo
 }
 
 size_t decode_chunks(int max_blocks) { return (static_cast<size_t>(max_blocks) + attn::kChunkPages - 1) / attn::kChunkPages; }
+
+// FP8 prefill: e4m3 Q, K, V with per-tensor descales; the persistent kernel's kFp8 instance.
+attn_status launch_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                           int N, int causal, int window, float scale, float descale_v, cudaStream_t stream, int dev) {
+    constexpr int D = 128;
+    using C = attn::FwdCfg<D, true>;
+    attn::FwdParams p{};
+    CUtensorMap tq, tk, tv;
+    attn_status st;
+    if ((st = make_map_3d(&tq, q, D, N, static_cast<uint64_t>(B) * Hq, 128, 1)) != ATTN_OK) return st;
+    if ((st = make_map_3d(&tk, k, D, N, static_cast<uint64_t>(B) * Hkv, 128, 1)) != ATTN_OK) return st;
+    if ((st = make_map_3d(&tv, v, D, N, static_cast<uint64_t>(B) * Hkv, 128, 1)) != ATTN_OK) return st;
+    p.o = static_cast<__nv_bfloat16*>(o);
+    p.lse = lse;
+    p.o_scale = descale_v;
+    p.B = B;
+    p.Hq = Hq;
+    p.Hkv = Hkv;
+    p.N = N;
+    p.causal = causal;
+    p.window = window > 0 ? window : 0;
+    p.scale_log2 = scale * attn::kLog2e;
+    p.nblk = (N + C::QT * C::BM - 1) / (C::QT * C::BM);
+    p.n_items = B * Hq * p.nblk;
+    int sms = 148;
+    CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+    const int grid = p.n_items < sms ? p.n_items : sms;
+    if ((st = ensure_smem(attn::attn_fwd_kernel<D, false, true>, C::SMEM_BYTES, dev)) != ATTN_OK) return st;
+    attn::attn_fwd_kernel<D, false, true><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+    CUDA_TRY(cudaGetLastError());
+    return ATTN_OK;
+}
 
 template <int D>
 attn_status launch_step_prep(const void* q, void* q_rot, const void* k_new, const void* v_new, void* k_pages,
@@ -459,6 +494,33 @@ attn_status attn_fwd_pos(const void* q, const void* k, const void* v, void* o, f
     pv.alibi = alibi_slopes;
     if (D == 64) return launch_fwd<64>(q, k, v, o, lse, B, Hq, Hkv, N, causal, window, rope_base, scale, s, dev, pv);
     return launch_fwd<128>(q, k, v, o, lse, B, Hq, Hkv, N, causal, window, rope_base, scale, s, dev, pv);
+}
+
+attn_status attn_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                         int N, int D, int causal, int window, float descale_q, float descale_k, float descale_v,
+                         float scale, void* stream) {
+    g_last_error.clear();
+    if (!q || !k || !v || !o) return fail(ATTN_ERR_INVALID_ARG, "q, k, v and o must be non-NULL");
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || (lse && !aligned16(lse)))
+        return fail(ATTN_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+    if (B < 1 || Hq < 1 || Hkv < 1 || N < 1) return fail(ATTN_ERR_INVALID_ARG, "B, Hq, Hkv, N must be >= 1");
+    if (Hq % Hkv != 0) return fail(ATTN_ERR_INVALID_ARG, "Hq (%d) must be a multiple of Hkv (%d)", Hq, Hkv);
+    if (causal != 0 && causal != 1) return fail(ATTN_ERR_INVALID_ARG, "causal must be 0 or 1");
+    if (window > 0 && !causal) return fail(ATTN_ERR_INVALID_ARG, "a sliding window requires causal = 1");
+    if (!std::isfinite(scale)) return fail(ATTN_ERR_INVALID_ARG, "scale must be finite");
+    if (!(std::isfinite(descale_q) && descale_q > 0.f) || !(std::isfinite(descale_k) && descale_k > 0.f) ||
+        !(std::isfinite(descale_v) && descale_v > 0.f))
+        return fail(ATTN_ERR_INVALID_ARG, "descale factors must be finite and > 0");
+    if (D != 128) return fail(ATTN_ERR_UNSUPPORTED, "the FP8 path supports head dim 128, got %d", D);
+    if (static_cast<long long>(B) * Hq * ((N + 255) / 256) > 0x7fffffffLL)
+        return fail(ATTN_ERR_UNSUPPORTED, "too many 256-query work items");
+    if (static_cast<double>(B) * Hq * N * D * 2 >= 1099511627776.0)
+        return fail(ATTN_ERR_UNSUPPORTED, "tensor larger than 1 TiB");
+    if (scale <= 0.f) scale = 1.0f / std::sqrt(static_cast<float>(D));
+    int dev = 0;
+    CUDA_TRY(cudaGetDevice(&dev));
+    return launch_fwd_fp8(q, k, v, o, lse, B, Hq, Hkv, N, causal, window, scale * descale_q * descale_k, descale_v,
+                          static_cast<cudaStream_t>(stream), dev);
 }
 
 attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,

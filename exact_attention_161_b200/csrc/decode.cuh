@@ -77,7 +77,7 @@ struct DecCfg {
     static constexpr int STAGE_BYTES = 2 * SLAB_BYTES;      // K then V
     static constexpr int WARP_BYTES = STAGES * STAGE_BYTES;
     static constexpr int NT = D / 8;                        // 8-wide output column tiles
-    static constexpr int COMBINE_BYTES = kDecodeWarps * 16 * (D + 2) * 4;
+    static constexpr int COMBINE_BYTES = (kDecodeWarps * 16 * (D + 3) + 32) * 4;
     static constexpr int SMEM_BYTES = kDecodeWarps * WARP_BYTES + 1024 /*align*/ + 256 /*barriers*/;
     static_assert(COMBINE_BYTES <= kDecodeWarps * WARP_BYTES, "combine buffer reuses the stages");
 };
@@ -327,7 +327,9 @@ __global__ void __launch_bounds__(kDecodeThreads)
     // ---- combine the 4 warps' states for this chunk (shared memory reuses the stage ring)
     float* cm = reinterpret_cast<float*>(smem);                 // [warps][16] max
     float* cl = cm + kDecodeWarps * 16;                          // [warps][16] sum
-    float* co = cl + kDecodeWarps * 16;                          // [warps][16][D]
+    float* cwt = cl + kDecodeWarps * 16;                         // [warps][16] merge weight
+    float* crow = cwt + kDecodeWarps * 16;                       // [16][2] merged (max, sum)
+    float* co = crow + 32;                                       // [warps][16][D]
 #pragma unroll
     for (int hr = 0; hr < 2; ++hr) {
         float lsum = l[hr];
@@ -347,26 +349,36 @@ __global__ void __launch_bounds__(kDecodeThreads)
     __syncthreads();
     if (!ok) return;
     const int rows_here = kStep ? min(16, p.G * T - mt * 16) : p.G;
-    for (int idx = threadIdx.x; idx < rows_here * D; idx += kDecodeThreads) {
-        const int row = idx / D, d = idx % D;
+    // per row, once: M = max of the warps' maxima, the warps' weights 2^(m_w - M) and the merged sum
+    if (threadIdx.x < rows_here) {
+        const int row = threadIdx.x;
         float M = -INFINITY;
 #pragma unroll
         for (int w = 0; w < kDecodeWarps; ++w) M = fmaxf(M, cm[w * 16 + row]);
-        float acc = 0.f, lacc = 0.f;
+        float lacc = 0.f;
 #pragma unroll
         for (int w = 0; w < kDecodeWarps; ++w) {
             const float mw = cm[w * 16 + row];
             const float sw = mw == -INFINITY ? 0.f : ptx::ex2(mw - M);
-            acc += sw * co[(w * 16 + row) * D + d];
+            cwt[w * 16 + row] = sw;
             lacc += sw * cl[w * 16 + row];
         }
+        crow[2 * row] = M;
+        crow[2 * row + 1] = lacc;
+    }
+    __syncthreads();
+    for (int idx = threadIdx.x; idx < rows_here * D; idx += kDecodeThreads) {
+        const int row = idx / D, d = idx % D;
+        float acc = 0.f;
+#pragma unroll
+        for (int w = 0; w < kDecodeWarps; ++w) acc += cwt[w * 16 + row] * co[(w * 16 + row) * D + d];
         const int R = mt * 16 + row, t = kStep ? R / p.G : 0;
         const size_t out_row = (static_cast<size_t>(s) * T + t) * p.Hq + g * p.G + (kStep ? R % p.G : R);
         const size_t prow = out_row * p.max_chunks + chunk;
         p.ws_o[prow * D + d] = acc;
         if (d == 0) {
-            p.ws_ml[prow * 2] = M;
-            p.ws_ml[prow * 2 + 1] = lacc;
+            p.ws_ml[prow * 2] = crow[2 * row];
+            p.ws_ml[prow * 2 + 1] = crow[2 * row + 1];
         }
     }
 }

@@ -44,6 +44,7 @@ struct FwdParams {
     const float2* rope;     // [>= N, D/2] (cos, sin) of pair i at pos, or nullptr (no RoPE)
     const float* alibi;     // [Hq] ALiBi slopes m_h (logit minus m_h (i - j)), read when kAlibi
     int rope_half;          // 1: half-split pairing (i, i + D/2); the key pass permutes to match
+    float o_scale;          // output multiplier (the FP8 path's V descale; 1 otherwise)
     int B, Hq, Hkv, N;
     int causal, window;     // window > 0 only together with causal
     float scale_log2;       // softmax scale * log2(e)
@@ -51,17 +52,25 @@ struct FwdParams {
     int n_items;            // B * Hq * nblk work items
 };
 
-template <int D>
+template <int D, bool kFp8 = false>
 struct FwdCfg {
     static_assert(D == 64 || D == 128, "head dim 64 or 128");
+    static_assert(!kFp8 || D == 128, "the FP8 path takes D = 128");
+    static constexpr int ELEM = kFp8 ? 1 : 2;         // bytes per Q/K/V element (e4m3 or bf16)
     static constexpr int BM = 128;                    // query rows per tile
     static constexpr int BN = 128;                    // keys per tile
     static constexpr int QT = 2;                      // query tiles per CTA
-    static constexpr int NREG = D / 64;               // 128-byte swizzle regions per row
+    static constexpr int ROW_BYTES = D * ELEM;
+    static constexpr int NREG = ROW_BYTES / 128;      // 128-byte swizzle regions per row
+    static constexpr int TMA_X = 128 / ELEM;          // elements per region row (TMA box width)
     static constexpr int REGION_BYTES = 128 * 128;    // 128 rows x 128 bytes
-    static constexpr int TILE_BYTES = 128 * D * 2;    // one Q, K or V tile in bf16
-    static constexpr int NK = (D == 128) ? 3 : 4;     // K pipeline stages
-    static constexpr int NV = (D == 128) ? 2 : 4;     // V pipeline stages
+    static constexpr int TILE_BYTES = 128 * ROW_BYTES;  // one Q, K or V tile
+    static constexpr int S_KSTEPS = ROW_BYTES / 32;   // MMAs per score tile (32 bytes of K each)
+    static constexpr int O_KSTEPS = BN * ELEM / 32;   // MMAs per P V (32 bytes of P per row each)
+    static constexpr int O_ROWS = 32 / ELEM;          // keys (V rows) per P V MMA
+    static constexpr int P_COLS = BN * ELEM / 4;      // TMEM columns that hold P
+    static constexpr int NK = kFp8 ? 4 : (D == 128) ? 3 : 4;  // K pipeline stages
+    static constexpr int NV = kFp8 ? 4 : (D == 128) ? 2 : 4;  // V pipeline stages
     static constexpr int SMEM_TILES = QT + NK + NV;
     static constexpr int SMEM_BYTES = SMEM_TILES * TILE_BYTES + 1024 /*barriers*/ + 1024 /*align*/;
     static constexpr uint32_t TMEM_COLS = 512;
@@ -196,11 +205,14 @@ __device__ __forceinline__ Item make_item(const FwdParams& p, int it) {
     return x;
 }
 
-template <int D, bool kAlibi>
-__global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
+// kFp8: Q, K, V in e4m3; both products run as kind::f8f6f4 (K = 32 per MMA) and P is packed to
+// e4m3 for the second one; the scores' scale carries the Q and K descales (scale_log2) and the
+// output the V descale (o_scale). No RoPE on this path.
+template <int D, bool kAlibi, bool kFp8 = false>
+__global__ void __launch_bounds__(FwdCfg<D, kFp8>::THREADS, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
-    using C = FwdCfg<D>;
+    using C = FwdCfg<D, kFp8>;
     constexpr int NK = C::NK, NV = C::NV;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -266,7 +278,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
 #pragma unroll
                     for (int r = 0; r < C::NREG; ++r)
                         ptx::tma_load_3d(sQ + i * C::TILE_BYTES + r * C::REGION_BYTES, &tm_q, &bar->q_loaded[i],
-                                         r * 64, x.rng[i].q0, zq);
+                                         r * C::TMA_X, x.rng[i].q0, zq);
                     ++kq[i];
                 }
                 for (int u = 0; u < x.T && ok; ++u, ++g) {
@@ -277,14 +289,14 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
 #pragma unroll
                     for (int r = 0; r < C::NREG; ++r)
                         ptx::tma_load_3d(sK + sk * C::TILE_BYTES + r * C::REGION_BYTES, &tm_k, &bar->k_full[sk],
-                                         r * 64, k0, zk);
+                                         r * C::TMA_X, k0, zk);
                     k_issued = g + 1;
                     if (g >= NV && !ptx::mbar_wait(&bar->v_empty[sv], ((g / NV) - 1) & 1, abort_flag)) { ok = false; break; }
                     ptx::mbar_arrive_expect_tx(&bar->v_full[sv], C::TILE_BYTES);
 #pragma unroll
                     for (int r = 0; r < C::NREG; ++r)
                         ptx::tma_load_3d(sV + sv * C::TILE_BYTES + r * C::REGION_BYTES, &tm_v, &bar->v_full[sv],
-                                         r * 64, k0, zk);
+                                         r * C::TMA_X, k0, zk);
                     v_issued = g + 1;
                 }
             }
@@ -305,8 +317,9 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     } else if (warp == C::MMA_WARP) {
         // ------------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            constexpr uint32_t IDESC_S = ptx::idesc_bf16_f32(128, C::BN, 0, 0);  // Q, K both K-major
-            constexpr uint32_t IDESC_O = ptx::idesc_bf16_f32(128, D, 0, 1);      // P K-major, V MN-major
+            // Q, K both K-major; P K-major, V MN-major
+            constexpr uint32_t IDESC_S = kFp8 ? ptx::idesc_e4m3_f32(128, C::BN, 0, 0) : ptx::idesc_bf16_f32(128, C::BN, 0, 0);
+            constexpr uint32_t IDESC_O = kFp8 ? ptx::idesc_e4m3_f32(128, D, 0, 1) : ptx::idesc_bf16_f32(128, D, 0, 1);
             constexpr uint32_t HI = ptx::sw128_desc_hi(1024);                    // 8-row groups 1024 B apart
             constexpr uint32_t TILE16 = C::TILE_BYTES >> 4;
             // low descriptor words of Q tile 0, K stage 0 and V stage 0 (K-major LBO unused = 16;
@@ -337,9 +350,13 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
                             ptx::tc_fence_after();  // P was written to TMEM by the softmax warps
                             const uint32_t vb = v_lo + ((g + u) % NV) * TILE16;
 #pragma unroll
-                            for (int kk = 0; kk < C::BN / 16; ++kk)
-                                ptx::mma_ts(d_o, d_s + kk * 8, ptx::desc64(vb + kk * (2048 >> 4), HI), IDESC_O,
-                                            (c > 0 || kk > 0) ? 1u : 0u);
+                            for (int kk = 0; kk < C::O_KSTEPS; ++kk) {
+                                const uint64_t bd = ptx::desc64(vb + kk * ((C::O_ROWS * 128) >> 4), HI);
+                                if constexpr (kFp8)
+                                    ptx::mma_ts_f8(d_o, d_s + kk * 8, bd, IDESC_O, (c > 0 || kk > 0) ? 1u : 0u);
+                                else
+                                    ptx::mma_ts(d_o, d_s + kk * 8, bd, IDESC_O, (c > 0 || kk > 0) ? 1u : 0u);
+                            }
                             if (c == R.n - 1) ptx::mma_commit(&bar->o_final[i]);
                         }
                         if (u + 1 < x.T && x.active(i, u + 1)) {
@@ -353,9 +370,12 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
                             if (!ptx::mbar_wait(&bar->k_full[(g + u + 1) % NK], ((g + u + 1) / NK) & 1, abort_flag)) { ok = false; break; }
                             const uint32_t qa = q_lo + i * TILE16, kb = k_lo + ((g + u + 1) % NK) * TILE16;
 #pragma unroll
-                            for (int kk = 0; kk < D / 16; ++kk) {
+                            for (int kk = 0; kk < C::S_KSTEPS; ++kk) {
                                 const uint32_t off = ((kk >> 2) * C::REGION_BYTES + (kk & 3) * 32) >> 4;
-                                ptx::mma_ss(d_s, ptx::desc64(qa + off, HI), ptx::desc64(kb + off, HI), IDESC_S, kk > 0);
+                                if constexpr (kFp8)
+                                    ptx::mma_ss_f8(d_s, ptx::desc64(qa + off, HI), ptx::desc64(kb + off, HI), IDESC_S, kk > 0);
+                                else
+                                    ptx::mma_ss(d_s, ptx::desc64(qa + off, HI), ptx::desc64(kb + off, HI), IDESC_S, kk > 0);
                             }
                             ptx::mma_commit(&bar->s_full[i]);
                             if (c == R.n - 1) ptx::mma_commit(&bar->q_empty[i]);  // Q_i no longer read
@@ -398,7 +418,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
             const int i_pos = R.q0 + r;  // query position
             ok = ptx::mbar_wait(&bar->q_loaded[wg], kq & 1, abort_flag);
             if (!ok) break;
-            if (p.rope != nullptr && i_pos < p.N) {
+            if (!kFp8 && p.rope != nullptr && i_pos < p.N) {
                 if (p.rope_half)
                     rope_rotate_smem_row_half<D>(sQ + wg * C::TILE_BYTES, r, p.rope + static_cast<size_t>(i_pos) * (D / 2));
                 else
@@ -481,7 +501,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
                                   : nm2;
                 };
                 float2 acc0 = make_float2(0.f, 0.f), acc1 = acc0, acc2 = acc0, acc3 = acc0;
-                uint32_t pk[C::BN / 2];
+                uint32_t pk[C::P_COLS];
 #pragma unroll
                 for (int k = 0; k < C::BN; k += 8) {
                     float2 x0 = ptx::ffma2(make_float2(s[k], s[k + 1]), sl2, addend(k));
@@ -496,16 +516,24 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
                     acc1 = ptx::fadd2(acc1, x1);
                     acc2 = ptx::fadd2(acc2, x2);
                     acc3 = ptx::fadd2(acc3, x3);
-                    pk[k / 2] = ptx::pack_bf16x2(x0.x, x0.y);
-                    pk[k / 2 + 1] = ptx::pack_bf16x2(x1.x, x1.y);
-                    pk[k / 2 + 2] = ptx::pack_bf16x2(x2.x, x2.y);
-                    pk[k / 2 + 3] = ptx::pack_bf16x2(x3.x, x3.y);
+                    if constexpr (kFp8) {
+                        pk[k / 4] = ptx::pack_e4m3x4(x0.x, x0.y, x1.x, x1.y);
+                        pk[k / 4 + 1] = ptx::pack_e4m3x4(x2.x, x2.y, x3.x, x3.y);
+                    } else {
+                        pk[k / 2] = ptx::pack_bf16x2(x0.x, x0.y);
+                        pk[k / 2 + 1] = ptx::pack_bf16x2(x1.x, x1.y);
+                        pk[k / 2 + 2] = ptx::pack_bf16x2(x2.x, x2.y);
+                        pk[k / 2 + 3] = ptx::pack_bf16x2(x3.x, x3.y);
+                    }
                 }
                 const float2 a01 = ptx::fadd2(acc0, acc1), a23 = ptx::fadd2(acc2, acc3);
                 const float2 a = ptx::fadd2(a01, a23);
                 l = l * alpha + (a.x + a.y);
-                // P (bf16 pairs) over the first 64 columns of this tile's score buffer.
-                ptx::tmem_st64(t_s, pk);
+                // P (bf16 pairs, or e4m3 quadruples) over the first columns of this tile's score buffer.
+                if constexpr (kFp8)
+                    ptx::tmem_st32(t_s, pk);
+                else
+                    ptx::tmem_st64(t_s, pk);
                 if (c > 0 && __any_sync(0xffffffffu, rescale)) {
                     // The product with the previous P has completed (it was issued before this
                     // tile's scores), so O_i is stable here.
@@ -533,7 +561,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
             if (!ptx::mbar_wait(&bar->o_final[wg], kq & 1, abort_flag)) { ok = false; break; }
             ptx::tc_fence_after();
             uint32_t w[D / 2];
-            const float inv_l = l > 0.f ? 1.f / l : 0.f;
+            const float inv_l = l > 0.f ? p.o_scale / l : 0.f;
 #pragma unroll
             for (int cc = 0; cc < D / 32; ++cc) {
                 uint32_t v[32];

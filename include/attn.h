@@ -103,6 +103,22 @@ attn_status attn_fwd_pos(const void* q, const void* k, const void* v, void* o, f
                          void* stream);
 
 /*
+ * attn_fwd_fp8 -- attn_fwd on FP8 e4m3 inputs ("Why is attention O(n^2), how does FlashAttention help,
+ * ...": newer hardware's FP8). The value of an element of q is its e4m3 value times descale_q (per
+ * tensor), likewise k and v. Both products run on the tensor cores in e4m3 with fp32 accumulation;
+ * the probabilities P are rounded to e4m3 (nearest even) for the P V product, so O carries their
+ * ~2.6% relative rounding (the LSE does not: the row sums stay fp32).
+ *   q            e4m3 bytes [B, Hq, N, 128]; k, v e4m3 bytes [B, Hkv, N, 128]; device, 16-byte aligned
+ *   descale_q, descale_k, descale_v   finite, > 0
+ *   o, lse, B, Hq, Hkv, N, causal, window, scale, stream   as attn_fwd (scale applies to q.k of
+ *                the dequantised values)
+ * D must be 128 (else ATTN_ERR_UNSUPPORTED). No RoPE on this path: rotate before quantising.
+ */
+attn_status attn_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                         int N, int D, int causal, int window, float descale_q, float descale_k, float descale_v,
+                         float scale, void* stream);
+
+/*
  * attn_bwd_workspace_size -- bytes of device workspace attn_bwd needs: fp32 (-LSE*log2 e, -D_i)
  * per query row padded to 128-row tiles, plus, with RoPE, the rotated Q and K (bf16). 0 for invalid sizes.
  */

@@ -22,7 +22,7 @@ def api():
 def declared_functions():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(attn_[a-z_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(attn_[a-z0-9_]+)\s*\(", text)))
 
 
 def test_header_and_binding_agree(api):
@@ -71,6 +71,18 @@ def _fwd_pos(api, causal=1, half=0, ps=1.0, ntk=1.0, alibi=None, rope=10000.0):
 ])
 def test_fwd_pos_validation(api, kw, expect):
     assert _fwd_pos(api, **kw) == expect
+
+
+def _fwd_fp8(api, D=128, dq=1.0, dk=1.0, dv=1.0, causal=1, window=0):
+    return api.lib.attn_fwd_fp8(FAKE, FAKE, FAKE, FAKE, None, 1, 4, 2, 128, D, causal, window, dq, dk, dv, 0.0, None)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(dq=0.0), 1), (dict(dv=float("nan")), 1), (dict(dk=-1.0), 1), (dict(causal=0, window=8), 1),
+    (dict(D=64), 2),
+])
+def test_fwd_fp8_validation(api, kw, expect):
+    assert _fwd_fp8(api, **kw) == expect
 
 
 def _dec(api, num_seqs=2, max_blocks=8, num_pages=16, page_size=16, Hq=8, Hkv=2, D=128, ws_bytes=None,
