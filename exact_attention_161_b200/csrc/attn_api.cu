@@ -21,7 +21,7 @@
 #include "fwd_sm100.cuh"
 #include "rope.cuh"
 
-#define ATTN_VERSION_STRING "exact_attention_161_b200 0.1.0 (sm_100a)"
+#define ATTN_VERSION_STRING "exact_attention_161_b200 0.2.0 (sm_100a)"
 
 namespace {
 
