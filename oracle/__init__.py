@@ -49,6 +49,9 @@ def _declare(lib):
     lib.oracle_attention_pos.restype = i32
     lib.oracle_e4m3_to_f64.argtypes = [p, i64, p]
     lib.oracle_e4m3_to_f64.restype = None
+    lib.oracle_attention_bwd_dq_rows.argtypes = [p, p, p, p, i32, i32, i32, i32, i32, i32, i32, f64, f64, p, i64, p,
+                                                 i32]
+    lib.oracle_attention_bwd_dq_rows.restype = i32
     lib.oracle_rope_bf16.argtypes = [p, p, i64, i32, f64, p]
     lib.oracle_rope_bf16.restype = i32
     lib.oracle_round_bf16_array.argtypes = [p, i64, p]
@@ -318,6 +321,28 @@ def attention_fp8(q8, k8, v8, descale_q, descale_k, descale_v, causal=False, win
     o, lse = attention(conv[0], conv[1], conv[2], causal=causal, window=window, rope_base=0.0,
                        scale=float(scale) * float(descale_q) * float(descale_k), rows=rows, nthreads=nthreads, lib=lib)
     return o * float(descale_v), lse
+
+
+def attention_bwd_dq_rows(q, k, v, dout, rows, causal=False, window=0, rope_base=0.0, scale=None, nthreads=0,
+                          lib=None):
+    """dq of the given query rows (flat ids (b*Hq + h)*N + i) for bf16 inputs, in fp64, with the steps
+    of ``attention_bwd`` for one row. Returns [len(rows), D]."""
+    lib = lib or _lib()
+    q, k, v, dout = _bits(q), _bits(k), _bits(v), _bits(dout)
+    B, Hq, N, D = q.shape
+    Hkv = k.shape[1]
+    if D > 512:
+        raise ValueError("D above 512")
+    if scale is None:
+        scale = 1.0 / np.sqrt(D)
+    rws = np.ascontiguousarray(rows, dtype=np.int64)
+    dq = np.empty((rws.shape[0], D), dtype=np.float64)
+    st = lib.oracle_attention_bwd_dq_rows(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), B, Hq, Hkv, N, D, int(causal),
+                                          int(window), float(rope_base), float(scale), _ptr(rws), rws.shape[0],
+                                          _ptr(dq), int(nthreads))
+    if st != 0:
+        raise OracleError("oracle_attention_bwd_dq_rows failed with status %d" % st)
+    return dq
 
 
 def rope_bf16(x, pos, base, lib=None):

@@ -671,6 +671,102 @@ int oracle_attention_bwd_f64(const double* q, const double* k, const double* v, 
 }
 
 /* Backward on bf16 inputs (the GPU's bits), rotated values rounded to bf16 as in the forward. */
+/*
+ * dq of selected query rows only (bf16 inputs, rotated values rounded to bf16 as in the forward):
+ * the same steps as oracle_attention_bwd_f64 for one row -- its full score row, P, dP_ij = dO_i . v_j,
+ * D_i = sum_j P_ij dP_ij, dS = P (dP - D_i), dq_i = scale sum_j dS_ij k_j rotated back -- which
+ * needs only that row, so rows of large problems can be checked one by one.
+ * rows: flat ids ((b*Hq + h)*N + i); dq: [n_rows, D].
+ */
+int oracle_attention_bwd_dq_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v, const uint16_t* dout,
+                                 int B, int Hq, int Hkv, int N, int D, int causal, int window, double rope_base,
+                                 double scale, const int64_t* rows, int64_t n_rows, double* dq, int nthreads) {
+    if (!q || !k || !v || !dout || !rows || !dq) return ORACLE_ERR_ARG;
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || N <= 0 || D <= 0 || Hq % Hkv != 0) return ORACLE_ERR_ARG;
+    if (window > 0 && !causal) return ORACLE_ERR_ARG;
+    const int G = Hq / Hkv;
+    const int64_t total = (int64_t)B * Hq * N;
+    for (int64_t r = 0; r < n_rows; ++r)
+        if (rows[r] < 0 || rows[r] >= total) return ORACLE_ERR_INDEX;
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#else
+    (void)nthreads;
+#endif
+    const size_t ND = (size_t)N * D;
+    double* kk = (double*)malloc(sizeof(double) * ND);
+    double* vv = (double*)malloc(sizeof(double) * ND);
+    if (!kk || !vv) {
+        free(kk); free(vv);
+        return ORACLE_ERR_NOMEM;
+    }
+    int status = ORACLE_OK;
+    for (int b = 0; b < B && status == ORACLE_OK; ++b)
+        for (int g = 0; g < Hkv && status == ORACLE_OK; ++g) {
+            int needed = 0;
+            for (int64_t r = 0; r < n_rows && !needed; ++r) {
+                const int rb = (int)(rows[r] / ((int64_t)Hq * N)), rh = (int)((rows[r] / N) % Hq);
+                if (rb == b && rh / G == g) needed = 1;
+            }
+            if (!needed) continue;
+            const size_t kv_off = ((size_t)b * Hkv + g) * ND;
+#pragma omp parallel for schedule(static)
+            for (int j = 0; j < N; ++j) {
+                double tmp[512];
+                for (int d = 0; d < D; ++d) tmp[d] = bf16_value(k[kv_off + (size_t)j * D + d]);
+                rope_row_f64(tmp, D, j, rope_base, 0, 1, kk + (size_t)j * D);
+                for (int d = 0; d < D; ++d) vv[(size_t)j * D + d] = bf16_value(v[kv_off + (size_t)j * D + d]);
+            }
+#pragma omp parallel
+            {
+                double* s_row = (double*)malloc(sizeof(double) * (size_t)N);
+                double* dp = (double*)malloc(sizeof(double) * (size_t)N);
+                double* buf = (double*)malloc(sizeof(double) * (size_t)D * 4);
+                if (!s_row || !dp || !buf) {
+#pragma omp atomic write
+                    status = ORACLE_ERR_NOMEM;
+                } else {
+                    double *qq = buf, *dqr = buf + D, *o_row = buf + 2 * D, *dO = buf + 3 * D;
+#pragma omp for schedule(dynamic, 1)
+                    for (int64_t r = 0; r < n_rows; ++r) {
+                        const int64_t id = rows[r];
+                        const int rb = (int)(id / ((int64_t)Hq * N)), rh = (int)((id / N) % Hq);
+                        const long i = (long)(id % N);
+                        if (rb != b || rh / G != g) continue;
+                        double lse_i;
+                        for (int d = 0; d < D; ++d) {
+                            dqr[d] = bf16_value(q[(size_t)id * D + d]);
+                            dO[d] = bf16_value(dout[(size_t)id * D + d]);
+                        }
+                        rope_row_f64(dqr, D, i, rope_base, 0, 1, qq);
+                        attend_row(qq, kk, vv, N, D, i, causal, window, scale, 0.0, s_row, o_row, &lse_i);
+                        double lsum = 0.0;
+                        for (int j = 0; j < N; ++j) lsum += s_row[j];
+                        for (int j = 0; j < N; ++j) s_row[j] /= lsum;
+                        double dsum = 0.0;
+                        for (int j = 0; j < N; ++j) {
+                            dp[j] = 0.0;
+                            if (s_row[j] == 0.0) continue;
+                            for (int d = 0; d < D; ++d) dp[j] += dO[d] * vv[(size_t)j * D + d];
+                            dsum += s_row[j] * dp[j];
+                        }
+                        for (int d = 0; d < D; ++d) dqr[d] = 0.0;
+                        for (int j = 0; j < N; ++j) {
+                            const double pj = s_row[j];
+                            if (pj == 0.0) continue;
+                            const double ds = pj * (dp[j] - dsum);
+                            for (int d = 0; d < D; ++d) dqr[d] += scale * ds * kk[(size_t)j * D + d];
+                        }
+                        rope_row_f64(dqr, D, i, rope_base, 1, 0, dq + (size_t)r * D);
+                    }
+                }
+                free(s_row); free(dp); free(buf);
+            }
+        }
+    free(kk); free(vv);
+    return status;
+}
+
 int oracle_attention_bwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, const uint16_t* dout, int B,
                          int Hq, int Hkv, int N, int D, int causal, int window, double rope_base, double scale,
                          double* dq, double* dk, double* dv, int nthreads) {

@@ -730,5 +730,17 @@ def check_bwd_bf16_entry(lib):
     assert all(np.array_equal(a, b) for a, b in zip(g1, g2))
 
 
+def check_bwd_dq_rows_match_full(lib):
+    """dq of selected rows equals the full backward's dq at those rows (bf16 entry, RoPE, GQA, window)."""
+    q, k, v = (synth.bits(t) for t in synth.prefill_inputs(1, 4, 2, 70, 16, 35))
+    do = synth.bits(synth.randn_bf16((1, 4, 70, 16), torch.Generator().manual_seed(36)))
+    for causal, window in ((1, 0), (1, 9), (0, 0)):
+        dq, _, _ = oracle.attention_bwd(q, k, v, do, causal=causal, window=window, rope_base=100.0, scale=0.25, lib=lib)
+        rows = np.array([0, 5, 69, 70, 139, 200, 279])
+        got = oracle.attention_bwd_dq_rows(q, k, v, do, rows, causal=causal, window=window, rope_base=100.0, scale=0.25,
+                                           lib=lib)
+        assert np.abs(got - dq.reshape(-1, 16)[rows]).max() < 1e-13
+
+
 ALL_CHECKS += [check_bwd_finite_differences, check_bwd_torch_autograd, check_bwd_gqa_is_sum_over_group,
-               check_bwd_bf16_entry]
+               check_bwd_bf16_entry, check_bwd_dq_rows_match_full]

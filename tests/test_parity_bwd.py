@@ -14,6 +14,7 @@ import torch
 
 import oracle
 from exact_attention_161_b200 import synth
+from parity import sample_rows
 
 pytestmark = pytest.mark.gpu
 
@@ -84,3 +85,43 @@ def test_backward_gqa_equals_repeated_heads(cuda_api):
     for a, b in ((dk, dk2), (dv, dv2)):
         summed = b.float().reshape(1, 2, 2, 300, 128).sum(dim=2)
         assert float((a.float() - summed).abs().max()) <= 2.0 ** -7 * float(summed.abs().max())
+
+
+def test_backward_workload_full_size(cuda_api):
+    """The backward the benchmark times (GQA causal N=8192, RoPE 5e5), checked where the oracle can
+    reach at that size:
+    - dq on sampled rows against the oracle's per-row backward;
+    - sum_j dV[b, g, j] = sum over the group's heads and rows of dO (each row of P sums to 1);
+    - sum_j R_j dK[b, g, j] = 0 with R_j the rotation at position j (each row of dS sums to 0).
+    The two sums are compared within 6 standard deviations of independent per-element errors of
+    2^-8 relative (the bf16 rounding of P, dS and the stored gradient)."""
+    cfg = synth.GQA_CAUSAL_N8192
+    q, k, v = synth.prefill_inputs_for(cfg)
+    dout = synth.randn_bf16(tuple(q.shape), torch.Generator().manual_seed(cfg.seed + 1))
+    qd, kd, vd, dod = q.cuda(), k.cuda(), v.cuda(), dout.cuda()
+    o, lse = cuda_api.attn_fwd(qd, kd, vd, causal=True, rope_base=cfg.rope_base)
+    dq, dk, dv = cuda_api.attn_bwd(qd, kd, vd, o, lse, dod, causal=True, rope_base=cfg.rope_base)
+    torch.cuda.synchronize()
+    assert cuda_api.device_status() == 0
+    rows = sample_rows(cfg.B, cfg.Hq, cfg.N, per_head=3, seed=12)
+    ref = oracle.attention_bwd_dq_rows(synth.bits(q), synth.bits(k), synth.bits(v), synth.bits(dout), rows,
+                                       causal=True, rope_base=cfg.rope_base, scale=cfg.scale)
+    check_grad("dq rows", dq.reshape(-1, cfg.D)[torch.from_numpy(rows).cuda()], ref)
+    G = cfg.Hq // cfg.Hkv
+    dv64 = dv.double().cpu()
+    lhs = dv64.sum(dim=2)                                                   # [B, Hkv, D]
+    rhs = dout.double().reshape(cfg.B, cfg.Hkv, G, cfg.N, cfg.D).sum(dim=(2, 3))
+    bound = 6 * 2.0 ** -8 * dv64.pow(2).sum(dim=2).sqrt() + 1e-6
+    assert bool(((lhs - rhs).abs() <= bound).all()), float(((lhs - rhs).abs() / bound).max())
+    dk64 = dk.double().cpu().numpy()
+    half = cfg.D // 2
+    theta = cfg.rope_base ** (-2.0 * np.arange(half) / cfg.D)
+    ang = np.arange(cfg.N)[:, None] * theta[None, :]
+    c, s = np.cos(ang), np.sin(ang)
+    x0, x1 = dk64[..., 0::2], dk64[..., 1::2]
+    rot = np.empty_like(dk64)
+    rot[..., 0::2] = x0 * c - x1 * s
+    rot[..., 1::2] = x0 * s + x1 * c
+    total = rot.sum(axis=2)
+    bound_k = 6 * 2.0 ** -8 * np.sqrt((dk64 ** 2).sum(axis=2)) + 1e-6
+    assert np.all(np.abs(total) <= bound_k), float((np.abs(total) / bound_k).max())
