@@ -496,7 +496,8 @@ def run_ours(args, rank, world, local):
     if fp8 is not None:
         fp8_peak = 2.0 * tensor_peak
         fp8["roofline"].update({"peak": fp8_peak, "frac": round(fp8["roofline"]["achieved"] / fp8_peak, 4),
-                                "peak_kind": "2 x %s bf16 GEMM sustained (nominal fp8:bf16 ratio 4.5:2.25)" % peaks_kind})
+                                "peak_kind": "2 x %s bf16 GEMM sustained (nominal fp8:bf16 ratio 4.5:2.25)" % peaks_kind,
+                                "traffic": profiled_traffic("attn_fwd_fp8")})
     if variants is not None:
         for vv in variants.values():
             vv["roofline"].update({"peak": tensor_peak, "frac": round(vv["roofline"]["achieved"] / tensor_peak, 4),
