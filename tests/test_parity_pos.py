@@ -1,12 +1,33 @@
 """Position-variant parity (GPU only): half-split RoPE pairing, Position Interpolation, NTK-aware
-base scaling and ALiBi in the prefill kernel, against the fp64 oracle's attention_pos."""
+base scaling and ALiBi in the prefill kernel, against the fp64 oracle's attention_pos.
+
+Tolerances are those of attn_fwd, except the max-abs bound with ALiBi. Steep slopes concentrate a
+row's weight on a few keys, so outputs reach the size of single V entries (up to ~4.5 for N(0,1)
+data), where one bf16 step of the stored output is up to 2^-5. There the bound is per element,
+max(2e-2, 2^-7 |reference|): two half-steps of bf16 at the reference value.
+"""
 import numpy as np
 import pytest
 import torch
 
 import oracle
 from exact_attention_161_b200 import synth
-from parity import assert_close, bits, f64, sample_rows
+from parity import LSE_MAX_ABS, O_MAX_ABS, O_REL_RMS, assert_close, bits, f64, sample_rows
+
+
+def assert_close_alibi(o, lse, o_ref, lse_ref, what):
+    o = np.asarray(o, np.float64)
+    assert np.all(np.isfinite(o)), what
+    d = o - o_ref
+    rel_rms = np.sqrt((d ** 2).sum() / (o_ref ** 2).sum())
+    worst = (np.abs(d) / np.maximum(O_MAX_ABS, 2.0 ** -7 * np.abs(o_ref))).max()
+    assert rel_rms <= O_REL_RMS, "%s rel-RMS %.3e" % (what, rel_rms)
+    assert worst <= 1.0, "%s max-abs over its per-element bound by %.2fx" % (what, worst)
+    assert np.abs(np.asarray(lse, np.float64) - lse_ref).max() <= LSE_MAX_ABS, what
+
+
+def _close(case, o, lse, o_ref, lse_ref, what):
+    (assert_close_alibi if case[-1] else assert_close)(o, lse, o_ref, lse_ref, what)
 
 pytestmark = pytest.mark.gpu
 
@@ -52,7 +73,7 @@ def test_variant_vs_oracle(cuda_api, case):
     o, lse = _gpu(cuda_api, q, k, v, case)
     assert cuda_api.device_status() == 0
     o_ref, lse_ref = _oracle(q, k, v, case)
-    assert_close(f64(o), f64(lse), o_ref, lse_ref, _ids(case))
+    _close(case, f64(o), f64(lse), o_ref, lse_ref, _ids(case))
 
 
 def test_neutral_variants_are_attn_fwd(cuda_api):
@@ -86,4 +107,4 @@ def test_alibi_full_size_sampled(cuda_api):
     o_ref, lse_ref = _oracle(q, k, v, case, rows=rows)
     og = f64(o).reshape(-1, cfg.D)[rows]
     lg = f64(lse).reshape(-1)[rows]
-    assert_close(og, lg, o_ref, lse_ref, "alibi full size")
+    _close(case, og, lg, o_ref, lse_ref, "alibi full size")
