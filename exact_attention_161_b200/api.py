@@ -37,6 +37,7 @@ SIGNATURES = {
     "attn_decode_step_workspace_size": (_sz, [_i, _i, _i, _i, _i, _i]),
     "attn_decode_step": (_i, [_p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _f, _f, _p, _p, _p, _sz,
                               _p]),
+    "attn_debug_drop_copy": (None, [_i]),
     "attn_get_device_status": (_i, [_p, ctypes.POINTER(ctypes.c_int)]),
     "attn_last_error": (ctypes.c_char_p, []),
     "attn_version": (ctypes.c_char_p, []),
@@ -284,6 +285,12 @@ def attn_decode_paged_noalloc(q, k_pages, v_pages, block_table, seq_lens, scale=
                                          _dev_tensor(lse, "lse", torch.float32) if lse is not None else None,
                                          _stream(stream)))
     return o, lse
+
+
+def debug_drop_copy(enable: bool) -> None:
+    """Test hook: make the next decode calls' first split CTA skip one page copy, so its bounded
+    wait runs out and the device status reports a timeout (see attn.h)."""
+    lib.attn_debug_drop_copy(1 if enable else 0)
 
 
 def device_status(stream=None) -> int:

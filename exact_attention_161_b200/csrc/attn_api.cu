@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -87,6 +88,8 @@ struct DevBuf {
     size_t bytes = 0;
     int dev = 0;
 };
+
+std::atomic<bool> g_debug_drop_copy{false};  // test hook of attn_debug_drop_copy
 
 std::mutex g_cache_mu;
 // (device, base, D, position scale, NTK factor, fp64?) -> cos/sin table covering positions [0, capacity)
@@ -338,6 +341,7 @@ attn_status launch_decode(const void* q, const void* k_pages, const void* v_page
     p.ws_ml = p.ws_o + static_cast<size_t>(S) * T * Hq * max_chunks * D;
     p.T = T;
     p.mtiles = (Hq / Hkv * T + 15) / 16;
+    p.debug_drop_copy = g_debug_drop_copy.load() ? 1 : 0;
     p.S = S;
     p.Hq = Hq;
     p.Hkv = Hkv;
@@ -695,6 +699,8 @@ attn_status attn_get_device_status(void* stream, int* flags_out) {
     if (word) return fail(ATTN_ERR_DEVICE_CHECK, "a device-side check fired (flags 0x%x)", word);
     return ATTN_OK;
 }
+
+void attn_debug_drop_copy(int enable) { g_debug_drop_copy.store(enable != 0); }
 
 const char* attn_last_error(void) { return g_last_error.c_str(); }
 

@@ -49,6 +49,7 @@ struct DecodeParams {
     float* ws_ml;                // [S, T*Hq, max_chunks, 2] partial (max in log2 units, sum)
     int S, Hq, Hkv, G, max_blocks, num_pages, max_chunks;
     int T, mtiles;               // new tokens per sequence; 16-row tiles per KV head = ceil(G*T / 16)
+    int debug_drop_copy;         // test hook: CTA (0,0,0) skips its first page copy (see attn.h)
     float scale_log2;
 };
 
@@ -162,6 +163,9 @@ __global__ void __launch_bounds__(kDecodeThreads)
                 const int z = phys * p.Hkv + g;
                 ptx::fence_proxy_async_smem();
                 ptx::mbar_arrive_expect_tx(bar, C::STAGE_BYTES);
+                // test hook: expect the bytes but never copy them, so this stage's wait runs out
+                if (p.debug_drop_copy && i == 0 && warp == 0 && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0)
+                    return valid;
 #pragma unroll
                 for (int r = 0; r < C::NREG; ++r) {
                     ptx::tma_load_3d(st + r * kPageSize * 128, &tm_k, bar, r * 64, 0, z);
@@ -347,7 +351,9 @@ __global__ void __launch_bounds__(kDecodeThreads)
         }
     }
     __syncthreads();
-    if (!ok) return;
+    // every warp that gave up set the shared abort flag before the barrier above, so this exit is
+    // the same for the whole CTA (the combine below has another barrier)
+    if (*abort_flag) return;
     const int rows_here = kStep ? min(16, p.G * T - mt * 16) : p.G;
     // per row, once: M = max of the warps' maxima, the warps' weights 2^(m_w - M) and the merged sum
     if (threadIdx.x < rows_here) {

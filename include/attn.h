@@ -269,6 +269,17 @@ attn_status attn_decode_paged_noalloc(const void* q, const void* k_pages, const 
  */
 attn_status attn_get_device_status(void* stream, int* flags_out);
 
+/*
+ * attn_debug_drop_copy -- test hook for the timeout path (not for production use). While enabled,
+ * the paged-decode split kernel's first CTA sets up its first page copy but never issues it, so
+ * that stage's bounded wait (about 2 s of SM clocks) runs out: the CTA raises
+ * ATTN_DEVICE_TIMEOUT in the device status word, drains its own copies, and returns; the call's
+ * output for that chunk is then undefined. No memory outside the inputs is touched and the CUDA
+ * context stays usable. Applies to calls launched while enabled (attn_decode_paged,
+ * attn_decode_paged_noalloc, attn_decode_step).
+ */
+void attn_debug_drop_copy(int enable);
+
 /* Message of the last failure on the calling thread ("" if none). Owned by the library. */
 const char* attn_last_error(void);
 
