@@ -417,8 +417,10 @@ __global__ void __launch_bounds__(FwdCfg<D, kFp8>::THREADS, 1)
             if (R.n == 0) continue;
             const int i_pos = R.q0 + r;  // query position
             ok = ptx::mbar_wait(&bar->q_loaded[wg], kq & 1, abort_flag);
-            if (!ok) break;
-            if (!kFp8 && p.rope != nullptr && i_pos < p.N) {
+            // every thread of the warpgroup reaches the named barrier below, even after a wait
+            // gave up (threads may disagree at the moment the abort flag is raised); they leave
+            // the item loop only after it
+            if (!kFp8 && p.rope != nullptr && i_pos < p.N && ok) {
                 if (p.rope_half)
                     rope_rotate_smem_row_half<D>(sQ + wg * C::TILE_BYTES, r, p.rope + static_cast<size_t>(i_pos) * (D / 2));
                 else
@@ -428,6 +430,7 @@ __global__ void __launch_bounds__(FwdCfg<D, kFp8>::THREADS, 1)
             const float slope2 = kAlibi ? p.alibi[x.h] * kLog2e : 0.f;
             ptx::fence_proxy_async_smem();
             ptx::named_barrier_sync(1 + wg, 128);
+            if (!ok) break;
             if (r == 0) ptx::mbar_arrive(&bar->q_ready[wg]);
 
             float m_used = -INFINITY, l = 0.f;
@@ -494,20 +497,27 @@ __global__ void __launch_bounds__(FwdCfg<D, kFp8>::THREADS, 1)
                 }
                 const float m_eff = (m_used == -INFINITY) ? 0.f : m_used;
                 const float2 sl2 = make_float2(sl, sl), nm2 = make_float2(-m_eff, -m_eff);
-                // ALiBi: per pair, the addend is slope2*(k, k+1) + b0 - m instead of -m
-                const float2 sp2 = make_float2(slope2, slope2), bm2 = make_float2(b0 - m_eff, b0 - m_eff);
-                auto addend = [&](int k) {
-                    return kAlibi ? ptx::ffma2(sp2, make_float2(static_cast<float>(k), static_cast<float>(k + 1)), bm2)
-                                  : nm2;
-                };
+                // ALiBi: the addend of column k is slope2*k + b0 - m instead of -m; per group of 8
+                // columns one FMA gives the group's base, the other columns follow from it
+                const float bm = b0 - m_eff;
                 float2 acc0 = make_float2(0.f, 0.f), acc1 = acc0, acc2 = acc0, acc3 = acc0;
                 uint32_t pk[C::P_COLS];
 #pragma unroll
                 for (int k = 0; k < C::BN; k += 8) {
-                    float2 x0 = ptx::ffma2(make_float2(s[k], s[k + 1]), sl2, addend(k));
-                    float2 x1 = ptx::ffma2(make_float2(s[k + 2], s[k + 3]), sl2, addend(k + 2));
-                    float2 x2 = ptx::ffma2(make_float2(s[k + 4], s[k + 5]), sl2, addend(k + 4));
-                    float2 x3 = ptx::ffma2(make_float2(s[k + 6], s[k + 7]), sl2, addend(k + 6));
+                    float2 a0, a1, a2, a3;
+                    if constexpr (!kAlibi) {
+                        a0 = a1 = a2 = a3 = nm2;
+                    } else {
+                        const float bg = fmaf(slope2, static_cast<float>(k), bm);
+                        a0 = make_float2(bg, bg + slope2);
+                        a1 = make_float2(fmaf(slope2, 2.f, bg), fmaf(slope2, 3.f, bg));
+                        a2 = make_float2(fmaf(slope2, 4.f, bg), fmaf(slope2, 5.f, bg));
+                        a3 = make_float2(fmaf(slope2, 6.f, bg), fmaf(slope2, 7.f, bg));
+                    }
+                    float2 x0 = ptx::ffma2(make_float2(s[k], s[k + 1]), sl2, a0);
+                    float2 x1 = ptx::ffma2(make_float2(s[k + 2], s[k + 3]), sl2, a1);
+                    float2 x2 = ptx::ffma2(make_float2(s[k + 4], s[k + 5]), sl2, a2);
+                    float2 x3 = ptx::ffma2(make_float2(s[k + 6], s[k + 7]), sl2, a3);
                     x0 = make_float2(ptx::ex2(x0.x), ptx::ex2(x0.y));
                     x1 = make_float2(ptx::ex2(x1.x), ptx::ex2(x1.y));
                     x2 = make_float2(ptx::ex2(x2.x), ptx::ex2(x2.y));
