@@ -1,5 +1,7 @@
 """The seeded input generator: determinism, the 1/sqrt(d) variance argument, and the paged
 cache's structure (CPU only)."""
+import math
+
 import numpy as np
 import torch
 
@@ -59,3 +61,41 @@ def test_contiguous_copy_and_identity_order_hold_the_same_tokens():
             ta = pa.permute(1, 0, 2, 3).reshape(2, -1, 64)[:, :n]
             tx = px.permute(1, 0, 2, 3).reshape(2, -1, 64)[:, :n]
             assert torch.equal(ta.view(torch.int16), tx.view(torch.int16))
+
+
+def test_decode_step_inputs_poison_only_the_new_slots():
+    """The new tokens' slots (positions len-T .. len-1) hold NaN until an append fills them; every
+    earlier token is the plain cache's."""
+    lens = [3, 16, 17, 40]
+    plain = synth.paged_decode_inputs(len(lens), 8, 2, 64, 16, seq_lens=lens, seed=9, spare_frac=0.5)
+    st = synth.decode_step_inputs(len(lens), 3, 8, 2, 64, 16, seq_lens=lens, seed=9, spare_frac=0.5)
+    assert st.q.shape == (4, 3, 8, 64) and st.k_new.shape == (4, 3, 2, 64) and st.T == 3
+    for s, n in enumerate(lens):
+        for pos in range(n):
+            page, slot = int(st.cache.block_table[s, pos // 16]), pos % 16
+            got = st.cache.k_pages[page, :, slot]
+            if pos >= n - 3:
+                assert bool(torch.isnan(got.float()).all())
+            else:
+                assert torch.equal(got.view(torch.int16), plain.k_pages[page, :, slot].view(torch.int16))
+
+
+def test_fp8_inputs_are_exact_scaled_e4m3():
+    """Per-tensor descales are powers of two covering max|x| with e4m3's largest value 448, and the
+    e4m3 codes decode (through torch) to values within e4m3 rounding of the fp32 draws."""
+    f = synth.fp8_inputs(1, 2, 1, 64, 128, seed=3)
+    g = torch.Generator().manual_seed(3)
+    for x8, d in ((f.q8, f.descale_q), (f.k8, f.descale_k), (f.v8, f.descale_v)):
+        assert x8.dtype == torch.uint8
+        assert math.log2(d) == int(math.log2(d))
+        vals = x8.view(torch.float8_e4m3fn).double()
+        assert float(vals.abs().max()) <= 448.0 and not bool(torch.isnan(vals).any())
+    x = torch.randn((1, 2, 64, 128), generator=g, dtype=torch.float32).double()
+    back = f.q8.view(torch.float8_e4m3fn).double() * f.descale_q
+    assert float(((back - x).abs() - 2.0 ** -4 * x.abs() - 2.0 ** -9 * f.descale_q).max()) <= 0.0
+
+
+def test_alibi_slopes_are_the_geometric_sequence():
+    s = synth.alibi_slopes(8)
+    assert s.dtype == torch.float32 and s.shape == (8,)
+    assert torch.equal(s, torch.tensor([2.0 ** -(h + 1) for h in range(8)], dtype=torch.float32))
