@@ -41,7 +41,7 @@ def _check_pages(kp, vp, kp_ref, vp_ref):
 
 @pytest.mark.parametrize("T,Hq,Hkv,D,rope", [
     (1, 8, 2, 128, 10000.0), (2, 8, 2, 128, 10000.0), (4, 32, 8, 128, 500000.0), (3, 8, 2, 64, 10000.0),
-    (4, 16, 1, 128, 0.0), (8, 4, 4, 64, 10000.0), (16, 8, 2, 128, 10000.0)])
+    (4, 16, 1, 128, 0.0), (8, 4, 4, 64, 10000.0), (16, 8, 2, 128, 10000.0), (33, 8, 2, 64, 10000.0)])
 def test_step_vs_oracle(cuda_api, T, Hq, Hkv, D, rope):
     lens = [max(n, T) for n in LENS]
     inp = synth.decode_step_inputs(len(lens), T, Hq, Hkv, D, 16, seq_lens=lens, spare_frac=0.25, seed=T * 100 + Hq + D)
