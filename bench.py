@@ -57,8 +57,19 @@ def visible_pairs(N, causal, window):
     return w * (w + 1) // 2 + (N - w) * w
 
 
-def prefill_flops(cfg=PREFILL):
+def prefill_flops(cfg=None):
+    cfg = cfg or PREFILL
     return 4 * cfg.D * visible_pairs(cfg.N, cfg.causal, cfg.window) * cfg.B * cfg.Hq
+
+
+def prefill_label():
+    """Metric label of the timed prefill workload (the default is the causal GQA N=8192 one)."""
+    c = PREFILL
+    if c is synth.GQA_CAUSAL_N8192:
+        return "causal GQA prefill B2 Hq32 Hkv8 N8192 D128, RoPE 5e5"
+    mask = ("causal, window %d" % c.window) if c.window else ("causal" if c.causal else "no mask")
+    rope = (", RoPE %g" % c.rope_base) if c.rope_base > 0 else ""
+    return "prefill B%d Hq%d Hkv%d N%d D%d, %s%s" % (c.B, c.Hq, c.Hkv, c.N, c.D, mask, rope)
 
 
 def decode_bytes(cache):
@@ -206,7 +217,7 @@ def oracle_prefill_sample(q, k, v, budget_s):
         rows = np.linspace(0, total - 1, n_rows).astype(np.int64)
         flops = int((4 * D * ((rows % N) + 1)).sum())
         t0 = time.perf_counter()
-        oracle.attention(qb, kb, vb, causal=True, rope_base=PREFILL.rope_base, scale=PREFILL.scale, rows=rows)
+        oracle.attention(qb, kb, vb, causal=PREFILL.causal, window=PREFILL.window, rope_base=PREFILL.rope_base, scale=PREFILL.scale, rows=rows)
         return flops, time.perf_counter() - t0
 
     f, t = run(256)  # calibration (includes the one-off key rotation of every KV head)
@@ -503,8 +514,7 @@ def run_ours(args, rank, world, local):
             vv["roofline"].update({"peak": tensor_peak, "frac": round(vv["roofline"]["achieved"] / tensor_peak, 4),
                                    "peak_kind": "%s bf16 GEMM, sustained" % peaks_kind})
     line = {
-        "metric": "attn fwd TFLOP/s (causal GQA prefill B2 Hq32 Hkv8 N8192 D128, RoPE 5e5) "
-                  "& paged-decode KV GB/s",
+        "metric": "attn fwd TFLOP/s (%s) & paged-decode KV GB/s" % prefill_label(),
         "value": round(value, 2) if do_prefill else None,
         "unit": "TFLOP/s",
         "n_gpus": world,
@@ -585,7 +595,7 @@ def run_reference(args, rank, world):
     N, D = PREFILL.N, PREFILL.D
     rows_probe = np.linspace(0, N - 1, 16).astype(np.int64)
     t0 = time.perf_counter()
-    oracle.attention(qb, kb, vb, causal=True, rope_base=PREFILL.rope_base, scale=PREFILL.scale, rows=rows_probe)
+    oracle.attention(qb, kb, vb, causal=PREFILL.causal, window=PREFILL.window, rope_base=PREFILL.rope_base, scale=PREFILL.scale, rows=rows_probe)
     t_probe = time.perf_counter() - t0
     n_rows = int(max(4, min(N, 16 * per_step / max(t_probe, 1e-4))))
     rng = np.random.default_rng(0)
@@ -593,7 +603,7 @@ def run_reference(args, rank, world):
     for s in range(args.warmup + args.steps):
         rows = np.sort(rng.choice(N, size=n_rows, replace=False)).astype(np.int64)
         t0 = time.perf_counter()
-        oracle.attention(qb, kb, vb, causal=True, rope_base=PREFILL.rope_base, scale=PREFILL.scale, rows=rows)
+        oracle.attention(qb, kb, vb, causal=PREFILL.causal, window=PREFILL.window, rope_base=PREFILL.rope_base, scale=PREFILL.scale, rows=rows)
         dt = time.perf_counter() - t0
         if s >= args.warmup:
             flops_total += sum(4 * D * (int(i) + 1) for i in rows)
@@ -603,7 +613,7 @@ def run_reference(args, rank, world):
               "the oracle rotates that head's keys each step" % n_rows)
     return {
         "impl": "reference",
-        "metric": "attn fwd TFLOP/s (causal GQA prefill B2 Hq32 Hkv8 N8192 D128, RoPE 5e5) & paged-decode KV GB/s",
+        "metric": "attn fwd TFLOP/s (%s) & paged-decode KV GB/s" % prefill_label(),
         "value": round(value, 6),
         "unit": "TFLOP/s",
         "n_gpus": world,
@@ -633,6 +643,9 @@ def parse_args(argv=None):
     ap.add_argument("--step-calls", type=int, default=50, help="decode-step calls timed per q_len; 0 skips")
     ap.add_argument("--variant-calls", type=int, default=20, help="position-variant prefill calls timed each; 0 skips")
     ap.add_argument("--fp8-calls", type=int, default=20, help="FP8 prefill calls timed; 0 skips")
+    ap.add_argument("--prefill-workload", choices=[c.name for c in synth.PREFILL_CONFIGS],
+                    default=synth.GQA_CAUSAL_N8192.name,
+                    help="prefill workload to time (default: the causal GQA N=8192 one)")
     ap.add_argument("--only", choices=["all", "prefill", "decode"], default="all",
                     help="time one half of the step only (profiling runs); the JSON line is then partial")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle time for the CPU baseline")
@@ -644,7 +657,9 @@ def parse_args(argv=None):
 
 
 def main(argv=None):
+    global PREFILL
     args = parse_args(argv)
+    PREFILL = next(c for c in synth.PREFILL_CONFIGS if c.name == args.prefill_workload)
     rank, world, local = dist_env()
     if world != args.gpus:
         print("warning: --gpus %d but WORLD_SIZE %d; using WORLD_SIZE" % (args.gpus, world), file=sys.stderr)
