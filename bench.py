@@ -2,8 +2,8 @@
 """Benchmark of the exact-attention hot path on B200.
 
 One step is one pass of the whole hot path over one batch of synthetic input:
-  prefill  causal GQA attention with RoPE, B=2, Hq=32, Hkv=8, N=8192, D=128 (attn_fwd: the key
-           rotation pass plus the attention kernel), and
+  prefill  causal GQA attention with RoPE, B=2, Hq=32, Hkv=8, N=8192, D=128 (attn_fwd: the
+           query/key rotation pass plus the attention kernel), and
   decode   one paged-KV decode token for 64 sequences with lengths uniform in [512, 16384],
            Hq=32, Hkv=8, D=128, 16-token pages (attn_decode_paged: split kernel plus merge).
 The headline value is prefill TFLOP/s (algorithmic FLOPs = 4*D per unmasked (query, key) pair per
@@ -550,7 +550,8 @@ def run_ours(args, rank, world, local):
                      "peak_kind": "%s bf16 GEMM, sustained" % peaks_kind,
                      "frac_of_2250": round(tflops_launch / DATASHEET_BF16_TFLOPS, 4),
                      "traffic": profiled_traffic("attn_fwd"),
-                     "kernel": "attn_fwd_kernel<128> (+ key rotation pass, inside the timed call)"},
+                     "rotation_pass_traffic": profiled_traffic("rope_rows"),
+                     "kernel": "attn_fwd_kernel<128> (+ query/key rotation pass, inside the timed call)"},
         "e2e": {"value": round(e2e_value, 2) if E else None, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": (2 * do_prefill + 2 * do_decode) * K,

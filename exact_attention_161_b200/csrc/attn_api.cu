@@ -92,24 +92,28 @@ struct DevBuf {
 std::atomic<bool> g_debug_drop_copy{false};  // test hook of attn_debug_drop_copy
 
 std::mutex g_cache_mu;
-// (device, base, D, position scale, NTK factor, fp64?) -> cos/sin table covering positions [0, capacity)
-std::map<std::tuple<int, double, int, double, double, bool>, std::pair<DevBuf, int>> g_rope_tables;
+// Layouts of a cos/sin table covering positions [0, cap): (cos, sin) pairs, [cap][D/2], one
+// position's pairs contiguous, in fp32 (kTab32) or fp64 (kTab64)
+enum TabLayout { kTab32 = 0, kTab64 = 1 };
+// (device, base, D, position scale, NTK factor, layout) -> table and its capacity
+std::map<std::tuple<int, double, int, double, double, int>, std::pair<DevBuf, int>> g_rope_tables;
 // (device, stream) -> rotated-key scratch
 std::map<std::pair<int, void*>, DevBuf> g_key_scratch;
 std::vector<DevBuf> g_retired;  // outgrown buffers; a launch still queued may read them
 
 // (cos, sin) of (pos / pos_scale) * b^(-2i/D), b = base * ntk^(D/(D-2)), for pos < n, i < D/2:
 // angles and trigonometry in fp64 (Position Interpolation divides the positions; NTK-aware scaling
-// raises the base), stored as fp64 pairs (wide) or rounded to fp32 pairs.
-attn_status rope_table_any(int dev, double base, int D, int n, double pos_scale, double ntk, bool wide,
+// raises the base), stored in fp64 or rounded to fp32.
+attn_status rope_table_any(int dev, double base, int D, int n, double pos_scale, double ntk, int layout,
                            const void** out) {
     std::lock_guard<std::mutex> lock(g_cache_mu);
-    auto key = std::make_tuple(dev, base, D, pos_scale, ntk, wide);
+    auto key = std::make_tuple(dev, base, D, pos_scale, ntk, layout);
     auto it = g_rope_tables.find(key);
     if (it != g_rope_tables.end() && it->second.second >= n) {
         *out = it->second.first.ptr;
         return ATTN_OK;
     }
+    const bool wide = layout == kTab64;
     const int cap = ((n + 1023) / 1024) * 1024;
     const size_t pairs = static_cast<size_t>(cap) * (D / 2);
     std::vector<double2> host64(wide ? pairs : 0);
@@ -144,18 +148,17 @@ attn_status rope_table_any(int dev, double base, int D, int n, double pos_scale,
 attn_status rope_table(int dev, double base, int D, int n, const float2** out, double pos_scale = 1.0,
                        double ntk = 1.0) {
     const void* p = nullptr;
-    attn_status st = rope_table_any(dev, base, D, n, pos_scale, ntk, false, &p);
+    attn_status st = rope_table_any(dev, base, D, n, pos_scale, ntk, kTab32, &p);
     *out = static_cast<const float2*>(p);
     return st;
 }
 attn_status rope_table64(int dev, double base, int D, int n, const double2** out, double pos_scale = 1.0,
                          double ntk = 1.0) {
     const void* p = nullptr;
-    attn_status st = rope_table_any(dev, base, D, n, pos_scale, ntk, true, &p);
+    attn_status st = rope_table_any(dev, base, D, n, pos_scale, ntk, kTab64, &p);
     *out = static_cast<const double2*>(p);
     return st;
 }
-
 attn_status key_scratch(int dev, void* stream, size_t bytes, void** out) {
     std::lock_guard<std::mutex> lock(g_cache_mu);
     DevBuf& b = g_key_scratch[std::make_pair(dev, stream)];
@@ -185,6 +188,38 @@ attn_status ensure_smem(K kernel, int bytes, int dev) {
     return ATTN_OK;
 }
 
+// Rotate Q (bhq rows of N positions) and K (bhk rows) into qr and kr with one launch of
+// rope_rotate_rows_kernel: x covers the N * D/8 (position, chunk) pairs with 256 threads a block,
+// at most 8 blocks per SM (the x loop strides over the rest); z picks the tensor; y splits the
+// rows so that about 8 blocks per SM are resident however few positions there are.
+template <int D>
+attn_status launch_rope_rows(bool half, const void* q, void* qr, long long bhq, const void* k, void* kr, long long bhk,
+                             const double2* cs, int N, int sms, cudaStream_t stream) {
+    attn::RopeRowsArgs a{};
+    a.src[0] = static_cast<const uint4*>(q);
+    a.dst[0] = static_cast<uint4*>(qr);
+    a.bh[0] = bhq;
+    a.src[1] = static_cast<const uint4*>(k);
+    a.dst[1] = static_cast<uint4*>(kr);
+    a.bh[1] = bhk;
+    a.cs = cs;
+    a.N = N;
+    const long long want = (static_cast<long long>(N) * (D / 8) + 255) / 256;
+    const long long gx = want < 8LL * sms ? want : 8LL * sms;
+    const long long bh_max = bhq > bhk ? bhq : bhk;
+    long long gy = (8LL * sms + 2 * gx - 1) / (2 * gx);
+    if (gy > bh_max) gy = bh_max;
+    if (gy > 65535) gy = 65535;
+    if (gy < 1) gy = 1;
+    const dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(gy), 2);
+    if (half)
+        attn::rope_rotate_rows_kernel<D, true><<<grid, 256, 0, stream>>>(a);
+    else
+        attn::rope_rotate_rows_kernel<D, false><<<grid, 256, 0, stream>>>(a);
+    CUDA_TRY(cudaGetLastError());
+    return ATTN_OK;
+}
+
 struct PosVariant {
     int half_split = 0;
     double pos_scale = 1.0, ntk = 1.0;
@@ -196,41 +231,35 @@ attn_status launch_fwd(const void* q, const void* k, const void* v, void* o, flo
                        int N, int causal, int window, float rope_base, float scale, cudaStream_t stream, int dev,
                        const PosVariant& pv = PosVariant()) {
     using C = attn::FwdCfg<D>;
+    const void* q_use = q;
     const void* k_use = k;
     attn::FwdParams p{};
     if (rope_base > 0.f) {
-        const float2* table = nullptr;
-        attn_status st = rope_table(dev, static_cast<double>(rope_base), D, N, &table, pv.pos_scale, pv.ntk);
-        if (st != ATTN_OK) return st;
         const double2* table64 = nullptr;
-        st = rope_table64(dev, static_cast<double>(rope_base), D, N, &table64, pv.pos_scale, pv.ntk);
+        attn_status st = rope_table64(dev, static_cast<double>(rope_base), D, N, &table64, pv.pos_scale, pv.ntk);
         if (st != ATTN_OK) return st;
-        void* k_rot = nullptr;
+        // rotated Q, then rotated K (256-byte aligned), in the stream's scratch
+        const size_t qbytes = static_cast<size_t>(B) * Hq * N * D * 2;
         const size_t kbytes = static_cast<size_t>(B) * Hkv * N * D * 2;
-        st = key_scratch(dev, stream, kbytes, &k_rot);
+        const size_t koff = (qbytes + 255) / 256 * 256;
+        void* scratch = nullptr;
+        st = key_scratch(dev, stream, koff + kbytes, &scratch);
         if (st != ATTN_OK) return st;
-        const long long rows = static_cast<long long>(B) * Hkv * N;
-        const long long chunks = static_cast<long long>(N) * (D / 8);  // one thread per (position, chunk)
+        void* q_rot = scratch;
+        void* k_rot = static_cast<char*>(scratch) + koff;
         int sms = 148;
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        const long long want = (chunks + 255) / 256;
-        const int grid = static_cast<int>(want < 8LL * sms ? want : 8LL * sms);
-        if (pv.half_split)
-            attn::rope_rotate_rows_kernel<D, true><<<grid, 256, 0, stream>>>(static_cast<const uint4*>(k),
-                                                                             static_cast<uint4*>(k_rot), table64, rows, N);
-        else
-            attn::rope_rotate_rows_kernel<D><<<grid, 256, 0, stream>>>(static_cast<const uint4*>(k),
-                                                                       static_cast<uint4*>(k_rot), table64, rows, N);
-        CUDA_TRY(cudaGetLastError());
+        st = launch_rope_rows<D>(pv.half_split != 0, q, q_rot, static_cast<long long>(B) * Hq, k, k_rot,
+                                 static_cast<long long>(B) * Hkv, table64, N, sms, stream);
+        if (st != ATTN_OK) return st;
+        q_use = q_rot;
         k_use = k_rot;
-        p.rope = table;
-        p.rope_half = pv.half_split;
     }
     p.alibi = pv.alibi;
     p.o_scale = 1.f;
     CUtensorMap tq, tk, tv;
     attn_status st;
-    if ((st = make_map_3d(&tq, q, D, N, static_cast<uint64_t>(B) * Hq, 128)) != ATTN_OK) return st;
+    if ((st = make_map_3d(&tq, q_use, D, N, static_cast<uint64_t>(B) * Hq, 128)) != ATTN_OK) return st;
     if ((st = make_map_3d(&tk, k_use, D, N, static_cast<uint64_t>(B) * Hkv, 128)) != ATTN_OK) return st;
     if ((st = make_map_3d(&tv, v, D, N, static_cast<uint64_t>(B) * Hkv, 128)) != ATTN_OK) return st;
     p.o = static_cast<__nv_bfloat16*>(o);
@@ -421,17 +450,9 @@ attn_status launch_bwd(const void* q, const void* k, const void* v, const void* 
         p.rope = table;
         void* qr = w + L.qrot;
         void* kr = w + L.krot;
-        const long long qrows = static_cast<long long>(B) * Hq * N, krows = static_cast<long long>(B) * Hkv * N;
-        auto grid_for = [&](long long) {  // one thread per (position, chunk); rows loop inside
-            const long long want = (static_cast<long long>(N) * (D / 8) + 255) / 256;
-            return static_cast<int>(want < 8LL * sms ? want : 8LL * sms);
-        };
-        attn::rope_rotate_rows_kernel<D><<<grid_for(qrows), 256, 0, stream>>>(static_cast<const uint4*>(q),
-                                                                              static_cast<uint4*>(qr), table64, qrows, N);
-        CUDA_TRY(cudaGetLastError());
-        attn::rope_rotate_rows_kernel<D><<<grid_for(krows), 256, 0, stream>>>(static_cast<const uint4*>(k),
-                                                                              static_cast<uint4*>(kr), table64, krows, N);
-        CUDA_TRY(cudaGetLastError());
+        st = launch_rope_rows<D>(false, q, qr, static_cast<long long>(B) * Hq, k, kr, static_cast<long long>(B) * Hkv,
+                                 table64, N, sms, stream);
+        if (st != ATTN_OK) return st;
         q_use = qr;
         k_use = kr;
     }

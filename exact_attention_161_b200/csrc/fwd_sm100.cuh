@@ -12,11 +12,11 @@
 //
 // Roles (320 threads):
 //   warps 0-3, 4-7  softmax warpgroup i (i = 0, 1) owns query tile i; thread r owns row r (TMEM
-//              lane r). It rotates its Q row (RoPE) once, then per key tile reads its 128 scores
-//              from TMEM with one load, masks them, updates m and l, writes P (bf16) back into
-//              TMEM over the first half of its score buffer, rescales its row of O when the max
-//              moved by more than 2^8, and finally reads O out of TMEM (releasing it for the
-//              next item's products) and writes O and LSE.
+//              lane r). Per key tile it reads its 128 scores from TMEM with one load, masks them,
+//              updates m and l, writes P (bf16) back into TMEM over the first half of its score
+//              buffer, rescales its row of O when the max moved by more than 2^8, and finally
+//              reads O out of TMEM (releasing it for the next item's products) and writes O and
+//              LSE. Q and K arrive already rotated (RoPE) by a streaming pass before the kernel.
 //   warp 8     TMA producer: the Q tiles once, then K tiles into a NK-stage ring and V tiles into
 //              a NV-stage ring.
 //   warp 9     MMA issuer (one thread) and TMEM owner.
@@ -41,9 +41,7 @@ namespace attn {
 struct FwdParams {
     __nv_bfloat16* o;       // [B, Hq, N, D]
     float* lse;             // [B, Hq, N] natural-log row logsumexp, or nullptr
-    const float2* rope;     // [>= N, D/2] (cos, sin) of pair i at pos, or nullptr (no RoPE)
     const float* alibi;     // [Hq] ALiBi slopes m_h (logit minus m_h (i - j)), read when kAlibi
-    int rope_half;          // 1: half-split pairing (i, i + D/2); the key pass permutes to match
     float o_scale;          // output multiplier (the FP8 path's V descale; 1 otherwise)
     int B, Hq, Hkv, N;
     int causal, window;     // window > 0 only together with causal
@@ -86,7 +84,7 @@ struct FwdCfg {
 
 template <int NK, int NV>
 struct FwdBarriers {
-    uint64_t q_loaded[2], q_ready[2], q_empty[2];
+    uint64_t q_loaded[2], q_empty[2];
     uint64_t k_full[NK], k_empty[NK], v_full[NV], v_empty[NV];
     uint64_t s_full[2], p_full[2], o_final[2], o_empty[2];
     uint64_t drain;
@@ -107,71 +105,6 @@ __device__ __forceinline__ TileRange tile_range(int q0, int N, int causal, int w
     t.jb = lo / 128;
     t.n = (hi + 127) / 128 - t.jb;
     return t;
-}
-
-// Rotate one 128-byte-swizzled row of a Q tile in place: pairs (2i, 2i+1) by pos * theta_i, in
-// fp32 with the (cos, sin) table, rounded back to bf16 ("attention-transformers", Q "How does
-// Rotary Position Embedding (RoPE) work?"). The table loads of each 64-column region are issued
-// together, so their latency is paid once per region rather than once per 16-byte chunk.
-template <int D>
-__device__ __forceinline__ void rope_rotate_smem_row(uint8_t* tile, int r, const float2* __restrict__ cs_row) {
-    using C = FwdCfg<D>;
-#pragma unroll
-    for (int reg = 0; reg < C::NREG; ++reg) {
-        float4 cs[16];
-#pragma unroll
-        for (int c = 0; c < 16; ++c) cs[c] = __ldg(reinterpret_cast<const float4*>(cs_row + reg * 32 + 2 * c));
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-            uint4* p = reinterpret_cast<uint4*>(tile + reg * C::REGION_BYTES + r * 128 + ((c ^ (r & 7)) << 4));
-            uint4 w = *p;
-            uint32_t* wv = reinterpret_cast<uint32_t*>(&w);
-            const float t[8] = {cs[2 * c].x, cs[2 * c].y, cs[2 * c].z, cs[2 * c].w,
-                                cs[2 * c + 1].x, cs[2 * c + 1].y, cs[2 * c + 1].z, cs[2 * c + 1].w};
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const float x0 = ptx::bf16lo_to_f32(wv[k]), x1 = ptx::bf16hi_to_f32(wv[k]);
-                const float cth = t[2 * k], sth = t[2 * k + 1];
-                wv[k] = ptx::pack_bf16x2(fmaf(x0, cth, -x1 * sth), fmaf(x0, sth, x1 * cth));
-            }
-            *p = w;
-        }
-    }
-}
-
-// Half-split pairing: the row's pairs (i, i + D/2) are rotated and written back interleaved, at
-// (2i, 2i+1). The key rotation pass applies the same permutation, and a score q.k is unchanged when
-// the dimensions of q and k are permuted alike, so the rest of the kernel is the interleaved one.
-// The whole row is read into registers before anything is written back.
-template <int D>
-__device__ __forceinline__ void rope_rotate_smem_row_half(uint8_t* tile, int r, const float2* __restrict__ cs_row) {
-    using C = FwdCfg<D>;
-    uint32_t w[D / 2];
-#pragma unroll
-    for (int reg = 0; reg < C::NREG; ++reg)
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-            const uint4 v = *reinterpret_cast<const uint4*>(tile + reg * C::REGION_BYTES + r * 128 + ((c ^ (r & 7)) << 4));
-            w[reg * 32 + c * 4 + 0] = v.x;
-            w[reg * 32 + c * 4 + 1] = v.y;
-            w[reg * 32 + c * 4 + 2] = v.z;
-            w[reg * 32 + c * 4 + 3] = v.w;
-        }
-#pragma unroll
-    for (int oc = 0; oc < D / 8; ++oc) {  // output chunk: pairs 4 oc .. 4 oc + 3
-        uint32_t ow[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const int pi = oc * 4 + k;
-            const uint32_t a = w[pi / 2], b = w[pi / 2 + D / 4];
-            const float x0 = (pi & 1) ? ptx::bf16hi_to_f32(a) : ptx::bf16lo_to_f32(a);
-            const float x1 = (pi & 1) ? ptx::bf16hi_to_f32(b) : ptx::bf16lo_to_f32(b);
-            const float2 t = __ldg(cs_row + pi);
-            ow[k] = ptx::pack_bf16x2(fmaf(x0, t.x, -x1 * t.y), fmaf(x0, t.y, x1 * t.x));
-        }
-        *reinterpret_cast<uint4*>(tile + (oc / 8) * C::REGION_BYTES + r * 128 + (((oc % 8) ^ (r & 7)) << 4)) =
-            make_uint4(ow[0], ow[1], ow[2], ow[3]);
-    }
 }
 
 // One work item: (batch b, query head h, block of 256 queries); the longest causal blocks come
@@ -227,7 +160,6 @@ __global__ void __launch_bounds__(FwdCfg<D, kFp8>::THREADS, 1)
     if (threadIdx.x == 0) {
         for (int i = 0; i < 2; ++i) {
             ptx::mbar_init(&bar->q_loaded[i], 1);
-            ptx::mbar_init(&bar->q_ready[i], 1);
             ptx::mbar_init(&bar->q_empty[i], 1);
             ptx::mbar_init(&bar->s_full[i], 1);
             ptx::mbar_init(&bar->p_full[i], 128);
@@ -362,11 +294,8 @@ __global__ void __launch_bounds__(FwdCfg<D, kFp8>::THREADS, 1)
                         if (u + 1 < x.T && x.active(i, u + 1)) {
                             // S_i(u+1) = Q_i K(u+1)^T into score buffer i
                             const int c = x.J0 + u + 1 - R.jb;
-                            if (c == 0) {
-                                if (!ptx::mbar_wait(&bar->q_ready[i], kq & 1, abort_flag)) { ok = false; break; }
-                                ptx::tc_fence_after();
-                            }
-                            // K arrives by TMA: the barrier alone orders it before the MMA's reads
+                            // Q and K arrive by TMA: the barriers alone order them before the MMA's reads
+                            if (c == 0 && !ptx::mbar_wait(&bar->q_loaded[i], kq & 1, abort_flag)) { ok = false; break; }
                             if (!ptx::mbar_wait(&bar->k_full[(g + u + 1) % NK], ((g + u + 1) / NK) & 1, abort_flag)) { ok = false; break; }
                             const uint32_t qa = q_lo + i * TILE16, kb = k_lo + ((g + u + 1) % NK) * TILE16;
 #pragma unroll
@@ -409,6 +338,12 @@ __global__ void __launch_bounds__(FwdCfg<D, kFp8>::THREADS, 1)
         const uint32_t t_s = tmem + lane_base + C::tmem_s(wg);
         const uint32_t t_o = tmem + lane_base + C::tmem_o(wg);
         const float sl = p.scale_log2;
+        // The warpgroup never touches Q: the MMA warp computes an item's first scores as soon as
+        // its query tile has landed (the tile's buffer was freed by the previous item's last score
+        // MMA), which overlaps them with this warpgroup's epilogue of the previous item. Score
+        // buffer reuse is ordered by the MMA warp issuing P(n, last) V before S(n+1, 0), and item
+        // n+1's first P V waits for o_empty, which the epilogue arrives on. Waits are made uniform
+        // per warp, because the tile loop holds warp-wide votes.
         bool ok = true;
         int kq = 0, cw = 0;
         for (int rnd = 0, it = blockIdx.x; ok && it < p.n_items; it = item_of_round(++rnd, blockIdx.x, gridDim.x)) {
@@ -416,27 +351,13 @@ __global__ void __launch_bounds__(FwdCfg<D, kFp8>::THREADS, 1)
             const TileRange R = x.rng[wg];
             if (R.n == 0) continue;
             const int i_pos = R.q0 + r;  // query position
-            ok = ptx::mbar_wait(&bar->q_loaded[wg], kq & 1, abort_flag);
-            // every thread of the warpgroup reaches the named barrier below, even after a wait
-            // gave up (threads may disagree at the moment the abort flag is raised); they leave
-            // the item loop only after it
-            if (!kFp8 && p.rope != nullptr && i_pos < p.N && ok) {
-                if (p.rope_half)
-                    rope_rotate_smem_row_half<D>(sQ + wg * C::TILE_BYTES, r, p.rope + static_cast<size_t>(i_pos) * (D / 2));
-                else
-                    rope_rotate_smem_row<D>(sQ + wg * C::TILE_BYTES, r, p.rope + static_cast<size_t>(i_pos) * (D / 2));
-            }
             // ALiBi: this head's slope in log2 units
             const float slope2 = kAlibi ? p.alibi[x.h] * kLog2e : 0.f;
-            ptx::fence_proxy_async_smem();
-            ptx::named_barrier_sync(1 + wg, 128);
-            if (!ok) break;
-            if (r == 0) ptx::mbar_arrive(&bar->q_ready[wg]);
 
             float m_used = -INFINITY, l = 0.f;
             for (int c = 0; ok && c < R.n; ++c) {
                 const int j0 = (R.jb + c) * C::BN;
-                if (!ptx::mbar_wait(&bar->s_full[wg], (cw + c) & 1, abort_flag)) { ok = false; break; }
+                if (!__all_sync(0xffffffffu, ptx::mbar_wait(&bar->s_full[wg], (cw + c) & 1, abort_flag))) { ok = false; break; }
                 ptx::tc_fence_after();
                 uint32_t sv[C::BN];
                 ptx::tmem_ld128(t_s, sv);
@@ -568,7 +489,7 @@ __global__ void __launch_bounds__(FwdCfg<D, kFp8>::THREADS, 1)
             if (!ok) break;
             cw += R.n;
             // ---- epilogue: O_i out of TMEM (then the next item may overwrite it), O = o / l, LSE
-            if (!ptx::mbar_wait(&bar->o_final[wg], kq & 1, abort_flag)) { ok = false; break; }
+            if (!__all_sync(0xffffffffu, ptx::mbar_wait(&bar->o_final[wg], kq & 1, abort_flag))) { ok = false; break; }
             ptx::tc_fence_after();
             uint32_t w[D / 2];
             const float inv_l = l > 0.f ? p.o_scale / l : 0.f;

@@ -1,14 +1,14 @@
-// rope.cuh -- rotary position embedding of the key rows, once per call.
+// rope.cuh -- rotary position embedding of the query and key rows, once per call.
 //
 // RoPE rotates each pair (2i, 2i+1) of a query or key vector by the angle pos * base^(-2i/D)
 // ("attention-transformers", Q "How does Rotary Position Embedding (RoPE) work?"; pairs are the
-// interleaved 2-D subspaces). Queries are rotated inside the attention kernel right after their
-// tile lands in shared memory (once per query tile). Keys are rotated here, by one streaming
-// pass over K: every key tile is read by many query tiles (all of its query heads, and every
-// later query tile under a causal mask), so rotating it inside the attention kernel would
-// repeat the same rotation tens of times per tile and compete with the softmax for the FP32
-// pipes. This pass moves 2 bytes in and 2 bytes out per element, about 1% of the attention
-// kernel's time at N = 8192.
+// interleaved 2-D subspaces). Queries and keys are rotated here, by one streaming pass over Q and
+// K in one launch, before the attention kernel reads them. Every key tile is read by many query
+// tiles, so rotating keys inside the attention kernel would repeat the same rotation tens of
+// times per tile; a query tile is used once, but rotating it inside the kernel puts 64 KB of
+// cos/sin table per query tile through the SM and the rotation on the tensor core's critical
+// path at every work item, which measured slower than this pass's extra read and write of Q.
+// The rotation itself is exact (fp64, below), so rotated operands equal an fp64 reference's.
 #pragma once
 #include "ptx.cuh"
 
@@ -28,49 +28,71 @@ __device__ __forceinline__ uint32_t rope_rotate_pair(uint32_t w, double cth, dou
     return lo | (hi << 16);
 }
 
-// k, k_rot: [rows, D] bf16 with row r at position r % N (rows = BH * N); cs: [>= N, D/2] (cos, sin)
-// in fp64. A thread takes one 16-byte output chunk (4 pairs) of one position, loads that chunk's 4
-// table entries once and applies them to the chunk in every one of the BH rows at the position;
-// consecutive threads take consecutive chunks, so each row's loads and stores are coalesced.
+// Up to two tensors per launch, blockIdx.z selecting one: src[z], dst[z]: [bh[z] * N, D] bf16
+// with row r at position r % N; cs: [>= N, D/2] (cos, sin) in fp64.
+struct RopeRowsArgs {
+    const uint4* src[2];
+    uint4* dst[2];
+    long long bh[2];
+    const double2* cs;
+    int N;
+};
+
+// A thread takes one 16-byte output chunk (4 pairs) of one position, loads that chunk's 4 table
+// entries once and applies them to the chunk in rows blockIdx.y, blockIdx.y + gridDim.y, ... of
+// the bh rows at that position, loading 4 such rows before it stores any, so that several loads
+// are in flight per thread. Consecutive threads take consecutive chunks, so each row's loads and
+// stores are coalesced; the y split keeps a short sequence (few positions, many rows) from
+// running on fewer blocks than there are SMs.
 // kHalf: the pairs are (i, i + D/2) and the rotated pair i is written interleaved at (2i, 2i+1) --
-// the dimensions are permuted so that the attention kernel, which rotates its queries the same
-// way, can treat both pairings alike.
+// the dimensions are permuted, the same for queries and keys, which leaves every score q.k
+// unchanged, so the attention kernel treats both pairings alike.
 template <int D, bool kHalf = false>
-__global__ void __launch_bounds__(256) rope_rotate_rows_kernel(const uint4* __restrict__ k, uint4* __restrict__ k_rot,
-                                                               const double2* __restrict__ cs, long long rows, int N) {
+__global__ void __launch_bounds__(256) rope_rotate_rows_kernel(RopeRowsArgs a) {
     constexpr int CHUNKS = D / 8;
-    const long long bh_count = rows / N;
+    constexpr int U = 4;  // rows in flight per thread
+    const int z = blockIdx.z;
+    const uint4* __restrict__ src = z ? a.src[1] : a.src[0];
+    uint4* __restrict__ dst = z ? a.dst[1] : a.dst[0];
+    const long long bh_count = z ? a.bh[1] : a.bh[0];
+    const int N = a.N;
     const long long total = static_cast<long long>(N) * CHUNKS;
+    const long long ys = gridDim.y;
     for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
          idx += (long long)gridDim.x * blockDim.x) {
         const int pos = static_cast<int>(idx / CHUNKS);
         const int c = static_cast<int>(idx % CHUNKS);
         double2 t[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) t[e] = __ldg(cs + static_cast<size_t>(pos) * (D / 2) + c * 4 + e);
-#pragma unroll 4
-        for (long long bh = 0; bh < bh_count; ++bh) {
-            const long long row = bh * N + pos;
-            uint4 w;
-            if constexpr (kHalf) {
-                // pairs 4c .. 4c+3: first members at elements 4c.., second members at D/2 + 4c..
-                const uint2* src = reinterpret_cast<const uint2*>(k + row * CHUNKS);
-                const uint2 a = __ldg(src + c), b = __ldg(src + c + D / 8);
-                const uint32_t av[2] = {a.x, a.y}, bv[2] = {b.x, b.y};
-                uint32_t* wv = reinterpret_cast<uint32_t*>(&w);
+        for (int e = 0; e < 4; ++e) t[e] = __ldg(a.cs + static_cast<size_t>(pos) * (D / 2) + c * 4 + e);
+        for (long long bh0 = blockIdx.y; bh0 < bh_count; bh0 += U * ys) {
+            uint4 w[U];
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const uint32_t lo = (e & 1) ? (av[e / 2] >> 16) : (av[e / 2] & 0xFFFFu);
-                    const uint32_t hi = (e & 1) ? (bv[e / 2] >> 16) : (bv[e / 2] & 0xFFFFu);
-                    wv[e] = lo | (hi << 16);
+            for (int j = 0; j < U; ++j) {
+                const long long bh = bh0 + j * ys;
+                if (bh >= bh_count) continue;
+                const long long row = bh * N + pos;
+                if constexpr (kHalf) {
+                    // pairs 4c .. 4c+3: first members at elements 4c.., second members at D/2 + 4c..
+                    const uint2* s2 = reinterpret_cast<const uint2*>(src + row * CHUNKS);
+                    const uint2 lo = __ldg(s2 + c), hi = __ldg(s2 + c + D / 8);
+                    w[j].x = (lo.x & 0xFFFFu) | (hi.x << 16);
+                    w[j].y = (lo.x >> 16) | (hi.x & 0xFFFF0000u);
+                    w[j].z = (lo.y & 0xFFFFu) | (hi.y << 16);
+                    w[j].w = (lo.y >> 16) | (hi.y & 0xFFFF0000u);
+                } else {
+                    w[j] = __ldg(src + row * CHUNKS + c);
                 }
-            } else {
-                w = __ldg(k + row * CHUNKS + c);
             }
-            uint32_t* wv = reinterpret_cast<uint32_t*>(&w);
 #pragma unroll
-            for (int e = 0; e < 4; ++e) wv[e] = rope_rotate_pair(wv[e], t[e].x, t[e].y);
-            k_rot[row * CHUNKS + c] = w;
+            for (int j = 0; j < U; ++j) {
+                const long long bh = bh0 + j * ys;
+                if (bh >= bh_count) continue;
+                uint32_t* wv = reinterpret_cast<uint32_t*>(&w[j]);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) wv[e] = rope_rotate_pair(wv[e], t[e].x, t[e].y);
+                dst[(bh * N + pos) * CHUNKS + c] = w[j];
+            }
         }
     }
 }

@@ -16,9 +16,9 @@
  *     message readable with attn_last_error(). Faults detected on the device (a bounded wait
  *     that gave up, an out-of-range block-table entry) set bits of a device status word read
  *     with attn_get_device_status().
- *   - The library owns only its caches (RoPE cos/sin tables per (device, base, head dim); key
- *     scratch per (device, stream) for the rotated keys; the device status word); attn_shutdown
- *     releases them.
+ *   - The library owns only its caches (RoPE cos/sin tables per (device, base, head dim); a
+ *     scratch per (device, stream) for the rotated queries and keys of attn_fwd and
+ *     attn_fwd_pos; the device status word); attn_shutdown releases them.
  *   - There is no CPU fallback: without a B200 every compute call returns ATTN_ERR_CUDA.
  */
 #ifndef ATTN_B200_H
@@ -68,7 +68,9 @@ typedef enum {
  *          requires causal = 1. <=0: no window.
  *   rope_base  >0: rotate q and k pairwise, pairs (2t, 2t+1) by pos * rope_base^(-2t/D), pos =
  *          the token index 0..N-1, counter-clockwise, then round to bf16 ("attention-transformers",
- *          Q "How does Rotary Position Embedding (RoPE) work?"). <=0: no rotation.
+ *          Q "How does Rotary Position Embedding (RoPE) work?"); the rotation is computed in
+ *          fp64 and rounded once, into the library's scratch, before the attention kernel.
+ *          <=0: no rotation.
  *   scale  >0: softmax scale; <=0: 1/sqrt(D) ("Why is attention scaled by 1/sqrt(dk)?").
  * Constraints: B, Hq, Hkv, N >= 1; Hq % Hkv == 0; D in {64, 128} (else ATTN_ERR_UNSUPPORTED);
  * B * Hq * ceil(N/256) < 2^31. Fully masked key tiles are skipped, not computed.
@@ -286,7 +288,7 @@ const char* attn_last_error(void);
 /* Library version string. */
 const char* attn_version(void);
 
-/* Frees every cache the library allocated (RoPE tables, key scratch), on every device.
+/* Frees every cache the library allocated (RoPE tables, query/key scratch), on every device.
  * The caller must ensure no call is still running on the GPU. */
 void attn_shutdown(void);
 
