@@ -96,6 +96,30 @@ def test_half_split_is_interleaved_on_permuted_dims(cuda_api, D):
     assert torch.equal(o1.view(torch.int16), o2.view(torch.int16)) and torch.equal(l1, l2)
 
 
+@pytest.mark.parametrize("D,half,ps,ntk", [(128, False, 1.0, 1.0), (64, False, 1.0, 1.0), (128, True, 2.0, 4.0)])
+def test_rope_pass_rotates_exactly(cuda_api, D, half, ps, ntk):
+    """With RoPE, the forward equals bit for bit the forward without RoPE on q and k rotated by the
+    oracle (for half-split pairing with the dimensions permuted to the interleaved order the
+    library uses): the library rotates each element in fp64 and rounds it once to bf16, as the
+    oracle does, so the attention kernel sees the oracle's rotated operands."""
+    B, Hq, Hkv, N, base = 2, 4, 2, 333, 10000.0
+    q, k, v = synth.prefill_inputs(B, Hq, Hkv, N, D, seed=523)
+    perm = torch.stack([torch.arange(D // 2), torch.arange(D // 2) + D // 2], 1).reshape(-1)
+
+    def rotated(x):
+        rows = bits(x).reshape(-1, D)
+        pos = np.tile(np.arange(N, dtype=np.int64), rows.shape[0] // N)
+        r = oracle.rope_bf16_ex(rows, pos, base, half_split=half, pos_scale=ps, ntk_factor=ntk)
+        t = torch.from_numpy(np.ascontiguousarray(r).view(np.int16)).view(torch.bfloat16).reshape(x.shape)
+        return t[..., perm].contiguous() if half else t
+
+    o1, l1 = _gpu(cuda_api, q, k, v, (B, Hq, Hkv, N, D, 1, 0, base, half, ps, ntk, False))
+    o2, l2 = cuda_api.attn_fwd(rotated(q).cuda(), rotated(k).cuda(), v.cuda(), causal=True, rope_base=0.0)
+    torch.cuda.synchronize()
+    assert cuda_api.device_status() == 0
+    assert torch.equal(o1.view(torch.int16), o2.view(torch.int16)) and torch.equal(l1, l2)
+
+
 def test_alibi_full_size_sampled(cuda_api):
     """ALiBi (with half-split RoPE and NTK scaling) on the GQA causal N=8192 workload, sampled rows."""
     cfg = synth.GQA_CAUSAL_N8192
