@@ -74,6 +74,34 @@ def test_no_lse_pointer(cuda_api):
     assert lse is None and torch.equal(o.view(torch.int16), o2.view(torch.int16))
 
 
+def test_deterministic_and_stream_independent(cuda_api):
+    """Two calls, and a call on a side stream (which has its own rotation scratch), give the same
+    bits: the work schedule is static and no result depends on timing."""
+    q, k, v = (x.cuda() for x in synth.prefill_inputs(2, 8, 2, 1100, 128, seed=8))
+    o1, l1 = cuda_api.attn_fwd(q, k, v, causal=True, rope_base=10000.0)
+    o2, l2 = cuda_api.attn_fwd(q, k, v, causal=True, rope_base=10000.0)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        o3, l3 = torch.empty_like(o1), torch.empty_like(l1)
+        cuda_api.attn_fwd(q, k, v, causal=True, rope_base=10000.0, o=o3, lse=l3, stream=side)
+    side.synchronize()
+    torch.cuda.synchronize()
+    assert cuda_api.device_status() == 0
+    for o, lse in ((o2, l2), (o3, l3)):
+        assert torch.equal(o1.view(torch.int16), o.view(torch.int16)) and torch.equal(l1, lse)
+
+
+def test_explicit_scale(cuda_api):
+    """A softmax scale other than 1/sqrt(D) (0.2 at D = 64, against the default 0.125)."""
+    q, k, v = synth.prefill_inputs(1, 4, 2, 333, 64, seed=9)
+    o, lse = cuda_api.attn_fwd(q.cuda(), k.cuda(), v.cuda(), causal=True, rope_base=10000.0, scale=0.2)
+    torch.cuda.synchronize()
+    assert cuda_api.device_status() == 0
+    o_ref, lse_ref = oracle_prefill(q, k, v, 1, 0, 10000.0, 0.2)
+    assert_close(f64(o), f64(lse), o_ref, lse_ref, "scale 0.2")
+
+
 @pytest.mark.parametrize("cfg", synth.PREFILL_CONFIGS, ids=lambda c: c.name)
 def test_workload_full_size_sampled(cuda_api, cfg):
     """The workloads at full size, in the benchmark's launch configuration, on sampled rows."""
