@@ -87,6 +87,20 @@ def test_backward_gqa_equals_repeated_heads(cuda_api):
         assert float((a.float() - summed).abs().max()) <= 2.0 ** -7 * float(summed.abs().max())
 
 
+def test_backward_deterministic(cuda_api):
+    """Two backward calls give the same bits: dQ, dK and dV are each written by one CTA (no
+    atomics), so no result depends on timing."""
+    q, k, v = (x.cuda() for x in synth.prefill_inputs(1, 8, 2, 700, 128, seed=79))
+    dout = synth.randn_bf16((1, 8, 700, 128), torch.Generator().manual_seed(80)).cuda()
+    o, lse = cuda_api.attn_fwd(q, k, v, causal=True, rope_base=10000.0)
+    first = cuda_api.attn_bwd(q, k, v, o, lse, dout, causal=True, rope_base=10000.0)
+    second = cuda_api.attn_bwd(q, k, v, o, lse, dout, causal=True, rope_base=10000.0)
+    torch.cuda.synchronize()
+    assert cuda_api.device_status() == 0
+    for a, b in zip(first, second):
+        assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
 def test_backward_workload_full_size(cuda_api):
     """The backward the benchmark times (GQA causal N=8192, RoPE 5e5), checked where the oracle can
     reach at that size:
