@@ -92,6 +92,20 @@ def test_deterministic_and_stream_independent(cuda_api):
         assert torch.equal(o1.view(torch.int16), o.view(torch.int16)) and torch.equal(l1, lse)
 
 
+def test_cache_growth_leaves_results_unchanged(cuda_api):
+    """The RoPE tables and the rotation scratch are cached and grow on demand: a call repeated
+    after larger calls (which regrow both) and a call with another base gives the same bits."""
+    a = [x.cuda() for x in synth.prefill_inputs(1, 4, 2, 900, 128, seed=10)]
+    b = [x.cuda() for x in synth.prefill_inputs(2, 4, 4, 3100, 128, seed=11)]
+    o1, l1 = cuda_api.attn_fwd(*a, causal=True, rope_base=10000.0)
+    cuda_api.attn_fwd(*b, causal=True, rope_base=10000.0)
+    cuda_api.attn_fwd(*b, causal=True, rope_base=500000.0)
+    o2, l2 = cuda_api.attn_fwd(*a, causal=True, rope_base=10000.0)
+    torch.cuda.synchronize()
+    assert cuda_api.device_status() == 0
+    assert torch.equal(o1.view(torch.int16), o2.view(torch.int16)) and torch.equal(l1, l2)
+
+
 def test_explicit_scale(cuda_api):
     """A softmax scale other than 1/sqrt(D) (0.2 at D = 64, against the default 0.125)."""
     q, k, v = synth.prefill_inputs(1, 4, 2, 333, 64, seed=9)
