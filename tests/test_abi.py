@@ -109,6 +109,36 @@ def test_workspace_size(api):
     assert api.decode_workspace_size(0, 1, 16, 1, 64) == 0
 
 
+def _bwd(api, q=FAKE, lse=FAKE, dq=FAKE, ws=FAKE, B=1, Hq=4, Hkv=2, N=128, D=128, causal=1, window=0, rope=0.0,
+         scale=0.0, ws_bytes=None):
+    if ws_bytes is None:
+        ws_bytes = api.bwd_workspace_size(B, Hq, Hkv, N, D, rope) if B > 0 and Hq > 0 and Hkv > 0 and N > 0 else 0
+    return api.lib.attn_bwd(q, FAKE, FAKE, FAKE, lse, FAKE, dq, FAKE, FAKE, B, Hq, Hkv, N, D, causal, window, rope,
+                            scale, ws, ws_bytes, None)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(q=None), 1), (dict(dq=None), 1), (dict(ws=None), 1), (dict(lse=ctypes.c_void_p(0x10002)), 1),
+    (dict(dq=MISALIGNED), 1), (dict(N=0), 1), (dict(Hq=3, Hkv=2), 1), (dict(causal=0, window=8), 1),
+    (dict(scale=float("inf")), 1), (dict(ws_bytes=256), 1), (dict(rope=10000.0, ws_bytes=70000), 1),
+    (dict(D=96), 2), (dict(B=65535, Hq=65535, Hkv=1), 2),
+])
+def test_bwd_validation(api, kw, expect):
+    assert _bwd(api, **kw) == expect
+    assert api.last_error() != ""
+
+
+def test_bwd_workspace_size(api):
+    # fp32 (-LSE log2 e, -D_i) per query row padded to 128-row tiles, 256-B rounded; with RoPE
+    # also the rotated Q and K in bf16, each 256-B rounded
+    assert api.bwd_workspace_size(1, 4, 2, 128, 128) == 4 * 128 * 2 * 4
+    assert api.bwd_workspace_size(1, 1, 1, 1, 64) == 1024
+    assert api.bwd_workspace_size(2, 32, 8, 8192, 128, 10000.0) == (2 * 32 * 8192 * 2 * 4 + 2 * 32 * 8192 * 128 * 2
+                                                                     + 2 * 8 * 8192 * 128 * 2)
+    assert api.bwd_workspace_size(1, 2, 1, 3, 64, 10000.0) == 2 * 128 * 2 * 4 + 768 + 512
+    assert api.bwd_workspace_size(0, 4, 2, 128, 128) == 0
+
+
 def _step(api, q_len=2, Hq=8, Hkv=2, D=128, k_new=FAKE, v_new=FAKE, ws_bytes=None, rope=0.0):
     if ws_bytes is None:
         ws_bytes = api.decode_step_workspace_size(2, q_len, 8, 16, Hq, D)
