@@ -139,6 +139,16 @@ def test_bwd_workspace_size(api):
     assert api.bwd_workspace_size(0, 4, 2, 128, 128) == 0
 
 
+def test_decode_noalloc_limit_is_checked_before_any_launch(api):
+    """2048 sequences x 32 heads x 32 splits x (128 + 2) floats exceed the fixed 40 MiB array: the
+    call is rejected on the host, naming the limit; smaller requests pass that check."""
+    st = api.lib.attn_decode_paged_noalloc(FAKE, FAKE, FAKE, FAKE, FAKE, 2048, 1024, 100, 16, 32, 8, 128, 0.0, FAKE,
+                                           None, None)
+    assert st == api.ATTN_ERR_INVALID_ARG and "no-alloc limit" in api.last_error()
+    assert api.decode_workspace_size(2048, 1024, 16, 32, 128) > 40 << 20
+    assert api.decode_workspace_size(64, 1024, 16, 32, 128) <= 40 << 20
+
+
 def _step(api, q_len=2, Hq=8, Hkv=2, D=128, k_new=FAKE, v_new=FAKE, ws_bytes=None, rope=0.0):
     if ws_bytes is None:
         ws_bytes = api.decode_step_workspace_size(2, q_len, 8, 16, Hq, D)
