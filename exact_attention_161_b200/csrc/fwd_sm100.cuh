@@ -19,7 +19,7 @@
 //              LSE. Q and K arrive already rotated (RoPE) by a streaming pass before the kernel.
 //   warp 8     TMA producer: the Q tiles once, then K tiles into a NK-stage ring and V tiles into
 //              a NV-stage ring.
-//   warp 9     MMA issuer (one thread) and TMEM owner.
+//   warp 9     MMA issuer and TMEM owner: the warp walks the schedule, one elected lane issues.
 //
 // Tensor Memory (512 columns): S0 at 0, S1 at 128, O0 at 256, O1 at 256 + D. The MMA thread
 // issues, per key tile j:  O0 += P0(j) V(j);  S0(j+1) = Q0 K(j+1)^T;  O1 += P1(j) V(j);
@@ -248,39 +248,43 @@ __global__ void __launch_bounds__(FwdCfg<D, kFp8>::THREADS, 1)
         }
     } else if (warp == C::MMA_WARP) {
         // ------------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            // Q, K both K-major; P K-major, V MN-major
-            constexpr uint32_t IDESC_S = kFp8 ? ptx::idesc_e4m3_f32(128, C::BN, 0, 0) : ptx::idesc_bf16_f32(128, C::BN, 0, 0);
-            constexpr uint32_t IDESC_O = kFp8 ? ptx::idesc_e4m3_f32(128, D, 0, 1) : ptx::idesc_bf16_f32(128, D, 0, 1);
-            constexpr uint32_t HI = ptx::sw128_desc_hi(1024);                    // 8-row groups 1024 B apart
-            constexpr uint32_t TILE16 = C::TILE_BYTES >> 4;
-            // low descriptor words of Q tile 0, K stage 0 and V stage 0 (K-major LBO unused = 16;
-            // V is MN-major with its 64-column halves one region apart)
-            const uint32_t q_lo = ptx::sw128_desc_lo(ptx::smem_u32(sQ), 16);
-            const uint32_t k_lo = ptx::sw128_desc_lo(ptx::smem_u32(sK), 16);
-            const uint32_t v_lo = ptx::sw128_desc_lo(ptx::smem_u32(sV), C::REGION_BYTES);
-            bool ok = true, issued_any = false;
-            int kq0 = 0, kq1 = 0;  // items of query tile 0 / 1 started so far
-            int cw0 = 0, cw1 = 0;  // score tiles of query tile 0 / 1 computed so far (all items)
-            int g = 0;             // key tiles consumed so far (ring position)
-            for (int rnd = 0, it = blockIdx.x; ok && it < p.n_items; it = item_of_round(++rnd, blockIdx.x, gridDim.x)) {
-                const Item x = make_item(p, it);
-                for (int u = -1; ok && u < x.T; ++u) {
-                    // u = -1: the prologue (scores of the first key tile only)
-                    if (u >= 0) {
-                        if (!ptx::mbar_wait(&bar->v_full[(g + u) % NV], ((g + u) / NV) & 1, abort_flag)) { ok = false; break; }
-                    }
-                    for (int i = 0; i < 2; ++i) {
-                        const int kq = i ? kq1 : kq0, cw = i ? cw1 : cw0;
-                        const TileRange& R = x.rng[i];
-                        const uint32_t d_s = tmem + C::tmem_s(i), d_o = tmem + C::tmem_o(i);
-                        if (u >= 0 && x.active(i, u)) {
-                            // O_i += P_i(u) V(u); P_i in TMEM over the first 64 columns of score buffer i
-                            const int c = x.J0 + u - R.jb;
-                            if (c == 0 && kq > 0 && !ptx::mbar_wait(&bar->o_empty[i], (kq - 1) & 1, abort_flag)) { ok = false; break; }
-                            if (!ptx::mbar_wait(&bar->p_full[i], (cw + c) & 1, abort_flag)) { ok = false; break; }
-                            ptx::tc_fence_after();  // P was written to TMEM by the softmax warps
-                            const uint32_t vb = v_lo + ((g + u) % NV) * TILE16;
+        // The whole warp walks the schedule and takes the waits, so every index, TMEM address and
+        // descriptor is warp-uniform; one elected lane issues the tcgen05 instructions.
+        const bool leader = ptx::elect_one();
+        const uint32_t tm = __shfl_sync(0xffffffffu, tmem, 0);
+        // Q, K both K-major; P K-major, V MN-major
+        constexpr uint32_t IDESC_S = kFp8 ? ptx::idesc_e4m3_f32(128, C::BN, 0, 0) : ptx::idesc_bf16_f32(128, C::BN, 0, 0);
+        constexpr uint32_t IDESC_O = kFp8 ? ptx::idesc_e4m3_f32(128, D, 0, 1) : ptx::idesc_bf16_f32(128, D, 0, 1);
+        constexpr uint32_t HI = ptx::sw128_desc_hi(1024);                    // 8-row groups 1024 B apart
+        constexpr uint32_t TILE16 = C::TILE_BYTES >> 4;
+        // low descriptor words of Q tile 0, K stage 0 and V stage 0 (K-major LBO unused = 16;
+        // V is MN-major with its 64-column halves one region apart)
+        const uint32_t q_lo = ptx::sw128_desc_lo(ptx::smem_u32(sQ), 16);
+        const uint32_t k_lo = ptx::sw128_desc_lo(ptx::smem_u32(sK), 16);
+        const uint32_t v_lo = ptx::sw128_desc_lo(ptx::smem_u32(sV), C::REGION_BYTES);
+        bool ok = true, issued_any = false;
+        int kq0 = 0, kq1 = 0;  // items of query tile 0 / 1 started so far
+        int cw0 = 0, cw1 = 0;  // score tiles of query tile 0 / 1 computed so far (all items)
+        int g = 0;             // key tiles consumed so far (ring position)
+        for (int rnd = 0, it = blockIdx.x; ok && it < p.n_items; it = item_of_round(++rnd, blockIdx.x, gridDim.x)) {
+            const Item x = make_item(p, it);
+            for (int u = -1; ok && u < x.T; ++u) {
+                // u = -1: the prologue (scores of the first key tile only)
+                if (u >= 0) {
+                    if (!ptx::mbar_wait_warp(&bar->v_full[(g + u) % NV], ((g + u) / NV) & 1, abort_flag)) { ok = false; break; }
+                }
+                for (int i = 0; i < 2; ++i) {
+                    const int kq = i ? kq1 : kq0, cw = i ? cw1 : cw0;
+                    const TileRange& R = x.rng[i];
+                    const uint32_t d_s = tm + C::tmem_s(i), d_o = tm + C::tmem_o(i);
+                    if (u >= 0 && x.active(i, u)) {
+                        // O_i += P_i(u) V(u); P_i in TMEM over the first 64 columns of score buffer i
+                        const int c = x.J0 + u - R.jb;
+                        if (c == 0 && kq > 0 && !ptx::mbar_wait_warp(&bar->o_empty[i], (kq - 1) & 1, abort_flag)) { ok = false; break; }
+                        if (!ptx::mbar_wait_warp(&bar->p_full[i], (cw + c) & 1, abort_flag)) { ok = false; break; }
+                        ptx::tc_fence_after();  // P was written to TMEM by the softmax warps
+                        const uint32_t vb = v_lo + ((g + u) % NV) * TILE16;
+                        if (leader) {
 #pragma unroll
                             for (int kk = 0; kk < C::O_KSTEPS; ++kk) {
                                 const uint64_t bd = ptx::desc64(vb + kk * ((C::O_ROWS * 128) >> 4), HI);
@@ -291,13 +295,16 @@ __global__ void __launch_bounds__(FwdCfg<D, kFp8>::THREADS, 1)
                             }
                             if (c == R.n - 1) ptx::mma_commit(&bar->o_final[i]);
                         }
-                        if (u + 1 < x.T && x.active(i, u + 1)) {
-                            // S_i(u+1) = Q_i K(u+1)^T into score buffer i
-                            const int c = x.J0 + u + 1 - R.jb;
-                            // Q and K arrive by TMA: the barriers alone order them before the MMA's reads
-                            if (c == 0 && !ptx::mbar_wait(&bar->q_loaded[i], kq & 1, abort_flag)) { ok = false; break; }
-                            if (!ptx::mbar_wait(&bar->k_full[(g + u + 1) % NK], ((g + u + 1) / NK) & 1, abort_flag)) { ok = false; break; }
-                            const uint32_t qa = q_lo + i * TILE16, kb = k_lo + ((g + u + 1) % NK) * TILE16;
+                        __syncwarp();
+                    }
+                    if (u + 1 < x.T && x.active(i, u + 1)) {
+                        // S_i(u+1) = Q_i K(u+1)^T into score buffer i
+                        const int c = x.J0 + u + 1 - R.jb;
+                        // Q and K arrive by TMA: the barriers alone order them before the MMA's reads
+                        if (c == 0 && !ptx::mbar_wait_warp(&bar->q_loaded[i], kq & 1, abort_flag)) { ok = false; break; }
+                        if (!ptx::mbar_wait_warp(&bar->k_full[(g + u + 1) % NK], ((g + u + 1) / NK) & 1, abort_flag)) { ok = false; break; }
+                        const uint32_t qa = q_lo + i * TILE16, kb = k_lo + ((g + u + 1) % NK) * TILE16;
+                        if (leader) {
 #pragma unroll
                             for (int kk = 0; kk < C::S_KSTEPS; ++kk) {
                                 const uint32_t off = ((kk >> 2) * C::REGION_BYTES + (kk & 3) * 32) >> 4;
@@ -308,18 +315,24 @@ __global__ void __launch_bounds__(FwdCfg<D, kFp8>::THREADS, 1)
                             }
                             ptx::mma_commit(&bar->s_full[i]);
                             if (c == R.n - 1) ptx::mma_commit(&bar->q_empty[i]);  // Q_i no longer read
-                            issued_any = true;
                         }
+                        __syncwarp();
+                        issued_any = true;
                     }
-                    if (!ok) break;
+                }
+                if (!ok) break;
+                if (leader) {
                     if (u >= 0) ptx::mma_commit(&bar->v_empty[(g + u) % NV]);
                     if (u + 1 < x.T) ptx::mma_commit(&bar->k_empty[(g + u + 1) % NK]);
                 }
-                if (x.rng[0].n > 0) { ++kq0; cw0 += x.rng[0].n; }
-                if (x.rng[1].n > 0) { ++kq1; cw1 += x.rng[1].n; }
-                g += x.T;
+                __syncwarp();
             }
-            if (!ok) {
+            if (x.rng[0].n > 0) { ++kq0; cw0 += x.rng[0].n; }
+            if (x.rng[1].n > 0) { ++kq1; cw1 += x.rng[1].n; }
+            g += x.T;
+        }
+        if (!ok) {
+            if (leader) {
                 *abort_flag = 1;
                 raise_status(kStatusTimeout);
                 if (issued_any) {  // wait for the MMAs in flight before TMEM is released

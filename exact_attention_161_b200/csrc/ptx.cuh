@@ -78,23 +78,23 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-__device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t nthreads) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+// The same wait taken by a whole warp: every lane polls the barrier and the result is made
+// warp-uniform, so that code after it stays converged.
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+    return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
 }
 
-// Named barrier that also returns the OR of `pred` over the nthreads participants, so that all of
-// them take the same branch afterwards.
-__device__ __forceinline__ bool named_barrier_or(uint32_t id, uint32_t nthreads, bool pred) {
-    uint32_t r;
+// One lane of a converged warp (the same lane every time for a full mask): the issuing thread of
+// the single-thread tcgen05 and TMA instructions, while the warp around it computes the
+// warp-uniform operands.
+__device__ __forceinline__ bool elect_one() {
+    uint32_t is_leader;
     asm volatile(
-        "{\n\t.reg .pred p, q;\n\t"
-        "setp.ne.u32 p, %1, 0;\n\t"
-        "barrier.cta.red.or.pred q, %2, %3, p;\n\t"
-        "selp.u32 %0, 1, 0, q;\n\t}"
-        : "=r"(r)
-        : "r"(static_cast<uint32_t>(pred)), "r"(id), "r"(nthreads)
-        : "memory");
-    return r != 0;
+        "{\n\t.reg .pred P;\n\t"
+        "elect.sync _|P, 0xffffffff;\n\t"
+        "selp.u32 %0, 1, 0, P;\n\t}"
+        : "=r"(is_leader));
+    return is_leader != 0;
 }
 
 // ------------------------------------------------------------------------------ TMA
