@@ -249,90 +249,89 @@ __global__ void __launch_bounds__(FwdCfg<D, kFp8>::THREADS, 1)
     } else if (warp == C::MMA_WARP) {
         // ------------------------------------------------------------------ MMA issuer
         // The whole warp walks the schedule and takes the waits, so every index, TMEM address and
-        // descriptor is warp-uniform; one elected lane issues the tcgen05 instructions.
-        const bool leader = ptx::elect_one();
+        // descriptor is warp-uniform; the tcgen05 instructions carry a lane predicate, so that one
+        // elected lane issues them without the warp leaving the converged path. Descriptors are
+        // 64-bit words built once; stepping through a tile adds a constant to their address field.
+        const uint32_t issue = ptx::elect_one() ? 1u : 0u;
         const uint32_t tm = __shfl_sync(0xffffffffu, tmem, 0);
         // Q, K both K-major; P K-major, V MN-major
         constexpr uint32_t IDESC_S = kFp8 ? ptx::idesc_e4m3_f32(128, C::BN, 0, 0) : ptx::idesc_bf16_f32(128, C::BN, 0, 0);
         constexpr uint32_t IDESC_O = kFp8 ? ptx::idesc_e4m3_f32(128, D, 0, 1) : ptx::idesc_bf16_f32(128, D, 0, 1);
         constexpr uint32_t HI = ptx::sw128_desc_hi(1024);                    // 8-row groups 1024 B apart
-        constexpr uint32_t TILE16 = C::TILE_BYTES >> 4;
-        // low descriptor words of Q tile 0, K stage 0 and V stage 0 (K-major LBO unused = 16;
-        // V is MN-major with its 64-column halves one region apart)
-        const uint32_t q_lo = ptx::sw128_desc_lo(ptx::smem_u32(sQ), 16);
-        const uint32_t k_lo = ptx::sw128_desc_lo(ptx::smem_u32(sK), 16);
-        const uint32_t v_lo = ptx::sw128_desc_lo(ptx::smem_u32(sV), C::REGION_BYTES);
+        constexpr uint64_t TILE16 = C::TILE_BYTES >> 4;
+        // descriptors of Q tile 0, K stage 0 and V stage 0 (K-major LBO unused = 16; V is MN-major
+        // with its 64-column halves one region apart)
+        const uint64_t q_d = ptx::desc64(__shfl_sync(0xffffffffu, ptx::sw128_desc_lo(ptx::smem_u32(sQ), 16), 0), HI);
+        const uint64_t k_d = ptx::desc64(__shfl_sync(0xffffffffu, ptx::sw128_desc_lo(ptx::smem_u32(sK), 16), 0), HI);
+        const uint64_t v_d =
+            ptx::desc64(__shfl_sync(0xffffffffu, ptx::sw128_desc_lo(ptx::smem_u32(sV), C::REGION_BYTES), 0), HI);
         bool ok = true, issued_any = false;
         int kq0 = 0, kq1 = 0;  // items of query tile 0 / 1 started so far
         int cw0 = 0, cw1 = 0;  // score tiles of query tile 0 / 1 computed so far (all items)
         int g = 0;             // key tiles consumed so far (ring position)
         for (int rnd = 0, it = blockIdx.x; ok && it < p.n_items; it = item_of_round(++rnd, blockIdx.x, gridDim.x)) {
             const Item x = make_item(p, it);
+            // per tile: first and one-past-last u of its key tiles (empty when the tile is past N)
+            const int a0 = x.rng[0].jb - x.J0, e0 = x.rng[0].n > 0 ? a0 + x.rng[0].n : a0;
+            const int a1 = x.rng[1].jb - x.J0, e1 = x.rng[1].n > 0 ? a1 + x.rng[1].n : a1;
             for (int u = -1; ok && u < x.T; ++u) {
                 // u = -1: the prologue (scores of the first key tile only)
                 if (u >= 0) {
                     if (!ptx::mbar_wait_warp(&bar->v_full[(g + u) % NV], ((g + u) / NV) & 1, abort_flag)) { ok = false; break; }
                 }
+                bool k_ready = false;
                 for (int i = 0; i < 2; ++i) {
                     const int kq = i ? kq1 : kq0, cw = i ? cw1 : cw0;
-                    const TileRange& R = x.rng[i];
+                    const int a = i ? a1 : a0, e = i ? e1 : e0;
                     const uint32_t d_s = tm + C::tmem_s(i), d_o = tm + C::tmem_o(i);
-                    if (u >= 0 && x.active(i, u)) {
+                    if (u >= a && u < e) {
                         // O_i += P_i(u) V(u); P_i in TMEM over the first 64 columns of score buffer i
-                        const int c = x.J0 + u - R.jb;
+                        const int c = u - a;
                         if (c == 0 && kq > 0 && !ptx::mbar_wait_warp(&bar->o_empty[i], (kq - 1) & 1, abort_flag)) { ok = false; break; }
                         if (!ptx::mbar_wait_warp(&bar->p_full[i], (cw + c) & 1, abort_flag)) { ok = false; break; }
                         ptx::tc_fence_after();  // P was written to TMEM by the softmax warps
-                        const uint32_t vb = v_lo + ((g + u) % NV) * TILE16;
-                        if (leader) {
+                        const uint64_t vb = v_d + ((g + u) % NV) * TILE16;
 #pragma unroll
-                            for (int kk = 0; kk < C::O_KSTEPS; ++kk) {
-                                const uint64_t bd = ptx::desc64(vb + kk * ((C::O_ROWS * 128) >> 4), HI);
-                                if constexpr (kFp8)
-                                    ptx::mma_ts_f8(d_o, d_s + kk * 8, bd, IDESC_O, (c > 0 || kk > 0) ? 1u : 0u);
-                                else
-                                    ptx::mma_ts(d_o, d_s + kk * 8, bd, IDESC_O, (c > 0 || kk > 0) ? 1u : 0u);
-                            }
-                            if (c == R.n - 1) ptx::mma_commit(&bar->o_final[i]);
+                        for (int kk = 0; kk < C::O_KSTEPS; ++kk) {
+                            const uint64_t bd = vb + kk * ((C::O_ROWS * 128) >> 4);
+                            if constexpr (kFp8)
+                                ptx::mma_ts_f8_if(issue, d_o, d_s + kk * 8, bd, IDESC_O, (c > 0 || kk > 0) ? 1u : 0u);
+                            else
+                                ptx::mma_ts_if(issue, d_o, d_s + kk * 8, bd, IDESC_O, (c > 0 || kk > 0) ? 1u : 0u);
                         }
-                        __syncwarp();
+                        if (c == e - a - 1) ptx::mma_commit_if(issue, &bar->o_final[i]);
                     }
-                    if (u + 1 < x.T && x.active(i, u + 1)) {
+                    if (u + 1 >= a && u + 1 < e) {
                         // S_i(u+1) = Q_i K(u+1)^T into score buffer i
-                        const int c = x.J0 + u + 1 - R.jb;
+                        const int c = u + 1 - a;
                         // Q and K arrive by TMA: the barriers alone order them before the MMA's reads
                         if (c == 0 && !ptx::mbar_wait_warp(&bar->q_loaded[i], kq & 1, abort_flag)) { ok = false; break; }
-                        if (!ptx::mbar_wait_warp(&bar->k_full[(g + u + 1) % NK], ((g + u + 1) / NK) & 1, abort_flag)) { ok = false; break; }
-                        const uint32_t qa = q_lo + i * TILE16, kb = k_lo + ((g + u + 1) % NK) * TILE16;
-                        if (leader) {
+                        if (!k_ready && !ptx::mbar_wait_warp(&bar->k_full[(g + u + 1) % NK], ((g + u + 1) / NK) & 1, abort_flag)) { ok = false; break; }
+                        k_ready = true;
+                        const uint64_t qa = q_d + i * TILE16, kb = k_d + ((g + u + 1) % NK) * TILE16;
 #pragma unroll
-                            for (int kk = 0; kk < C::S_KSTEPS; ++kk) {
-                                const uint32_t off = ((kk >> 2) * C::REGION_BYTES + (kk & 3) * 32) >> 4;
-                                if constexpr (kFp8)
-                                    ptx::mma_ss_f8(d_s, ptx::desc64(qa + off, HI), ptx::desc64(kb + off, HI), IDESC_S, kk > 0);
-                                else
-                                    ptx::mma_ss(d_s, ptx::desc64(qa + off, HI), ptx::desc64(kb + off, HI), IDESC_S, kk > 0);
-                            }
-                            ptx::mma_commit(&bar->s_full[i]);
-                            if (c == R.n - 1) ptx::mma_commit(&bar->q_empty[i]);  // Q_i no longer read
+                        for (int kk = 0; kk < C::S_KSTEPS; ++kk) {
+                            const uint64_t off = ((kk >> 2) * C::REGION_BYTES + (kk & 3) * 32) >> 4;
+                            if constexpr (kFp8)
+                                ptx::mma_ss_f8_if(issue, d_s, qa + off, kb + off, IDESC_S, kk > 0);
+                            else
+                                ptx::mma_ss_if(issue, d_s, qa + off, kb + off, IDESC_S, kk > 0);
                         }
-                        __syncwarp();
+                        ptx::mma_commit_if(issue, &bar->s_full[i]);
+                        if (c == e - a - 1) ptx::mma_commit_if(issue, &bar->q_empty[i]);  // Q_i no longer read
                         issued_any = true;
                     }
                 }
                 if (!ok) break;
-                if (leader) {
-                    if (u >= 0) ptx::mma_commit(&bar->v_empty[(g + u) % NV]);
-                    if (u + 1 < x.T) ptx::mma_commit(&bar->k_empty[(g + u + 1) % NK]);
-                }
-                __syncwarp();
+                if (u >= 0) ptx::mma_commit_if(issue, &bar->v_empty[(g + u) % NV]);
+                if (u + 1 < x.T) ptx::mma_commit_if(issue, &bar->k_empty[(g + u + 1) % NK]);
             }
             if (x.rng[0].n > 0) { ++kq0; cw0 += x.rng[0].n; }
             if (x.rng[1].n > 0) { ++kq1; cw1 += x.rng[1].n; }
             g += x.T;
         }
         if (!ok) {
-            if (leader) {
+            if (issue) {
                 *abort_flag = 1;
                 raise_status(kStatusTimeout);
                 if (issued_any) {  // wait for the MMAs in flight before TMEM is released
