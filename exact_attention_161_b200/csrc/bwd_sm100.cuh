@@ -200,8 +200,10 @@ __device__ __forceinline__ void dscores32_row(const float* pr, const uint32_t (&
 
 // =============================================================================== dK, dV
 // CTA (key tile jt, K/V head g, batch b); block numbers run over key tiles slowest, so the causal
-// key tiles with the most visible queries start first. Steps t walk (query head of the group,
-// visible query tile). TMEM: S^T at 0 (P^T packed into columns 0-31 and 64-95), dP^T at 128 (dS^T
+// key tiles with the most visible queries start first. Steps t walk the visible query tiles from
+// the last one down, and the query heads of the group for each: under a causal mask every key
+// tile's walk starts at the same query tile, so the CTAs of one K/V head that run side by side read
+// each Q and dO tile at about the same time, and the repeats come from L2. TMEM: S^T at 0 (P^T packed into columns 0-31 and 64-95), dP^T at 128 (dS^T
 // packed likewise), dV at 256, dK at 256 + D.
 //
 // Issue order per step t: dV(t) once P^T(t) is written, S^T(t+1), dK(t) once dS^T(t) is written,
@@ -275,7 +277,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
             for (int t = 0; t < T && ok; ++t) {
                 const int s = t & 1;
                 if (t >= 2 && !ptx::mbar_wait(&bar->empty[s], ((t >> 1) - 1) & 1, abort_flag)) { ok = false; break; }
-                const int h = g * G + t / per_head, qt = ib + t % per_head;
+                const int qt = ie - 1 - t / G, h = g * G + t % G;
                 const int zq = b * p.Hq + h;
                 ptx::mbar_arrive_expect_tx(&bar->full[s], 2 * C::TILE_BYTES + C::VEC_BYTES);
                 for (int r = 0; r < C::NREG; ++r) {
@@ -298,7 +300,11 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         }
     } else if (warp == C::MMA_WARP) {
         // ------------------------------------------------------------------ MMA issuer
-        if (lane == 0 && T > 0) {
+        // The whole warp walks the steps and takes the waits, so operands stay warp-uniform; one
+        // elected lane issues the tcgen05 instructions.
+        if (T > 0) {
+            const bool leader = ptx::elect_one();
+            const uint32_t tm = __shfl_sync(0xffffffffu, tmem, 0);
             constexpr uint32_t ID_S = ptx::idesc_bf16_f32(128, 128, 0, 0);  // K (keys) x Q^T, both K-major
             constexpr uint32_t ID_G = ptx::idesc_bf16_f32(128, D, 0, 1);    // P^T/dS^T (TMEM) x dO/Q (MN-major)
             constexpr uint32_t HI = ptx::sw128_desc_hi(1024);
@@ -315,7 +321,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = ((kk >> 2) * C::REGION_BYTES + (kk & 3) * 32) >> 4;
-                    ptx::mma_ss(tmem + T_S, ptx::desc64(k_lo + off, HI), ptx::desc64(q_lo + st + off, HI), ID_S, kk > 0);
+                    ptx::mma_ss(tm + T_S, ptx::desc64(k_lo + off, HI), ptx::desc64(q_lo + st + off, HI), ID_S, kk > 0);
                 }
             };
             // dP^T = V dO^T
@@ -324,7 +330,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = ((kk >> 2) * C::REGION_BYTES + (kk & 3) * 32) >> 4;
-                    ptx::mma_ss(tmem + T_DP, ptx::desc64(v_lo + off, HI), ptx::desc64(do_lo + st + off, HI), ID_S, kk > 0);
+                    ptx::mma_ss(tm + T_DP, ptx::desc64(v_lo + off, HI), ptx::desc64(do_lo + st + off, HI), ID_S, kk > 0);
                 }
             };
             // dV += P^T dO, dK += dS^T Q (M = 128 keys, N = D, K = 128 queries)
@@ -332,39 +338,50 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
                 const uint32_t st = (t & 1) * TILE16;
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    ptx::mma_ts(tmem + acc_col, tmem + a_col + packed_col(kk), ptx::desc64(b_lo + st + ((kk * 2048) >> 4), HI),
+                    ptx::mma_ts(tm + acc_col, tm + a_col + packed_col(kk), ptx::desc64(b_lo + st + ((kk * 2048) >> 4), HI),
                                 ID_G, (t > 0 || kk > 0) ? 1u : 0u);
             };
-            bool ok = ptx::mbar_wait(&bar->fixed_loaded, 0, abort_flag) && ptx::mbar_wait(&bar->full[0], 0, abort_flag);
+            bool ok = ptx::mbar_wait_warp(&bar->fixed_loaded, 0, abort_flag) &&
+                      ptx::mbar_wait_warp(&bar->full[0], 0, abort_flag);
             bool issued_any = false;
             if (ok) {
-                issue_s(0);
-                ptx::mma_commit(&bar->s_full[0]);
-                issue_dp(0);
-                ptx::mma_commit(&bar->dp_full);
+                if (leader) {
+                    issue_s(0);
+                    ptx::mma_commit(&bar->s_full[0]);
+                    issue_dp(0);
+                    ptx::mma_commit(&bar->dp_full);
+                }
+                __syncwarp();
                 issued_any = true;
             }
             for (int t = 0; ok && t < T; ++t) {
-                if (!ptx::mbar_wait(&bar->p_full, t & 1, abort_flag)) { ok = false; break; }
+                if (!ptx::mbar_wait_warp(&bar->p_full, t & 1, abort_flag)) { ok = false; break; }
                 ptx::tc_fence_after();
-                issue_grad(t, T_DV, T_S, domn_lo);
+                if (leader) issue_grad(t, T_DV, T_S, domn_lo);
+                __syncwarp();
                 if (t + 1 < T) {
-                    if (!ptx::mbar_wait(&bar->full[(t + 1) & 1], ((t + 1) >> 1) & 1, abort_flag)) { ok = false; break; }
-                    issue_s(t + 1);
-                    ptx::mma_commit(&bar->s_full[0]);
+                    if (!ptx::mbar_wait_warp(&bar->full[(t + 1) & 1], ((t + 1) >> 1) & 1, abort_flag)) { ok = false; break; }
+                    if (leader) {
+                        issue_s(t + 1);
+                        ptx::mma_commit(&bar->s_full[0]);
+                    }
+                    __syncwarp();
                 }
-                if (!ptx::mbar_wait(&bar->ds_full, t & 1, abort_flag)) { ok = false; break; }
+                if (!ptx::mbar_wait_warp(&bar->ds_full, t & 1, abort_flag)) { ok = false; break; }
                 ptx::tc_fence_after();
-                issue_grad(t, T_DK, T_DP, qmn_lo);
-                ptx::mma_commit(&bar->empty[t & 1]);
-                if (t + 1 < T) {
-                    issue_dp(t + 1);
-                    ptx::mma_commit(&bar->dp_full);
-                } else {
-                    ptx::mma_commit(&bar->acc_done);
+                if (leader) {
+                    issue_grad(t, T_DK, T_DP, qmn_lo);
+                    ptx::mma_commit(&bar->empty[t & 1]);
+                    if (t + 1 < T) {
+                        issue_dp(t + 1);
+                        ptx::mma_commit(&bar->dp_full);
+                    } else {
+                        ptx::mma_commit(&bar->acc_done);
+                    }
                 }
+                __syncwarp();
             }
-            if (!ok) {
+            if (!ok && leader) {
                 *abort_flag = 1;
                 raise_status(kStatusTimeout);
                 if (issued_any) {
@@ -385,7 +402,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         bool ok = true;
         for (int t = 0; ok && t < T; ++t) {
             const int s = t & 1;
-            const int c0 = (ib + t % per_head) * 128 + 64 * wg;  // first query of this warpgroup's columns
+            const int c0 = (ie - 1 - t / G) * 128 + 64 * wg;  // first query of this warpgroup's columns
             if (!ptx::mbar_wait(&bar->full[s], (t >> 1) & 1, abort_flag)) { ok = false; break; }
             if (!ptx::mbar_wait(&bar->s_full[0], t & 1, abort_flag)) { ok = false; break; }
             ptx::tc_fence_after();
@@ -545,7 +562,10 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
             }
         }
     } else if (warp == C::MMA_WARP) {
-        if (lane == 0 && T > 0) {
+        // The whole warp walks the steps and takes the waits; one elected lane issues.
+        if (T > 0) {
+            const bool leader = ptx::elect_one();
+            const uint32_t tm = __shfl_sync(0xffffffffu, tmem, 0);
             constexpr uint32_t ID_S = ptx::idesc_bf16_f32(128, 128, 0, 0);  // Q K^T, dO V^T: K-major
             constexpr uint32_t ID_G = ptx::idesc_bf16_f32(128, D, 0, 1);    // dS (TMEM) x K (MN-major)
             constexpr uint32_t HI = ptx::sw128_desc_hi(1024);
@@ -561,7 +581,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = ((kk >> 2) * C::REGION_BYTES + (kk & 3) * 32) >> 4;
-                    ptx::mma_ss(tmem + T_S + 128 * (t & 1), ptx::desc64(q_lo + off, HI), ptx::desc64(k_lo + st + off, HI),
+                    ptx::mma_ss(tm + T_S + 128 * (t & 1), ptx::desc64(q_lo + off, HI), ptx::desc64(k_lo + st + off, HI),
                                 ID_S, kk > 0);
                 }
             };
@@ -571,41 +591,51 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = ((kk >> 2) * C::REGION_BYTES + (kk & 3) * 32) >> 4;
-                    ptx::mma_ss(tmem + T_DP, ptx::desc64(do_lo + off, HI), ptx::desc64(v_lo + st + off, HI), ID_S, kk > 0);
+                    ptx::mma_ss(tm + T_DP, ptx::desc64(do_lo + off, HI), ptx::desc64(v_lo + st + off, HI), ID_S, kk > 0);
                 }
             };
-            bool ok = ptx::mbar_wait(&bar->fixed_loaded, 0, abort_flag) && ptx::mbar_wait(&bar->full[0], 0, abort_flag);
+            bool ok = ptx::mbar_wait_warp(&bar->fixed_loaded, 0, abort_flag) &&
+                      ptx::mbar_wait_warp(&bar->full[0], 0, abort_flag);
             bool issued_any = false;
             if (ok) {
-                issue_s(0);
-                ptx::mma_commit(&bar->s_full[0]);
-                issue_dp(0);
-                ptx::mma_commit(&bar->dp_full);
+                if (leader) {
+                    issue_s(0);
+                    ptx::mma_commit(&bar->s_full[0]);
+                    issue_dp(0);
+                    ptx::mma_commit(&bar->dp_full);
+                }
+                __syncwarp();
                 issued_any = true;
             }
             for (int t = 0; ok && t < T; ++t) {
                 if (t + 1 < T) {
-                    if (!ptx::mbar_wait(&bar->full[(t + 1) & 1], ((t + 1) >> 1) & 1, abort_flag)) { ok = false; break; }
-                    issue_s(t + 1);
-                    ptx::mma_commit(&bar->s_full[(t + 1) & 1]);
+                    if (!ptx::mbar_wait_warp(&bar->full[(t + 1) & 1], ((t + 1) >> 1) & 1, abort_flag)) { ok = false; break; }
+                    if (leader) {
+                        issue_s(t + 1);
+                        ptx::mma_commit(&bar->s_full[(t + 1) & 1]);
+                    }
+                    __syncwarp();
                 }
-                if (!ptx::mbar_wait(&bar->ds_full, t & 1, abort_flag)) { ok = false; break; }
+                if (!ptx::mbar_wait_warp(&bar->ds_full, t & 1, abort_flag)) { ok = false; break; }
                 ptx::tc_fence_after();
-                // dQ += dS K (M = 128 queries, N = D, K = 128 keys)
-                const uint32_t st = (t & 1) * TILE16;
+                if (leader) {
+                    // dQ += dS K (M = 128 queries, N = D, K = 128 keys)
+                    const uint32_t st = (t & 1) * TILE16;
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    ptx::mma_ts(tmem + T_DQ, tmem + T_DP + packed_col(kk),
-                                ptx::desc64(kmn_lo + st + ((kk * 2048) >> 4), HI), ID_G, (t > 0 || kk > 0) ? 1u : 0u);
-                ptx::mma_commit(&bar->empty[t & 1]);
-                if (t + 1 < T) {
-                    issue_dp(t + 1);
-                    ptx::mma_commit(&bar->dp_full);
-                } else {
-                    ptx::mma_commit(&bar->acc_done);
+                    for (int kk = 0; kk < 8; ++kk)
+                        ptx::mma_ts(tm + T_DQ, tm + T_DP + packed_col(kk),
+                                    ptx::desc64(kmn_lo + st + ((kk * 2048) >> 4), HI), ID_G, (t > 0 || kk > 0) ? 1u : 0u);
+                    ptx::mma_commit(&bar->empty[t & 1]);
+                    if (t + 1 < T) {
+                        issue_dp(t + 1);
+                        ptx::mma_commit(&bar->dp_full);
+                    } else {
+                        ptx::mma_commit(&bar->acc_done);
+                    }
                 }
+                __syncwarp();
             }
-            if (!ok) {
+            if (!ok && leader) {
                 *abort_flag = 1;
                 raise_status(kStatusTimeout);
                 if (issued_any) {
