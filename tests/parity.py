@@ -34,6 +34,11 @@ def assert_close(o_gpu, lse_gpu, o_ref, lse_ref, what=""):
     return max_abs, rel_rms, lse_abs
 
 
+def report(what, max_abs, rel_rms, lse_abs):
+    """Print the measured errors of a parity case (shown with pytest -s)."""
+    print("PARITY %s max_abs=%.3e rel_rms=%.3e lse_max_abs=%.3e" % (what, max_abs, rel_rms, lse_abs))
+
+
 def sample_rows(B, Hq, N, per_head=12, heads=None, seed=0):
     """Flat row ids ((b*Hq + h)*N + i): every head (or the given ones), the first and last
     rows, both sides of every tile boundary near the start and end, and random rows."""

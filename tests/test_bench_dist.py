@@ -65,3 +65,15 @@ def test_two_gloo_ranks_take_the_max_and_sum_the_work():
         assert (rr, w, local) == (r, world, r)
         assert mx == 15.0                      # slowest rank
         assert value == 1000.0 * world / 15.0  # all ranks' units over the slowest time
+
+
+def test_peak_choice_follows_the_timed_region():
+    """A leg timed for under a second is compared with the burst GEMM rate, a longer one with the
+    sustained rate (the clocks settle under the power cap only after a while)."""
+    peaks = {"bf16_tflops": 1615.5, "bf16_tflops_sustained": 1379.5, "hbm_gbs": 6559.4}
+    p, kind = bench.tensor_peak_for(peaks, "measured", 0.03)
+    assert p == 1615.5 and "burst" in kind
+    p, kind = bench.tensor_peak_for(peaks, "measured", 2.5)
+    assert p == 1379.5 and "sustained" in kind
+    p, kind = bench.tensor_peak_for({"bf16_tflops": 1590.0, "hbm_gbs": 6650.0}, "fallback", 5.0)
+    assert p == 1590.0
