@@ -91,15 +91,39 @@ struct DevBuf {
 
 std::atomic<bool> g_debug_drop_copy{false};  // test hook of attn_debug_drop_copy
 
+// Caches. A table or scratch buffer that is outgrown is replaced by a larger one; the old one is
+// freed at once, after a device synchronisation (a launch still queued on any stream may read
+// it). Growth is geometric, so this happens a few times in a process's life, not per call.
 std::mutex g_cache_mu;
 // Layouts of a cos/sin table covering positions [0, cap): (cos, sin) pairs, [cap][D/2], one
 // position's pairs contiguous, in fp32 (kTab32) or fp64 (kTab64)
 enum TabLayout { kTab32 = 0, kTab64 = 1 };
 // (device, base, D, position scale, NTK factor, layout) -> table and its capacity
 std::map<std::tuple<int, double, int, double, double, int>, std::pair<DevBuf, int>> g_rope_tables;
-// (device, stream) -> rotated-key scratch
+// (device, stream) -> scratch for the rotated queries and keys of attn_fwd; at most
+// kMaxScratchStreams streams per device keep one (a new stream beyond that frees the device's
+// others first, after a device synchronisation)
 std::map<std::pair<int, void*>, DevBuf> g_key_scratch;
-std::vector<DevBuf> g_retired;  // outgrown buffers; a launch still queued may read them
+constexpr int kMaxScratchStreams = 8;
+
+// Frees an outgrown buffer of device `dev` once every launch queued on that device has finished.
+cudaError_t free_after_device_sync(const DevBuf& b) {
+    if (!b.ptr) return cudaSuccess;
+    int cur = 0;
+    cudaError_t e = cudaGetDevice(&cur);
+    if (e != cudaSuccess) return e;
+    if (cur != b.dev && (e = cudaSetDevice(b.dev)) != cudaSuccess) return e;
+    e = cudaDeviceSynchronize();
+    if (e == cudaSuccess) e = cudaFree(b.ptr);
+    if (cur != b.dev) cudaSetDevice(cur);
+    return e;
+}
+
+size_t grow_geometric(size_t need, size_t have) {
+    size_t cap = have > 0 ? have : 1;
+    while (cap < need) cap *= 2;
+    return cap;
+}
 
 // (cos, sin) of (pos / pos_scale) * b^(-2i/D), b = base * ntk^(D/(D-2)), for pos < n, i < D/2:
 // angles and trigonometry in fp64 (Position Interpolation divides the positions; NTK-aware scaling
@@ -114,7 +138,11 @@ attn_status rope_table_any(int dev, double base, int D, int n, double pos_scale,
         return ATTN_OK;
     }
     const bool wide = layout == kTab64;
-    const int cap = ((n + 1023) / 1024) * 1024;
+    // capacity: a power of two of at least 1024 positions (so regrowth is rare), never beyond the
+    // int range of positions
+    int cap = 1024;
+    while (cap < n && cap < (1 << 30)) cap *= 2;
+    if (cap < n) cap = n;
     const size_t pairs = static_cast<size_t>(cap) * (D / 2);
     std::vector<double2> host64(wide ? pairs : 0);
     std::vector<float2> host32(wide ? 0 : pairs);
@@ -140,7 +168,13 @@ attn_status rope_table_any(int dev, double base, int D, int n, double pos_scale,
         cudaFree(buf.ptr);
         return fail(ATTN_ERR_CUDA, "rope table upload: %s", cudaGetErrorString(e));
     }
-    if (it != g_rope_tables.end()) g_retired.push_back(it->second.first);
+    if (it != g_rope_tables.end()) {
+        e = free_after_device_sync(it->second.first);
+        if (e != cudaSuccess) {
+            cudaFree(buf.ptr);
+            return fail(ATTN_ERR_CUDA, "freeing an outgrown rope table: %s", cudaGetErrorString(e));
+        }
+    }
     g_rope_tables[key] = std::make_pair(buf, cap);
     *out = buf.ptr;
     return ATTN_OK;
@@ -161,12 +195,27 @@ attn_status rope_table64(int dev, double base, int D, int n, const double2** out
 }
 attn_status key_scratch(int dev, void* stream, size_t bytes, void** out) {
     std::lock_guard<std::mutex> lock(g_cache_mu);
-    DevBuf& b = g_key_scratch[std::make_pair(dev, stream)];
+    const auto key = std::make_pair(dev, stream);
+    if (g_key_scratch.find(key) == g_key_scratch.end()) {
+        int on_dev = 0;
+        for (const auto& kv : g_key_scratch) on_dev += kv.first.first == dev;
+        if (on_dev >= kMaxScratchStreams) {
+            for (auto it = g_key_scratch.begin(); it != g_key_scratch.end();) {
+                if (it->first.first != dev) { ++it; continue; }
+                const cudaError_t e = free_after_device_sync(it->second);
+                if (e != cudaSuccess) return fail(ATTN_ERR_CUDA, "freeing stream scratch: %s", cudaGetErrorString(e));
+                it = g_key_scratch.erase(it);
+            }
+        }
+    }
+    DevBuf& b = g_key_scratch[key];
     if (b.bytes < bytes) {
-        if (b.ptr) g_retired.push_back(b);
+        const size_t cap = grow_geometric(bytes, b.bytes);
+        const cudaError_t e = free_after_device_sync(b);
+        if (e != cudaSuccess) return fail(ATTN_ERR_CUDA, "freeing outgrown scratch: %s", cudaGetErrorString(e));
         b = DevBuf();
-        CUDA_TRY(cudaMalloc(&b.ptr, bytes));
-        b.bytes = bytes;
+        CUDA_TRY(cudaMalloc(&b.ptr, cap));
+        b.bytes = cap;
         b.dev = dev;
     }
     *out = b.ptr;
@@ -480,6 +529,9 @@ attn_status launch_bwd(const void* q, const void* k, const void* v, const void* 
     return ATTN_OK;
 }
 
+// Forgets the cached device addresses of the no-alloc decode's array (defined with it below).
+void noalloc_forget();
+
 }  // namespace
 
 extern "C" {
@@ -736,11 +788,10 @@ void attn_shutdown(void) {
     };
     for (auto& kv : g_rope_tables) release(kv.second.first);
     for (auto& kv : g_key_scratch) release(kv.second);
-    for (auto& b : g_retired) release(b);
     if (have_dev) cudaSetDevice(cur);
     g_rope_tables.clear();
     g_key_scratch.clear();
-    g_retired.clear();
+    noalloc_forget();
 }
 
 }  // extern "C"
@@ -773,6 +824,11 @@ attn_status noalloc_scratch(int dev, void** out) {
     }
     *out = g_noalloc_ptr[dev];
     return ATTN_OK;
+}
+
+void noalloc_forget() {
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    for (auto& ptr : g_noalloc_ptr) ptr = nullptr;
 }
 
 }  // namespace

@@ -18,7 +18,9 @@
  *     with attn_get_device_status().
  *   - The library owns only its caches (RoPE cos/sin tables per (device, base, head dim); a
  *     scratch per (device, stream) for the rotated queries and keys of attn_fwd and
- *     attn_fwd_pos; the device status word); attn_shutdown releases them.
+ *     attn_fwd_pos, kept for at most 8 streams per device; the device status word);
+ *     attn_shutdown releases them. A cache grows geometrically when a call needs more; the
+ *     outgrown buffer is freed at once after a device synchronisation, so memory stays bounded.
  *   - There is no CPU fallback: without a B200 every compute call returns ATTN_ERR_CUDA.
  */
 #ifndef ATTN_B200_H
@@ -76,7 +78,8 @@ typedef enum {
  * B * Hq * ceil(N/256) < 2^31. Fully masked key tiles are skipped, not computed.
  * Errors: ATTN_ERR_INVALID_ARG for NULL/misaligned pointers or inconsistent sizes/flags;
  * ATTN_ERR_CUDA when a runtime call or the launch fails. With RoPE, the first call for a new
- * (device, rope_base, D, N) or a new stream allocates cached device memory (cudaMalloc).
+ * (device, rope_base, D), a longer N than cached, or a new stream allocates cached device memory
+ * (cudaMalloc) and synchronises the device; later calls of the same or smaller size do neither.
  */
 attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
                      int N, int D, int causal, int window, float rope_base, float scale, void* stream);
@@ -206,7 +209,8 @@ size_t attn_decode_step_workspace_size(int num_seqs, int q_len, int max_blocks_p
  * The new tokens of sequence s sit at positions seq_lens[s]-q_len .. seq_lens[s]-1 (seq_lens
  * count them). With rope_base > 0, every new query and key is rotated at its position, on
  * interleaved pairs (2i, 2i+1) by pos * rope_base^(-2i/D) ("attention-transformers", Q "How does
- * Rotary Position Embedding (RoPE) work?"), in fp32 and rounded to bf16; values are never rotated.
+ * Rotary Position Embedding (RoPE) work?"), in fp64 (an fp64 cos/sin table, unfused products) and
+ * rounded once to bf16; values are never rotated.
  * 1. Append (when k_new is given): new token t's rotated key and its value go to page
  *    block_table[s][pos / page_size], slot pos % page_size ("Self-Attention Complexity,
  *    FlashAttention, PagedAttention, and RoPE in Code", Part 3: the cache grows one block-table
@@ -249,14 +253,19 @@ attn_status attn_decode_step(const void* q, const void* k_new, const void* v_new
  * Same arguments, computation, results and checks as attn_decode_paged, without the workspace:
  * the partial softmax states live in one fixed device array of ATTN_DECODE_NOALLOC_MAX_BYTES
  * compiled into the library (every GPU that loads the library holds it until the process exits).
- * The call allocates nothing. Limits and sharing:
+ * The call itself allocates nothing. The array is reserved when the library's device code is
+ * loaded on a device, which with CUDA's lazy module loading happens at the first call into the
+ * library on that device, whichever entry point it is, and may synchronise the device: make one
+ * warm-up call per device before the latency-sensitive path. Limits and sharing:
  *   - requests whose attn_decode_workspace_size(...) exceeds ATTN_DECODE_NOALLOC_MAX_BYTES are
  *     rejected with ATTN_ERR_INVALID_ARG and a message naming the limit;
  *   - every call, on every stream, uses the same array and leaves its contents behind; nothing in
  *     it needs to start at zero (each call writes every partial state it reads), but calls that
  *     overlap on the GPU race on it and must be serialised by the caller;
  *   - the first call on each device looks up the array's device address (cudaGetSymbolAddress,
- *     with that device current); make that first call before any stream capture.
+ *     with that device current) and caches it; make that first call before any stream capture;
+ *   - after a device reset (cudaDeviceReset) the cached address is stale: call attn_shutdown,
+ *     which forgets it, before calling in again.
  */
 #define ATTN_DECODE_NOALLOC_MAX_BYTES ((size_t)40 << 20)
 attn_status attn_decode_paged_noalloc(const void* q, const void* k_pages, const void* v_pages,
@@ -288,8 +297,9 @@ const char* attn_last_error(void);
 /* Library version string. */
 const char* attn_version(void);
 
-/* Frees every cache the library allocated (RoPE tables, query/key scratch), on every device.
- * The caller must ensure no call is still running on the GPU. */
+/* Frees every cache the library allocated (RoPE tables, query/key scratch), on every device, and
+ * forgets the cached device address of the no-alloc decode's array. The caller must ensure no call
+ * is still running on the GPU. */
 void attn_shutdown(void);
 
 #ifdef __cplusplus
