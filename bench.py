@@ -173,6 +173,54 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
+class NvmlSampler:
+    """SM clock samples from NVML every few milliseconds in a thread, for timed regions that are
+    too short for nvidia-smi's interval."""
+
+    def __init__(self, device_index, interval_s=0.005):
+        self.device_index, self.interval_s = device_index, interval_s
+        self.samples, self.thread, self.stop_flag = [], None, False
+
+    def start(self):
+        try:
+            import threading
+            import pynvml
+            pynvml.nvmlInit()
+            handle = pynvml.nvmlDeviceGetHandleByIndex(self.device_index)
+        except Exception:
+            return
+
+        def run():
+            import pynvml
+            while not self.stop_flag:
+                try:
+                    self.samples.append(pynvml.nvmlDeviceGetClockInfo(handle, pynvml.NVML_CLOCK_SM))
+                except Exception:
+                    return
+                time.sleep(self.interval_s)
+
+        self.thread = threading.Thread(target=run, daemon=True)
+        self.thread.start()
+
+    def stop(self):
+        if self.thread is None:
+            return None
+        self.stop_flag = True
+        self.thread.join(timeout=1.0)
+        if not self.samples:
+            return None
+        return {"sm_mhz_median": statistics.median(self.samples), "sm_mhz_min": min(self.samples),
+                "samples": len(self.samples), "interval_ms": self.interval_s * 1e3}
+
+
+def tensor_peak_for(peaks, peaks_kind, timed_s):
+    """The bf16 GEMM peak that applies to a leg: the burst figure for a timed region under a second
+    (clocks have not settled under the power cap yet), the sustained one for longer regions."""
+    if timed_s < 1.0 or "bf16_tflops_sustained" not in peaks:
+        return peaks["bf16_tflops"], "%s bf16 GEMM, burst (timed region %.3f s)" % (peaks_kind, timed_s)
+    return peaks["bf16_tflops_sustained"], "%s bf16 GEMM, sustained (timed region %.1f s)" % (peaks_kind, timed_s)
+
+
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -246,6 +294,55 @@ def oracle_decode_sample(cache, budget_s):
 
 
 # ------------------------------------------------------------------------------ our arm
+def time_loop(fn, calls, stream, world, dev):
+    """Mean ms per call of `calls` back-to-back calls on `stream` (events on that stream), after
+    the caller's warm-up; the max over ranks."""
+    barrier(world)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(calls):
+        fn()
+    b.record(stream)
+    torch.cuda.synchronize()
+    return reduce_max(a.elapsed_time(b), world, dev) / calls
+
+
+def e2e_pipeline(steps, h2d, compute, d2h, dev):
+    """End-to-end rate through the public API: step i's host->device copies (pinned host buffers),
+    its compute and its device->host copies run on three streams, so step i+1's upload, step i's
+    compute and step i-1's download overlap. Two device buffer sets alternate; events order each
+    reuse. h2d(i, stream), compute(i, stream), d2h(i, stream) enqueue step i's work for buffer set
+    i % 2. Returns ms for `steps` steps, from the first upload to the last download (one untimed
+    pass first)."""
+    s_up, s_run, s_down = (torch.cuda.Stream(device=dev) for _ in range(3))
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+
+    def run(n):
+        up, ran, down = [ev() for _ in range(n)], [ev() for _ in range(n)], [ev() for _ in range(n)]
+        t0, t1 = ev(), ev()
+        t0.record(s_up)
+        for i in range(n):
+            if i >= 2:
+                s_up.wait_event(ran[i - 2])     # buffer set i % 2 is free once step i-2 computed
+            h2d(i, s_up)
+            up[i].record(s_up)
+            s_run.wait_event(up[i])
+            if i >= 2:
+                s_run.wait_event(down[i - 2])   # its outputs were read back
+            compute(i, s_run)
+            ran[i].record(s_run)
+            s_down.wait_event(ran[i])
+            d2h(i, s_down)
+            down[i].record(s_down)
+        t1.record(s_down)
+        torch.cuda.synchronize()
+        return t0.elapsed_time(t1)
+
+    run(2)
+    return run(steps)
+
+
 def run_ours(args, rank, world, local):
     from exact_attention_161_b200 import api
     dev = torch.device("cuda", local)
@@ -288,10 +385,12 @@ def run_ours(args, rank, world, local):
     K = args.steps
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
     clocks = ClockSampler(local)
+    nvml = NvmlSampler(local)
     barrier(world)
     torch.cuda.synchronize()
     clocks.start()
     time.sleep(0.3)  # let the sampler take its first reading
+    nvml.start()
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     t_start.record(stream)
@@ -305,8 +404,11 @@ def run_ours(args, rank, world, local):
         ev[s][2].record(stream)
     t_end.record(stream)
     torch.cuda.synchronize()
+    nvml_clk = nvml.stop()
     barrier(world)
     clk = clocks.stop()
+    if clk is not None and nvml_clk is not None:
+        clk["nvml"] = nvml_clk
     total_ms = t_start.elapsed_time(t_end)
     prefill_ms = [ev[s][0].elapsed_time(ev[s][1]) for s in range(K)]
     decode_ms = [ev[s][1].elapsed_time(ev[s][2]) for s in range(K)]
@@ -319,6 +421,50 @@ def run_ours(args, rank, world, local):
     dbytes = decode_bytes(cache_h) if do_decode else 0
     value = job_throughput(flops * K, world, prefill_sum_max / 1e3) / 1e12 if do_prefill else None
     decode_value = job_throughput(dbytes * K, world, decode_sum_max / 1e3) / 1e9 if do_decode else None
+
+    # ---- the attention kernel alone: the same call without RoPE launches only attn_fwd_kernel (the
+    # same instance; the rotation pass is skipped), so its event time is that kernel's launch time
+    kern = None
+    if do_prefill and args.kernel_calls > 0:
+        def kernel_only():
+            api.attn_fwd(q, k, v, causal=PREFILL.causal, window=PREFILL.window, rope_base=0.0, o=o, lse=lse,
+                         stream=stream)
+
+        for _ in range(args.warmup):
+            kernel_only()
+        kern_ms = time_loop(kernel_only, args.kernel_calls, stream, world, dev)
+        kern = {"ms_per_launch": round(kern_ms, 4), "launches": args.kernel_calls,
+                "timed_s": kern_ms * args.kernel_calls / 1e3}
+
+    # ---- the other prefill workloads through the same call (own loops; not part of the step)
+    configs_out = None
+    if do_prefill and args.config_calls > 0:
+        configs_out = {}
+        for cfg in synth.PREFILL_CONFIGS:
+            if cfg is PREFILL:
+                continue
+            cq, ck, cv = (t.to(dev) for t in synth.prefill_inputs_for(cfg))
+            co = torch.empty_like(cq)
+            cl = torch.empty((cfg.B, cfg.Hq, cfg.N), dtype=torch.float32, device=dev)
+
+            def cfg_call():
+                api.attn_fwd(cq, ck, cv, causal=cfg.causal, window=cfg.window, rope_base=cfg.rope_base, o=co,
+                             lse=cl, stream=stream)
+
+            for _ in range(args.warmup):
+                cfg_call()
+            n_calls = args.config_calls * (20 if cfg.N <= 128 else 1)
+            cms = time_loop(cfg_call, n_calls, stream, world, dev)
+            if api.device_status() != 0:
+                raise RuntimeError("device status raised during the %s loop" % cfg.name)
+            cf = prefill_flops(cfg)
+            configs_out[cfg.name] = {
+                "value": round(job_throughput(cf, world, cms / 1e3) / 1e12, 3), "unit": "TFLOP/s",
+                "ms_per_call": round(cms, 5), "calls": n_calls, "flops_per_call": cf,
+                "timed_s": cms * n_calls / 1e3,
+                "config": {"B": cfg.B, "Hq": cfg.Hq, "Hkv": cfg.Hkv, "N": cfg.N, "D": cfg.D, "causal": cfg.causal,
+                           "window": cfg.window, "rope_base": cfg.rope_base}}
+            del cq, ck, cv, co, cl
 
     # ---- backward of the prefill workload (its own loop; not part of the step)
     bwd = None
@@ -335,23 +481,16 @@ def run_ours(args, rank, world, local):
         prefill()
         for _ in range(args.warmup):
             backward()
-        barrier(world)
-        torch.cuda.synchronize()
-        b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        b0.record(stream)
-        for _ in range(args.bwd_steps):
-            backward()
-        b1.record(stream)
-        torch.cuda.synchronize()
+        bwd_ms = time_loop(backward, args.bwd_steps, stream, world, dev)
         if api.device_status() != 0:
             raise RuntimeError("device status raised during the backward loop")
-        bwd_ms = reduce_max(b0.elapsed_time(b1), world, dev) / args.bwd_steps
         bwd_flops = flops * 5 // 2  # five products per unmasked pair (S, dP, dV, dK, dQ) vs two forward
         bwd = {"metric": "attn bwd TFLOP/s (same workload; algorithmic FLOPs = 2.5 x forward)",
                "value": round(job_throughput(bwd_flops, world, bwd_ms / 1e3) / 1e12, 2), "unit": "TFLOP/s",
-               "ms_per_call": round(bwd_ms, 4), "calls": args.bwd_steps,
+               "ms_per_call": round(bwd_ms, 4), "calls": args.bwd_steps, "timed_s": bwd_ms * args.bwd_steps / 1e3,
                "roofline": {"bound": "tensor", "achieved": round(bwd_flops / (bwd_ms / 1e3) / 1e12, 2),
-                            "unit": "TFLOP/s", "note": "five-kernel call: rotation x2, prep, dK/dV, dQ"}}
+                            "unit": "TFLOP/s", "note": "five-kernel call: rotation pass, prep, dK/dV, dQ"}}
+        del dout, gq, gk, gv, bws
 
     # ---- position variants of the prefill workload (own loops; not part of the step)
     variants = None
@@ -366,19 +505,12 @@ def run_ours(args, rank, world, local):
 
             for _ in range(args.warmup):
                 variant_call()
-            barrier(world)
-            torch.cuda.synchronize()
-            v0, v1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            v0.record(stream)
-            for _ in range(args.variant_calls):
-                variant_call()
-            v1.record(stream)
-            torch.cuda.synchronize()
+            vms = time_loop(variant_call, args.variant_calls, stream, world, dev)
             if api.device_status() != 0:
                 raise RuntimeError("device status raised during the %s loop" % name)
-            vms = reduce_max(v0.elapsed_time(v1), world, dev) / args.variant_calls
             variants[name] = {"value": round(job_throughput(flops, world, vms / 1e3) / 1e12, 2), "unit": "TFLOP/s",
                               "ms_per_call": round(vms, 4), "calls": args.variant_calls,
+                              "timed_s": vms * args.variant_calls / 1e3,
                               "roofline": {"bound": "tensor", "achieved": round(flops / (vms / 1e3) / 1e12, 2),
                                            "unit": "TFLOP/s"}}
 
@@ -394,58 +526,72 @@ def run_ours(args, rank, world, local):
 
         for _ in range(args.warmup):
             fp8_call()
-        barrier(world)
-        torch.cuda.synchronize()
-        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        f0.record(stream)
-        for _ in range(args.fp8_calls):
-            fp8_call()
-        f1.record(stream)
-        torch.cuda.synchronize()
+        fms = time_loop(fp8_call, args.fp8_calls, stream, world, dev)
         if api.device_status() != 0:
             raise RuntimeError("device status raised during the FP8 loop")
-        fms = reduce_max(f0.elapsed_time(f1), world, dev) / args.fp8_calls
         fp8 = {"metric": "attn fwd TFLOP/s, e4m3 Q/K/V (per-tensor scales), same shape and mask, no RoPE",
                "value": round(job_throughput(flops, world, fms / 1e3) / 1e12, 2), "unit": "TFLOP/s", "dtype": "e4m3",
-               "ms_per_call": round(fms, 4), "calls": args.fp8_calls,
+               "ms_per_call": round(fms, 4), "calls": args.fp8_calls, "timed_s": fms * args.fp8_calls / 1e3,
                "roofline": {"bound": "tensor", "achieved": round(flops / (fms / 1e3) / 1e12, 2), "unit": "TFLOP/s"}}
+        del q8, k8, v8
 
-    # ---- end to end through the public API with pinned host buffers
+    # ---- end to end through the public API: pinned host buffers, uploads, compute and downloads of
+    # successive steps overlapped on three streams (prefill and decode timed as separate pipelines)
     E = min(args.e2e_steps, K) if (args.e2e_steps > 0 and args.only == "all") else 0
+    e2e_value = e2e_decode = None
     if E:
         q_p, k_p, v_p = q_h.pin_memory(), k_h.pin_memory(), v_h.pin_memory()
-        o_p = torch.empty(o.shape, dtype=o.dtype).pin_memory()
-        lse_p = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+        bufs = [(q, k, v, o, lse), tuple(torch.empty_like(t) for t in (q, k, v, o, lse))]
+        outs_p = [(torch.empty(o.shape, dtype=o.dtype).pin_memory(), torch.empty(lse.shape, dtype=lse.dtype).pin_memory())
+                  for _ in range(2)]
+
+        def p_up(i, st):
+            with torch.cuda.stream(st):
+                for dst, src in zip(bufs[i % 2][:3], (q_p, k_p, v_p)):
+                    dst.copy_(src, non_blocking=True)
+
+        def p_run(i, st):
+            bq, bk, bv, bo, bl = bufs[i % 2]
+            api.attn_fwd(bq, bk, bv, causal=PREFILL.causal, window=PREFILL.window, rope_base=PREFILL.rope_base,
+                         o=bo, lse=bl, stream=st)
+
+        def p_down(i, st):
+            with torch.cuda.stream(st):
+                outs_p[i % 2][0].copy_(bufs[i % 2][3], non_blocking=True)
+                outs_p[i % 2][1].copy_(bufs[i % 2][4], non_blocking=True)
+
+        e_pre = reduce_max(e2e_pipeline(E, p_up, p_run, p_down, dev), world, dev)
+        e2e_value = job_throughput(flops * E, world, e_pre / 1e3) / 1e12
+        del bufs, outs_p
         dq_p, bt_p, sl_p = cache_h.q.pin_memory(), cache_h.block_table.pin_memory(), cache_h.seq_lens.pin_memory()
-        do_p = torch.empty(do.shape, dtype=do.dtype).pin_memory()
-        dlse_p = torch.empty(dlse.shape, dtype=dlse.dtype).pin_memory()
-    e_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(E)]
-    for s in range(E + 1 if E else 0):  # the first pass is a warm-up
-        r = e_ev[s - 1] if s > 0 else [torch.cuda.Event(enable_timing=True) for _ in range(3)]
-        r[0].record(stream)
-        q.copy_(q_p, non_blocking=True)
-        k.copy_(k_p, non_blocking=True)
-        v.copy_(v_p, non_blocking=True)
-        prefill()
-        o_p.copy_(o, non_blocking=True)
-        lse_p.copy_(lse, non_blocking=True)
-        r[1].record(stream)
-        dq.copy_(dq_p, non_blocking=True)
-        bt.copy_(bt_p, non_blocking=True)
-        sl.copy_(sl_p, non_blocking=True)
-        decode()
-        do_p.copy_(do, non_blocking=True)
-        dlse_p.copy_(dlse, non_blocking=True)
-        r[2].record(stream)
-    torch.cuda.synchronize()
-    e_pre = reduce_max(sum(e[0].elapsed_time(e[1]) for e in e_ev), world, dev) if E else float("nan")
-    e_dec = reduce_max(sum(e[1].elapsed_time(e[2]) for e in e_ev), world, dev) if E else float("nan")
+        dbufs = [(dq, bt, sl, do, dlse, ws),
+                 tuple(torch.empty_like(t) for t in (dq, bt, sl, do, dlse, ws))]
+        douts_p = [(torch.empty(do.shape, dtype=do.dtype).pin_memory(),
+                    torch.empty(dlse.shape, dtype=dlse.dtype).pin_memory()) for _ in range(2)]
+
+        def d_up(i, st):
+            with torch.cuda.stream(st):
+                for dst, src in zip(dbufs[i % 2][:3], (dq_p, bt_p, sl_p)):
+                    dst.copy_(src, non_blocking=True)
+
+        def d_run(i, st):
+            bq, bbt, bsl, bo, bl, bws = dbufs[i % 2]
+            api.attn_decode_paged(bq, kp, vp, bbt, bsl, o=bo, lse=bl, workspace=bws, stream=st)
+
+        def d_down(i, st):
+            with torch.cuda.stream(st):
+                douts_p[i % 2][0].copy_(dbufs[i % 2][3], non_blocking=True)
+                douts_p[i % 2][1].copy_(dbufs[i % 2][4], non_blocking=True)
+
+        e_dec = reduce_max(e2e_pipeline(E, d_up, d_run, d_down, dev), world, dev)
+        e2e_decode = job_throughput(dbytes * E, world, e_dec / 1e3) / 1e9
+        del dbufs, douts_p
+        if api.device_status() != 0:
+            raise RuntimeError("device status raised during the end-to-end legs")
     h2d = sum(t.numel() * t.element_size() for t in (q_h, k_h, v_h)) if do_prefill else 0
     d2h = o.numel() * 2 + lse.numel() * 4 if do_prefill else 0
     dh2d = sum(t.numel() * t.element_size() for t in (cache_h.q, cache_h.block_table, cache_h.seq_lens)) if do_decode else 0
     dd2h = do.numel() * 2 + dlse.numel() * 4 if do_decode else 0
-    e2e_value = job_throughput(flops * E, world, e_pre / 1e3) / 1e12 if E else None
-    e2e_decode = job_throughput(dbytes * E, world, e_dec / 1e3) / 1e9 if E else None
 
     # ---- decode step: append one or four new tokens per sequence (keys rotated, RoPE 1e4) and attend
     # with their rotated queries, on the same cache (runs after the legs above: it writes the cache)
@@ -469,17 +615,9 @@ def run_ours(args, rank, world, local):
 
             for _ in range(args.warmup):
                 step_call()
-            barrier(world)
-            torch.cuda.synchronize()
-            a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a0.record(stream)
-            for _ in range(args.step_calls):
-                step_call()
-            a1.record(stream)
-            torch.cuda.synchronize()
+            ms = time_loop(step_call, args.step_calls, stream, world, dev)
             if api.device_status() != 0:
                 raise RuntimeError("device status raised during the decode-step loop")
-            ms = reduce_max(a0.elapsed_time(a1), world, dev) / args.step_calls
             sbytes = step_bytes(cache_h, T)
             steps_out["q_len=%d" % T] = {
                 "value": round(job_throughput(sbytes, world, ms / 1e3) / 1e9, 1), "unit": "GB/s",
@@ -489,30 +627,57 @@ def run_ours(args, rank, world, local):
     if rank != 0:
         return None
     peaks, peaks_kind = measured_peaks()
+    hbm = peaks["hbm_gbs"]
     if steps_out is not None:
         for key, v in steps_out.items():
-            v["roofline"].update({"peak": peaks["hbm_gbs"], "frac": round(v["roofline"]["achieved"] / peaks["hbm_gbs"], 4),
-                                  "peak_kind": peaks_kind,
+            v["roofline"].update({"peak": hbm, "frac": round(v["roofline"]["achieved"] / hbm, 4),
+                                  "peak_kind": "%s HBM copy" % peaks_kind,
                                   "traffic": profiled_traffic("decode_split" if key == "q_len=1" else "decode_step_split_q4")})
     pre_launch_ms = statistics.mean(prefill_ms)
     dec_launch_ms = statistics.mean(decode_ms)
-    tflops_launch = flops / (pre_launch_ms / 1e3) / 1e12 if do_prefill else float("nan")
+    tflops_call = flops / (pre_launch_ms / 1e3) / 1e12 if do_prefill else float("nan")
     gbs_launch = dbytes / (dec_launch_ms / 1e3) / 1e9 if do_decode else float("nan")
-    tensor_peak = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
+    step_peak, step_peak_kind = tensor_peak_for(peaks, peaks_kind, prefill_sum_max / 1e3)
+    if kern is not None:
+        k_peak, k_kind = tensor_peak_for(peaks, peaks_kind, kern["timed_s"])
+        k_tf = flops / (kern["ms_per_launch"] / 1e3) / 1e12
+        roof = {"bound": "tensor", "achieved": round(k_tf, 2), "peak": k_peak, "unit": "TFLOP/s",
+                "frac": round(k_tf / k_peak, 4), "peak_kind": k_kind, "frac_of_2250": round(k_tf / DATASHEET_BF16_TFLOPS, 4),
+                "traffic": profiled_traffic("attn_fwd"),
+                "kernel": "attn_fwd_kernel<128, 0, 0>, its own launches (%d, %.4f ms each) timed in a loop of the "
+                          "same call without RoPE (the rotation pass is the only launch RoPE adds)"
+                          % (kern["launches"], kern["ms_per_launch"]),
+                "call": {"achieved": round(tflops_call, 2), "frac": round(tflops_call / step_peak, 4),
+                         "peak_kind": step_peak_kind,
+                         "note": "the whole attn_fwd call with RoPE in the timed step (rotation pass + attention kernel)",
+                         "rotation_pass_traffic": profiled_traffic("rope_rows")}}
+    else:
+        roof = {"bound": "tensor", "achieved": round(tflops_call, 2), "peak": step_peak, "unit": "TFLOP/s",
+                "frac": round(tflops_call / step_peak, 4), "peak_kind": step_peak_kind,
+                "traffic": profiled_traffic("attn_fwd"), "kernel": "attn_fwd call (rotation pass + attention kernel)"}
+    if configs_out is not None:
+        for cname, cv in configs_out.items():
+            cp, ck = tensor_peak_for(peaks, peaks_kind, cv["timed_s"])
+            if cv["config"]["N"] <= 128:
+                cv["latency_us"] = round(cv["ms_per_call"] * 1e3, 2)
+                cv["roofline"] = {"bound": "latency", "note": "one CTA; no roofline claim"}
+            else:
+                cv["roofline"] = {"bound": "tensor", "achieved": cv["value"], "peak": cp, "unit": "TFLOP/s",
+                                  "frac": round(cv["value"] / cp, 4), "peak_kind": ck}
     if bwd is not None:
-        bwd["roofline"].update({"peak": tensor_peak, "frac": round(bwd["roofline"]["achieved"] / tensor_peak, 4),
-                                "peak_kind": "%s bf16 GEMM, sustained" % peaks_kind,
+        bp, bk = tensor_peak_for(peaks, peaks_kind, bwd["timed_s"])
+        bwd["roofline"].update({"peak": bp, "frac": round(bwd["roofline"]["achieved"] / bp, 4), "peak_kind": bk,
                                 "traffic": profiled_traffic("attn_bwd_dkdv"),
                                 "traffic_kernel": "attn_bwd_dkdv_kernel<128> (the larger of the two backward kernels)"})
     if fp8 is not None:
-        fp8_peak = 2.0 * tensor_peak
-        fp8["roofline"].update({"peak": fp8_peak, "frac": round(fp8["roofline"]["achieved"] / fp8_peak, 4),
-                                "peak_kind": "2 x %s bf16 GEMM sustained (nominal fp8:bf16 ratio 4.5:2.25)" % peaks_kind,
+        fp, fk = tensor_peak_for(peaks, peaks_kind, fp8["timed_s"])
+        fp8["roofline"].update({"peak": 2.0 * fp, "frac": round(fp8["roofline"]["achieved"] / (2.0 * fp), 4),
+                                "peak_kind": "2 x (%s) (nominal fp8:bf16 ratio 4.5:2.25)" % fk,
                                 "traffic": profiled_traffic("attn_fwd_fp8")})
     if variants is not None:
         for vv in variants.values():
-            vv["roofline"].update({"peak": tensor_peak, "frac": round(vv["roofline"]["achieved"] / tensor_peak, 4),
-                                   "peak_kind": "%s bf16 GEMM, sustained" % peaks_kind})
+            vp_, vk = tensor_peak_for(peaks, peaks_kind, vv["timed_s"])
+            vv["roofline"].update({"peak": vp_, "frac": round(vv["roofline"]["achieved"] / vp_, 4), "peak_kind": vk})
     line = {
         "metric": "attn fwd TFLOP/s (%s) & paged-decode KV GB/s" % prefill_label(),
         "value": round(value, 2) if do_prefill else None,
@@ -539,22 +704,18 @@ def run_ours(args, rank, world, local):
         },
         "decode": {"metric": "paged-decode KV GB/s", "value": round(decode_value, 1) if do_decode else None, "unit": "GB/s",
                    "ms_per_step": round(decode_sum_max / K, 4),
-                   "roofline": {"bound": "hbm", "achieved": round(gbs_launch, 1), "peak": peaks["hbm_gbs"],
-                                "unit": "GB/s", "frac": round(gbs_launch / peaks["hbm_gbs"], 4),
-                                "peak_kind": peaks_kind, "frac_of_8TBs": round(gbs_launch / DATASHEET_HBM_GBS, 4),
+                   "roofline": {"bound": "hbm", "achieved": round(gbs_launch, 1), "peak": hbm,
+                                "unit": "GB/s", "frac": round(gbs_launch / hbm, 4),
+                                "peak_kind": "%s HBM copy" % peaks_kind, "frac_of_8TBs": round(gbs_launch / DATASHEET_HBM_GBS, 4),
                                 "traffic": profiled_traffic("decode_split")},
                    "e2e": {"value": round(e2e_decode, 2) if E else None, "unit": "GB/s", "h2d_bytes_per_step": dh2d,
-                           "d2h_bytes_per_step": dd2h}},
-        "roofline": {"bound": "tensor", "achieved": round(tflops_launch, 2), "peak": tensor_peak, "unit": "TFLOP/s",
-                     "frac": round(tflops_launch / tensor_peak, 4),
-                     "peak_kind": "%s bf16 GEMM, sustained" % peaks_kind,
-                     "frac_of_2250": round(tflops_launch / DATASHEET_BF16_TFLOPS, 4),
-                     "traffic": profiled_traffic("attn_fwd"),
-                     "rotation_pass_traffic": profiled_traffic("rope_rows"),
-                     "kernel": "attn_fwd_kernel<128> (+ query/key rotation pass, inside the timed call)"},
+                           "d2h_bytes_per_step": dd2h, "overlap": "upload, compute and download on three streams"}},
+        "roofline": roof,
         "e2e": {"value": round(e2e_value, 2) if E else None, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h},
+                "d2h_bytes_per_step": d2h, "steps": E,
+                "overlap": "step i+1's upload, step i's compute and step i-1's download on three streams"},
         "gpu_launches": (2 * do_prefill + 2 * do_decode) * K,
+        "prefill_configs": configs_out,
         "backward": bwd,
         "fp8": fp8,
         "position_variants": None if variants is None else dict(
@@ -640,6 +801,10 @@ def parse_args(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--e2e-steps", type=int, default=10, help="0 skips the end-to-end leg")
+    ap.add_argument("--kernel-calls", type=int, default=20,
+                    help="attention-kernel-only launches timed for the roofline; 0 skips")
+    ap.add_argument("--config-calls", type=int, default=20,
+                    help="calls timed per other prefill workload (x20 for the N=128 one); 0 skips")
     ap.add_argument("--bwd-steps", type=int, default=20, help="backward calls timed after the step loop; 0 skips")
     ap.add_argument("--step-calls", type=int, default=50, help="decode-step calls timed per q_len; 0 skips")
     ap.add_argument("--variant-calls", type=int, default=20, help="position-variant prefill calls timed each; 0 skips")
