@@ -238,7 +238,7 @@ attn_status ensure_smem(K kernel, int bytes, int dev) {
 }
 
 // Rotate Q (bhq rows of N positions) and K (bhk rows) into qr and kr with one launch of
-// rope_rotate_rows_kernel: x covers the N * D/8 (position, chunk) pairs with 256 threads a block,
+// rope_rotate_rows_kernel: x covers the N * units (position, unit) pairs with 256 threads a block,
 // at most 8 blocks per SM (the x loop strides over the rest); z picks the tensor; y splits the
 // rows so that about 8 blocks per SM are resident however few positions there are.
 template <int D>
@@ -253,7 +253,8 @@ attn_status launch_rope_rows(bool half, const void* q, void* qr, long long bhq, 
     a.bh[1] = bhk;
     a.cs = cs;
     a.N = N;
-    const long long want = (static_cast<long long>(N) * (D / 8) + 255) / 256;
+    const long long units = half ? D / 16 : D / 8;  // thread units per position (see the kernel)
+    const long long want = (static_cast<long long>(N) * units + 255) / 256;
     const long long gx = want < 8LL * sms ? want : 8LL * sms;
     const long long bh_max = bhq > bhk ? bhq : bhk;
     long long gy = (8LL * sms + 2 * gx - 1) / (2 * gx);
@@ -325,12 +326,24 @@ attn_status launch_fwd(const void* q, const void* k, const void* v, void* o, flo
     int sms = 148;
     CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
     const int grid = p.n_items < sms ? p.n_items : sms;  // persistent: one CTA per SM
+    // With RoPE the kernel is the rotation pass's programmatic dependent (see the kernel's set-up):
+    // it is scheduled while the pass finishes and waits for it on the device.
+    cudaLaunchConfig_t lc{};
+    lc.gridDim = dim3(static_cast<unsigned>(grid));
+    lc.blockDim = dim3(C::THREADS);
+    lc.dynamicSmemBytes = C::SMEM_BYTES;
+    lc.stream = stream;
+    cudaLaunchAttribute la[1];
+    la[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    la[0].val.programmaticStreamSerializationAllowed = 1;
+    lc.attrs = la;
+    lc.numAttrs = rope_base > 0.f ? 1 : 0;
     if (pv.alibi != nullptr) {
         if ((st = ensure_smem(attn::attn_fwd_kernel<D, true>, C::SMEM_BYTES, dev)) != ATTN_OK) return st;
-        attn::attn_fwd_kernel<D, true><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+        CUDA_TRY(cudaLaunchKernelEx(&lc, attn::attn_fwd_kernel<D, true, false>, tq, tk, tv, p));
     } else {
         if ((st = ensure_smem(attn::attn_fwd_kernel<D, false>, C::SMEM_BYTES, dev)) != ATTN_OK) return st;
-        attn::attn_fwd_kernel<D, false><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+        CUDA_TRY(cudaLaunchKernelEx(&lc, attn::attn_fwd_kernel<D, false, false>, tq, tk, tv, p));
     }
     CUDA_TRY(cudaGetLastError());
     return ATTN_OK;
@@ -408,8 +421,17 @@ attn_status launch_decode(const void* q, const void* k_pages, const void* v_page
     const uint64_t slabs = static_cast<uint64_t>(num_pages) * Hkv;
     if ((st = make_map_3d(&tk, k_pages, D, attn::kPageSize, slabs, attn::kPageSize)) != ATTN_OK) return st;
     if ((st = make_map_3d(&tv, v_pages, D, attn::kPageSize, slabs, attn::kPageSize)) != ATTN_OK) return st;
-    const int max_chunks = static_cast<int>(decode_chunks(max_blocks));
+    // chunk length: the longest that still gives at least 8 CTAs per SM (the grid's upper bound,
+    // from max_blocks; the workspace is sized for the shortest chunk, so any choice fits)
+    int sms = 148;
+    CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+    const long long rows = static_cast<long long>(S) * Hkv * ((Hq / Hkv * T + 15) / 16);
+    int chunk_pages = attn::kMaxChunkPages;
+    while (chunk_pages > attn::kChunkPages && rows * ((max_blocks + chunk_pages - 1) / chunk_pages) < 8LL * sms)
+        chunk_pages /= 2;
+    const int max_chunks = (max_blocks + chunk_pages - 1) / chunk_pages;  // never more than decode_chunks()
     attn::DecodeParams p{};
+    p.chunk_pages = chunk_pages;
     p.q = static_cast<const __nv_bfloat16*>(q);
     p.block_table = block_table;
     p.seq_lens = seq_lens;

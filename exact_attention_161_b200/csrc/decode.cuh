@@ -7,7 +7,7 @@
 // sequence and does little arithmetic per byte, so this path is bound by HBM bandwidth ("Why is
 // attention O(n^2), how does FlashAttention help, ...", follow-up "Why is decode memory-bound").
 //
-// Split: the logical token range of every sequence is cut into chunks of kChunkPages pages.
+// Split: the logical token range of every sequence is cut into chunks of 32 to 128 pages.
 // One CTA handles one (chunk, KV head, sequence) and produces, for each of the G query heads
 // of that KV head, a partial online-softmax state (m, l, o) over its chunk -- the recurrence of
 // "Deep dive: FlashAttention" applied to a slice of the keys. A second kernel merges the
@@ -35,7 +35,12 @@
 namespace attn {
 
 constexpr int kPageSize = 16;
-constexpr int kChunkPages = 32;                    // 512 tokens per split
+// Chunk lengths in pages: the host takes the longest of 128, 64 and 32 pages (2048, 1024, 512
+// tokens) that still gives every SM several CTAs. Longer chunks spread a CTA's fixed cost (its
+// set-up, the combine of its four warps' states and the partial states it writes) over more
+// pages; the workspace is sized for the shortest.
+constexpr int kChunkPages = 32;
+constexpr int kMaxChunkPages = 128;
 constexpr int kDecodeWarps = 4;
 constexpr int kDecodeThreads = kDecodeWarps * 32;
 
@@ -49,6 +54,7 @@ struct DecodeParams {
     float* ws_ml;                // [S, T*Hq, max_chunks, 2] partial (max in log2 units, sum)
     int S, Hq, Hkv, G, max_blocks, num_pages, max_chunks;
     int T, mtiles;               // new tokens per sequence; 16-row tiles per KV head = ceil(G*T / 16)
+    int chunk_pages;             // pages per split chunk
     int debug_drop_copy;         // test hook: CTA (0,0,0) skips its first page copy (see attn.h)
     float scale_log2;
 };
@@ -130,9 +136,9 @@ __global__ void __launch_bounds__(kDecodeThreads)
         return;
     }
     const int n_pages = (len + kPageSize - 1) / kPageSize;
-    const int pg_begin = chunk * kChunkPages;
+    const int pg_begin = chunk * p.chunk_pages;
     if (pg_begin >= n_pages) return;
-    const int pg_end = min(n_pages, pg_begin + kChunkPages);
+    const int pg_end = min(n_pages, pg_begin + p.chunk_pages);
     const int my_count = (pg_end - pg_begin - warp + kDecodeWarps - 1) / kDecodeWarps;  // may be <= 0
 
     if (threadIdx.x == 0) {
@@ -408,7 +414,7 @@ __global__ void __launch_bounds__(128) decode_merge_kernel(const DecodeParams p)
         if (p.lse != nullptr && lane == 0) p.lse[out_row] = __int_as_float(0x7fc00000);
         return;
     }
-    const int n_chunks = (len + kChunkPages * kPageSize - 1) / (kChunkPages * kPageSize);
+    const int n_chunks = (len + p.chunk_pages * kPageSize - 1) / (p.chunk_pages * kPageSize);
     const size_t base = out_row * p.max_chunks;
     float M = -INFINITY;
     for (int c = 0; c < n_chunks; ++c) M = fmaxf(M, p.ws_ml[(base + c) * 2]);

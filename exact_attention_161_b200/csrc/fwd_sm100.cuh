@@ -187,6 +187,10 @@ __global__ void __launch_bounds__(FwdCfg<D, kFp8>::THREADS, 1)
         ptx::tmem_alloc(&bar->tmem_base, C::TMEM_COLS);
         ptx::tmem_relinquish();
     }
+    // Launched right behind the query/key rotation pass, the kernel may start before that pass
+    // has finished: the set-up above overlaps its tail, and every thread waits here for it (and its
+    // writes) to complete before any global memory is read or written.
+    ptx::grid_dependency_wait();
     ptx::tc_fence_before();
     __syncthreads();
     ptx::tc_fence_after();

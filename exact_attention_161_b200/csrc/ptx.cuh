@@ -97,6 +97,14 @@ __device__ __forceinline__ bool elect_one() {
     return is_leader != 0;
 }
 
+// Programmatic dependent launch: a kernel launched with programmatic stream serialisation may
+// start while the kernel before it on the stream is still running; launch_dependents (in the
+// earlier kernel) lets it be scheduled, and wait (in the later kernel) blocks until the earlier
+// kernel has completed and its memory writes are visible. Without such a predecessor, wait returns
+// at once.
+__device__ __forceinline__ void grid_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ------------------------------------------------------------------------------ TMA
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");

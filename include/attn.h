@@ -155,7 +155,8 @@ attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o,
 
 /*
  * attn_decode_workspace_size -- bytes of device workspace attn_decode_paged needs: fp32 partial
- * (max, sum, output) states for every (sequence, query head, 512-token split). Returns 0 for
+ * (max, sum, output) states for every (sequence, query head, 512-token split) -- the shortest split
+ * the call may use, so the size covers every choice. Returns 0 for
  * invalid sizes.
  */
 size_t attn_decode_workspace_size(int num_seqs, int max_blocks_per_seq, int page_size, int Hq, int D);
@@ -168,7 +169,9 @@ size_t attn_decode_workspace_size(int num_seqs, int max_blocks_per_seq, int page
  * FlashAttention, PagedAttention, and RoPE in Code", Part 3: fixed-size blocks, block tables).
  * The single query of sequence s (its newest token, position seq_lens[s]-1, already rotated)
  * attends to all seq_lens[s] cached tokens, which include that token itself. The key range is
- * split into chunks of 512 tokens whose partial softmax states are merged in ascending order,
+ * split into chunks of 512, 1024 or 2048 tokens (the longest that still gives every SM several
+ * CTAs for the call's num_seqs, heads and max_blocks_per_seq) whose partial softmax states are
+ * merged in ascending order,
  * so the result depends only on logical token positions: a paged cache and a contiguous copy
  * of it give bit-identical outputs.
  *
@@ -197,7 +200,8 @@ attn_status attn_decode_paged(const void* q, const void* k_pages, const void* v_
 
 /*
  * attn_decode_step_workspace_size -- bytes of device workspace attn_decode_step needs: fp32 partial
- * outputs and (max, sum) per (sequence, new token, query head, 512-token chunk), rounded up to
+ * outputs and (max, sum) per (sequence, new token, query head, 512-token chunk, the shortest a call
+ * may use), rounded up to
  * 256 bytes. 0 for invalid sizes.
  */
 size_t attn_decode_step_workspace_size(int num_seqs, int q_len, int max_blocks_per_seq, int page_size, int Hq, int D);
