@@ -238,7 +238,7 @@ attn_status ensure_smem(K kernel, int bytes, int dev) {
 }
 
 // Rotate Q (bhq rows of N positions) and K (bhk rows) into qr and kr with one launch of
-// rope_rotate_rows_kernel: x covers the N * units (position, unit) pairs with 256 threads a block,
+// rope_rotate_rows_kernel: x covers the N * D/8 (position, chunk) pairs with 256 threads a block,
 // at most 8 blocks per SM (the x loop strides over the rest); z picks the tensor; y splits the
 // rows so that about 8 blocks per SM are resident however few positions there are.
 template <int D>
@@ -253,8 +253,7 @@ attn_status launch_rope_rows(bool half, const void* q, void* qr, long long bhq, 
     a.bh[1] = bhk;
     a.cs = cs;
     a.N = N;
-    const long long units = half ? D / 16 : D / 8;  // thread units per position (see the kernel)
-    const long long want = (static_cast<long long>(N) * units + 255) / 256;
+    const long long want = (static_cast<long long>(N) * (D / 8) + 255) / 256;
     const long long gx = want < 8LL * sms ? want : 8LL * sms;
     const long long bh_max = bhq > bhk ? bhq : bhk;
     long long gy = (8LL * sms + 2 * gx - 1) / (2 * gx);

@@ -38,10 +38,10 @@ struct RopeRowsArgs {
     int N;
 };
 
-// A thread takes one 16-byte output chunk (4 pairs) of one position (half-split: two chunks, from
-// one full 16-byte load of each half), loads that unit's table entries once and applies them to
-// it in rows blockIdx.y, blockIdx.y + gridDim.y, ... of the bh rows at that position, loading
-// several such rows before it stores any, so that several loads are in flight per thread. Consecutive threads take consecutive chunks, so each row's loads and
+// A thread takes one 16-byte output chunk (4 pairs) of one position, loads that chunk's 4 table
+// entries once and applies them to the chunk in rows blockIdx.y, blockIdx.y + gridDim.y, ... of
+// the bh rows at that position, loading 4 such rows before it stores any, so that several loads
+// are in flight per thread. Consecutive threads take consecutive chunks, so each row's loads and
 // stores are coalesced; the y split keeps a short sequence (few positions, many rows) from
 // running on fewer blocks than there are SMs.
 // kHalf: the pairs are (i, i + D/2) and the rotated pair i is written interleaved at (2i, 2i+1) --
@@ -49,12 +49,8 @@ struct RopeRowsArgs {
 // unchanged, so the attention kernel treats both pairings alike.
 template <int D, bool kHalf = false>
 __global__ void __launch_bounds__(256) rope_rotate_rows_kernel(RopeRowsArgs a) {
-    // half-split: a thread takes 8 pairs (i, i + D/2), i = 8c .. 8c+7: one full 16-byte chunk of
-    // each half, written as two interleaved output chunks 2c and 2c+1
     constexpr int CHUNKS = D / 8;
-    constexpr int UNITS = kHalf ? D / 16 : D / 8;  // thread units per position
-    constexpr int PAIRS = kHalf ? 8 : 4;           // pairs per unit
-    constexpr int U = kHalf ? 2 : 4;               // rows in flight per thread
+    constexpr int U = 4;  // rows in flight per thread
     // The attention kernel that reads the rotated rows is launched as this kernel's programmatic
     // dependent: it may be scheduled now and run its set-up, and it waits for this grid to
     // complete before it touches global memory.
@@ -64,49 +60,42 @@ __global__ void __launch_bounds__(256) rope_rotate_rows_kernel(RopeRowsArgs a) {
     uint4* __restrict__ dst = z ? a.dst[1] : a.dst[0];
     const long long bh_count = z ? a.bh[1] : a.bh[0];
     const int N = a.N;
-    const long long total = static_cast<long long>(N) * UNITS;
+    const long long total = static_cast<long long>(N) * CHUNKS;
     const long long ys = gridDim.y;
     for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
          idx += (long long)gridDim.x * blockDim.x) {
-        const int pos = static_cast<int>(idx / UNITS);
-        const int c = static_cast<int>(idx % UNITS);
-        double2 t[PAIRS];
+        const int pos = static_cast<int>(idx / CHUNKS);
+        const int c = static_cast<int>(idx % CHUNKS);
+        double2 t[4];
 #pragma unroll
-        for (int e = 0; e < PAIRS; ++e) t[e] = __ldg(a.cs + static_cast<size_t>(pos) * (D / 2) + c * PAIRS + e);
+        for (int e = 0; e < 4; ++e) t[e] = __ldg(a.cs + static_cast<size_t>(pos) * (D / 2) + c * 4 + e);
         for (long long bh0 = blockIdx.y; bh0 < bh_count; bh0 += U * ys) {
-            uint4 w[U][kHalf ? 2 : 1];
+            uint4 w[U];
 #pragma unroll
             for (int j = 0; j < U; ++j) {
                 const long long bh = bh0 + j * ys;
                 if (bh >= bh_count) continue;
                 const long long row = bh * N + pos;
                 if constexpr (kHalf) {
-                    const uint4 lo = __ldg(src + row * CHUNKS + c);               // elements 8c .. 8c+7
-                    const uint4 hi = __ldg(src + row * CHUNKS + c + CHUNKS / 2);  // elements D/2 + 8c ..
-                    const uint32_t lv[4] = {lo.x, lo.y, lo.z, lo.w}, hv[4] = {hi.x, hi.y, hi.z, hi.w};
-                    uint32_t o[8];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {  // pair 2e, 2e+1 of the unit: (lo[k], hi[k]) interleaved
-                        o[2 * e] = (lv[e] & 0xFFFFu) | (hv[e] << 16);
-                        o[2 * e + 1] = (lv[e] >> 16) | (hv[e] & 0xFFFF0000u);
-                    }
-                    w[j][0] = make_uint4(o[0], o[1], o[2], o[3]);
-                    w[j][1] = make_uint4(o[4], o[5], o[6], o[7]);
+                    // pairs 4c .. 4c+3: first members at elements 4c.., second members at D/2 + 4c..
+                    const uint2* s2 = reinterpret_cast<const uint2*>(src + row * CHUNKS);
+                    const uint2 lo = __ldg(s2 + c), hi = __ldg(s2 + c + D / 8);
+                    w[j].x = (lo.x & 0xFFFFu) | (hi.x << 16);
+                    w[j].y = (lo.x >> 16) | (hi.x & 0xFFFF0000u);
+                    w[j].z = (lo.y & 0xFFFFu) | (hi.y << 16);
+                    w[j].w = (lo.y >> 16) | (hi.y & 0xFFFF0000u);
                 } else {
-                    w[j][0] = __ldg(src + row * CHUNKS + c);
+                    w[j] = __ldg(src + row * CHUNKS + c);
                 }
             }
 #pragma unroll
             for (int j = 0; j < U; ++j) {
                 const long long bh = bh0 + j * ys;
                 if (bh >= bh_count) continue;
+                uint32_t* wv = reinterpret_cast<uint32_t*>(&w[j]);
 #pragma unroll
-                for (int h = 0; h < (kHalf ? 2 : 1); ++h) {
-                    uint32_t* wv = reinterpret_cast<uint32_t*>(&w[j][h]);
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) wv[e] = rope_rotate_pair(wv[e], t[4 * h + e].x, t[4 * h + e].y);
-                    dst[(bh * N + pos) * CHUNKS + (kHalf ? 2 * c + h : c)] = w[j][h];
-                }
+                for (int e = 0; e < 4; ++e) wv[e] = rope_rotate_pair(wv[e], t[e].x, t[e].y);
+                dst[(bh * N + pos) * CHUNKS + c] = w[j];
             }
         }
     }
