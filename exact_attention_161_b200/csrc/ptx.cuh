@@ -415,6 +415,23 @@ __device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
         : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
     return d;
 }
+// 2^x on the FMA and ALU pipes instead of the SFU, by the range reduction of
+// Cody and Waite: x = j + f with j = round(x) and f in [-1/2, 1/2], 2^x = p(f) * 2^j, the power of
+// two entering as j added to the exponent field. p is a degree-3 polynomial with p(0) = 1, fitted
+// for this kernel by minimax in relative error on [-1/2, 1/2] (Lawson's iteration): largest
+// relative error 1.0e-4, far below the bf16 rounding of the probabilities. x is clamped at -127,
+// where the result is exactly +0 (j = -127, p(0) = 1), so masked scores (-inf) give 0.
+__device__ __forceinline__ float ex2_poly(float x) {
+    x = fmaxf(x, -127.f);
+    const float t = x + 12582912.f;  // 1.5 * 2^23: t holds round(x) in its low mantissa bits
+    const float f = x - (t - 12582912.f);
+    float q = fmaf(0x1.c2a15cp-5f, f, 0x1.f00bfep-3f);
+    q = fmaf(q, f, 0x1.62f5fap-1f);
+    q = fmaf(q, f, 1.f);
+    return __int_as_float(__float_as_int(q) + (__float_as_int(t) << 23));
+}
+__device__ __forceinline__ float2 ex2_poly2(float2 x) { return make_float2(ex2_poly(x.x), ex2_poly(x.y)); }
+
 // max(a, b, c) in one instruction (sm_100a).
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
     float d;
