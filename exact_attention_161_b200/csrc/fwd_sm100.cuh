@@ -17,8 +17,8 @@
 //              buffer, rescales its row of O when the max moved by more than 2^8, and finally
 //              reads O out of TMEM (releasing it for the next item's products) and writes O and
 //              LSE. Q and K arrive already rotated (RoPE) by a streaming pass before the kernel.
-//   warp 8     TMA producer: the Q tiles once, then K tiles into a NK-stage ring and V tiles into
-//              a NV-stage ring.
+//   warp 8     TMA producer: the Q tiles once, then K tiles into an NK-stage ring and V tiles into
+//              an NV-stage ring.
 //   warp 9     MMA issuer and TMEM owner: the warp walks the schedule, one elected lane issues.
 //
 // Tensor Memory (512 columns): S0 at 0, S1 at 128, O0 at 256, O1 at 256 + D. The MMA thread
@@ -67,8 +67,10 @@ struct FwdCfg {
     static constexpr int O_KSTEPS = BN * ELEM / 32;   // MMAs per P V (32 bytes of P per row each)
     static constexpr int O_ROWS = 32 / ELEM;          // keys (V rows) per P V MMA
     static constexpr int P_COLS = BN * ELEM / 4;      // TMEM columns that hold P
-    static constexpr int NK = kFp8 ? 4 : (D == 128) ? 3 : 4;  // K pipeline stages
-    static constexpr int NV = kFp8 ? 4 : (D == 128) ? 2 : 4;  // V pipeline stages
+    // K and V pipeline stages. K(u) is read one step before V(u) and both stages of a step are
+    // released together, so at D = 128 (five 32 KB tiles fit beside Q) V gets the deeper ring.
+    static constexpr int NK = kFp8 ? 4 : (D == 128) ? 2 : 4;
+    static constexpr int NV = kFp8 ? 4 : (D == 128) ? 3 : 4;
     static constexpr int SMEM_TILES = QT + NK + NV;
     static constexpr int SMEM_BYTES = SMEM_TILES * TILE_BYTES + 1024 /*barriers*/ + 1024 /*align*/;
     static constexpr uint32_t TMEM_COLS = 512;
