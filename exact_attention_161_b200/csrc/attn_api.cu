@@ -82,6 +82,21 @@ attn_status make_map_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_
     return ATTN_OK;
 }
 
+// 2-D fp32 map [d1 rows][d0 columns] with 32 x 32 boxes, 128-byte swizzled (reduce targets).
+attn_status make_map_2d_f32(CUtensorMap* map, void* base, uint64_t d0, uint64_t d1) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return fail(ATTN_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable (no CUDA driver?)");
+    const cuuint64_t dims[2] = {d0, d1};
+    const cuuint64_t strides[1] = {d0 * 4};
+    const cuuint32_t box[2] = {32, 32};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base, dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(ATTN_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+    return ATTN_OK;
+}
+
 // ------------------------------------------------------------------ caches
 struct DevBuf {
     void* ptr = nullptr;
@@ -467,7 +482,7 @@ attn_status launch_decode(const void* q, const void* k_pages, const void* v_page
 }
 
 struct BwdLayout {
-    size_t vec, qrot, krot, total;  // byte offsets within the workspace
+    size_t vec, dqacc, qrot, krot, total;  // byte offsets within the workspace
 };
 
 BwdLayout bwd_layout(int B, int Hq, int Hkv, int N, int D, bool rope) {
@@ -475,7 +490,8 @@ BwdLayout bwd_layout(int B, int Hq, int Hkv, int N, int D, bool rope) {
     const size_t npad = static_cast<size_t>((N + 127) / 128) * 128;
     BwdLayout L{};
     L.vec = 0;
-    L.qrot = up(static_cast<size_t>(B) * Hq * npad * 2 * sizeof(float));
+    L.dqacc = up(static_cast<size_t>(B) * Hq * npad * 2 * sizeof(float));
+    L.qrot = L.dqacc + up(static_cast<size_t>(B) * Hq * npad * D * sizeof(float));
     L.krot = L.qrot + (rope ? up(static_cast<size_t>(B) * Hq * N * D * 2) : 0);
     L.total = L.krot + (rope ? up(static_cast<size_t>(B) * Hkv * N * D * 2) : 0);
     return L;
@@ -495,6 +511,7 @@ attn_status launch_bwd(const void* q, const void* k, const void* v, const void* 
     p.lse = lse;
     p.vec = reinterpret_cast<float*>(w + L.vec);
     p.dq = static_cast<__nv_bfloat16*>(dq);
+    p.dqacc = reinterpret_cast<float*>(w + L.dqacc);
     p.dk = static_cast<__nv_bfloat16*>(dk);
     p.dv = static_cast<__nv_bfloat16*>(dv);
     p.B = B;
@@ -531,21 +548,25 @@ attn_status launch_bwd(const void* q, const void* k, const void* v, const void* 
     attn::bwd_prep_kernel<D><<<static_cast<unsigned>(prep_blocks < 16LL * sms ? prep_blocks : 16LL * sms), 256, 0,
                                stream>>>(p);
     CUDA_TRY(cudaGetLastError());
-    CUtensorMap tq, tk, tv, tdo;
+    CUtensorMap tq, tk, tv, tdo, tdq;
     attn_status st;
     if ((st = make_map_3d(&tq, q_use, D, N, static_cast<uint64_t>(B) * Hq, 128)) != ATTN_OK) return st;
     if ((st = make_map_3d(&tk, k_use, D, N, static_cast<uint64_t>(B) * Hkv, 128)) != ATTN_OK) return st;
     if ((st = make_map_3d(&tv, v, D, N, static_cast<uint64_t>(B) * Hkv, 128)) != ATTN_OK) return st;
     if ((st = make_map_3d(&tdo, dout, D, N, static_cast<uint64_t>(B) * Hq, 128)) != ATTN_OK) return st;
-    if ((st = ensure_smem(attn::attn_bwd_dkdv_kernel<D>, C::SMEM_BYTES, dev)) != ATTN_OK) return st;
-    if ((st = ensure_smem(attn::attn_bwd_dq_kernel<D>, C::SMEM_BYTES, dev)) != ATTN_OK) return st;
-    // one-dimensional grids, tile index slowest (the kernels start the longest causal tiles first)
+    if ((st = make_map_2d_f32(&tdq, p.dqacc, D, static_cast<uint64_t>(B) * Hq * p.ntiles * 128)) != ATTN_OK) return st;
+    if ((st = ensure_smem(attn::attn_bwd_kernel<D>, C::SMEM_BYTES, dev)) != ATTN_OK) return st;
+    // the dq sums start from zero; every (key tile, query tile) pair adds its part
+    CUDA_TRY(cudaMemsetAsync(p.dqacc, 0, static_cast<size_t>(B) * Hq * p.ntiles * 128 * D * sizeof(float), stream));
+    // one-dimensional grid, key tile index slowest (the longest causal walks start first)
     const unsigned nt = static_cast<unsigned>(p.ntiles);
-    attn::attn_bwd_dkdv_kernel<D><<<nt * static_cast<unsigned>(B * Hkv), C::THREADS, C::SMEM_BYTES, stream>>>(
-        tq, tk, tv, tdo, p);
+    attn::attn_bwd_kernel<D><<<nt * static_cast<unsigned>(B * Hkv), C::THREADS, C::SMEM_BYTES, stream>>>(
+        tq, tk, tv, tdo, tdq, p);
     CUDA_TRY(cudaGetLastError());
-    attn::attn_bwd_dq_kernel<D><<<nt * static_cast<unsigned>(B * Hq), C::THREADS, C::SMEM_BYTES, stream>>>(
-        tq, tk, tv, tdo, p);
+    const long long dq_threads = static_cast<long long>(B) * Hq * N * (D / 8);
+    const long long dq_blocks = (dq_threads + 255) / 256;
+    attn::bwd_dq_store_kernel<D><<<static_cast<unsigned>(dq_blocks < 16LL * sms ? dq_blocks : 16LL * sms), 256, 0,
+                                   stream>>>(p);
     CUDA_TRY(cudaGetLastError());
     return ATTN_OK;
 }
@@ -647,8 +668,8 @@ attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o,
     if (window > 0 && !causal) return fail(ATTN_ERR_INVALID_ARG, "a sliding window requires causal = 1");
     if (!std::isfinite(scale) || !std::isfinite(rope_base)) return fail(ATTN_ERR_INVALID_ARG, "scale and rope_base must be finite");
     if (D != 64 && D != 128) return fail(ATTN_ERR_UNSUPPORTED, "head dim %d not supported (64 or 128)", D);
-    if (static_cast<double>(B) * Hq * ((N + 127) / 128) >= 2147483648.0)
-        return fail(ATTN_ERR_UNSUPPORTED, "grid too large: B * Hq * ceil(N/128) must be < 2^31");
+    if (static_cast<double>(B) * Hq * ((N + 127) / 128) * 128 >= 2147483648.0)
+        return fail(ATTN_ERR_UNSUPPORTED, "too many query rows: B * Hq * ceil(N/128) * 128 must be < 2^31");
     if (static_cast<double>(B) * Hq * N * D * 2 >= 1099511627776.0) return fail(ATTN_ERR_UNSUPPORTED, "tensor larger than 1 TiB");
     const size_t need = attn_bwd_workspace_size(B, Hq, Hkv, N, D, rope_base);
     if (workspace_bytes < need)

@@ -11,14 +11,16 @@
 //   dq_i  = scale sum_j dS_ij k_j       dk_j  = scale sum_i dS_ij q_i
 // with q, k the rotated vectors; RoPE's gradient rotates dq, dk back by -angle.
 //
-// Three kernels: a prep pass (D_i and the log2-scaled LSE, padded per 128-row tile), a dK/dV
+// Three kernels: a prep pass (D_i and the log2-scaled LSE, padded per 128-row tile), the main
 // kernel with one CTA per (128-key tile, K/V head) that walks every query head of the group and
-// every query tile that sees the keys, and a dQ kernel with one CTA per (128-query tile, query
-// head) that walks the visible key tiles. All five products per tile pair run on tcgen05 with
-// fp32 accumulators in Tensor Memory. Eight elementwise warps (two warpgroups, each owning 64 of
-// the 128 columns of a tile) turn scores into P and dS; the products are issued in an order that
-// lets the tensor core work on the next tile while they do (see each kernel's issue loop).
-// CTAs are numbered so that the ones with the most work start first.
+// every query tile that sees the keys, and a pass that turns the fp32 dq sums into bf16. The five
+// products of a tile pair (S^T, dP^T, dV, dK, dQ) run on tcgen05 with fp32 accumulators in Tensor
+// Memory: dK and dV accumulate there over the whole walk; the dQ of each tile pair is added into an
+// fp32 array in device memory by TMA reductions, since every key tile contributes to it.
+// Eight elementwise warps (two warpgroups, each owning 64 of the 128 query columns of a tile)
+// turn scores into P and dS and move the dQ partials out; the products are issued in an order that
+// lets the tensor core work while they do (see the issue loop). CTAs are numbered so that the
+// ones with the most work start first.
 #pragma once
 #include "common.cuh"
 #include "fwd_sm100.cuh"
@@ -33,6 +35,7 @@ struct BwdParams {
     float* vec;                 // [B*Hq, ntiles, 2, 128]: per 128-row tile -LSE*log2 e, then -D_i;
                                 // rows >= N hold (-inf, 0)
     __nv_bfloat16* dq;          // [B, Hq, N, D]
+    float* dqacc;               // [B*Hq, ntiles*128, D] fp32 sums of dS K, zeroed before the main kernel
     __nv_bfloat16* dk;          // [B, Hkv, N, D]
     __nv_bfloat16* dv;          // [B, Hkv, N, D]
     const float2* rope;         // (cos, sin) table or nullptr
@@ -85,11 +88,15 @@ struct BwdCfg {
     static constexpr int NREG = D / 64;
     static constexpr int REGION_BYTES = 128 * 128;
     static constexpr int TILE_BYTES = 128 * D * 2;
+    static constexpr int DS_BYTES = 2 * REGION_BYTES;  // dS^T of one tile pair: 128 keys x 128 queries, bf16
     static constexpr int VEC_BYTES = 256 * 4;  // -LSE*log2 e and -D of the 128 rows of a query tile
-    // fixed pair (K,V or Q,dO) + two stages of the streamed pair, with their vectors
-    static constexpr int SMEM_BYTES = 6 * TILE_BYTES + 2 * VEC_BYTES + 1024 /*barriers*/ + 1024 /*align*/;
-    static constexpr int THREADS = 320;  // warps 0-7 elementwise, 8 TMA producer, 9 MMA issuer
-    static constexpr int PRODUCER_WARP = 8, MMA_WARP = 9;
+    // K, V fixed + two stages of Q, dO + dS + two stages of the vectors, from a 1024-byte boundary
+    // (128-byte swizzled tiles), + 1024 bytes for the gap in front of that boundary and the barriers:
+    // the barriers (128 bytes) sit in the gap when it is at least that large, else after the vectors
+    static constexpr int SMEM_BYTES = 6 * TILE_BYTES + DS_BYTES + 2 * VEC_BYTES + 1024;
+    static_assert(SMEM_BYTES <= 232448, "backward shared memory above 227 KiB per CTA");
+    static constexpr int THREADS = 352;  // warps 0-7 elementwise, 8 TMA producer, 9 MMA issuer, 10 dQ reduce
+    static constexpr int PRODUCER_WARP = 8, MMA_WARP = 9, REDUCE_WARP = 10;
     static constexpr int EW_THREADS = 256;
     static constexpr uint32_t TMEM_COLS = 512;
 };
@@ -97,10 +104,12 @@ struct BwdCfg {
 struct BwdBarriers {
     uint64_t fixed_loaded;
     uint64_t full[2], empty[2];
-    uint64_t s_full[2], dp_full, p_full, ds_full, acc_done, drain;
+    uint64_t staged[2];  // the dQ partial of the step held in stage s is in shared memory
+    uint64_t s_full, dp_full, p_full, ds_full, dq_full, dq_free, acc_done, drain;
     uint32_t tmem_base;
     int abort;
 };
+static_assert(sizeof(BwdBarriers) <= 128, "barrier block larger than its reserved bytes");
 
 // 32 consecutive columns [c0, c0 + 32) of a gradient row held in registers (fp32, pairs (2t, 2t+1)):
 // rotate each pair by -angle at position pos (the gradient of the unrotated vector is the
@@ -140,7 +149,7 @@ __device__ __forceinline__ void query_tiles_for_keys(int j0, int N, int causal, 
 __device__ __forceinline__ constexpr uint32_t packed_col(int kk) { return (kk >> 2) * 64 + (kk & 3) * 8; }
 
 // P = 2^(s * scale_log2 + nlse) for 64 consecutive fp32 scores, the (-LSE*log2 e) values given per
-// element (dK/dV: per query column, from shared memory) or as one value (dQ: per row).
+// query column (from shared memory).
 __device__ __forceinline__ void probs64_cols(const uint32_t (&sv)[64], float scale_log2, const float* nlse,
                                              float (&pr)[64]) {
     const float2 sc = make_float2(scale_log2, scale_log2);
@@ -157,22 +166,12 @@ __device__ __forceinline__ void probs64_cols(const uint32_t (&sv)[64], float sca
         pr[c + 3] = ptx::ex2(b.y);
     }
 }
-__device__ __forceinline__ void probs64_row(const uint32_t (&sv)[64], float scale_log2, float nlse,
-                                            float (&pr)[64]) {
-    const float2 sc = make_float2(scale_log2, scale_log2), nl = make_float2(nlse, nlse);
-#pragma unroll
-    for (int c = 0; c < 64; c += 2) {
-        const float2 a = ptx::ffma2(make_float2(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])), sc, nl);
-        pr[c] = ptx::ex2(a.x);
-        pr[c + 1] = ptx::ex2(a.y);
-    }
-}
 // Zero the probabilities of columns outside [lo, hi] (column indices relative to the 64-column block).
 __device__ __forceinline__ void mask64(float (&pr)[64], int lo, int hi) {
 #pragma unroll
     for (int c = 0; c < 64; ++c) pr[c] = (c < lo || c > hi) ? 0.f : pr[c];
 }
-// dS = P (dP - D) for 32 columns, packed to 16 bf16 pairs. nd: -D per element (pointer) or per row.
+// dS = P (dP - D) for 32 columns, packed to 16 bf16 pairs; nd holds -D per column.
 __device__ __forceinline__ void dscores32_cols(const float* pr, const uint32_t (&dp)[32], const float* nd,
                                                uint32_t* out) {
 #pragma unroll
@@ -188,34 +187,44 @@ __device__ __forceinline__ void dscores32_cols(const float* pr, const uint32_t (
         out[c / 2 + 1] = ptx::pack_bf16x2(b.x, b.y);
     }
 }
-__device__ __forceinline__ void dscores32_row(const float* pr, const uint32_t (&dp)[32], float nd, uint32_t* out) {
-    const float2 n2 = make_float2(nd, nd);
-#pragma unroll
-    for (int c = 0; c < 32; c += 2) {
-        const float2 a = ptx::fmul2(make_float2(pr[c], pr[c + 1]),
-                                    ptx::fadd2(make_float2(__uint_as_float(dp[c]), __uint_as_float(dp[c + 1])), n2));
-        out[c / 2] = ptx::pack_bf16x2(a.x, a.y);
-    }
-}
 
-// =============================================================================== dK, dV
+// A warp's 32 x 32 fp32 block (lane = row, 32 columns in registers) into 4 KB of shared memory:
+// 128-byte rows, 16-byte chunk e of row r at position e ^ (r & 7), so the eight lanes of each
+// store phase hit distinct banks.
+// blk is the 32-bit shared address of a 1024-byte aligned block, so chunk e of row r sits at
+// (blk + 128 r + 16 (r & 7)) ^ 16 e.
+__device__ __forceinline__ void stage_rows32(uint32_t blk, const uint32_t (&v)[32], int lane) {
+    const uint32_t row = blk + lane * 128 + ((lane & 7) << 4);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) ptx::st_shared_v4(row ^ (e << 4), v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
+}
+// =============================================================================== dQ, dK, dV
 // CTA (key tile jt, K/V head g, batch b); block numbers run over key tiles slowest, so the causal
 // key tiles with the most visible queries start first. Steps t walk the visible query tiles from
 // the last one down, and the query heads of the group for each: under a causal mask every key
 // tile's walk starts at the same query tile, so the CTAs of one K/V head that run side by side read
-// each Q and dO tile at about the same time, and the repeats come from L2. TMEM: S^T at 0 (P^T packed into columns 0-31 and 64-95), dP^T at 128 (dS^T
-// packed likewise), dV at 256, dK at 256 + D.
+// each Q and dO tile at about the same time, and the repeats come from L2.
 //
-// Issue order per step t: dV(t) once P^T(t) is written, S^T(t+1), dK(t) once dS^T(t) is written,
-// dP^T(t+1). MMAs of one thread run in issue order, so S^T(t+1) may overwrite the scores that P^T(t)
-// was packed over once dV(t) is issued, and dP^T(t+1) the dS^T(t) buffer once dK(t) is issued; the
-// elementwise warps compute P^T(t+1) while the tensor core runs dK(t) and dP^T(t+1), and dS^T(t)
-// while it runs dV(t) and S^T(t+1).
+// TMEM: S^T at 0 (P^T packed into columns 0-31 and 64-95), dP^T at 128, which also takes the dQ
+// partial of the step once dS^T has been formed, dV at 256, dK at 256 + D. Shared memory holds dS^T
+// once per step (keys as 128-byte swizzled rows, queries along them); dK reads it K-major as
+// dS^T and dQ reads the same bytes MN-major as dS. The dQ partial (128 x D fp32) leaves through the
+// step's Q and dO buffers, which the tensor core is done with by then: each elementwise warp
+// stages its 32 rows there as 32 x 32 fp32 boxes; a reduce warp has the TMA add them into the fp32
+// sums and hands the stage back to the producer once the TMA has read it. That read takes about a
+// step's worth of time under load, so no warp on the per-step chain waits for it.
+//
+// Issue order per step t: dV(t) once P^T(t) is written; dK(t) and dQ(t) once dS^T(t) is written;
+// S^T(t+1); dP^T(t+1) once the dQ(t) partial has been read out of TMEM. MMAs of one thread run in
+// issue order, so S^T(t+1) may overwrite the scores that P^T(t) was packed over once dV(t) is
+// issued. The tensor core runs S^T(t+1) while the elementwise warps move dQ(t) out, and dV(t+1)
+// while they form dS^T(t+1). S^T(t+1) comes after dQ(t) so that the next stage of the ring, which
+// the dQ reduce of two steps back holds until the TMA has read it, has that long to load.
 template <int D>
 __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
-    attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                         const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                         const BwdParams p) {
+    attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                    const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
     using C = BwdCfg<D>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -223,8 +232,10 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     uint8_t* sV = sK + C::TILE_BYTES;
     uint8_t* sQ = sV + C::TILE_BYTES;          // [2] stages
     uint8_t* sDO = sQ + 2 * C::TILE_BYTES;     // [2] stages
-    float* sVec = reinterpret_cast<float*>(sDO + 2 * C::TILE_BYTES);  // [2][256]
-    auto* bar = reinterpret_cast<BwdBarriers*>(reinterpret_cast<uint8_t*>(sVec) + 2 * C::VEC_BYTES);
+    uint8_t* sDS = sDO + 2 * C::TILE_BYTES;    // dS^T, two 64-query regions
+    float* sVec = reinterpret_cast<float*>(sDS + C::DS_BYTES);  // [2][256]
+    auto* bar = reinterpret_cast<BwdBarriers*>(smem - smem_raw >= 128 ? smem_raw
+                                                                      : reinterpret_cast<uint8_t*>(sVec) + 2 * C::VEC_BYTES);
     volatile int* abort_flag = &bar->abort;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int groups = p.B * p.Hkv;
@@ -242,12 +253,15 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         ptx::mbar_init(&bar->fixed_loaded, 1);
         for (int s = 0; s < 2; ++s) {
             ptx::mbar_init(&bar->full[s], 1);
-            ptx::mbar_init(&bar->empty[s], 1);
-            ptx::mbar_init(&bar->s_full[s], 1);
+            ptx::mbar_init(&bar->empty[s], 1);  // the reduce warp, after the TMA has read the dQ staged there
+            ptx::mbar_init(&bar->staged[s], C::EW_THREADS);
         }
+        ptx::mbar_init(&bar->s_full, 1);
         ptx::mbar_init(&bar->dp_full, 1);
         ptx::mbar_init(&bar->p_full, C::EW_THREADS);
         ptx::mbar_init(&bar->ds_full, C::EW_THREADS);
+        ptx::mbar_init(&bar->dq_full, 1);
+        ptx::mbar_init(&bar->dq_free, C::EW_THREADS);
         ptx::mbar_init(&bar->acc_done, 1);
         ptx::mbar_init(&bar->drain, 1);
         bar->abort = 0;
@@ -305,41 +319,62 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         if (T > 0) {
             const bool leader = ptx::elect_one();
             const uint32_t tm = __shfl_sync(0xffffffffu, tmem, 0);
-            constexpr uint32_t ID_S = ptx::idesc_bf16_f32(128, 128, 0, 0);  // K (keys) x Q^T, both K-major
-            constexpr uint32_t ID_G = ptx::idesc_bf16_f32(128, D, 0, 1);    // P^T/dS^T (TMEM) x dO/Q (MN-major)
+            constexpr uint32_t ID_S = ptx::idesc_bf16_f32(128, 128, 0, 0);  // K Q^T, V dO^T: both K-major
+            constexpr uint32_t ID_G = ptx::idesc_bf16_f32(128, D, 0, 1);    // P^T (TMEM) / dS^T x dO / Q (MN-major)
+            constexpr uint32_t ID_Q = ptx::idesc_bf16_f32(128, D, 1, 1);    // dS x K, both MN-major
             constexpr uint32_t HI = ptx::sw128_desc_hi(1024);
             constexpr uint32_t TILE16 = C::TILE_BYTES >> 4;
             const uint32_t k_lo = ptx::sw128_desc_lo(ptx::smem_u32(sK), 16);
             const uint32_t v_lo = ptx::sw128_desc_lo(ptx::smem_u32(sV), 16);
             const uint32_t q_lo = ptx::sw128_desc_lo(ptx::smem_u32(sQ), 16);
             const uint32_t do_lo = ptx::sw128_desc_lo(ptx::smem_u32(sDO), 16);
+            const uint32_t ds_lo = ptx::sw128_desc_lo(ptx::smem_u32(sDS), 16);
             const uint32_t qmn_lo = ptx::sw128_desc_lo(ptx::smem_u32(sQ), C::REGION_BYTES);
             const uint32_t domn_lo = ptx::sw128_desc_lo(ptx::smem_u32(sDO), C::REGION_BYTES);
+            const uint32_t dsmn_lo = ptx::sw128_desc_lo(ptx::smem_u32(sDS), C::REGION_BYTES);
+            const uint32_t kmn_lo = ptx::sw128_desc_lo(ptx::smem_u32(sK), C::REGION_BYTES);
+            // K-major 16-element slice kk of a tile stored as 64-column regions of 128-byte rows
+            auto kslice = [](int kk) -> uint32_t {
+                return static_cast<uint32_t>(((kk >> 2) * C::REGION_BYTES + (kk & 3) * 32) >> 4);
+            };
             // S^T = K Q^T (M = 128 keys, N = 128 queries, K = D)
             auto issue_s = [&](int t) {
                 const uint32_t st = (t & 1) * TILE16;
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = ((kk >> 2) * C::REGION_BYTES + (kk & 3) * 32) >> 4;
-                    ptx::mma_ss(tm + T_S, ptx::desc64(k_lo + off, HI), ptx::desc64(q_lo + st + off, HI), ID_S, kk > 0);
-                }
+                for (int kk = 0; kk < D / 16; ++kk)
+                    ptx::mma_ss(tm + T_S, ptx::desc64(k_lo + kslice(kk), HI), ptx::desc64(q_lo + st + kslice(kk), HI),
+                                ID_S, kk > 0);
             };
             // dP^T = V dO^T
             auto issue_dp = [&](int t) {
                 const uint32_t st = (t & 1) * TILE16;
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = ((kk >> 2) * C::REGION_BYTES + (kk & 3) * 32) >> 4;
-                    ptx::mma_ss(tm + T_DP, ptx::desc64(v_lo + off, HI), ptx::desc64(do_lo + st + off, HI), ID_S, kk > 0);
-                }
+                for (int kk = 0; kk < D / 16; ++kk)
+                    ptx::mma_ss(tm + T_DP, ptx::desc64(v_lo + kslice(kk), HI), ptx::desc64(do_lo + st + kslice(kk), HI),
+                                ID_S, kk > 0);
             };
-            // dV += P^T dO, dK += dS^T Q (M = 128 keys, N = D, K = 128 queries)
-            auto issue_grad = [&](int t, uint32_t acc_col, uint32_t a_col, uint32_t b_lo) {
+            // dV += P^T dO (M = 128 keys, N = D, K = 128 queries; P^T packed in TMEM)
+            auto issue_dv = [&](int t) {
                 const uint32_t st = (t & 1) * TILE16;
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
-                    ptx::mma_ts(tm + acc_col, tm + a_col + packed_col(kk), ptx::desc64(b_lo + st + ((kk * 2048) >> 4), HI),
+                    ptx::mma_ts(tm + T_DV, tm + T_S + packed_col(kk), ptx::desc64(domn_lo + st + kk * 128, HI), ID_G,
+                                (t > 0 || kk > 0) ? 1u : 0u);
+            };
+            // dK += dS^T Q (M = 128 keys, N = D, K = 128 queries)
+            auto issue_dk = [&](int t) {
+                const uint32_t st = (t & 1) * TILE16;
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    ptx::mma_ss(tm + T_DK, ptx::desc64(ds_lo + kslice(kk), HI), ptx::desc64(qmn_lo + st + kk * 128, HI),
                                 ID_G, (t > 0 || kk > 0) ? 1u : 0u);
+            };
+            // dQ partial = dS K (M = 128 queries, N = D, K = 128 keys), into the dP^T columns
+            auto issue_dq = [&]() {
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    ptx::mma_ss(tm + T_DP, ptx::desc64(dsmn_lo + kk * 128, HI), ptx::desc64(kmn_lo + kk * 128, HI), ID_Q,
+                                kk > 0);
             };
             bool ok = ptx::mbar_wait_warp(&bar->fixed_loaded, 0, abort_flag) &&
                       ptx::mbar_wait_warp(&bar->full[0], 0, abort_flag);
@@ -347,7 +382,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
             if (ok) {
                 if (leader) {
                     issue_s(0);
-                    ptx::mma_commit(&bar->s_full[0]);
+                    ptx::mma_commit(&bar->s_full);
                     issue_dp(0);
                     ptx::mma_commit(&bar->dp_full);
                 }
@@ -357,29 +392,32 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
             for (int t = 0; ok && t < T; ++t) {
                 if (!ptx::mbar_wait_warp(&bar->p_full, t & 1, abort_flag)) { ok = false; break; }
                 ptx::tc_fence_after();
-                if (leader) issue_grad(t, T_DV, T_S, domn_lo);
+                if (leader) issue_dv(t);
+                __syncwarp();
+                if (!ptx::mbar_wait_warp(&bar->ds_full, t & 1, abort_flag)) { ok = false; break; }
+                ptx::tc_fence_after();
+                if (leader) {
+                    issue_dk(t);
+                    issue_dq();
+                    ptx::mma_commit(&bar->dq_full);
+                    if (t + 1 == T) ptx::mma_commit(&bar->acc_done);
+                }
                 __syncwarp();
                 if (t + 1 < T) {
                     if (!ptx::mbar_wait_warp(&bar->full[(t + 1) & 1], ((t + 1) >> 1) & 1, abort_flag)) { ok = false; break; }
                     if (leader) {
                         issue_s(t + 1);
-                        ptx::mma_commit(&bar->s_full[0]);
+                        ptx::mma_commit(&bar->s_full);
+                    }
+                    __syncwarp();
+                    if (!ptx::mbar_wait_warp(&bar->dq_free, t & 1, abort_flag)) { ok = false; break; }
+                    ptx::tc_fence_after();
+                    if (leader) {
+                        issue_dp(t + 1);
+                        ptx::mma_commit(&bar->dp_full);
                     }
                     __syncwarp();
                 }
-                if (!ptx::mbar_wait_warp(&bar->ds_full, t & 1, abort_flag)) { ok = false; break; }
-                ptx::tc_fence_after();
-                if (leader) {
-                    issue_grad(t, T_DK, T_DP, qmn_lo);
-                    ptx::mma_commit(&bar->empty[t & 1]);
-                    if (t + 1 < T) {
-                        issue_dp(t + 1);
-                        ptx::mma_commit(&bar->dp_full);
-                    } else {
-                        ptx::mma_commit(&bar->acc_done);
-                    }
-                }
-                __syncwarp();
             }
             if (!ok && leader) {
                 *abort_flag = 1;
@@ -392,19 +430,50 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
             }
         }
         __syncwarp();
+    } else if (warp == C::REDUCE_WARP) {
+        // ------------------------------------------------------------------ dQ reduce
+        // Per step: the TMA adds the staged boxes into the fp32 sums; once it has read them the
+        // stage goes back to the producer. The additions complete before the CTA exits.
+        if (lane == 0 && T > 0) {
+            bool ok = true;
+            for (int t = 0; t < T; ++t) {
+                const int s = t & 1;
+                const int qt = ie - 1 - t / G, h = g * G + t % G;
+                if (!ptx::mbar_wait(&bar->staged[s], (t >> 1) & 1, abort_flag)) { ok = false; break; }
+                const int row0 = ((b * p.Hq + h) * p.ntiles + qt) * 128;
+#pragma unroll 1
+                for (int w = 0; w < C::EW_THREADS / 32; ++w) {
+                    const uint32_t box = ptx::smem_u32((w >> 2) == 0 ? sQ : sDO) + s * C::TILE_BYTES + (w & 3) * (D / 64) * 4096;
+#pragma unroll
+                    for (int c = 0; c < D / 64; ++c)
+                        ptx::tma_reduce_add_2d(&tm_dq, box + c * 4096, (w >> 2) * (D / 2) + 32 * c, row0 + (w & 3) * 32);
+                }
+                ptx::bulk_commit_group();
+                ptx::bulk_wait_read_all();
+                ptx::mbar_arrive(&bar->empty[s]);
+            }
+            ptx::bulk_wait_all();
+            if (!ok) {
+                *abort_flag = 1;
+                raise_status(kStatusTimeout);
+            }
+        }
     } else {
         // ------------------------------------------------------------------ elementwise warps
         const int wg = warp >> 2;                  // query columns [64 wg, 64 wg + 64) of each tile
-        const int r = (warp & 3) * 32 + lane;      // key row == TMEM lane
+        const int r = (warp & 3) * 32 + lane;      // TMEM lane: key row of S^T, dP^T; query row of dQ
         const int key = j0 + r;
         const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
         const uint32_t t_s = tmem + lane_base + T_S + 64 * wg, t_dp = tmem + lane_base + T_DP + 64 * wg;
+        // this thread's dS^T row: region wg, 128-byte row r, 16-byte chunk c stored at c ^ (r & 7)
+        uint4* ds_row = reinterpret_cast<uint4*>(sDS + wg * C::REGION_BYTES + r * 128);
         bool ok = true;
         for (int t = 0; ok && t < T; ++t) {
             const int s = t & 1;
-            const int c0 = (ie - 1 - t / G) * 128 + 64 * wg;  // first query of this warpgroup's columns
+            const int qt = ie - 1 - t / G, h = g * G + t % G;
+            const int c0 = qt * 128 + 64 * wg;  // first query of this warpgroup's columns
             if (!ptx::mbar_wait(&bar->full[s], (t >> 1) & 1, abort_flag)) { ok = false; break; }
-            if (!ptx::mbar_wait(&bar->s_full[0], t & 1, abort_flag)) { ok = false; break; }
+            if (!ptx::mbar_wait(&bar->s_full, t & 1, abort_flag)) { ok = false; break; }
             ptx::tc_fence_after();
             const float* vec = sVec + s * 256 + 64 * wg;
             float pr[64];
@@ -427,16 +496,39 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
             ptx::mbar_arrive(&bar->p_full);
             if (!ptx::mbar_wait(&bar->dp_full, t & 1, abort_flag)) { ok = false; break; }
             ptx::tc_fence_after();
-            uint32_t dsk[32];
+            {
+                uint32_t dsk[32];
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                uint32_t dp[32];
-                ptx::tmem_ld32(t_dp + 32 * half, dp);
-                dscores32_cols(pr + 32 * half, dp, vec + 128 + 32 * half, dsk + 16 * half);
+                for (int half = 0; half < 2; ++half) {
+                    uint32_t dp[32];
+                    ptx::tmem_ld32(t_dp + 32 * half, dp);
+                    dscores32_cols(pr + 32 * half, dp, vec + 128 + 32 * half, dsk + 16 * half);
+                }
+#pragma unroll
+                for (int c = 0; c < 8; ++c)
+                    ds_row[c ^ (r & 7)] = make_uint4(dsk[4 * c], dsk[4 * c + 1], dsk[4 * c + 2], dsk[4 * c + 3]);
             }
-            ptx::tmem_st32(t_dp, dsk);
+            ptx::fence_proxy_async_smem();
             ptx::tc_fence_before();
             ptx::mbar_arrive(&bar->ds_full);
+            // dQ partial of this step: query row qt * 128 + r, columns [wg D/2, wg D/2 + D/2). The
+            // step's Q (warpgroup 0) or dO (warpgroup 1) buffer takes it, this warp's rows as D/64
+            // boxes of 32 x 32; the TMEM columns are released once the last chunk is in registers.
+            if (!ptx::mbar_wait(&bar->dq_full, t & 1, abort_flag)) { ok = false; break; }
+            ptx::tc_fence_after();
+            {
+                const uint32_t box = ptx::smem_u32(wg == 0 ? sQ : sDO) + s * C::TILE_BYTES + (warp & 3) * (D / 64) * 4096;
+                const uint32_t t_dq = tmem + lane_base + T_DP + wg * (D / 2);
+                uint32_t v[32];
+                ptx::tmem_ld32(t_dq, v);
+                stage_rows32(box, v, lane);
+                if constexpr (D == 128) ptx::tmem_ld32(t_dq + 32, v);
+                ptx::tc_fence_before();
+                ptx::mbar_arrive(&bar->dq_free);
+                if constexpr (D == 128) stage_rows32(box + 4096, v, lane);
+            }
+            ptx::fence_proxy_async_smem();
+            ptx::mbar_arrive(&bar->staged[s]);
         }
         if (ok && T > 0) ok = ptx::mbar_wait(&bar->acc_done, 0, abort_flag);
         if (ok && T > 0) {
@@ -474,237 +566,36 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     }
 }
 
-// =============================================================================== dQ
-// CTA (query tile it, query head h, batch b); block numbers run over query tiles slowest, the last
-// (causal: longest) tiles first. Steps walk the visible key tiles. TMEM: S in two buffers at 0 and
-// 128, dP at 256 (dS packed into columns 256-287 and 320-351), dQ at 384.
-//
-// Issue order per step t: S(t+1) into the other buffer, dQ(t) once dS(t) is written, dP(t+1). P
-// stays in registers, so the elementwise warps compute P(t+1) while the tensor core runs dQ(t) and
-// dP(t+1).
+// dq = scale * (the fp32 sums) rotated back by -angle (RoPE), stored bf16. Eight columns per
+// thread (one 16-byte store), grid-stride over the B * Hq * N rows.
 template <int D>
-__global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
-    attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                       const BwdParams p) {
-    using C = BwdCfg<D>;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t* sQ = smem;
-    uint8_t* sDO = sQ + C::TILE_BYTES;
-    uint8_t* sK = sDO + C::TILE_BYTES;        // [2] stages
-    uint8_t* sV = sK + 2 * C::TILE_BYTES;     // [2] stages
-    auto* bar = reinterpret_cast<BwdBarriers*>(sV + 2 * C::TILE_BYTES + 2 * C::VEC_BYTES);
-    volatile int* abort_flag = &bar->abort;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int groups = p.B * p.Hq;
-    const int rank = static_cast<int>(blockIdx.x / groups);
-    const int hb = static_cast<int>(blockIdx.x - static_cast<unsigned>(rank) * groups);
-    const int h = hb % p.Hq, b = hb / p.Hq;
-    const int qt = p.ntiles - 1 - rank;
-    const int q0 = qt * 128;
-    const int g = h / (p.Hq / p.Hkv);
-    const TileRange R = tile_range(q0, p.N, p.causal, p.window);
-    const int T = R.n;
-
-    if (threadIdx.x == 0) {
-        ptx::mbar_init(&bar->fixed_loaded, 1);
-        for (int s = 0; s < 2; ++s) {
-            ptx::mbar_init(&bar->full[s], 1);
-            ptx::mbar_init(&bar->empty[s], 1);
-            ptx::mbar_init(&bar->s_full[s], 1);
-        }
-        ptx::mbar_init(&bar->dp_full, 1);
-        ptx::mbar_init(&bar->p_full, 1);
-        ptx::mbar_init(&bar->ds_full, C::EW_THREADS);
-        ptx::mbar_init(&bar->acc_done, 1);
-        ptx::mbar_init(&bar->drain, 1);
-        bar->abort = 0;
-        ptx::fence_mbar_init();
-    }
-    if (warp == C::MMA_WARP) {
-        ptx::tmem_alloc(&bar->tmem_base, C::TMEM_COLS);
-        ptx::tmem_relinquish();
-    }
-    ptx::tc_fence_before();
-    __syncthreads();
-    ptx::tc_fence_after();
-    const uint32_t tmem = bar->tmem_base;
-    constexpr uint32_t T_S = 0, T_DP = 256, T_DQ = 384;
-
-    if (warp == C::PRODUCER_WARP) {
-        if (lane == 0 && T > 0) {
-            const int zq = b * p.Hq + h, zk = b * p.Hkv + g;
-            ptx::mbar_arrive_expect_tx(&bar->fixed_loaded, 2 * C::TILE_BYTES);
-            for (int r = 0; r < C::NREG; ++r) {
-                ptx::tma_load_3d(sQ + r * C::REGION_BYTES, &tm_q, &bar->fixed_loaded, r * 64, q0, zq);
-                ptx::tma_load_3d(sDO + r * C::REGION_BYTES, &tm_do, &bar->fixed_loaded, r * 64, q0, zq);
-            }
-            int issued = 0;
-            bool ok = true;
-            for (int t = 0; t < T && ok; ++t) {
-                const int s = t & 1;
-                if (t >= 2 && !ptx::mbar_wait(&bar->empty[s], ((t >> 1) - 1) & 1, abort_flag)) { ok = false; break; }
-                const int k0 = (R.jb + t) * 128;
-                ptx::mbar_arrive_expect_tx(&bar->full[s], 2 * C::TILE_BYTES);
-                for (int r = 0; r < C::NREG; ++r) {
-                    ptx::tma_load_3d(sK + s * C::TILE_BYTES + r * C::REGION_BYTES, &tm_k, &bar->full[s], r * 64, k0, zk);
-                    ptx::tma_load_3d(sV + s * C::TILE_BYTES + r * C::REGION_BYTES, &tm_v, &bar->full[s], r * 64, k0, zk);
-                }
-                issued = t + 1;
-            }
-            if (!ok) {
-                *abort_flag = 1;
-                raise_status(kStatusTimeout);
-                volatile int never = 0;
-                ptx::mbar_wait(&bar->fixed_loaded, 0, &never);
-                for (int t = max(0, issued - 2); t < issued; ++t) ptx::mbar_wait(&bar->full[t & 1], (t >> 1) & 1, &never);
-            }
-        }
-    } else if (warp == C::MMA_WARP) {
-        // The whole warp walks the steps and takes the waits; one elected lane issues.
-        if (T > 0) {
-            const bool leader = ptx::elect_one();
-            const uint32_t tm = __shfl_sync(0xffffffffu, tmem, 0);
-            constexpr uint32_t ID_S = ptx::idesc_bf16_f32(128, 128, 0, 0);  // Q K^T, dO V^T: K-major
-            constexpr uint32_t ID_G = ptx::idesc_bf16_f32(128, D, 0, 1);    // dS (TMEM) x K (MN-major)
-            constexpr uint32_t HI = ptx::sw128_desc_hi(1024);
-            constexpr uint32_t TILE16 = C::TILE_BYTES >> 4;
-            const uint32_t q_lo = ptx::sw128_desc_lo(ptx::smem_u32(sQ), 16);
-            const uint32_t do_lo = ptx::sw128_desc_lo(ptx::smem_u32(sDO), 16);
-            const uint32_t k_lo = ptx::sw128_desc_lo(ptx::smem_u32(sK), 16);
-            const uint32_t v_lo = ptx::sw128_desc_lo(ptx::smem_u32(sV), 16);
-            const uint32_t kmn_lo = ptx::sw128_desc_lo(ptx::smem_u32(sK), C::REGION_BYTES);
-            // S = Q K^T into buffer t & 1 (M = 128 queries, N = 128 keys, K = D)
-            auto issue_s = [&](int t) {
-                const uint32_t st = (t & 1) * TILE16;
+__global__ void __launch_bounds__(256) bwd_dq_store_kernel(const BwdParams p) {
+    constexpr int CPR = D / 8;  // threads per row
+    const long long total = static_cast<long long>(p.B) * p.Hq * p.N * CPR;
+    const size_t npad = static_cast<size_t>(p.ntiles) * 128;
+    for (long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
+         idx += static_cast<long long>(gridDim.x) * blockDim.x) {
+        const long long row = idx / CPR;
+        const int c0 = static_cast<int>(idx - row * CPR) * 8;
+        const long long bh = row / p.N;
+        const int i = static_cast<int>(row - bh * p.N);
+        const float4* src = reinterpret_cast<const float4*>(p.dqacc + (static_cast<size_t>(bh) * npad + i) * D + c0);
+        const float4 a = src[0], c = src[1];
+        float g[8] = {a.x * p.scale, a.y * p.scale, a.z * p.scale, a.w * p.scale,
+                      c.x * p.scale, c.y * p.scale, c.z * p.scale, c.w * p.scale};
+        if (p.rope != nullptr) {
+            const float2* cs = p.rope + static_cast<size_t>(i) * (D / 2) + c0 / 2;
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = ((kk >> 2) * C::REGION_BYTES + (kk & 3) * 32) >> 4;
-                    ptx::mma_ss(tm + T_S + 128 * (t & 1), ptx::desc64(q_lo + off, HI), ptx::desc64(k_lo + st + off, HI),
-                                ID_S, kk > 0);
-                }
-            };
-            // dP = dO V^T
-            auto issue_dp = [&](int t) {
-                const uint32_t st = (t & 1) * TILE16;
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = ((kk >> 2) * C::REGION_BYTES + (kk & 3) * 32) >> 4;
-                    ptx::mma_ss(tm + T_DP, ptx::desc64(do_lo + off, HI), ptx::desc64(v_lo + st + off, HI), ID_S, kk > 0);
-                }
-            };
-            bool ok = ptx::mbar_wait_warp(&bar->fixed_loaded, 0, abort_flag) &&
-                      ptx::mbar_wait_warp(&bar->full[0], 0, abort_flag);
-            bool issued_any = false;
-            if (ok) {
-                if (leader) {
-                    issue_s(0);
-                    ptx::mma_commit(&bar->s_full[0]);
-                    issue_dp(0);
-                    ptx::mma_commit(&bar->dp_full);
-                }
-                __syncwarp();
-                issued_any = true;
-            }
-            for (int t = 0; ok && t < T; ++t) {
-                if (t + 1 < T) {
-                    if (!ptx::mbar_wait_warp(&bar->full[(t + 1) & 1], ((t + 1) >> 1) & 1, abort_flag)) { ok = false; break; }
-                    if (leader) {
-                        issue_s(t + 1);
-                        ptx::mma_commit(&bar->s_full[(t + 1) & 1]);
-                    }
-                    __syncwarp();
-                }
-                if (!ptx::mbar_wait_warp(&bar->ds_full, t & 1, abort_flag)) { ok = false; break; }
-                ptx::tc_fence_after();
-                if (leader) {
-                    // dQ += dS K (M = 128 queries, N = D, K = 128 keys)
-                    const uint32_t st = (t & 1) * TILE16;
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        ptx::mma_ts(tm + T_DQ, tm + T_DP + packed_col(kk),
-                                    ptx::desc64(kmn_lo + st + ((kk * 2048) >> 4), HI), ID_G, (t > 0 || kk > 0) ? 1u : 0u);
-                    ptx::mma_commit(&bar->empty[t & 1]);
-                    if (t + 1 < T) {
-                        issue_dp(t + 1);
-                        ptx::mma_commit(&bar->dp_full);
-                    } else {
-                        ptx::mma_commit(&bar->acc_done);
-                    }
-                }
-                __syncwarp();
-            }
-            if (!ok && leader) {
-                *abort_flag = 1;
-                raise_status(kStatusTimeout);
-                if (issued_any) {
-                    ptx::mma_commit(&bar->drain);
-                    volatile int never = 0;
-                    ptx::mbar_wait(&bar->drain, 0, &never);
-                }
+            for (int t = 0; t < 4; ++t) {
+                const float2 r = __ldg(cs + t);
+                const float x0 = g[2 * t], x1 = g[2 * t + 1];
+                g[2 * t] = fmaf(x0, r.x, x1 * r.y);
+                g[2 * t + 1] = fmaf(-x0, r.y, x1 * r.x);
             }
         }
-        __syncwarp();
-    } else {
-        const int wg = warp >> 2;              // key columns [64 wg, 64 wg + 64) of each tile
-        const int r = (warp & 3) * 32 + lane;  // query row == TMEM lane
-        const int qpos = q0 + r;
-        const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-        const uint32_t t_dp = tmem + lane_base + T_DP + 64 * wg;
-        const float* vrow = p.vec + (static_cast<size_t>(b * p.Hq + h) * p.ntiles + qt) * 256 + r;
-        const float nlse = vrow[0], nd = vrow[128];
-        bool ok = true;
-        for (int t = 0; ok && t < T; ++t) {
-            const int c0 = (R.jb + t) * 128 + 64 * wg;  // first key of this warpgroup's columns
-            if (!ptx::mbar_wait(&bar->s_full[t & 1], (t >> 1) & 1, abort_flag)) { ok = false; break; }
-            ptx::tc_fence_after();
-            float pr[64];
-            {
-                uint32_t sv[64];
-                ptx::tmem_ld64(tmem + lane_base + T_S + 128 * (t & 1) + 64 * wg, sv);
-                probs64_row(sv, p.scale_log2, nlse, pr);
-            }
-            // key kpos is visible iff kpos <= qpos (causal) and qpos - kpos < window; keys past N
-            // have zero K and V rows (zero-filled loads), so their dS meets a zero K row
-            const int hi = p.causal ? qpos - c0 : 64;
-            const int lo = p.window > 0 ? qpos - p.window + 1 - c0 : -1;
-            if (lo > 0 || hi < 63) mask64(pr, lo, hi);
-            if (!ptx::mbar_wait(&bar->dp_full, t & 1, abort_flag)) { ok = false; break; }
-            ptx::tc_fence_after();
-            uint32_t dsk[32];
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                uint32_t dp[32];
-                ptx::tmem_ld32(t_dp + 32 * half, dp);
-                dscores32_row(pr + 32 * half, dp, nd, dsk + 16 * half);
-            }
-            ptx::tmem_st32(t_dp, dsk);
-            ptx::tc_fence_before();
-            ptx::mbar_arrive(&bar->ds_full);
-        }
-        if (ok && T > 0) ok = ptx::mbar_wait(&bar->acc_done, 0, abort_flag);
-        if (ok && T > 0) {
-            // each warpgroup writes half of the D columns
-            ptx::tc_fence_after();
-            __nv_bfloat16* dst = p.dq + ((static_cast<size_t>(b) * p.Hq + h) * p.N + min(qpos, p.N - 1)) * D;
-#pragma unroll 1
-            for (int c = wg * (D / 64); c < (wg + 1) * (D / 64); ++c) {
-                uint32_t v[32];
-                ptx::tmem_ld32(tmem + lane_base + T_DQ + c * 32, v);
-                if (qpos < p.N) store_chunk_unrotated(v, p.scale, p.rope, D, qpos, c * 32, dst);
-            }
-        }
-        if (!ok) {
-            *abort_flag = 1;
-            raise_status(kStatusTimeout);
-        }
-    }
-    ptx::tc_fence_before();
-    __syncthreads();
-    if (warp == C::MMA_WARP) {
-        ptx::tc_fence_after();
-        ptx::tmem_dealloc(tmem, C::TMEM_COLS);
+        *reinterpret_cast<uint4*>(p.dq + static_cast<size_t>(row) * D + c0) =
+            make_uint4(ptx::pack_bf16x2(g[0], g[1]), ptx::pack_bf16x2(g[2], g[3]), ptx::pack_bf16x2(g[4], g[5]),
+                       ptx::pack_bf16x2(g[6], g[7]));
     }
 }
 

@@ -125,7 +125,8 @@ attn_status attn_fwd_fp8(const void* q, const void* k, const void* v, void* o, f
 
 /*
  * attn_bwd_workspace_size -- bytes of device workspace attn_bwd needs: fp32 (-LSE*log2 e, -D_i)
- * per query row padded to 128-row tiles, plus, with RoPE, the rotated Q and K (bf16). 0 for invalid sizes.
+ * and the fp32 dq sums (D values) per query row padded to 128-row tiles, plus, with RoPE, the
+ * rotated Q and K (bf16). 0 for invalid sizes.
  */
 size_t attn_bwd_workspace_size(int B, int Hq, int Hkv, int N, int D, float rope_base);
 
@@ -139,7 +140,9 @@ size_t attn_bwd_workspace_size(int B, int Hq, int Hkv, int N, int D, float rope_
  *   dv_j = sum_i P_ij dO_i,  dS_ij = P_ij (dO_i . v_j - dO_i . O_i),
  *   dq_i = scale sum_j dS_ij k_j,  dk_j = scale sum_i dS_ij q_i,
  * with q, k rotated; the gradients of the unrotated inputs are rotated back. For GQA, dk and dv of a
- * K/V head sum over its query heads.
+ * K/V head sum over its query heads. dk and dv are accumulated in a fixed order and repeat bit for
+ * bit; dq is a sum of fp32 partials (one per 128-key tile) added in device memory in the order the
+ * tiles finish, so two calls may differ by one bf16 unit in the last place.
  *
  *   q, k, v, causal, window, rope_base, scale, B, Hq, Hkv, N, D   as given to attn_fwd
  *   o      bf16 [B, Hq, N, D] and lse fp32 [B, Hq, N]: attn_fwd's outputs for these inputs
@@ -147,7 +150,7 @@ size_t attn_bwd_workspace_size(int B, int Hq, int Hkv, int N, int D, float rope_
  *   dq     bf16 [B, Hq, N, D]; dk, dv bf16 [B, Hkv, N, D]: written
  *   workspace  device scratch of at least attn_bwd_workspace_size(...) bytes, 16-byte aligned,
  *          owned by the caller, any initial contents; overlapping calls need their own.
- * Constraints and errors as attn_fwd (D in {64, 128}), with B * Hq * ceil(N/128) < 2^31.
+ * Constraints and errors as attn_fwd (D in {64, 128}), with B * Hq * ceil(N/128) * 128 < 2^31.
  */
 attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
                      void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int N, int D, int causal, int window,

@@ -129,13 +129,14 @@ def test_bwd_validation(api, kw, expect):
 
 
 def test_bwd_workspace_size(api):
-    # fp32 (-LSE log2 e, -D_i) per query row padded to 128-row tiles, 256-B rounded; with RoPE
-    # also the rotated Q and K in bf16, each 256-B rounded
-    assert api.bwd_workspace_size(1, 4, 2, 128, 128) == 4 * 128 * 2 * 4
-    assert api.bwd_workspace_size(1, 1, 1, 1, 64) == 1024
-    assert api.bwd_workspace_size(2, 32, 8, 8192, 128, 10000.0) == (2 * 32 * 8192 * 2 * 4 + 2 * 32 * 8192 * 128 * 2
+    # fp32 (-LSE log2 e, -D_i) and fp32 dq sums per query row padded to 128-row tiles, each 256-B
+    # rounded; with RoPE also the rotated Q and K in bf16, each 256-B rounded
+    assert api.bwd_workspace_size(1, 4, 2, 128, 128) == 4 * 128 * 2 * 4 + 4 * 128 * 128 * 4
+    assert api.bwd_workspace_size(1, 1, 1, 1, 64) == 1024 + 128 * 64 * 4
+    assert api.bwd_workspace_size(2, 32, 8, 8192, 128, 10000.0) == (2 * 32 * 8192 * 2 * 4 + 2 * 32 * 8192 * 128 * 4
+                                                                     + 2 * 32 * 8192 * 128 * 2
                                                                      + 2 * 8 * 8192 * 128 * 2)
-    assert api.bwd_workspace_size(1, 2, 1, 3, 64, 10000.0) == 2 * 128 * 2 * 4 + 768 + 512
+    assert api.bwd_workspace_size(1, 2, 1, 3, 64, 10000.0) == 2 * 128 * 2 * 4 + 2 * 128 * 64 * 4 + 768 + 512
     assert api.bwd_workspace_size(0, 4, 2, 128, 128) == 0
 
 
