@@ -95,9 +95,11 @@ struct BwdCfg {
     // the barriers (128 bytes) sit in the gap when it is at least that large, else after the vectors
     static constexpr int SMEM_BYTES = 6 * TILE_BYTES + DS_BYTES + 2 * VEC_BYTES + 1024;
     static_assert(SMEM_BYTES <= 232448, "backward shared memory above 227 KiB per CTA");
-    static constexpr int THREADS = 352;  // warps 0-7 elementwise, 8 TMA producer, 9 MMA issuer, 10 dQ reduce
-    static constexpr int PRODUCER_WARP = 8, MMA_WARP = 9, REDUCE_WARP = 10;
-    static constexpr int EW_THREADS = 256;
+    // warps 0-15 elementwise (four groups of 32 query columns), 16 TMA producer, 17 MMA issuer,
+    // 18 dQ reduce
+    static constexpr int THREADS = 608;
+    static constexpr int PRODUCER_WARP = 16, MMA_WARP = 17, REDUCE_WARP = 18;
+    static constexpr int EW_THREADS = 512;
     static constexpr uint32_t TMEM_COLS = 512;
 };
 
@@ -144,17 +146,17 @@ __device__ __forceinline__ void query_tiles_for_keys(int j0, int N, int causal, 
     if (window > 0) ie = min(nq, (j0 + 127 + window - 1) / 128 + 1);
 }
 
-// TMEM column of the k-th 16-element slice of a packed bf16 operand: each warpgroup packs its 64
-// columns of a 128-column fp32 buffer into the first 32 columns of its own half.
-__device__ __forceinline__ constexpr uint32_t packed_col(int kk) { return (kk >> 2) * 64 + (kk & 3) * 8; }
+// TMEM column of the k-th 16-element slice of a packed bf16 operand: each group of elementwise
+// warps packs its 32 columns of a 128-column fp32 buffer into the first 16 of them.
+__device__ __forceinline__ constexpr uint32_t packed_col(int kk) { return (kk >> 1) * 32 + (kk & 1) * 8; }
 
-// P = 2^(s * scale_log2 + nlse) for 64 consecutive fp32 scores, the (-LSE*log2 e) values given per
+// P = 2^(s * scale_log2 + nlse) for 32 consecutive fp32 scores, the (-LSE*log2 e) values given per
 // query column (from shared memory).
-__device__ __forceinline__ void probs64_cols(const uint32_t (&sv)[64], float scale_log2, const float* nlse,
-                                             float (&pr)[64]) {
+__device__ __forceinline__ void probs32_cols(const uint32_t (&sv)[32], float scale_log2, const float* nlse,
+                                             float (&pr)[32]) {
     const float2 sc = make_float2(scale_log2, scale_log2);
 #pragma unroll
-    for (int c = 0; c < 64; c += 4) {
+    for (int c = 0; c < 32; c += 4) {
         const float4 l4 = *reinterpret_cast<const float4*>(nlse + c);
         const float2 a = ptx::ffma2(make_float2(__uint_as_float(sv[c]), __uint_as_float(sv[c + 1])), sc,
                                     make_float2(l4.x, l4.y));
@@ -166,10 +168,10 @@ __device__ __forceinline__ void probs64_cols(const uint32_t (&sv)[64], float sca
         pr[c + 3] = ptx::ex2(b.y);
     }
 }
-// Zero the probabilities of columns outside [lo, hi] (column indices relative to the 64-column block).
-__device__ __forceinline__ void mask64(float (&pr)[64], int lo, int hi) {
+// Zero the probabilities of columns outside [lo, hi] (column indices relative to the 32-column block).
+__device__ __forceinline__ void mask32(float (&pr)[32], int lo, int hi) {
 #pragma unroll
-    for (int c = 0; c < 64; ++c) pr[c] = (c < lo || c > hi) ? 0.f : pr[c];
+    for (int c = 0; c < 32; ++c) pr[c] = (c < lo || c > hi) ? 0.f : pr[c];
 }
 // dS = P (dP - D) for 32 columns, packed to 16 bf16 pairs; nd holds -D per column.
 __device__ __forceinline__ void dscores32_cols(const float* pr, const uint32_t (&dp)[32], const float* nd,
@@ -198,6 +200,15 @@ __device__ __forceinline__ void stage_rows32(uint32_t blk, const uint32_t (&v)[3
 #pragma unroll
     for (int e = 0; e < 8; ++e) ptx::st_shared_v4(row ^ (e << 4), v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
 }
+// Shared address of the 32 x 32 fp32 box that stages dQ columns [32 cg, 32 cg + 32), rows
+// [32 qw, 32 qw + 32) of a query tile: the first D / 64 column groups in the Q buffer of ring stage
+// s, the rest in its dO buffer, 4 KB per box.
+template <int D>
+__device__ __forceinline__ uint32_t dq_box(int cg, int qw, const uint8_t* sQ, const uint8_t* sDO, int s) {
+    constexpr int TILE = 128 * D * 2;
+    return ptx::smem_u32(cg < D / 64 ? sQ : sDO) + s * TILE + ((cg % (D / 64)) * 4 + qw) * 4096;
+}
+
 // =============================================================================== dQ, dK, dV
 // CTA (key tile jt, K/V head g, batch b); block numbers run over key tiles slowest, so the causal
 // key tiles with the most visible queries start first. Steps t walk the visible query tiles from
@@ -218,8 +229,9 @@ __device__ __forceinline__ void stage_rows32(uint32_t blk, const uint32_t (&v)[3
 // S^T(t+1); dP^T(t+1) once the dQ(t) partial has been read out of TMEM. MMAs of one thread run in
 // issue order, so S^T(t+1) may overwrite the scores that P^T(t) was packed over once dV(t) is
 // issued. The tensor core runs S^T(t+1) while the elementwise warps move dQ(t) out, and dV(t+1)
-// while they form dS^T(t+1). S^T(t+1) comes after dQ(t) so that the next stage of the ring, which
-// the dQ reduce of two steps back holds until the TMA has read it, has that long to load.
+// while they form dS^T(t+1). The ring stage that S^T(t+1) reads is held by the dQ reduce of two
+// steps back until the TMA has read it (about 64 KB at ~20 bytes per clock per SM under load), so
+// issuing it earlier in the step gains nothing.
 template <int D>
 __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -442,14 +454,12 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
                 if (!ptx::mbar_wait(&bar->staged[s], (t >> 1) & 1, abort_flag)) { ok = false; break; }
                 const int row0 = ((b * p.Hq + h) * p.ntiles + qt) * 128;
 #pragma unroll 1
-                for (int w = 0; w < C::EW_THREADS / 32; ++w) {
-                    const uint32_t box = ptx::smem_u32((w >> 2) == 0 ? sQ : sDO) + s * C::TILE_BYTES + (w & 3) * (D / 64) * 4096;
+                for (int cg = 0; cg < D / 32; ++cg)
 #pragma unroll
-                    for (int c = 0; c < D / 64; ++c)
-                        ptx::tma_reduce_add_2d(&tm_dq, box + c * 4096, (w >> 2) * (D / 2) + 32 * c, row0 + (w & 3) * 32);
-                }
+                    for (int qw = 0; qw < 4; ++qw)
+                        ptx::tma_reduce_add_2d(&tm_dq, dq_box<D>(cg, qw, sQ, sDO, s), 32 * cg, row0 + 32 * qw);
                 ptx::bulk_commit_group();
-                ptx::bulk_wait_read_all();
+                ptx::bulk_wait_read<0>();
                 ptx::mbar_arrive(&bar->empty[s]);
             }
             ptx::bulk_wait_all();
@@ -460,98 +470,96 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         }
     } else {
         // ------------------------------------------------------------------ elementwise warps
-        const int wg = warp >> 2;                  // query columns [64 wg, 64 wg + 64) of each tile
+        const int cg = warp >> 2;                  // query columns [32 cg, 32 cg + 32) of each tile
         const int r = (warp & 3) * 32 + lane;      // TMEM lane: key row of S^T, dP^T; query row of dQ
         const int key = j0 + r;
         const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-        const uint32_t t_s = tmem + lane_base + T_S + 64 * wg, t_dp = tmem + lane_base + T_DP + 64 * wg;
-        // this thread's dS^T row: region wg, 128-byte row r, 16-byte chunk c stored at c ^ (r & 7)
-        uint4* ds_row = reinterpret_cast<uint4*>(sDS + wg * C::REGION_BYTES + r * 128);
+        const uint32_t t_s = tmem + lane_base + T_S + 32 * cg, t_dp = tmem + lane_base + T_DP + 32 * cg;
+        // this thread's dS^T row, queries [32 cg, 32 cg + 32): 128-byte row r of region cg / 2,
+        // 16-byte chunks 4 (cg & 1) + c stored at (4 (cg & 1) + c) ^ (r & 7)
+        const uint32_t ds_row = ptx::smem_u32(sDS) + (cg >> 1) * C::REGION_BYTES + r * 128;
         bool ok = true;
         for (int t = 0; ok && t < T; ++t) {
             const int s = t & 1;
-            const int qt = ie - 1 - t / G, h = g * G + t % G;
-            const int c0 = qt * 128 + 64 * wg;  // first query of this warpgroup's columns
+            const int qt = ie - 1 - t / G;
+            const int c0 = qt * 128 + 32 * cg;  // first query of this group's columns
             if (!ptx::mbar_wait(&bar->full[s], (t >> 1) & 1, abort_flag)) { ok = false; break; }
             if (!ptx::mbar_wait(&bar->s_full, t & 1, abort_flag)) { ok = false; break; }
             ptx::tc_fence_after();
-            const float* vec = sVec + s * 256 + 64 * wg;
-            float pr[64];
+            const float* vec = sVec + s * 256 + 32 * cg;
+            float pr[32];
             {
-                uint32_t sv[64];
-                ptx::tmem_ld64(t_s, sv);
-                probs64_cols(sv, p.scale_log2, vec, pr);
+                uint32_t sv[32];
+                ptx::tmem_ld32(t_s, sv);
+                probs32_cols(sv, p.scale_log2, vec, pr);
             }
             // query qpos sees this key iff qpos >= key (causal) and qpos - key < window
             const int lo = p.causal ? key - c0 : -1;
-            const int hi = p.window > 0 ? key + p.window - 1 - c0 : 64;
-            if (lo > 0 || hi < 63) mask64(pr, lo, hi);
+            const int hi = p.window > 0 ? key + p.window - 1 - c0 : 32;
+            if (lo > 0 || hi < 31) mask32(pr, lo, hi);
             {
-                uint32_t pk[32];
+                uint32_t pk[16];
 #pragma unroll
-                for (int c = 0; c < 32; ++c) pk[c] = ptx::pack_bf16x2(pr[2 * c], pr[2 * c + 1]);
-                ptx::tmem_st32(t_s, pk);
+                for (int c = 0; c < 16; ++c) pk[c] = ptx::pack_bf16x2(pr[2 * c], pr[2 * c + 1]);
+                ptx::tmem_st16(t_s, pk);
             }
             ptx::tc_fence_before();
             ptx::mbar_arrive(&bar->p_full);
             if (!ptx::mbar_wait(&bar->dp_full, t & 1, abort_flag)) { ok = false; break; }
             ptx::tc_fence_after();
             {
-                uint32_t dsk[32];
+                uint32_t dp[32], dsk[16];
+                ptx::tmem_ld32(t_dp, dp);
+                dscores32_cols(pr, dp, vec + 128, dsk);
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    uint32_t dp[32];
-                    ptx::tmem_ld32(t_dp + 32 * half, dp);
-                    dscores32_cols(pr + 32 * half, dp, vec + 128 + 32 * half, dsk + 16 * half);
-                }
-#pragma unroll
-                for (int c = 0; c < 8; ++c)
-                    ds_row[c ^ (r & 7)] = make_uint4(dsk[4 * c], dsk[4 * c + 1], dsk[4 * c + 2], dsk[4 * c + 3]);
+                for (int c = 0; c < 4; ++c)
+                    ptx::st_shared_v4(ds_row + ((((cg & 1) * 4 + c) ^ (r & 7)) << 4), dsk[4 * c], dsk[4 * c + 1],
+                                      dsk[4 * c + 2], dsk[4 * c + 3]);
             }
             ptx::fence_proxy_async_smem();
             ptx::tc_fence_before();
             ptx::mbar_arrive(&bar->ds_full);
-            // dQ partial of this step: query row qt * 128 + r, columns [wg D/2, wg D/2 + D/2). The
-            // step's Q (warpgroup 0) or dO (warpgroup 1) buffer takes it, this warp's rows as D/64
-            // boxes of 32 x 32; the TMEM columns are released once the last chunk is in registers.
+            // dQ partial of this step: query row qt * 128 + r, columns [32 cg, 32 cg + 32) for the
+            // first D / 32 groups, staged as one 32 x 32 box in the step's Q or dO buffer; the TMEM
+            // columns are released as soon as it is in registers
             if (!ptx::mbar_wait(&bar->dq_full, t & 1, abort_flag)) { ok = false; break; }
             ptx::tc_fence_after();
-            {
-                const uint32_t box = ptx::smem_u32(wg == 0 ? sQ : sDO) + s * C::TILE_BYTES + (warp & 3) * (D / 64) * 4096;
-                const uint32_t t_dq = tmem + lane_base + T_DP + wg * (D / 2);
+            if (cg < D / 32) {
                 uint32_t v[32];
-                ptx::tmem_ld32(t_dq, v);
-                stage_rows32(box, v, lane);
-                if constexpr (D == 128) ptx::tmem_ld32(t_dq + 32, v);
+                ptx::tmem_ld32(tmem + lane_base + T_DP + 32 * cg, v);
                 ptx::tc_fence_before();
                 ptx::mbar_arrive(&bar->dq_free);
-                if constexpr (D == 128) stage_rows32(box + 4096, v, lane);
+                stage_rows32(dq_box<D>(cg, warp & 3, sQ, sDO, s), v, lane);
+            } else {
+                ptx::mbar_arrive(&bar->dq_free);
             }
             ptx::fence_proxy_async_smem();
             ptx::mbar_arrive(&bar->staged[s]);
         }
+        // groups 0 and 1 write dV columns [0, D/2) and [D/2, D), groups 2 and 3 dK likewise
+        const bool is_k = cg >= 2;
+        const int col0 = (cg & 1) * (D / 2);
         if (ok && T > 0) ok = ptx::mbar_wait(&bar->acc_done, 0, abort_flag);
         if (ok && T > 0) {
-            // warpgroup 0 writes dV, warpgroup 1 dK; every lane takes part in the warp-collective
-            // TMEM loads, rows past N store nothing
+            // every lane takes part in the warp-collective TMEM loads; rows past N store nothing
             ptx::tc_fence_after();
             const size_t row = (static_cast<size_t>(b) * p.Hkv + g) * p.N + min(key, p.N - 1);
 #pragma unroll 1
-            for (int c = 0; c < D / 32; ++c) {
+            for (int c = 0; c < D / 64; ++c) {
                 uint32_t v[32];
-                ptx::tmem_ld32(tmem + lane_base + (wg == 0 ? T_DV : T_DK) + c * 32, v);
+                ptx::tmem_ld32(tmem + lane_base + (is_k ? T_DK : T_DV) + col0 + c * 32, v);
                 if (key < p.N) {
-                    if (wg == 0)
-                        store_chunk_unrotated(v, 1.f, nullptr, D, key, c * 32, p.dv + row * D);
+                    if (is_k)
+                        store_chunk_unrotated(v, p.scale, p.rope, D, key, col0 + c * 32, p.dk + row * D);
                     else
-                        store_chunk_unrotated(v, p.scale, p.rope, D, key, c * 32, p.dk + row * D);
+                        store_chunk_unrotated(v, 1.f, nullptr, D, key, col0 + c * 32, p.dv + row * D);
                 }
             }
         } else if (T == 0 && key < p.N) {
             // no query sees these keys: zero gradients
             const size_t row = (static_cast<size_t>(b) * p.Hkv + g) * p.N + key;
-            uint4* d1 = reinterpret_cast<uint4*>((wg == 0 ? p.dv : p.dk) + row * D);
-            for (int k = 0; k < D / 8; ++k) d1[k] = make_uint4(0, 0, 0, 0);
+            uint4* d1 = reinterpret_cast<uint4*>((is_k ? p.dk : p.dv) + row * D + col0);
+            for (int k = 0; k < D / 16; ++k) d1[k] = make_uint4(0, 0, 0, 0);
         }
         if (!ok) {
             *abort_flag = 1;

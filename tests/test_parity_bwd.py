@@ -81,34 +81,30 @@ def test_backward_gqa_equals_repeated_heads(cuda_api):
     kr, vr = kd.repeat_interleave(2, dim=1), vd.repeat_interleave(2, dim=1)
     o2, lse2 = cuda_api.attn_fwd(qd, kr, vr, causal=True, rope_base=10000.0)
     dq2, dk2, dv2 = cuda_api.attn_bwd(qd, kr, vr, o2, lse2, dout, causal=True, rope_base=10000.0)
-    assert bf16_ulps_apart(dq, dq2) <= 1
+    assert_same_up_to_sum_order(dq, dq2)
     for a, b in ((dk, dk2), (dv, dv2)):
         summed = b.float().reshape(1, 2, 2, 300, 128).sum(dim=2)
         assert float((a.float() - summed).abs().max()) <= 2.0 ** -7 * float(summed.abs().max())
 
 
-def bf16_ulps_apart(a, b):
-    """Largest distance between two bf16 tensors in units in the last place (same-sign ordering of
-    the bit patterns; both tensors finite)."""
-    def ordered(x):
-        i = x.view(torch.int16).to(torch.int32)
-        return torch.where(i < 0, -32768 - i, i)
-    return int((ordered(a) - ordered(b)).abs().max())
-
-
-def test_bf16_ulps_apart():
-    x = torch.tensor([1.0, -1.0, 0.0, 2.0 ** -130], dtype=torch.bfloat16)
-    nxt = torch.tensor([1.0078125, -1.0078125, 2.0 ** -133, 2.0 ** -130], dtype=torch.bfloat16)
-    assert bf16_ulps_apart(x, x) == 0
-    assert bf16_ulps_apart(x, nxt) == 1
-    assert bf16_ulps_apart(torch.tensor([2.0 ** -133], dtype=torch.bfloat16),
-                           torch.tensor([-(2.0 ** -133)], dtype=torch.bfloat16)) == 2
+def assert_same_up_to_sum_order(a, b):
+    """a and b are dq from two calls: fp32 sums of the same partials (one per key tile) in different
+    orders, rounded to bf16. Reordering moves an fp32 sum by a few 2^-24 of the partials' size, and
+    the chain rule makes each row's dS sum to zero, so partials can cancel to a result far smaller
+    than they are: the bound is one bf16 ulp of the element or 2^-16 of the largest |dq|."""
+    af, bf = a.float(), b.float()
+    tol = torch.maximum(af.abs() * 2.0 ** -7, torch.full_like(af, 2.0 ** -16 * float(af.abs().max())))
+    bad = (af - bf).abs() > tol
+    if bool(bad.any()):
+        i = int(torch.nonzero(bad.flatten())[0])
+        raise AssertionError(f"dq repeats differ at flat index {i}: {float(af.flatten()[i])} vs "
+                             f"{float(bf.flatten()[i])}, max |dq| {float(af.abs().max())}")
 
 
 def test_backward_deterministic(cuda_api):
     """Two backward calls: dK and dV are each accumulated by one CTA in a fixed order, so their bits
     repeat. dQ is a sum of fp32 partials, one per key tile, added into device memory in the order
-    the CTAs get there; repeats agree to within one bf16 unit in the last place."""
+    the CTAs get there; repeats agree up to that summation order."""
     q, k, v = (x.cuda() for x in synth.prefill_inputs(1, 8, 2, 700, 128, seed=79))
     dout = synth.randn_bf16((1, 8, 700, 128), torch.Generator().manual_seed(80)).cuda()
     o, lse = cuda_api.attn_fwd(q, k, v, causal=True, rope_base=10000.0)
@@ -116,7 +112,7 @@ def test_backward_deterministic(cuda_api):
     second = cuda_api.attn_bwd(q, k, v, o, lse, dout, causal=True, rope_base=10000.0)
     torch.cuda.synchronize()
     assert cuda_api.device_status() == 0
-    assert bf16_ulps_apart(first[0], second[0]) <= 1
+    assert_same_up_to_sum_order(first[0], second[0])
     for a, b in zip(first[1:], second[1:]):
         assert torch.equal(a.view(torch.int16), b.view(torch.int16))
 
