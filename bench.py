@@ -489,7 +489,7 @@ def run_ours(args, rank, world, local):
                "value": round(job_throughput(bwd_flops, world, bwd_ms / 1e3) / 1e12, 2), "unit": "TFLOP/s",
                "ms_per_call": round(bwd_ms, 4), "calls": args.bwd_steps, "timed_s": bwd_ms * args.bwd_steps / 1e3,
                "roofline": {"bound": "tensor", "achieved": round(bwd_flops / (bwd_ms / 1e3) / 1e12, 2),
-                            "unit": "TFLOP/s", "note": "five-kernel call: rotation pass, prep, dK/dV, dQ"}}
+                            "unit": "TFLOP/s", "note": "the whole call: rotation pass, prep, zeroing of the dq sums, the gradient kernel, the dq store"}}
         del dout, gq, gk, gv, bws
 
     # ---- position variants of the prefill workload (own loops; not part of the step)
@@ -667,8 +667,8 @@ def run_ours(args, rank, world, local):
     if bwd is not None:
         bp, bk = tensor_peak_for(peaks, peaks_kind, bwd["timed_s"])
         bwd["roofline"].update({"peak": bp, "frac": round(bwd["roofline"]["achieved"] / bp, 4), "peak_kind": bk,
-                                "traffic": profiled_traffic("attn_bwd_dkdv"),
-                                "traffic_kernel": "attn_bwd_dkdv_kernel<128> (the larger of the two backward kernels)"})
+                                "traffic": profiled_traffic("attn_bwd"),
+                                "traffic_kernel": "attn_bwd_kernel<128> (dQ, dK and dV; five products per tile pair)"})
     if fp8 is not None:
         fp, fk = tensor_peak_for(peaks, peaks_kind, fp8["timed_s"])
         fp8["roofline"].update({"peak": 2.0 * fp, "frac": round(fp8["roofline"]["achieved"] / (2.0 * fp), 4),
