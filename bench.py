@@ -489,7 +489,7 @@ def run_ours(args, rank, world, local):
                "value": round(job_throughput(bwd_flops, world, bwd_ms / 1e3) / 1e12, 2), "unit": "TFLOP/s",
                "ms_per_call": round(bwd_ms, 4), "calls": args.bwd_steps, "timed_s": bwd_ms * args.bwd_steps / 1e3,
                "roofline": {"bound": "tensor", "achieved": round(bwd_flops / (bwd_ms / 1e3) / 1e12, 2),
-                            "unit": "TFLOP/s", "note": "the whole call: rotation pass, prep, zeroing of the dq sums, the gradient kernel, the dq store"}}
+                            "unit": "TFLOP/s", "note": "the whole call: rotation pass, prep (which also zeroes the dq sums), the gradient kernel, the dq store"}}
         del dout, gq, gk, gv, bws
 
     # ---- position variants of the prefill workload (own loops; not part of the step)

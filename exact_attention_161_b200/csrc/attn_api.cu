@@ -556,8 +556,6 @@ attn_status launch_bwd(const void* q, const void* k, const void* v, const void* 
     if ((st = make_map_3d(&tdo, dout, D, N, static_cast<uint64_t>(B) * Hq, 128)) != ATTN_OK) return st;
     if ((st = make_map_2d_f32(&tdq, p.dqacc, D, static_cast<uint64_t>(B) * Hq * p.ntiles * 128)) != ATTN_OK) return st;
     if ((st = ensure_smem(attn::attn_bwd_kernel<D>, C::SMEM_BYTES, dev)) != ATTN_OK) return st;
-    // the dq sums start from zero; every (key tile, query tile) pair adds its part
-    CUDA_TRY(cudaMemsetAsync(p.dqacc, 0, static_cast<size_t>(B) * Hq * p.ntiles * 128 * D * sizeof(float), stream));
     // one-dimensional grid, key tile index slowest (the longest causal walks start first)
     const unsigned nt = static_cast<unsigned>(p.ntiles);
     attn::attn_bwd_kernel<D><<<nt * static_cast<unsigned>(B * Hkv), C::THREADS, C::SMEM_BYTES, stream>>>(

@@ -17,8 +17,8 @@
 // products of a tile pair (S^T, dP^T, dV, dK, dQ) run on tcgen05 with fp32 accumulators in Tensor
 // Memory: dK and dV accumulate there over the whole walk; the dQ of each tile pair is added into an
 // fp32 array in device memory by TMA reductions, since every key tile contributes to it.
-// Eight elementwise warps (two warpgroups, each owning 64 of the 128 query columns of a tile)
-// turn scores into P and dS and move the dQ partials out; the products are issued in an order that
+// Sixteen elementwise warps (four groups, each owning 32 of the 128 query columns of a tile) turn
+// scores into P and dS and move the dQ partials out; the products are issued in an order that
 // lets the tensor core work while they do (see the issue loop). CTAs are numbered so that the
 // ones with the most work start first.
 #pragma once
@@ -35,7 +35,7 @@ struct BwdParams {
     float* vec;                 // [B*Hq, ntiles, 2, 128]: per 128-row tile -LSE*log2 e, then -D_i;
                                 // rows >= N hold (-inf, 0)
     __nv_bfloat16* dq;          // [B, Hq, N, D]
-    float* dqacc;               // [B*Hq, ntiles*128, D] fp32 sums of dS K, zeroed before the main kernel
+    float* dqacc;               // [B*Hq, ntiles*128, D] fp32 sums of dS K, zeroed by the prep kernel
     __nv_bfloat16* dk;          // [B, Hkv, N, D]
     __nv_bfloat16* dv;          // [B, Hkv, N, D]
     const float2* rope;         // (cos, sin) table or nullptr
@@ -45,8 +45,9 @@ struct BwdParams {
 };
 
 // Per query row: -D_i = -(dO_i . O_i) and -LSE_i * log2(e), stored negated so that the kernels add
-// them. D/8 lanes share a row (16-byte loads), grid-stride over all padded rows; rows past N get
-// (-inf, 0) so that their recomputed probabilities are exactly 0.
+// them, and the row's fp32 dq sums set to zero. D/8 lanes share a row (16-byte loads), grid-stride
+// over all padded rows; rows past N get (-inf, 0) so that their recomputed probabilities are
+// exactly 0.
 template <int D>
 __global__ void __launch_bounds__(256) bwd_prep_kernel(const BwdParams p) {
     constexpr int LPR = D / 8;     // lanes per row
@@ -72,6 +73,11 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const BwdParams p) {
                 acc = fmaf(ptx::bf16lo_to_f32(aw[e]), ptx::bf16lo_to_f32(bw[e]), acc);
                 acc = fmaf(ptx::bf16hi_to_f32(aw[e]), ptx::bf16hi_to_f32(bw[e]), acc);
             }
+        }
+        if (row < rows) {
+            float4* z = reinterpret_cast<float4*>(p.dqacc + static_cast<size_t>(row) * D + l * 8);
+            z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+            z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
         }
 #pragma unroll
         for (int m = LPR / 2; m >= 1; m >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, m);
@@ -216,7 +222,7 @@ __device__ __forceinline__ uint32_t dq_box(int cg, int qw, const uint8_t* sQ, co
 // tile's walk starts at the same query tile, so the CTAs of one K/V head that run side by side read
 // each Q and dO tile at about the same time, and the repeats come from L2.
 //
-// TMEM: S^T at 0 (P^T packed into columns 0-31 and 64-95), dP^T at 128, which also takes the dQ
+// TMEM: S^T at 0 (P^T packed into the first 16 of every 32 columns), dP^T at 128, which takes the dQ
 // partial of the step once dS^T has been formed, dV at 256, dK at 256 + D. Shared memory holds dS^T
 // once per step (keys as 128-byte swizzled rows, queries along them); dK reads it K-major as
 // dS^T and dQ reads the same bytes MN-major as dS. The dQ partial (128 x D fp32) leaves through the
