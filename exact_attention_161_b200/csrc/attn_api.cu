@@ -337,6 +337,7 @@ attn_status launch_fwd(const void* q, const void* k, const void* v, void* o, flo
     p.scale_log2 = scale * attn::kLog2e;
     p.nblk = (N + C::QT * C::BM - 1) / (C::QT * C::BM);
     p.n_items = B * Hq * p.nblk;
+    p.debug_drop_copy = g_debug_drop_copy.load() ? 1 : 0;
     int sms = 148;
     CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
     const int grid = p.n_items < sms ? p.n_items : sms;  // persistent: one CTA per SM
@@ -388,6 +389,7 @@ attn_status launch_fwd_fp8(const void* q, const void* k, const void* v, void* o,
     p.scale_log2 = scale * attn::kLog2e;
     p.nblk = (N + C::QT * C::BM - 1) / (C::QT * C::BM);
     p.n_items = B * Hq * p.nblk;
+    p.debug_drop_copy = g_debug_drop_copy.load() ? 1 : 0;
     int sms = 148;
     CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
     const int grid = p.n_items < sms ? p.n_items : sms;
@@ -523,6 +525,7 @@ attn_status launch_bwd(const void* q, const void* k, const void* v, const void* 
     p.window = window > 0 ? window : 0;
     p.scale = scale;
     p.scale_log2 = scale * attn::kLog2e;
+    p.debug_drop_copy = g_debug_drop_copy.load() ? 1 : 0;
     int sms = 148;
     CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
     const void* q_use = q;

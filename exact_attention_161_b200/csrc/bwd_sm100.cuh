@@ -42,6 +42,7 @@ struct BwdParams {
     int B, Hq, Hkv, N, ntiles;
     int causal, window;
     float scale, scale_log2;
+    int debug_drop_copy;        // test hook: CTA 0 skips its first Q / dO copy (see attn.h)
 };
 
 // Per query row: -D_i = -(dO_i . O_i) and -LSE_i * log2(e), stored negated so that the kernels add
@@ -312,14 +313,16 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
                 const int qt = ie - 1 - t / G, h = g * G + t % G;
                 const int zq = b * p.Hq + h;
                 ptx::mbar_arrive_expect_tx(&bar->full[s], 2 * C::TILE_BYTES + C::VEC_BYTES);
-                for (int r = 0; r < C::NREG; ++r) {
-                    ptx::tma_load_3d(sQ + s * C::TILE_BYTES + r * C::REGION_BYTES, &tm_q, &bar->full[s], r * 64,
-                                     qt * 128, zq);
-                    ptx::tma_load_3d(sDO + s * C::TILE_BYTES + r * C::REGION_BYTES, &tm_do, &bar->full[s], r * 64,
-                                     qt * 128, zq);
+                if (!(p.debug_drop_copy && t == 0 && blockIdx.x == 0)) {
+                    for (int r = 0; r < C::NREG; ++r) {
+                        ptx::tma_load_3d(sQ + s * C::TILE_BYTES + r * C::REGION_BYTES, &tm_q, &bar->full[s], r * 64,
+                                         qt * 128, zq);
+                        ptx::tma_load_3d(sDO + s * C::TILE_BYTES + r * C::REGION_BYTES, &tm_do, &bar->full[s], r * 64,
+                                         qt * 128, zq);
+                    }
+                    ptx::bulk_load(sVec + s * 256, p.vec + (static_cast<size_t>(zq) * p.ntiles + qt) * 256,
+                                   C::VEC_BYTES, &bar->full[s]);
                 }
-                ptx::bulk_load(sVec + s * 256, p.vec + (static_cast<size_t>(zq) * p.ntiles + qt) * 256, C::VEC_BYTES,
-                               &bar->full[s]);
                 issued = t + 1;
             }
             if (!ok) {

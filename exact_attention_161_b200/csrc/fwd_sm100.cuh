@@ -48,6 +48,7 @@ struct FwdParams {
     float scale_log2;       // softmax scale * log2(e)
     int nblk;               // 256-query blocks per (batch, head)
     int n_items;            // B * Hq * nblk work items
+    int debug_drop_copy;    // test hook: CTA 0 skips its first key-tile copy (see attn.h)
 };
 
 template <int D, bool kFp8 = false>
@@ -234,10 +235,12 @@ __global__ void __launch_bounds__(FwdCfg<D, kFp8>::THREADS, 1)
                     const int sk = g % NK, sv = g % NV;
                     if (g >= NK && !ptx::mbar_wait(&bar->k_empty[sk], ((g / NK) - 1) & 1, abort_flag)) { ok = false; break; }
                     ptx::mbar_arrive_expect_tx(&bar->k_full[sk], C::TILE_BYTES);
+                    if (!(p.debug_drop_copy && g == 0 && blockIdx.x == 0)) {
 #pragma unroll
-                    for (int r = 0; r < C::NREG; ++r)
-                        ptx::tma_load_3d(sK + sk * C::TILE_BYTES + r * C::REGION_BYTES, &tm_k, &bar->k_full[sk],
-                                         r * C::TMA_X, k0, zk);
+                        for (int r = 0; r < C::NREG; ++r)
+                            ptx::tma_load_3d(sK + sk * C::TILE_BYTES + r * C::REGION_BYTES, &tm_k, &bar->k_full[sk],
+                                             r * C::TMA_X, k0, zk);
+                    }
                     k_issued = g + 1;
                     if (g >= NV && !ptx::mbar_wait(&bar->v_empty[sv], ((g / NV) - 1) & 1, abort_flag)) { ok = false; break; }
                     ptx::mbar_arrive_expect_tx(&bar->v_full[sv], C::TILE_BYTES);

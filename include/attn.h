@@ -289,12 +289,14 @@ attn_status attn_get_device_status(void* stream, int* flags_out);
 
 /*
  * attn_debug_drop_copy -- test hook for the timeout path (not for production use). While enabled,
- * the paged-decode split kernel's first CTA sets up its first page copy but never issues it, so
- * that stage's bounded wait (about 2 s of SM clocks) runs out: the CTA raises
- * ATTN_DEVICE_TIMEOUT in the device status word, drains its own copies, and returns; the call's
- * output for that chunk is then undefined. No memory outside the inputs is touched and the CUDA
- * context stays usable. Applies to calls launched while enabled (attn_decode_paged,
- * attn_decode_paged_noalloc, attn_decode_step).
+ * the first CTA of a kernel sets up one copy but never issues it: its first page copy in the
+ * paged-decode split kernel (attn_decode_paged, attn_decode_paged_noalloc, attn_decode_step), its
+ * first key-tile copy in the prefill kernel (attn_fwd, attn_fwd_pos, attn_fwd_fp8), its first
+ * query/dO copy in the backward's main kernel (attn_bwd). The bounded wait on that copy (about
+ * 2 s of SM clocks) runs out: the CTA raises ATTN_DEVICE_TIMEOUT in the device status word, drains
+ * its own copies and products, and returns; the outputs that CTA owns are then undefined. No
+ * memory outside the call's buffers is touched and the CUDA context stays usable. Applies to
+ * calls launched while enabled.
  */
 void attn_debug_drop_copy(int enable);
 
