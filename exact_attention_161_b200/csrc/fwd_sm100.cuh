@@ -158,7 +158,7 @@ __global__ void __launch_bounds__(FwdCfg<D, kFp8>::THREADS, 1)
     using C = FwdCfg<D, kFp8>;
     constexpr int NK = C::NK, NV = C::NV;
     // the exponential pair of columns 6-7 of every kPolyEvery-th group of 8 is evaluated on the FMA
-    // pipe (0: none)
+    // pipe (0: none); FP8 also moves the pair of columns 4-5 of every second group there
     constexpr int kPolyEvery = kFp8 ? ATTN_FP8_POLY_EVERY : ATTN_BF16_POLY_EVERY;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -472,16 +472,21 @@ __global__ void __launch_bounds__(FwdCfg<D, kFp8>::THREADS, 1)
                     float2 x3 = ptx::ffma2(make_float2(s[k + 6], s[k + 7]), sl2, a3);
                     x0 = make_float2(ptx::ex2(x0.x), ptx::ex2(x0.y));
                     x1 = make_float2(ptx::ex2(x1.x), ptx::ex2(x1.y));
-                    x2 = make_float2(ptx::ex2(x2.x), ptx::ex2(x2.y));
-                    // One exponential pair of some groups of 8 columns goes to the FMA pipe, which
-                    // the softmax leaves mostly idle while the SFU is busy: every second group for
-                    // bf16 (1/8 of the exponentials), every group for FP8, whose SFU also packs P
-                    // to e4m3 (1/4). Larger shares measured slower. The polynomial's 1e-4 relative
-                    // error is far below the rounding of P to bf16 or e4m3; it gives exactly 1 at 0
-                    // and exactly 0 for masked scores.
+                    // Some exponential pairs go to the FMA pipe, which the softmax leaves mostly idle
+                    // while the SFU is busy. bf16: columns 6-7 of every second group of 8 (1/8 of
+                    // the exponentials), one lane at a time (the packed form's extra registers
+                    // spill there). FP8, whose SFU also packs P to e4m3 and whose P takes fewer
+                    // registers: columns 6-7 of every group and 4-5 of every second one (3/8), on
+                    // packed f32x2 instructions. Shares of 1/4, 5/16, 7/16 and 1/2 measured slower
+                    // for FP8. The polynomial's 1e-4 relative error is far below the rounding of P
+                    // to bf16 or e4m3; it gives exactly 1 at 0 and exactly 0 for masked scores.
+                    if (kFp8 && (k / 8) % 2 == 0) x2 = ptx::ex2_poly2(x2);
+                    else x2 = make_float2(ptx::ex2(x2.x), ptx::ex2(x2.y));
                     if constexpr (kPolyEvery > 0) {
-                        if ((k / 8) % kPolyEvery == 0) x3 = ptx::ex2_poly2(x3);
-                        else x3 = make_float2(ptx::ex2(x3.x), ptx::ex2(x3.y));
+                        if ((k / 8) % kPolyEvery == 0)
+                            x3 = kFp8 ? ptx::ex2_poly2(x3) : make_float2(ptx::ex2_poly(x3.x), ptx::ex2_poly(x3.y));
+                        else
+                            x3 = make_float2(ptx::ex2(x3.x), ptx::ex2(x3.y));
                     } else {
                         x3 = make_float2(ptx::ex2(x3.x), ptx::ex2(x3.y));
                     }

@@ -460,7 +460,20 @@ __device__ __forceinline__ float ex2_poly(float x) {
     q = fmaf(q, f, 1.f);
     return __int_as_float(__float_as_int(q) + (__float_as_int(t) << 23));
 }
-__device__ __forceinline__ float2 ex2_poly2(float2 x) { return make_float2(ex2_poly(x.x), ex2_poly(x.y)); }
+// The same for a pair, with the fp32 steps on packed f32x2 instructions (each lane rounds exactly as
+// the scalar version does, so the results are identical): x - round(x) as fma(round(x), -1, x),
+// the exact difference rounded once, as the scalar subtraction does.
+__device__ __forceinline__ float2 ex2_poly2(float2 x) {
+    x = make_float2(fmaxf(x.x, -127.f), fmaxf(x.y, -127.f));
+    const float2 t = fadd2(x, make_float2(12582912.f, 12582912.f));
+    const float2 rx = fadd2(t, make_float2(-12582912.f, -12582912.f));
+    const float2 f = ffma2(rx, make_float2(-1.f, -1.f), x);
+    float2 q = ffma2(make_float2(0x1.c2a15cp-5f, 0x1.c2a15cp-5f), f, make_float2(0x1.f00bfep-3f, 0x1.f00bfep-3f));
+    q = ffma2(q, f, make_float2(0x1.62f5fap-1f, 0x1.62f5fap-1f));
+    q = ffma2(q, f, make_float2(1.f, 1.f));
+    return make_float2(__int_as_float(__float_as_int(q.x) + (__float_as_int(t.x) << 23)),
+                       __int_as_float(__float_as_int(q.y) + (__float_as_int(t.y) << 23)));
+}
 
 // max(a, b, c) in one instruction (sm_100a).
 __device__ __forceinline__ float fmax3(float a, float b, float c) {

@@ -23,6 +23,16 @@ def shipped_coefficients():
     return c1, c2, c3
 
 
+def test_packed_pair_uses_the_same_coefficients():
+    # ex2_poly2 (FP8's pairs on f32x2 instructions) must evaluate the same polynomial
+    src = open(PTX).read()
+    body = src[src.index("float2 ex2_poly2(float2 x)"):]
+    body = body[:body.index("\n}")]
+    hexf = [float.fromhex(h) for h in re.findall(r"(0x1\.[0-9a-f]+p-?\d+)f", body)]
+    c1, c2, c3 = shipped_coefficients()
+    assert sorted(set(hexf)) == sorted({c1, c2, c3}), (hexf, (c1, c2, c3))
+
+
 def lawson_fit(deg=3, iters=200):
     f = np.linspace(-0.5, 0.5, 20001)
     y = 2.0 ** f
