@@ -34,6 +34,8 @@ CASES = [
     (1, 2, 1, 1, 64, 1, 0, 10000.0),
     (1, 4, 2, 640, 128, 0, 0, 10000.0),
     (4, 16, 16, 2048, 128, 1, 0, 10000.0),  # the N=2048 MHA workload's shape
+    (1, 4, 2, 700, 64, 1, 200, 10000.0),    # D = 64 through the dQ drain's two column groups, window
+    (2, 8, 2, 520, 64, 0, 0, 500000.0),     # D = 64, non-causal, 4 query heads per K/V head
 ]
 
 
