@@ -174,12 +174,18 @@ class ClockSampler:
 
 
 class NvmlSampler:
-    """SM clock samples from NVML every few milliseconds in a thread, for timed regions that are
-    too short for nvidia-smi's interval."""
+    """SM clock and clock-event (throttle) reasons from NVML every millisecond in a thread, for
+    timed regions that are too short for nvidia-smi's interval."""
 
-    def __init__(self, device_index, interval_s=0.005):
+    REASONS = (("nvmlClocksEventReasonSwPowerCap", "sw_power_cap"),
+               ("nvmlClocksEventReasonHwSlowdown", "hw_slowdown"),
+               ("nvmlClocksEventReasonHwThermalSlowdown", "hw_thermal_slowdown"),
+               ("nvmlClocksEventReasonSwThermalSlowdown", "sw_thermal_slowdown"),
+               ("nvmlClocksEventReasonHwPowerBrakeSlowdown", "hw_power_brake_slowdown"))
+
+    def __init__(self, device_index, interval_s=0.001):
         self.device_index, self.interval_s = device_index, interval_s
-        self.samples, self.thread, self.stop_flag = [], None, False
+        self.samples, self.reason_bits, self.thread, self.stop_flag = [], 0, None, False
 
     def start(self):
         try:
@@ -192,15 +198,30 @@ class NvmlSampler:
 
         def run():
             import pynvml
+            # the reasons query has two names across NVML versions; a driver may support neither
+            reason_fns = [getattr(pynvml, f) for f in ("nvmlDeviceGetCurrentClocksEventReasons",
+                                                        "nvmlDeviceGetCurrentClocksThrottleReasons")
+                          if hasattr(pynvml, f)]
             while not self.stop_flag:
                 try:
                     self.samples.append(pynvml.nvmlDeviceGetClockInfo(handle, pynvml.NVML_CLOCK_SM))
                 except Exception:
                     return
+                while reason_fns:
+                    try:
+                        self.reason_bits |= int(reason_fns[0](handle))
+                        break
+                    except Exception:
+                        reason_fns.pop(0)
                 time.sleep(self.interval_s)
 
         self.thread = threading.Thread(target=run, daemon=True)
         self.thread.start()
+
+    def reasons(self):
+        import pynvml
+        return sorted(label for attr, label in self.REASONS
+                      if hasattr(pynvml, attr) and self.reason_bits & int(getattr(pynvml, attr)))
 
     def stop(self):
         if self.thread is None:
@@ -210,7 +231,7 @@ class NvmlSampler:
         if not self.samples:
             return None
         return {"sm_mhz_median": statistics.median(self.samples), "sm_mhz_min": min(self.samples),
-                "samples": len(self.samples), "interval_ms": self.interval_s * 1e3}
+                "samples": len(self.samples), "interval_ms": self.interval_s * 1e3, "reasons": self.reasons()}
 
 
 def tensor_peak_for(peaks, peaks_kind, timed_s):
@@ -409,6 +430,8 @@ def run_ours(args, rank, world, local):
     clk = clocks.stop()
     if clk is not None and nvml_clk is not None:
         clk["nvml"] = nvml_clk
+        # the reasons either sampler saw during the timed region
+        clk["reasons"] = sorted(set(clk.get("reasons", [])) | set(nvml_clk.get("reasons", [])))
     total_ms = t_start.elapsed_time(t_end)
     prefill_ms = [ev[s][0].elapsed_time(ev[s][1]) for s in range(K)]
     decode_ms = [ev[s][1].elapsed_time(ev[s][2]) for s in range(K)]
