@@ -120,6 +120,48 @@ def test_rope_pass_rotates_exactly(cuda_api, D, half, ps, ntk):
     assert torch.equal(o1.view(torch.int16), o2.view(torch.int16)) and torch.equal(l1, l2)
 
 
+def _with_special_values(x, seed):
+    """x with a seeded share of its entries replaced by signed zeros (10%), bf16 subnormals (5%) and
+    normals of 2^-126 to 2^-120 (5%), whose rotations round into the bf16 subnormal range."""
+    rng = np.random.default_rng(seed)
+    b = bits(x).copy()
+    u = rng.random(b.shape)
+    sign = (rng.integers(0, 2, b.shape) << 15).astype(np.uint16)
+    sub = rng.integers(1, 0x80, b.shape).astype(np.uint16)
+    tiny = ((rng.integers(1, 8, b.shape) << 7) | rng.integers(0, 0x80, b.shape)).astype(np.uint16)
+    b = np.where(u < 0.10, sign, b)
+    b = np.where((u >= 0.10) & (u < 0.15), sign | sub, b)
+    b = np.where((u >= 0.15) & (u < 0.20), sign | tiny, b)
+    return torch.from_numpy(b.view(np.int16)).view(torch.bfloat16)
+
+
+@pytest.mark.parametrize("half", [False, True])
+def test_rope_pass_rotates_special_values_exactly(cuda_api, half):
+    """The rotation pass on signed zeros, subnormal inputs and results that round to subnormals
+    (the paths that leave the field-moving conversions) still equals the oracle's rotation bit for
+    bit, checked as in the test above."""
+    B, Hq, Hkv, N, D, base = 1, 2, 1, 200, 128, 10000.0
+    q, k, v = synth.prefill_inputs(B, Hq, Hkv, N, D, seed=524)
+    q, k = _with_special_values(q, 1), _with_special_values(k, 2)
+    perm = torch.stack([torch.arange(D // 2), torch.arange(D // 2) + D // 2], 1).reshape(-1)
+
+    def rotated(x):
+        rows = bits(x).reshape(-1, D)
+        pos = np.tile(np.arange(N, dtype=np.int64), rows.shape[0] // N)
+        r = oracle.rope_bf16_ex(rows, pos, base, half_split=half)
+        t = torch.from_numpy(np.ascontiguousarray(r).view(np.int16)).view(torch.bfloat16).reshape(x.shape)
+        return t[..., perm].contiguous() if half else t
+
+    qr = bits(rotated(q))
+    subnormal = ((qr & 0x7F80) == 0) & ((qr & 0x7F) != 0)
+    assert np.count_nonzero(subnormal) > 0.005 * qr.size and np.count_nonzero((qr & 0x7FFF) == 0) > 0
+    o1, l1 = _gpu(cuda_api, q, k, v, (B, Hq, Hkv, N, D, 1, 0, base, half, 1.0, 1.0, False))
+    o2, l2 = cuda_api.attn_fwd(rotated(q).cuda(), rotated(k).cuda(), v.cuda(), causal=True, rope_base=0.0)
+    torch.cuda.synchronize()
+    assert cuda_api.device_status() == 0
+    assert torch.equal(o1.view(torch.int16), o2.view(torch.int16)) and torch.equal(l1, l2)
+
+
 def test_alibi_full_size_all_rows(cuda_api):
     """ALiBi (with half-split RoPE and NTK scaling) on the GQA causal N=8192 workload, every row."""
     cfg = synth.GQA_CAUSAL_N8192
