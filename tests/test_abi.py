@@ -3,6 +3,7 @@ declares, and rejects bad arguments before any CUDA call (no compute call is mad
 import ctypes
 import os
 import re
+import subprocess
 
 import pytest
 
@@ -175,3 +176,45 @@ def test_decode_step_workspace_size(api):
 
 def test_device_status_needs_out_pointer(api):
     assert api.lib.attn_get_device_status(None, None) == 1
+
+
+def test_header_is_plain_c_and_a_c_program_links(api, tmp_path):
+    """include/attn.h compiles as strict C99 on its own (no CUDA or C++ header needed), and a C
+    program built against it links with the library, finds every declared function and gets the
+    documented answers from the calls that need no GPU: the version string, a null-pointer
+    rejection with its message, and the workspace sizes the Python binding also reports."""
+    table = ",\n    ".join("(fn)%s" % f for f in declared_functions())
+    src = tmp_path / "use_attn.c"
+    src.write_text("""#include "attn.h"
+#include <stdio.h>
+#include <string.h>
+typedef void (*fn)(void);
+static const fn every_entry_point[] = {
+    %s
+};
+int main(void) {
+    size_t i;
+    for (i = 0; i < sizeof every_entry_point / sizeof every_entry_point[0]; ++i)
+        if (!every_entry_point[i]) return 10;
+    if (!strstr(attn_version(), "sm_100a")) return 11;
+    if (attn_fwd(NULL, NULL, NULL, NULL, NULL, 1, 1, 1, 128, 64, 1, 0, 0.f, 0.f, NULL) != ATTN_ERR_INVALID_ARG)
+        return 12;
+    if (attn_last_error()[0] == 0) return 13;
+    printf("%%zu %%zu %%zu\\n", attn_bwd_workspace_size(2, 32, 8, 8192, 128, 5e5f),
+           attn_decode_workspace_size(64, 1024, 16, 32, 128),
+           attn_decode_step_workspace_size(64, 4, 1024, 16, 32, 128));
+    return 0;
+}
+""" % table)
+    exe = tmp_path / "use_attn"
+    lib_dir = os.path.dirname(api.LIB_PATH)
+    lib_name = os.path.basename(api.LIB_PATH)
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I",
+                    os.path.join(ROOT, "include"), str(src), "-o", str(exe), "-L", lib_dir,
+                    "-l:" + lib_name, "-Wl,-rpath," + lib_dir], check=True)
+    run = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert run.returncode == 0, (run.returncode, run.stderr)
+    sizes = [int(x) for x in run.stdout.split()]
+    assert sizes == [api.bwd_workspace_size(2, 32, 8, 8192, 128, 5e5),
+                     api.decode_workspace_size(64, 1024, 16, 32, 128),
+                     api.decode_step_workspace_size(64, 4, 1024, 16, 32, 128)]
