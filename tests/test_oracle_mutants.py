@@ -46,6 +46,17 @@ MUTANTS = {
     "e4m3_bias": ("v = ldexp(1.0 + (double)m / 8.0, e - 7);", "v = ldexp(1.0 + (double)m / 8.0, e - 8);"),
     "e4m3_subnormal": ("v = ldexp((double)m, -9);", "v = ldexp((double)m, -10);"),
     "normaliser_missing": ("for (int d = 0; d < D; ++d) o[d] /= l;", "for (int d = 0; d < D; ++d) o[d] /= (l + 1e-3);"),
+    "bwd_dv_uses_ds": ("my_dv[(size_t)j * D + d] += p * dO[d];", "my_dv[(size_t)j * D + d] += ds * dO[d];"),
+    "bwd_dp_uses_keys": ("dp[j] += dO[d] * vv[(size_t)j * D + d];", "dp[j] += dO[d] * kk[(size_t)j * D + d];"),
+    "bwd_p_unnormalised": ("for (int j = 0; j < N; ++j) s_row[j] /= lsum;", "for (int j = 0; j < N; ++j) s_row[j] /= 1.0;"),
+    "bwd_dk_not_rotated_back": ("rope_row_f64(dk_rot + (size_t)j * D, D, j, rope_base, 1, 0,",
+                                "rope_row_f64(dk_rot + (size_t)j * D, D, j, rope_base, 0, 0,"),
+    "bwd_row_term_unweighted": ("dsum += s_row[j] * dp[j];", "dsum += dp[j];"),
+    "bwd_gqa_interleaved_heads": ("const int h = g * G + r / N, i = r % N;", "const int h = g + (r / N) * Hkv, i = r % N;"),
+    "decode_block_table_skipped": ("int32_t pg = block_table[(size_t)s * max_blocks + t / page_size];",
+                                   "int32_t pg = (int32_t)((t / page_size) % num_pages);"),
+    "decode_cache_layout_head_major": ("(((size_t)pg * Hkv + g) * page_size", "(((size_t)g * num_pages + pg) * page_size"),
+    "decode_gqa_interleaved_heads": ("int h = g * G + hh;", "int h = hh * Hkv + g;"),
 }
 
 
