@@ -77,3 +77,27 @@ def test_peak_choice_follows_the_timed_region():
     assert p == 1379.5 and "sustained" in kind
     p, kind = bench.tensor_peak_for({"bf16_tflops": 1590.0, "hbm_gbs": 6650.0}, "fallback", 5.0)
     assert p == 1590.0
+
+
+def test_reference_arm_line(capsys):
+    """`--impl reference` (the fp64 oracle on the host cores) prints one JSON line with the
+    contract's keys, its e2e and cpu_baseline equal to its own value, and no host<->device bytes."""
+    import json
+    bench.main(["--impl", "reference", "--steps", "1", "--warmup", "3"])
+    lines = [ln for ln in capsys.readouterr().out.splitlines() if ln.strip()]
+    assert len(lines) == 1
+    line = json.loads(lines[0])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better", "scaling",
+                "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in line, key
+    assert line["impl"] == "reference" and line["n_gpus"] == 1 and line["steps"] == 1 and line["warmup"] == 3
+    assert line["value"] > 0 and line["higher_is_better"] is True and line["unit"] == "TFLOP/s"
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
+    assert line["cpu_baseline"]["cores"] >= 1 and line["cpu_baseline"]["sample"]
+    assert line["e2e"] == {"value": line["value"], "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+
+
+def test_reference_arm_other_ranks_do_no_work():
+    """Under torchrun only rank 0 runs the oracle and prints; the other ranks return at once."""
+    args = bench.parse_args(["--impl", "reference", "--steps", "1", "--warmup", "3"])
+    assert bench.run_reference(args, rank=1, world=2) is None
